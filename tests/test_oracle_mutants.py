@@ -1,0 +1,57 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case plants one mistake in a copy of oracle.c (a dropped term, a wrong
+sign or index, a transposed operand, a different rounding rule), builds it on
+the CPU, and runs the pin suites against that copy in a subprocess: the suites
+must fail.  The oracle itself is never modified.
+"""
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "oracle.c")
+
+MUTANTS = {
+    "rmsnorm_no_eps": ("ss / (double)n + RMS_EPS", "ss / (double)n"),
+    "rmsnorm_sum_not_mean": ("sqrt(ss / (double)n + RMS_EPS)", "sqrt(ss + RMS_EPS)"),
+    "matvec_transposed": ("v += (double)row[j] * (double)x[j];", "v += (double)W[(size_t)j * d + i] * (double)x[j];"),
+    "rope_sign": ("v[i] = (float)(a * c - b * s);", "v[i] = (float)(a * c + b * s);"),
+    "rope_freq_index": ("orc_rope_freq(i % head_size, head_size)", "orc_rope_freq(i, head_size)"),
+    "attn_no_scale": ("att[t] = s * scale;", "att[t] = s;"),
+    "gqa_mapping": ("int g = h / rep;", "int g = h % n_kv_heads;"),
+    "silu_sign": ("return z / (1.0 + exp(-z));", "return z / (1.0 + exp(z));"),
+    "quant_round_half_even": ("q[g * gs + i] = (int8_t)round((double)quot);", "q[g * gs + i] = (int8_t)rint((double)quot);"),
+    "quant_scale_128": ("float scale = wmax / 127.0f;", "float scale = wmax / 128.0f;"),
+    "q80_drop_sx": ("vd += (double)ival * (double)srow[g] * (double)sx[g];", "vd += (double)ival * (double)srow[g];"),
+    "no_attn_residual": ("for (int i = 0; i < d; i++) x[i] += m->xb2[i];", "for (int i = 0; i < d; i++) x[i] = m->xb2[i];"),
+    "no_rope_on_k": ("orc_rope(k, kvd, hs, pos);", ""),
+    "argmax_last_tie": ("if (x[i] > x[best]) best = i;", "if (x[i] >= x[best]) best = i;"),
+    "wrong_norm_weight": ("orc_rmsnorm(m->xb, x, m->w_att + l * d, d);", "orc_rmsnorm(m->xb, x, m->w_ffn + l * d, d);"),
+    "swiglu_operands_swapped": ("orc_swiglu(m->hb, m->hb2, h);", "orc_swiglu(m->hb2, m->hb, h); memcpy(m->hb, m->hb2, sizeof(float) * (size_t)h);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name):
+    find, repl = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(find) == 1, f"mutation anchor not found once: {find}"
+    with tempfile.TemporaryDirectory() as td:
+        msrc = os.path.join(td, "oracle.c")
+        with open(msrc, "w") as f:
+            f.write(src.replace(find, repl))
+        with open(os.path.join(td, "oracle.h"), "w") as f:
+            f.write(open(os.path.join(ROOT, "oracle", "oracle.h")).read())
+        so = os.path.join(td, "liboracle_mutant.so")
+        subprocess.check_call(["gcc", *oracle.CFLAGS, "-o", so, msrc, "-lm"])
+        env = dict(os.environ, ORACLE_LIB_PATH=so, OMP_NUM_THREADS="2")
+        r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                            "tests/test_oracle_pins.py", "tests/test_oracle_forward.py"],
+                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+        assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
