@@ -1,0 +1,421 @@
+"""Decode throughput of the B200 decode-step library on the 7B-shape Llama-2 workload.
+
+One step = six single-token decode steps through the C ABI: the fp32 path and
+the Q8_0 (GS=64) path, each at positions 0, 512 and 2048 of a KV cache
+prefilled with N(0,1), token 1 (dim 4096, hidden 11008, 32 layers, 32 heads,
+32 KV heads, vocab 32000, seq_len 4096, untied classifier, weights N(0,0.02)
+from seed 3; both weight sets resident).  value = tokens decoded per second,
+timed on the device with CUDA events between barriers, max over ranks.  Each
+rank (one per GPU) runs an independent replica: batch-1 decode does not shard.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+SPEC = synth.L7B  # --layers N swaps in the same widths with N layers (small profiling case)
+GS = 64
+POSITIONS = (0, 512, 2048)
+TOKEN = 1
+METRIC = "decode tokens/s at batch 1 (fp32 & Q8_0) on 1 B200; achieved HBM GB/s vs peak"
+UNIT = "tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------ byte accounting --
+
+def bytes_per_token(q80: bool, pos: int, spec=None, gs=GS) -> float:
+    """Algorithmic bytes of one decode step: every weight once, the KV cache for
+    positions 0..pos (K and V, fp32), the embedding row; activations ignored."""
+    d, h, L, H, Hkv, V, S = (spec or SPEC).cfg
+    kvd = Hkv * (d // H)
+    kv = 8.0 * L * (pos + 1) * kvd
+    mats = L * (2 * d * d + 2 * d * kvd + 3 * d * h) + V * d
+    if not q80:
+        return 4.0 * (mats + L * 2 * d + d + d) + kv
+    return (1 + 4.0 / gs) * (mats + d) + 4.0 * (2 * L * d + d) + kv
+
+
+def w13_bytes(q80: bool, spec=None, gs=GS) -> float:
+    """Algorithmic bytes of one W1/W3 launch: both weight matrices, the RMSNorm
+    gain, the input x and the output hb."""
+    spec = spec or SPEC
+    d, h = spec.dim, spec.hidden_dim
+    w = 2 * h * d * (1 + 4.0 / gs) if q80 else 2 * h * d * 4.0
+    return w + 4.0 * (2 * d + h)
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_record(kernel_key: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the kernel source as it is now (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    src = os.path.join(ROOT, "decode_llama_step_02_b200", "csrc", "kernels.cuh")
+    try:
+        rec = json.load(open(p))
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+        if rec.get("kernels_cuh_sha256") != sha:
+            return None
+        return rec["kernels"][kernel_key]["dram_bytes_per_launch_full"]
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ------------------------------------------------------------------ setup ----
+
+def device_blob(torch, spec=None, chunk=1 << 27):
+    """The seeded fp32 blob generated on the host in chunks and uploaded."""
+    spec = spec or SPEC
+    n = synth.blob_floats(spec)
+    dev = torch.empty(n, dtype=torch.float32, device="cuda")
+    host = torch.empty(chunk, dtype=torch.float32).pin_memory()
+    hn = host.numpy()
+    for s in range(0, n, chunk):
+        m = min(chunk, n - s)
+        synth.blob_into(spec, hn[:m], start=s)
+        dev[s:s + m].copy_(host[:m], non_blocking=False)
+    return dev
+
+
+def make_decoder(torch, l2c):
+    blob = device_blob(torch)
+    dec = l2c.Decoder(SPEC.cfg, blob, SPEC.shared_weights)
+    del blob
+    torch.cuda.empty_cache()
+    dec.enable_q80(GS)
+    k, v = synth.kv_prefill(SPEC, seq=0, n_pos=max(POSITIONS))
+    dec.kv_load(k, v)
+    del k, v
+    return dec
+
+
+def one_step(dec):
+    for q80 in (False, True):
+        for p in POSITIONS:
+            dec.forward_ptr(TOKEN, p, q80)
+
+
+# ----------------------------------------------------------- CPU oracle ------
+
+def oracle_sample(q80_also=True, pos=512):
+    """Seconds per token of the CPU oracle on the 7B-shape model at `pos`:
+    one fp32 step and (optionally) one Q8_0 step.  Returns (tokens, seconds, setup_s)."""
+    import oracle
+    t0 = time.perf_counter()
+    blob = synth.blob(SPEC)
+    m = oracle.Model(SPEC.cfg, blob, SPEC.shared_weights)
+    k, v = synth.kv_prefill(SPEC, seq=0, n_pos=pos)
+    m.kv_load(k, v)
+    del k, v
+    if q80_also:
+        m.enable_q80(GS)
+    setup = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    m.forward(TOKEN, pos, q80=False)
+    ntok = 1
+    if q80_also:
+        m.forward(TOKEN, pos, q80=True)
+        ntok += 1
+    dt = time.perf_counter() - t1
+    m.close()
+    return ntok, dt, setup
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ arms -----
+
+def run_reference(args, rank):
+    """The CPU oracle as the reference arm: each step decodes one fp32 and one
+    Q8_0 token of the 7B-shape model at pos 512 on the host cores."""
+    if rank != 0:
+        return 0
+    import oracle
+    cores = host_cores()
+    blob = synth.blob(SPEC)
+    m = oracle.Model(SPEC.cfg, blob, SPEC.shared_weights)
+    k, v = synth.kv_prefill(SPEC, seq=0, n_pos=512)
+    m.kv_load(k, v)
+    del k, v
+    m.enable_q80(GS)
+    for _ in range(args.warmup):
+        m.forward(TOKEN, 512, q80=False)
+        m.forward(TOKEN, 512, q80=True)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        m.forward(TOKEN, 512, q80=False)
+        m.forward(TOKEN, 512, q80=True)
+    dt = time.perf_counter() - t0
+    val = 2 * args.steps / dt
+    sample = "each step: one fp32 and one Q8_0 decode step of the 7B-shape model at pos 512 (KV prefilled N(0,1))"
+    out = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (CPU oracle)",
+        "data": "synthetic", "config": workload_config(),
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def workload_config():
+    return {
+        "workload": "Llama-2 7B-shape single-token decode, batch 1: dim 4096, hidden 11008, 32 layers, "
+                    "32 heads, 32 KV heads, vocab 32000, seq_len 4096, untied classifier; fp32 and Q8_0 "
+                    "GS=64 weight sets resident; KV cache prefilled N(0,1); token 1 at positions 0, 512, 2048",
+        "tokens_per_step": 2 * len(POSITIONS),
+        "positions": list(POSITIONS),
+        "variants": ["fp32", "q8_0 gs=64"],
+        "l2": "inputs larger than L2 (33.9 GB of weights streamed per step)",
+        "parallelism": "replicas (one independent decoder per GPU)",
+    }
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import __graft_entry__
+    __graft_entry__.build()
+    import decode_llama_step_02_b200 as l2c
+
+    torch.cuda.set_device(local_rank)
+    dec = make_decoder(torch, l2c)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up (captures both step graphs)
+    for _ in range(max(args.warmup, 1)):
+        one_step(dec)
+    dec.sync()
+
+    # ---- device-timed region
+    launches_per_token = 1 + 5 * SPEC.n_layers + 1
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            one_step(dec)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    dec.sync()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    tokens = 2 * len(POSITIONS) * args.steps * world
+    value = tokens / (ms / 1e3)
+
+    # ---- per (variant, position) breakdown
+    peak, peak_kind = measured_peak()
+    reps = max(3, args.steps)
+    variants = {}
+    for q80 in (False, True):
+        for p in POSITIONS:
+            for _ in range(2):
+                dec.forward_ptr(TOKEN, p, q80)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record(stream)
+            for _ in range(reps):
+                dec.forward_ptr(TOKEN, p, q80)
+            b.record(stream)
+            torch.cuda.synchronize()
+            t = a.elapsed_time(b) / reps
+            by = bytes_per_token(q80, p)
+            variants[f"{'q8_0' if q80 else 'fp32'}@pos{p}"] = {
+                "ms_per_token": t, "tokens_per_s": 1e3 / t, "bytes_per_token": by,
+                "gbs": by / t / 1e6, "frac_of_measured_hbm": by / t / 1e6 / peak,
+                "frac_of_8tbs_roofline": by / t / 1e6 / NOMINAL_HBM_GBS,
+                "roofline_tokens_per_s_8tbs": NOMINAL_HBM_GBS * 1e9 / by,
+            }
+    dec.sync()
+
+    # ---- dominant kernel: RMSNorm + W1/W3 + SwiGLU (44% of the fp32 step's bytes)
+    def kernel_roofline(q80: bool):
+        dec.forward_ptr(TOKEN, 512, q80)
+        iters = 2 * SPEC.n_layers
+        dec.time_kernel(l2c.K_W13, q80, SPEC.n_layers)  # warm
+        avg_ms = dec.time_kernel(l2c.K_W13, q80, iters)
+        ach = w13_bytes(q80) / avg_ms / 1e6
+        key = "k_gemv_q8<W13>" if q80 else "k_gemv_f32<W13>"
+        return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                "traffic": traffic_record(key), "kernel": key, "algorithmic_bytes_per_launch": w13_bytes(q80),
+                "avg_launch_ms": avg_ms, "peak_kind": peak_kind}
+
+    roof = kernel_roofline(False)
+    roof_q8 = kernel_roofline(True)
+
+    # ---- end to end through the public API: per token, logits back to pinned host memory
+    host = torch.empty(SPEC.vocab_size, dtype=torch.float32).pin_memory()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for q80 in (False, True):
+            for p in POSITIONS:
+                lg = dec.forward(TOKEN, p, q80)
+                host.copy_(lg, non_blocking=True)
+        torch.cuda.synchronize()
+    e2e_s = max_over_ranks(time.perf_counter() - t0)
+    barrier()
+    e2e = {"value": tokens / e2e_s, "unit": UNIT,
+           "h2d_bytes_per_step": 2 * len(POSITIONS) * 8,          # token + position per decode step
+           "d2h_bytes_per_step": 2 * len(POSITIONS) * SPEC.vocab_size * 4}
+
+    # ---- CPU oracle beside it (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ntok, dt, setup = oracle_sample()
+        cpu = {"value": ntok / dt, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
+               "sample": f"one fp32 and one Q8_0 decode step of the 7B-shape model at pos 512 "
+                         f"({dt:.1f} s of compute; {setup:.0f} s to generate the weights, prefill the cache "
+                         f"and quantize, not counted)"}
+
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 | i8*i8->i32 with f64 group sums", "data": "synthetic",
+        "config": workload_config(), "roofline": roof, "roofline_q8_0": roof_q8,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_token * 2 * len(POSITIONS) * args.steps,
+        "clocks": clk.summary(), "variants": variants,
+        "context": "pages' CPU figures: ~110 tok/s 15M int8 on an M1 MacBook Air; ~0.8 tok/s 7B fp32 on a "
+                   "16-core Ryzen 9 7950X; ~4 tok/s 7B on a 96-thread server",
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    dec.close()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling case: the 7B widths with this many layers (not a bench line)")
+    args = ap.parse_args()
+    if args.layers:
+        global SPEC
+        import dataclasses
+        SPEC = dataclasses.replace(synth.L7B, name=f"7B-width-{args.layers}L", n_layers=args.layers)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

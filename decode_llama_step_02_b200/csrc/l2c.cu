@@ -1,0 +1,723 @@
+// l2c.cu - host runtime and C ABI of the decode-step library (see include/l2c.h).
+//
+// Device layout (all sizes 64-bit):
+//   E [V][d]              embedding (also the classifier when tied)
+//   rms_att, rms_ffn [L][d], rms_final [d]
+//   Wqkv [L][d + 2 kvd][d]  Wq, Wk, Wv rows concatenated: one matvec per layer
+//   Wo [L][d][d], W2 [L][d][h]
+//   W13 [L][2h][d]        row 2i = W1 row i, row 2i+1 = W3 row i (SwiGLU pairs)
+//   Wcls [V][d]           only when untied
+//   Q8_0 copies: the same matrices as row records [K codes | K/gs scales | pad16]
+//   KV caches [max_batch][L][S][kvd] fp32 for K and for V
+// A step is captured once per variant as a CUDA graph; token and position
+// live in device memory, so one graph serves every position.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <vector>
+
+#include "../../include/l2c.h"
+#include "kernels.cuh"
+
+using namespace l2c;
+
+struct Q8Mat {
+    uint8_t* p = nullptr;
+    size_t rb = 0;  // record bytes per row
+};
+
+struct l2c_ctx {
+    l2c_config c{};
+    int shared = 1, max_batch = 1;
+    cudaStream_t stream = nullptr, cap = nullptr;
+    int dev = 0, sms = 148;
+    int d = 0, h = 0, L = 0, H = 0, Hkv = 0, hs = 0, kvd = 0, V = 0, S = 0, rep = 1;
+    // fp32 weights
+    float *E = nullptr, *rms_att = nullptr, *rms_ffn = nullptr, *rms_final = nullptr;
+    float *Wqkv = nullptr, *Wo = nullptr, *W13 = nullptr, *W2 = nullptr, *Wcls = nullptr, *freq = nullptr;
+    // Q8_0 weights
+    int gs = 0;
+    Q8Mat qE, qWqkv, qWo, qW13, qW2, qWcls;
+    // state
+    float *kc = nullptr, *vc = nullptr;
+    float *x = nullptr, *q = nullptr, *att = nullptr, *hb = nullptr, *logits = nullptr;
+    int* tp = nullptr;  // [max_batch][2]
+    unsigned long long* amax = nullptr;
+    int* err = nullptr;
+    int* gen_tokens = nullptr;  // [S]
+    int* gen_count = nullptr;
+    int* idx_out = nullptr;
+    unsigned long long* key_scratch = nullptr;
+    void* attn_part = nullptr;
+    int* attn_cnt = nullptr;
+    int attn_chunk = 64, attn_nchunks = 1;
+    // graphs: [q80][gen]
+    cudaGraphExec_t graph[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+    // tuning
+    size_t pf_f32 = 256 << 10, pf_q8 = 128 << 10;
+    int f32_ctas_per_sm = 1;
+    bool pdl = true;     // programmatic dependent launch between the step's kernels
+    bool graphs = true;  // replay the step as a CUDA graph (off: plain launches)
+    std::vector<void*> allocs;
+    char msg[512] = {0};
+    int status = L2C_OK;  // code of the last failure
+};
+
+// ------------------------------------------------------------------ helpers --
+
+static int fail(l2c_ctx* h, int code, const char* fmt, ...) {
+    if (h) {
+        h->status = code;
+        va_list ap;
+        va_start(ap, fmt);
+        vsnprintf(h->msg, sizeof(h->msg), fmt, ap);
+        va_end(ap);
+    }
+    return code;
+}
+
+#define CK(call)                                                                              \
+    do {                                                                                      \
+        cudaError_t e_ = (call);                                                              \
+        if (e_ != cudaSuccess)                                                                \
+            return fail(h, L2C_E_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));       \
+    } while (0)
+
+static int dalloc(l2c_ctx* h, void** p, size_t bytes) {
+    if (bytes == 0) bytes = 16;
+    cudaError_t e = cudaMalloc(p, bytes);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(h, L2C_E_OOM, "cudaMalloc(%zu) failed: %s", bytes, cudaGetErrorString(e));
+    }
+    h->allocs.push_back(*p);
+    return L2C_OK;
+}
+
+static size_t env_size(const char* name, size_t dflt) {
+    const char* v = getenv(name);
+    return v ? (size_t)strtoull(v, nullptr, 10) : dflt;
+}
+
+static bool is_device_ptr(const void* p) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+static bool g_pdl = true;  // launch attribute switch, set from the handle before each launch
+
+template <typename Kern, typename... Args>
+static cudaError_t launch(cudaStream_t s, bool pdl, Kern kernel, dim3 grid, dim3 block, size_t smem,
+                          Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = (pdl && g_pdl) ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+extern "C" size_t l2c_blob_floats(const l2c_config* c, int shared_weights) {
+    if (!c || c->n_heads <= 0) return 0;
+    size_t d = (size_t)c->dim, hh = (size_t)c->hidden_dim, L = (size_t)c->n_layers;
+    size_t hs = d / (size_t)c->n_heads, kvd = (size_t)c->n_kv_heads * hs;
+    size_t V = (size_t)c->vocab_size, S = (size_t)c->seq_len;
+    size_t n = V * d + L * d + 2 * L * d * d + 2 * L * kvd * d + L * d + 3 * L * hh * d + d + S * hs;
+    return shared_weights ? n : n + V * d;
+}
+
+// ------------------------------------------------------------ attention table --
+
+typedef void (*AttnKernel)(const AttnArgs);
+
+template <typename Acc>
+static AttnKernel attn_kernel_for(int hs, int rep) {
+#define L2C_ATTN(HS_, REP_) \
+    if (hs == HS_ && rep == REP_) return k_attention<Acc, HS_, REP_>;
+    L2C_ATTN(8, 1) L2C_ATTN(8, 2) L2C_ATTN(8, 3) L2C_ATTN(8, 4)
+    L2C_ATTN(16, 1) L2C_ATTN(16, 2) L2C_ATTN(16, 4)
+    L2C_ATTN(32, 1) L2C_ATTN(32, 2) L2C_ATTN(32, 4)
+    L2C_ATTN(48, 1) L2C_ATTN(48, 2) L2C_ATTN(48, 4)
+    L2C_ATTN(64, 1) L2C_ATTN(64, 2) L2C_ATTN(64, 4) L2C_ATTN(64, 8)
+    L2C_ATTN(96, 1) L2C_ATTN(96, 2) L2C_ATTN(96, 4)
+    L2C_ATTN(128, 1) L2C_ATTN(128, 2) L2C_ATTN(128, 4) L2C_ATTN(128, 8)
+#undef L2C_ATTN
+    return nullptr;
+}
+
+// ------------------------------------------------------------- step building --
+
+struct GemvShape {
+    int rows, K, unit;
+};
+
+static Q8Layout q8_layout(const l2c_ctx* h, int K, size_t rb, int unit, int* nwc_out) {
+    (void)h;
+    int nwc = (unit == 2) ? 4 : (K > 4096 ? 4 : 8);
+    Q8Layout L = {};
+    L.units_per_stage = nwc;
+    L.stage_bytes = (size_t)nwc * unit * rb;
+    size_t budget = 96 << 10;
+    int ns = (int)(budget / L.stage_bytes);
+    L.ns = ns < 2 ? 2 : (ns > 4 ? 4 : ns);
+    *nwc_out = nwc;
+    return L;
+}
+
+static size_t q8_smem(int K, int gs, const Q8Layout& L, bool stage_fp32) {
+    size_t b = (size_t)L.ns * L.stage_bytes;
+    if (stage_fp32) b += (size_t)K * 4;
+    b += ((size_t)K + 15) & ~size_t(15);
+    b += (size_t)(K / gs) * 4;
+    b = (b + 15) & ~size_t(15);
+    b += 16 * (size_t)L.ns;
+    return b;
+}
+
+template <int MODE>
+static cudaError_t launch_gemv(l2c_ctx* h, bool q80, GemvArgs a, int unit) {
+    const int units = a.rows / unit;
+    if (!q80) {
+        int grid = h->sms * h->f32_ctas_per_sm;
+        if (grid > units) grid = units;
+        a.prefetch_bytes = h->pf_f32;
+        return launch(h->cap, true, k_gemv_f32<MODE>, dim3(grid), dim3(F32_THREADS), (size_t)a.K * 4, a);
+    }
+    int nwc = 8;
+    Q8Layout L = q8_layout(h, a.K, a.ld, unit, &nwc);
+    L.stage_fp32 = (a.norm_w != nullptr || a.emb != nullptr) ? 1 : 0;
+    size_t smem = q8_smem(a.K, a.gs, L, L.stage_fp32 != 0);
+    int grid = h->sms;
+    if (grid > units) grid = units;
+    a.prefetch_bytes = h->pf_q8;
+    return launch(h->cap, true, k_gemv_q8<MODE>, dim3(grid), dim3(32 * (nwc + 1)), smem, a, L);
+}
+
+static int set_smem_limits(l2c_ctx* h) {
+    int maxopt = 0;
+    CK(cudaDeviceGetAttribute(&maxopt, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->dev));
+    CK(cudaFuncSetAttribute(k_gemv_f32<M_QKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+    CK(cudaFuncSetAttribute(k_gemv_f32<M_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+    CK(cudaFuncSetAttribute(k_gemv_f32<M_W13>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+    CK(cudaFuncSetAttribute(k_gemv_f32<M_CLS>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_QKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_W13>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+    return L2C_OK;
+}
+
+// Kernels of the step, in order within a layer.
+enum StepKernel : int { SK_QKV = 0, SK_ATTN = 1, SK_WO = 2, SK_W13 = 3, SK_W2 = 4, SK_CLS = 5 };
+
+// Enqueues kernel `kind` of layer l (sequence 0) on stream s.
+static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, int l) {
+    g_pdl = h->pdl;
+    const size_t d = h->d, kvd = h->kvd, hh = h->h, S = h->S;
+    float* kslot = h->kc + (size_t)l * S * kvd;
+    float* vslot = h->vc + (size_t)l * S * kvd;
+    cudaStream_t saved = h->cap;
+    h->cap = s;  // launch_gemv enqueues on h->cap
+    cudaError_t e = cudaSuccess;
+    GemvArgs a = {};
+    a.gs = h->gs; a.tp = h->tp; a.err = h->err; a.vocab = h->V; a.seq_len = h->S;
+    a.d = (int)d; a.kvd = (int)kvd; a.hs = h->hs;
+    switch (kind) {
+    case SK_QKV:  // RMSNorm + q/k/v + RoPE + cache write
+        a.rows = (int)(d + 2 * kvd);
+        a.K = (int)d;
+        if (q80) { a.W = h->qWqkv.p + (size_t)l * a.rows * h->qWqkv.rb; a.ld = h->qWqkv.rb; }
+        else { a.W = h->Wqkv + (size_t)l * a.rows * d; a.ld = d; }
+        a.in = h->x;
+        a.norm_w = h->rms_att + (size_t)l * d;
+        if (l == 0) {
+            a.emb = q80 ? (const void*)h->qE.p : (const void*)h->E;
+            a.x_resid = h->x;
+            a.amax = h->amax;
+        }
+        a.out = h->q;
+        a.kslot = kslot;
+        a.vslot = vslot;
+        a.freq = h->freq;
+        e = launch_gemv<M_QKV>(h, q80, a, 2);
+        break;
+    case SK_ATTN: {
+        AttnArgs t = {};
+        t.q = h->q; t.kc = kslot; t.vc = vslot; t.seq_stride = (size_t)h->L * S * kvd;
+        t.out = h->att; t.tp = h->tp; t.tp_stride = 2;
+        t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = (int)kvd; t.seq_len = h->S;
+        t.chunk = h->attn_chunk; t.nchunks = h->attn_nchunks;
+        t.part = h->attn_part; t.count = h->attn_cnt; t.err = h->err;
+        AttnKernel ak = q80 ? attn_kernel_for<double>(h->hs, h->rep) : attn_kernel_for<float>(h->hs, h->rep);
+        e = launch(s, true, ak, dim3(h->attn_nchunks, h->Hkv, 1), dim3(128), 0, t);
+        break;
+    }
+    case SK_WO:  // wo + residual
+        a.rows = (int)d; a.K = (int)d;
+        if (q80) { a.W = h->qWo.p + (size_t)l * d * h->qWo.rb; a.ld = h->qWo.rb; }
+        else { a.W = h->Wo + (size_t)l * d * d; a.ld = d; }
+        a.in = h->att; a.out = h->x;
+        e = launch_gemv<M_RESID>(h, q80, a, 1);
+        break;
+    case SK_W13:  // RMSNorm + W1/W3 + SwiGLU
+        a.rows = (int)(2 * hh); a.K = (int)d;
+        if (q80) { a.W = h->qW13.p + (size_t)l * 2 * hh * h->qW13.rb; a.ld = h->qW13.rb; }
+        else { a.W = h->W13 + (size_t)l * 2 * hh * d; a.ld = d; }
+        a.in = h->x; a.norm_w = h->rms_ffn + (size_t)l * d; a.out = h->hb;
+        e = launch_gemv<M_W13>(h, q80, a, 2);
+        break;
+    case SK_W2:  // W2 + residual
+        a.rows = (int)d; a.K = (int)hh;
+        if (q80) { a.W = h->qW2.p + (size_t)l * d * h->qW2.rb; a.ld = h->qW2.rb; }
+        else { a.W = h->W2 + (size_t)l * d * hh; a.ld = hh; }
+        a.in = h->hb; a.out = h->x;
+        e = launch_gemv<M_RESID>(h, q80, a, 1);
+        break;
+    default:  // final RMSNorm + classifier + argmax
+        a.rows = h->V; a.K = (int)d;
+        if (q80) { a.W = h->qWcls.p; a.ld = h->qWcls.rb; }
+        else { a.W = h->Wcls; a.ld = d; }
+        a.in = h->x; a.norm_w = h->rms_final; a.out = h->logits; a.amax = h->amax;
+        e = launch_gemv<M_CLS>(h, q80, a, 1);
+        break;
+    }
+    h->cap = saved;
+    if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "kernel %d launch: %s", kind, cudaGetErrorString(e));
+    return L2C_OK;
+}
+
+// Enqueues one decode step of sequence 0 on h->cap (being captured).
+static int enqueue_step(l2c_ctx* h, bool q80) {
+    int rc;
+    for (int l = 0; l < h->L; l++)
+        for (int k = SK_QKV; k <= SK_W2; k++)
+            if ((rc = launch_step_kernel(h, h->cap, k, q80, l)) != L2C_OK) return rc;
+    return launch_step_kernel(h, h->cap, SK_CLS, q80, 0);
+}
+
+static int build_graph(l2c_ctx* h, bool q80, bool gen) {
+    if (h->graph[q80][gen]) return L2C_OK;
+    CK(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
+    int rc = enqueue_step(h, q80);
+    if (rc == L2C_OK && gen) {
+        cudaError_t e = launch(h->cap, false, k_advance, dim3(1), dim3(1), 0, h->tp,
+                               (const unsigned long long*)h->amax, h->gen_tokens, h->gen_count);
+        if (e != cudaSuccess) rc = fail(h, L2C_E_CUDA, "advance launch: %s", cudaGetErrorString(e));
+    }
+    cudaGraph_t g = nullptr;
+    cudaError_t e = cudaStreamEndCapture(h->cap, &g);
+    if (rc != L2C_OK) {
+        if (g) cudaGraphDestroy(g);
+        return rc;
+    }
+    if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "capture failed: %s", cudaGetErrorString(e));
+    e = cudaGraphInstantiate(&h->graph[q80][gen], g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "graph instantiate: %s", cudaGetErrorString(e));
+    return L2C_OK;
+}
+
+// ------------------------------------------------------------------ create --
+
+static int copy_in(l2c_ctx* h, void* dst, const float* src, size_t n, cudaMemcpyKind kind) {
+    CK(cudaMemcpyAsync(dst, src, n * sizeof(float), kind, h->stream));
+    return L2C_OK;
+}
+
+// rows of `src` [rows][K] into every `stride`-th row of dst starting at row `first`
+static int copy_rows_strided(l2c_ctx* h, float* dst, int first, int stride, const float* src, size_t rows,
+                             size_t K, cudaMemcpyKind kind) {
+    CK(cudaMemcpy2DAsync(dst + (size_t)first * K, (size_t)stride * K * sizeof(float), src, K * sizeof(float),
+                         K * sizeof(float), rows, kind, h->stream));
+    return L2C_OK;
+}
+
+static int check_config(l2c_ctx* h, const l2c_config* c) {
+    if (c->dim <= 0 || c->hidden_dim <= 0 || c->n_layers <= 0 || c->n_heads <= 0 || c->n_kv_heads <= 0 ||
+        c->vocab_size <= 0 || c->seq_len <= 0)
+        return fail(h, L2C_E_ARG, "config fields must be positive");
+    if (c->dim % c->n_heads || c->n_heads % c->n_kv_heads)
+        return fail(h, L2C_E_ARG, "dim %% n_heads and n_heads %% n_kv_heads must be 0");
+    int hs = c->dim / c->n_heads;
+    if (hs % 2) return fail(h, L2C_E_ARG, "head_size must be even (RoPE rotates pairs)");
+    if (c->dim % 4 || c->hidden_dim % 4) return fail(h, L2C_E_ARG, "dim and hidden_dim must be multiples of 4");
+    if (!attn_kernel_for<float>(hs, c->n_heads / c->n_kv_heads))
+        return fail(h, L2C_E_ARG, "unsupported head_size %d / GQA ratio %d", hs, c->n_heads / c->n_kv_heads);
+    return L2C_OK;
+}
+
+extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_floats, int shared_weights,
+                          int max_batch, void* cuda_stream, l2c_ctx** out) {
+    if (!out) return L2C_E_ARG;
+    *out = nullptr;
+    if (!cfg || !blob || max_batch < 1) return L2C_E_ARG;
+    l2c_ctx* h = new (std::nothrow) l2c_ctx();
+    if (!h) return L2C_E_OOM;
+    int rc = check_config(h, cfg);
+    if (rc == L2C_OK && blob_floats != l2c_blob_floats(cfg, shared_weights))
+        rc = fail(h, L2C_E_ARG, "blob has %zu floats, the config needs %zu", blob_floats,
+                  l2c_blob_floats(cfg, shared_weights));
+    if (rc != L2C_OK) {
+        // keep the message reachable through a static handle-less error
+        fprintf(stderr, "l2c_create: %s\n", h->msg);
+        delete h;
+        return rc;
+    }
+    h->c = *cfg;
+    h->shared = shared_weights ? 1 : 0;
+    h->max_batch = max_batch;
+    h->stream = (cudaStream_t)cuda_stream;
+    h->d = cfg->dim; h->h = cfg->hidden_dim; h->L = cfg->n_layers; h->H = cfg->n_heads;
+    h->Hkv = cfg->n_kv_heads; h->hs = h->d / h->H; h->kvd = h->Hkv * h->hs; h->V = cfg->vocab_size;
+    h->S = cfg->seq_len; h->rep = h->H / h->Hkv;
+    h->pf_f32 = env_size("L2C_PREFETCH_F32", h->pf_f32);
+    h->pf_q8 = env_size("L2C_PREFETCH_Q8", h->pf_q8);
+    h->f32_ctas_per_sm = (int)env_size("L2C_F32_CTAS_PER_SM", 1);
+    h->attn_chunk = (int)env_size("L2C_ATTN_CHUNK", 64);
+    h->pdl = env_size("L2C_NO_PDL", 0) == 0;
+    h->graphs = env_size("L2C_NO_GRAPH", 0) == 0;
+    if (h->attn_chunk < 1) h->attn_chunk = 64;
+    h->attn_nchunks = (h->S + h->attn_chunk - 1) / h->attn_chunk;
+    auto bail = [&](int code) { l2c_destroy(h); return code; };
+    if (cudaGetDevice(&h->dev) != cudaSuccess) return bail(fail(h, L2C_E_CUDA, "no CUDA device"));
+    if (cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->dev) != cudaSuccess)
+        return bail(L2C_E_CUDA);
+    if (cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking) != cudaSuccess) return bail(L2C_E_CUDA);
+    if ((rc = set_smem_limits(h)) != L2C_OK) return bail(rc);
+
+    const size_t d = h->d, hh = h->h, L = h->L, kvd = h->kvd, V = h->V, S = h->S, B = max_batch;
+    const size_t rq = d + 2 * kvd;
+#define ALLOC(ptr, bytes)                                                  \
+    do {                                                                   \
+        if ((rc = dalloc(h, (void**)&(ptr), (bytes))) != L2C_OK) return bail(rc); \
+    } while (0)
+    ALLOC(h->E, V * d * 4);
+    ALLOC(h->rms_att, L * d * 4);
+    ALLOC(h->rms_ffn, L * d * 4);
+    ALLOC(h->rms_final, d * 4);
+    ALLOC(h->Wqkv, L * rq * d * 4);
+    ALLOC(h->Wo, L * d * d * 4);
+    ALLOC(h->W13, L * 2 * hh * d * 4);
+    ALLOC(h->W2, L * d * hh * 4);
+    if (!h->shared) {
+        ALLOC(h->Wcls, V * d * 4);
+    } else {
+        h->Wcls = h->E;
+    }
+    ALLOC(h->freq, (size_t)(h->hs / 2) * 4);
+    ALLOC(h->kc, B * L * S * kvd * 4);
+    ALLOC(h->vc, B * L * S * kvd * 4);
+    ALLOC(h->x, B * d * 4);
+    ALLOC(h->q, B * d * 4);
+    ALLOC(h->att, B * d * 4);
+    ALLOC(h->hb, B * hh * 4);
+    ALLOC(h->logits, B * V * 4);
+    ALLOC(h->tp, B * 2 * 4);
+    ALLOC(h->amax, B * 8);
+    ALLOC(h->err, 4);
+    ALLOC(h->gen_tokens, (S + 1) * 4);
+    ALLOC(h->gen_count, 4);
+    ALLOC(h->idx_out, 4);
+    ALLOC(h->key_scratch, 8);
+    ALLOC(h->attn_part, B * (size_t)h->Hkv * h->attn_nchunks * h->rep * (h->hs + 2) * sizeof(double));
+    ALLOC(h->attn_cnt, B * (size_t)h->Hkv * 4);
+#undef ALLOC
+    // zero state
+    if (cudaMemsetAsync(h->kc, 0, B * L * S * kvd * 4, h->stream) != cudaSuccess ||
+        cudaMemsetAsync(h->vc, 0, B * L * S * kvd * 4, h->stream) != cudaSuccess ||
+        cudaMemsetAsync(h->attn_cnt, 0, B * (size_t)h->Hkv * 4, h->stream) != cudaSuccess ||
+        cudaMemsetAsync(h->err, 0, 4, h->stream) != cudaSuccess ||
+        cudaMemsetAsync(h->tp, 0, B * 2 * 4, h->stream) != cudaSuccess ||
+        cudaMemsetAsync(h->x, 0, B * d * 4, h->stream) != cudaSuccess)
+        return bail(fail(h, L2C_E_CUDA, "memset failed"));
+
+    // weights in checkpoint order -> device layout
+    const cudaMemcpyKind kind = is_device_ptr(blob) ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+    const float* p = blob;
+    const float *pE = p; p += V * d;
+    const float *patt = p; p += L * d;
+    const float *pq = p; p += L * d * d;
+    const float *pk = p; p += L * kvd * d;
+    const float *pv = p; p += L * kvd * d;
+    const float *po = p; p += L * d * d;
+    const float *pffn = p; p += L * d;
+    const float *p1 = p; p += L * hh * d;
+    const float *p2 = p; p += L * d * hh;
+    const float *p3 = p; p += L * hh * d;
+    const float *pfin = p; p += d;
+    p += S * (size_t)h->hs;  // legacy freq_cis_real and freq_cis_imag, not used
+    const float* pcls = h->shared ? nullptr : p;
+    if ((rc = copy_in(h, h->E, pE, V * d, kind)) ||
+        (rc = copy_in(h, h->rms_att, patt, L * d, kind)) ||
+        (rc = copy_in(h, h->rms_ffn, pffn, L * d, kind)) ||
+        (rc = copy_in(h, h->rms_final, pfin, d, kind)) ||
+        (rc = copy_in(h, h->Wo, po, L * d * d, kind)) ||
+        (rc = copy_in(h, h->W2, p2, L * d * hh, kind)))
+        return bail(rc);
+    if (pcls && (rc = copy_in(h, h->Wcls, pcls, V * d, kind))) return bail(rc);
+    for (size_t l = 0; l < L; l++) {
+        float* qkv = h->Wqkv + l * rq * d;
+        if ((rc = copy_in(h, qkv, pq + l * d * d, d * d, kind)) ||
+            (rc = copy_in(h, qkv + d * d, pk + l * kvd * d, kvd * d, kind)) ||
+            (rc = copy_in(h, qkv + (d + kvd) * d, pv + l * kvd * d, kvd * d, kind)))
+            return bail(rc);
+        float* w13 = h->W13 + l * 2 * hh * d;
+        if ((rc = copy_rows_strided(h, w13, 0, 2, p1 + l * hh * d, hh, d, kind)) ||
+            (rc = copy_rows_strided(h, w13, 1, 2, p3 + l * hh * d, hh, d, kind)))
+            return bail(rc);
+    }
+    // RoPE frequencies of the even in-head indices j: 1 / 10000^(j/hs), fp32
+    // (the formula llama2.c evaluates inside forward; tabulated once here)
+    std::vector<float> fr(h->hs / 2);
+    for (int j = 0; j < h->hs; j += 2) fr[j / 2] = 1.0f / powf(10000.0f, (float)j / (float)h->hs);
+    if (cudaMemcpyAsync(h->freq, fr.data(), fr.size() * 4, cudaMemcpyHostToDevice, h->stream) != cudaSuccess)
+        return bail(fail(h, L2C_E_CUDA, "freq upload failed"));
+    if (cudaStreamSynchronize(h->stream) != cudaSuccess)
+        return bail(fail(h, L2C_E_CUDA, "upload failed: %s", cudaGetErrorString(cudaGetLastError())));
+    *out = h;
+    return L2C_OK;
+}
+
+// ---------------------------------------------------------------- Q8_0 set --
+
+static size_t record_bytes(int K, int gs) {
+    return (size_t)K + (((size_t)(K / gs) * 4 + 15) & ~size_t(15));
+}
+
+static int make_q8(l2c_ctx* h, Q8Mat& m, const float* W, size_t rows, int K) {
+    m.rb = record_bytes(K, h->gs);
+    int rc = dalloc(h, (void**)&m.p, rows * m.rb);
+    if (rc) return rc;
+    CK(cudaMemsetAsync(m.p, 0, rows * m.rb, h->stream));
+    long long groups = (long long)rows * (K / h->gs);
+    long long blocks = (groups + 7) / 8;
+    int grid = (int)(blocks < 65535LL * 16 ? blocks : 65535LL * 16);
+    k_quantize_rows<<<grid, 256, 0, h->stream>>>(W, (long long)rows, K, h->gs, m.p, m.rb);
+    CK(cudaGetLastError());
+    return L2C_OK;
+}
+
+extern "C" int l2c_enable_q80(l2c_ctx* h, int gs) {
+    if (!h) return L2C_E_ARG;
+    if (h->gs) return h->gs == gs ? L2C_OK : fail(h, L2C_E_STATE, "Q8_0 already enabled with gs=%d", h->gs);
+    if (gs < 16 || gs > 256 || gs % 16 || h->d % gs || h->h % gs)
+        return fail(h, L2C_E_ARG, "gs=%d must be a multiple of 16 in [16,256] dividing dim and hidden_dim", gs);
+    h->gs = gs;
+    const size_t d = h->d, hh = h->h, L = h->L, kvd = h->kvd, V = h->V;
+    int rc;
+    if ((rc = make_q8(h, h->qE, h->E, V, (int)d)) || (rc = make_q8(h, h->qWqkv, h->Wqkv, L * (d + 2 * kvd), (int)d)) ||
+        (rc = make_q8(h, h->qWo, h->Wo, L * d, (int)d)) || (rc = make_q8(h, h->qW13, h->W13, L * 2 * hh, (int)d)) ||
+        (rc = make_q8(h, h->qW2, h->W2, L * d, (int)hh))) {
+        h->gs = 0;
+        return rc;
+    }
+    if (h->shared) h->qWcls = h->qE;
+    else if ((rc = make_q8(h, h->qWcls, h->Wcls, V, (int)d))) {
+        h->gs = 0;
+        return rc;
+    }
+    CK(cudaStreamSynchronize(h->stream));
+    return L2C_OK;
+}
+
+// ------------------------------------------------------------------ forward --
+
+static const float* forward_impl(l2c_ctx* h, int token, int pos, bool q80) {
+    if (!h) return nullptr;
+    if (token < 0 || token >= h->V) { fail(h, L2C_E_ARG, "token %d not in [0,%d)", token, h->V); return nullptr; }
+    if (pos < 0 || pos >= h->S) { fail(h, L2C_E_ARG, "pos %d not in [0,%d)", pos, h->S); return nullptr; }
+    if (q80 && !h->gs) { fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)"); return nullptr; }
+    if (h->graphs && build_graph(h, q80, false) != L2C_OK) return nullptr;
+    k_set_tp<<<1, 1, 0, h->stream>>>(h->tp, token, pos);
+    cudaError_t e = cudaSuccess;
+    if (h->graphs) {
+        e = cudaGraphLaunch(h->graph[q80][0], h->stream);
+    } else {
+        cudaStream_t saved = h->cap;
+        h->cap = h->stream;
+        int rc = enqueue_step(h, q80);
+        h->cap = saved;
+        if (rc != L2C_OK) return nullptr;
+    }
+    if (e != cudaSuccess) { fail(h, L2C_E_CUDA, "graph launch: %s", cudaGetErrorString(e)); return nullptr; }
+    return h->logits;
+}
+
+extern "C" const float* l2c_forward(l2c_ctx* h, int token, int pos) { return forward_impl(h, token, pos, false); }
+extern "C" const float* l2c_forward_q80(l2c_ctx* h, int token, int pos) { return forward_impl(h, token, pos, true); }
+
+extern "C" int l2c_generate(l2c_ctx* h, int token0, int pos0, int steps, int q80, int32_t* tokens_out) {
+    if (!h || !tokens_out || steps < 0) return L2C_E_ARG;
+    if (token0 < 0 || token0 >= h->V) return fail(h, L2C_E_ARG, "token %d not in [0,%d)", token0, h->V);
+    if (pos0 < 0 || pos0 + steps > h->S) return fail(h, L2C_E_ARG, "pos0 + steps exceeds seq_len");
+    if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
+    if (steps == 0) return L2C_OK;
+    int rc = build_graph(h, q80 != 0, true);
+    if (rc) return rc;
+    k_set_tp<<<1, 1, 0, h->stream>>>(h->tp, token0, pos0);
+    CK(cudaMemsetAsync(h->gen_count, 0, 4, h->stream));
+    for (int t = 0; t < steps; t++) CK(cudaGraphLaunch(h->graph[q80 != 0][1], h->stream));
+    CK(cudaMemcpyAsync(tokens_out, h->gen_tokens, (size_t)steps * 4, cudaMemcpyDeviceToHost, h->stream));
+    return l2c_sync(h);
+}
+
+extern "C" int l2c_forward_batch(l2c_ctx* h, int B, const int32_t* tokens, const int32_t* pos, int q80,
+                                 float* logits_out) {
+    (void)B; (void)tokens; (void)pos; (void)q80; (void)logits_out;
+    return fail(h, L2C_E_STATE, "batched step not available in this build");
+}
+
+extern "C" int l2c_time_kernel(l2c_ctx* h, int kind, int q80, int iters, float* avg_ms) {
+    if (!h || kind < SK_QKV || kind > SK_CLS || iters < 1 || !avg_ms) return fail(h, L2C_E_ARG, "time_kernel: bad arguments");
+    if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
+    cudaEvent_t e0, e1;
+    CK(cudaEventCreate(&e0));
+    CK(cudaEventCreate(&e1));
+    int rc = L2C_OK;
+    cudaError_t er = cudaEventRecord(e0, h->stream);
+    for (int i = 0; i < iters && rc == L2C_OK && er == cudaSuccess; i++)
+        rc = launch_step_kernel(h, h->stream, kind, q80 != 0, kind == SK_CLS ? 0 : i % h->L);
+    if (er == cudaSuccess) er = cudaEventRecord(e1, h->stream);
+    if (er == cudaSuccess) er = cudaEventSynchronize(e1);
+    float ms = 0.f;
+    if (er == cudaSuccess) er = cudaEventElapsedTime(&ms, e0, e1);
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    if (rc != L2C_OK) return rc;
+    if (er != cudaSuccess) return fail(h, L2C_E_CUDA, "time_kernel: %s", cudaGetErrorString(er));
+    *avg_ms = ms / (float)iters;
+    return l2c_sync(h);
+}
+
+// ------------------------------------------------------------------- misc --
+
+extern "C" int l2c_argmax(l2c_ctx* h, const float* logits, int n, int* out_idx) {
+    if (!h || !logits || n <= 0 || !out_idx) return L2C_E_ARG;
+    CK(cudaMemsetAsync(h->key_scratch, 0, 8, h->stream));
+    int grid = (n + 1023) / 1024;
+    if (grid > h->sms) grid = h->sms;
+    k_argmax<<<grid, 256, 0, h->stream>>>(logits, n, h->key_scratch, h->err);
+    k_argmax_index<<<1, 1, 0, h->stream>>>(h->key_scratch, h->idx_out);
+    CK(cudaGetLastError());
+    int rc = l2c_sync(h);
+    if (rc) return rc;
+    CK(cudaMemcpy(out_idx, h->idx_out, 4, cudaMemcpyDeviceToHost));
+    return L2C_OK;
+}
+
+extern "C" int l2c_quantize_q80(l2c_ctx* h, const float* x, int64_t n, int gs, int8_t* q, float* s) {
+    if (!h || !x || !q || !s || n < 0 || gs < 1 || gs > 1024 || n % gs)
+        return fail(h, L2C_E_ARG, "quantize: need n %% gs == 0 and 1 <= gs <= 1024");
+    if (n == 0) return L2C_OK;
+    long long groups = n / gs;
+    long long blocks = (groups + 7) / 8;
+    int grid = (int)(blocks < 65535LL * 16 ? blocks : 65535LL * 16);
+    k_quantize<<<grid, 256, 0, h->stream>>>(x, groups, gs, q, s);
+    CK(cudaGetLastError());
+    return L2C_OK;
+}
+
+extern "C" int l2c_q80_group_dots(l2c_ctx* h, const int8_t* qw, const int8_t* qx, int rows, int K, int gs,
+                                  int32_t* out) {
+    if (!h || !qw || !qx || !out || rows < 0 || K <= 0 || gs < 16 || gs > 512 || gs % 16 || K % gs)
+        return fail(h, L2C_E_ARG, "group_dots: need K %% gs == 0 and gs a multiple of 16 in [16,512]");
+    if (rows == 0) return L2C_OK;
+    k_group_dots<<<(rows + 7) / 8, 256, 0, h->stream>>>(qw, qx, rows, K, gs, out);
+    CK(cudaGetLastError());
+    return L2C_OK;
+}
+
+extern "C" int l2c_kv_load(l2c_ctx* h, int seq, int n_pos, const float* k, const float* v) {
+    if (!h || seq < 0 || seq >= h->max_batch || n_pos < 0 || n_pos > h->S || (!k && !v))
+        return fail(h, L2C_E_ARG, "kv_load: bad sequence or n_pos");
+    if (n_pos == 0) return L2C_OK;
+    const size_t kvd = h->kvd, S = h->S, L = h->L;
+    const size_t base = (size_t)seq * L * S * kvd;
+    const cudaMemcpyKind kk = k && is_device_ptr(k) ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+    const cudaMemcpyKind kv = v && is_device_ptr(v) ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice;
+    for (size_t l = 0; l < L; l++) {
+        if (k) CK(cudaMemcpyAsync(h->kc + base + l * S * kvd, k + l * n_pos * kvd, n_pos * kvd * 4, kk, h->stream));
+        if (v) CK(cudaMemcpyAsync(h->vc + base + l * S * kvd, v + l * n_pos * kvd, n_pos * kvd * 4, kv, h->stream));
+    }
+    CK(cudaStreamSynchronize(h->stream));
+    return L2C_OK;
+}
+
+extern "C" int l2c_kv_read(l2c_ctx* h, int seq, int n_pos, float* k, float* v) {
+    if (!h || seq < 0 || seq >= h->max_batch || n_pos < 0 || n_pos > h->S)
+        return fail(h, L2C_E_ARG, "kv_read: bad sequence or n_pos");
+    const size_t kvd = h->kvd, S = h->S, L = h->L;
+    const size_t base = (size_t)seq * L * S * kvd;
+    for (size_t l = 0; l < L && n_pos > 0; l++) {
+        if (k) CK(cudaMemcpyAsync(k + l * n_pos * kvd, h->kc + base + l * S * kvd, n_pos * kvd * 4,
+                                  cudaMemcpyDeviceToHost, h->stream));
+        if (v) CK(cudaMemcpyAsync(v + l * n_pos * kvd, h->vc + base + l * S * kvd, n_pos * kvd * 4,
+                                  cudaMemcpyDeviceToHost, h->stream));
+    }
+    return l2c_sync(h);
+}
+
+extern "C" int l2c_kv_reset(l2c_ctx* h, int seq) {
+    if (!h || seq < -1 || seq >= h->max_batch) return fail(h, L2C_E_ARG, "kv_reset: bad sequence");
+    const size_t n = (size_t)h->L * h->S * h->kvd;
+    if (seq < 0) {
+        CK(cudaMemsetAsync(h->kc, 0, n * h->max_batch * 4, h->stream));
+        CK(cudaMemsetAsync(h->vc, 0, n * h->max_batch * 4, h->stream));
+    } else {
+        CK(cudaMemsetAsync(h->kc + (size_t)seq * n, 0, n * 4, h->stream));
+        CK(cudaMemsetAsync(h->vc + (size_t)seq * n, 0, n * 4, h->stream));
+    }
+    return L2C_OK;
+}
+
+extern "C" int l2c_sync(l2c_ctx* h) {
+    if (!h) return L2C_E_ARG;
+    CK(cudaStreamSynchronize(h->stream));
+    int e = 0;
+    CK(cudaMemcpy(&e, h->err, 4, cudaMemcpyDeviceToHost));
+    if (e) {
+        CK(cudaMemset(h->err, 0, 4));
+        return fail(h, L2C_E_DEVICE, "device error word 0x%x:%s%s%s%s", e, (e & DERR_TOKEN) ? " token" : "",
+                    (e & DERR_POS) ? " pos" : "", (e & DERR_TIMEOUT) ? " wait-timeout" : "",
+                    (e & DERR_NAN) ? " nan" : "");
+    }
+    return L2C_OK;
+}
+
+extern "C" void* l2c_stream(l2c_ctx* h) { return h ? (void*)h->stream : nullptr; }
+
+extern "C" int l2c_last_status(l2c_ctx* h) { return h ? h->status : L2C_E_ARG; }
+
+extern "C" int l2c_last_error(l2c_ctx* h, char* buf, int len) {
+    if (!h) return 0;
+    int n = (int)strlen(h->msg);
+    if (buf && len > 0) {
+        strncpy(buf, h->msg, (size_t)len - 1);
+        buf[len - 1] = 0;
+    }
+    return n;
+}
+
+extern "C" void l2c_destroy(l2c_ctx* h) {
+    if (!h) return;
+    if (h->stream || h->cap) cudaDeviceSynchronize();
+    for (int a = 0; a < 2; a++)
+        for (int b = 0; b < 2; b++)
+            if (h->graph[a][b]) cudaGraphExecDestroy(h->graph[a][b]);
+    for (void* p : h->allocs) cudaFree(p);
+    if (h->cap) cudaStreamDestroy(h->cap);
+    delete h;
+}

@@ -1,0 +1,219 @@
+/*
+ * l2c.h - C ABI of the B200 decode-step library for Llama-2 decoders.
+ *
+ * One call runs one autoregressive decode step of llama2.c's transformer:
+ * the single-token forward() of run.c (fp32 weights) or of runq.c (Q8_0
+ * weights and activations), on one GPU, as a CUDA graph of hand-written
+ * sm_100a kernels.  Sources: web pages about karpathy's llama2.c, cited by
+ * title and section:
+ *   [hub]  "Llama 2 in Pure C: 一个周末Hack的AI奇迹" (pomoai.com), sections
+ *          架构实现 (RMSNorm, SwiGLU, RoPE, GQA, KV cache), 数据格式 (the .bin
+ *          weight file), 量化支持 (Q8_0 with per-group scales).
+ *   [port] "超精简LLM部署：llama2.c嵌入式移植全攻略" (blog.gitcode.com),
+ *          §1 INT8量化压缩 (quantize()), §2 内存优化策略 (KV cache),
+ *          智能家居控制案例 (build_transformer / forward / sample_argmax).
+ *   [qa]   "Karpathy 技術學習庫 - Q&A 問答集", 技術細節 (KV cache indexing,
+ *          GQA, RoPE on the fly, skipped freq_cis, shared_weights) and
+ *          效能相關 (13B pointer overflow).
+ *
+ * Conventions for every entry point:
+ *   - Return value: L2C_OK (0) or a negative L2C_E_* code; l2c_last_error()
+ *     gives a one-line reason.  Nothing aborts the process.
+ *   - Pointers named *_dev are device pointers on the handle's GPU; *_host
+ *     are host pointers.  "host or device" arguments are detected with
+ *     cudaPointerGetAttributes.
+ *   - The library never keeps a caller pointer past the call: inputs are
+ *     copied, outputs written.  Buffers the library returns stay owned by
+ *     the handle and stay valid until the next call on the same handle.
+ *   - One handle, one CUDA stream.  Calls on one handle are not thread-safe.
+ *     Work is enqueued on the handle's stream; l2c_sync() waits for it and
+ *     reports device-side errors (bad token or position, a bounded wait that
+ *     gave up, a NaN logit) recorded by the kernels.
+ *   - Sizes and offsets are 64-bit internally ([qa] 效能相關: llama2.c's 13B
+ *     failure was int overflow in pointer arithmetic).
+ */
+#ifndef L2C_H
+#define L2C_H
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define L2C_API __attribute__((visibility("default")))
+#else
+#define L2C_API
+#endif
+
+#define L2C_OK 0
+#define L2C_E_ARG (-1)    /* invalid argument or unsupported shape */
+#define L2C_E_OOM (-2)    /* device allocation failed */
+#define L2C_E_CUDA (-3)   /* a CUDA runtime call failed */
+#define L2C_E_DEVICE (-4) /* a kernel recorded an error (see l2c_last_error) */
+#define L2C_E_STATE (-5)  /* call not valid in the handle's state (e.g. Q8_0 not enabled) */
+
+/* The model shape: the seven integers of llama2.c's checkpoint header
+ * ([hub] 数据格式: "layers, dimensions, heads ..."; [qa] GQA: kv heads).
+ * head_size = dim / n_heads, kv_dim = n_kv_heads * head_size. */
+typedef struct {
+    int32_t dim, hidden_dim, n_layers, n_heads, n_kv_heads, vocab_size, seq_len;
+} l2c_config;
+
+typedef struct l2c_ctx l2c_ctx;
+
+/* Number of fp32 values in a weight blob of this shape (see l2c_create). */
+L2C_API size_t l2c_blob_floats(const l2c_config* cfg, int shared_weights);
+
+/*
+ * l2c_create - build_transformer() of [port] 智能家居控制案例.
+ *
+ * blob: the fp32 weights in llama2.c's checkpoint order, without the header
+ *   ([hub] 数据格式: contiguous fp32 arrays after the config; [qa] 跳過
+ *   freq_cis): E[V][d], rms_att[L][d], Wq[L][d][d], Wk[L][kvd][d],
+ *   Wv[L][kvd][d], Wo[L][d][d], rms_ffn[L][d], W1[L][h][d], W2[L][d][h],
+ *   W3[L][h][d], rms_final[d], two legacy RoPE tables of seq_len*hs/2 floats
+ *   each (skipped), then Wcls[V][d] only when shared_weights == 0.
+ *   Host or device memory; blob_floats must equal l2c_blob_floats().  The
+ *   blob is copied (and re-tiled) into device memory; the caller keeps it.
+ * shared_weights: 1 = the classifier is the embedding table ([qa]
+ *   shared_weights: a positive vocab_size in the header), 0 = a separate
+ *   classifier follows the legacy tables.
+ * max_batch: sequences the handle serves (each gets its own KV cache of
+ *   n_layers*seq_len*kv_dim fp32 for K and for V, [port] §2); >= 1.
+ * cuda_stream: the cudaStream_t to enqueue on (NULL = the legacy stream).
+ * Errors: L2C_E_ARG for a bad shape (dim % n_heads, n_heads % n_kv_heads,
+ *   odd head_size, a row width not a multiple of 4, an unsupported
+ *   head_size/GQA ratio) or blob size; L2C_E_OOM; L2C_E_CUDA.
+ */
+L2C_API int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_floats, int shared_weights,
+               int max_batch, void* cuda_stream, l2c_ctx** out);
+
+/*
+ * l2c_enable_q80 - makes the Q8_0 weight set of runq.c ([hub] 量化支持).
+ * Every matvec weight (Wq, Wk, Wv, Wo, W1, W2, W3, the classifier) and the
+ * embedding table are quantized on the device with the rule of quantize()
+ * ([port] §1 INT8量化压缩): per group of gs consecutive values along a row,
+ * scale = max|x| / 127 (fp32) and code = round(x / scale).  The fp32 set is
+ * kept, so both paths stay usable.  gs must divide dim and hidden_dim and be
+ * a multiple of 16 (16..256).  Calling it again with the same gs is a no-op;
+ * another gs gives L2C_E_STATE.
+ */
+L2C_API int l2c_enable_q80(l2c_ctx* h, int gs);
+
+/*
+ * l2c_forward - forward(transformer, token, pos) of run.c ([port]
+ * 智能家居控制案例): one decode step of sequence 0 in fp32.  Embedding row,
+ * then per layer RMSNorm, q/k/v matvecs, RoPE as cos/sin(pos*freq) computed
+ * in the kernel ([qa] RoPE), the K/V write at cache[layer][pos] ([qa] KV
+ * Cache), grouped-query attention over positions 0..pos ([qa] GQA), wo plus
+ * residual, RMSNorm, SwiGLU FFN plus residual; final RMSNorm and classifier.
+ * Returns the handle-owned DEVICE logits [vocab_size] (valid until the next
+ * call on the handle; the step may still be running: use the handle's stream
+ * or l2c_sync()), or NULL if token is not in [0, vocab_size) or pos not in
+ * [0, seq_len) (l2c_last_error says which).
+ */
+L2C_API const float* l2c_forward(l2c_ctx* h, int token, int pos);
+
+/* l2c_forward_q80 - the same step through the Q8_0 weights (runq.c): every
+ * matvec input is quantized at the same group size and each output is the
+ * sum over groups of the exact int32 group dot times both scales.  NULL also
+ * when l2c_enable_q80 has not been called. */
+L2C_API const float* l2c_forward_q80(l2c_ctx* h, int token, int pos);
+
+/*
+ * l2c_argmax - sample_argmax() of [port] 智能家居控制案例: the index of the
+ * largest of n device floats, the lowest index among equal maxima.  Blocks
+ * until the result is on the host.  A NaN in the input gives L2C_E_DEVICE.
+ */
+L2C_API int l2c_argmax(l2c_ctx* h, const float* logits_dev, int n, int* out_idx_host);
+
+/*
+ * l2c_generate - greedy decoding with the token fed back on the device:
+ * tok_0 = token0; for t = 0..steps-1: logits = forward(tok_t, pos0 + t),
+ * tok_{t+1} = argmax(logits).  tokens_out_host[t] = tok_{t+1}.
+ * q80 selects the Q8_0 path.  pos0 + steps must not exceed seq_len.
+ * Blocks until the tokens are on the host.
+ */
+L2C_API int l2c_generate(l2c_ctx* h, int token0, int pos0, int steps, int q80, int32_t* tokens_out_host);
+
+/*
+ * l2c_forward_batch - B independent sequences, one token each: sequence b
+ * runs the step with tokens[b] at position pos[b] against its own KV cache.
+ * tokens, pos: host or device int32 [B]; B <= max_batch.  logits_out_dev:
+ * device [B][vocab_size].  q80 selects the Q8_0 path.
+ */
+L2C_API int l2c_forward_batch(l2c_ctx* h, int B, const int32_t* tokens, const int32_t* pos, int q80,
+                      float* logits_out_dev);
+
+/*
+ * l2c_quantize_q80 - quantize() of [port] §1 INT8量化压缩 on n device
+ * floats: for each group of gs values, s[g] = max|x| / 127 (fp32) and
+ * q[i] = round(x[i] / s[g]) (fp32 quotient, half away from zero); a group of
+ * zeros gets s = 0 and codes 0.  x_dev [n], q_dev [n], s_dev [n / gs];
+ * n % gs == 0, 1 <= gs <= 1024.  Asynchronous on the handle's stream.
+ */
+L2C_API int l2c_quantize_q80(l2c_ctx* h, const float* x_dev, int64_t n, int gs, int8_t* q_dev, float* s_dev);
+
+/*
+ * l2c_q80_group_dots - the exact int32 dot product of every (row, group) of
+ * Q8_0 codes, computed by the same dp4a chunk loop as the Q8_0 matvec:
+ * out[r][g] = sum_k qw[r][g*gs+k] * qx[g*gs+k].  qw_dev [rows][K] int8,
+ * qx_dev [K] int8, out_dev [rows][K/gs] int32; K % gs == 0, gs a multiple of
+ * 16 (16..512).  Asynchronous on the handle's stream.
+ */
+L2C_API int l2c_q80_group_dots(l2c_ctx* h, const int8_t* qw_dev, const int8_t* qx_dev, int rows, int K, int gs,
+                       int32_t* out_dev);
+
+/*
+ * l2c_kv_load - fills the KV cache of sequence seq at positions [0, n_pos)
+ * from k and v laid out [n_layers][n_pos][kv_dim] (host or device); slots
+ * from n_pos on are left as they are.  Used to start a step from a given
+ * context without decoding it.
+ */
+L2C_API int l2c_kv_load(l2c_ctx* h, int seq, int n_pos, const float* k, const float* v);
+
+/* l2c_kv_read - copies the cache slots [0, n_pos) of sequence seq into host
+ * buffers k_host, v_host laid out [n_layers][n_pos][kv_dim].  Blocks. */
+L2C_API int l2c_kv_read(l2c_ctx* h, int seq, int n_pos, float* k_host, float* v_host);
+
+/* l2c_kv_reset - zeroes the KV cache of sequence seq (-1: all sequences). */
+L2C_API int l2c_kv_reset(l2c_ctx* h, int seq);
+
+/*
+ * l2c_time_kernel - measurement hook: runs kernel `kind` of the fp32 (q80 = 0)
+ * or Q8_0 step alone, iters times back to back on the handle's stream, and
+ * stores the average time per launch in ms (two CUDA events around the
+ * loop).  Launch i uses layer i % n_layers, so consecutive launches stream
+ * different weights.  kind: 0 = RMSNorm+QKV+RoPE, 1 = attention, 2 = wo,
+ * 3 = RMSNorm+W1/W3+SwiGLU, 4 = W2, 5 = final RMSNorm+classifier.  The
+ * kernels use the handle's current token/position and update its state
+ * (KV slot, activations) as in a step.  Blocks.
+ */
+L2C_API int l2c_time_kernel(l2c_ctx* h, int kind, int q80, int iters, float* avg_ms);
+
+/* l2c_sync - waits for the handle's stream, then reads and clears the
+ * device error word: L2C_E_DEVICE if a kernel recorded an error since the
+ * last check. */
+L2C_API int l2c_sync(l2c_ctx* h);
+
+/* l2c_stream - the cudaStream_t the handle enqueues on. */
+L2C_API void* l2c_stream(l2c_ctx* h);
+
+/* l2c_last_status - the L2C_E_* code of the last failed call on the handle
+ * (L2C_OK if none failed); use it after l2c_forward / l2c_forward_q80 return
+ * NULL. */
+L2C_API int l2c_last_status(l2c_ctx* h);
+
+/* l2c_last_error - copies the last error message (NUL-terminated, at most
+ * len bytes) and returns its full length. */
+L2C_API int l2c_last_error(l2c_ctx* h, char* buf, int len);
+
+/* l2c_destroy - frees all device memory and graphs of the handle. */
+L2C_API void l2c_destroy(l2c_ctx* h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,94 @@
+"""Kernel-level parity through the C ABI: Q8_0 quantize and int32 group dots must be
+bit-exact with the oracle; argmax must return the first index of the maximum."""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import need_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def env():
+    torch, l2c = need_gpu()
+    spec = synth.TINY
+    b = synth.blob(spec)
+    dec = l2c.Decoder(spec.cfg, b, spec.shared_weights)
+    yield torch, l2c, dec
+    dec.close()
+
+
+def _quant_inputs(n, gs, seed):
+    rng = np.random.default_rng(seed)
+    x = (rng.standard_normal(n) * rng.uniform(1e-3, 10.0, n // gs).repeat(gs)).astype(np.float32)
+    x[:gs] = 0.0                                        # an all-zero group
+    x[gs:2 * gs] = np.float32(1.5) * np.arange(gs)       # exact values on .5 ties after scaling
+    x[2 * gs] = np.float32(-127.0)
+    return x
+
+
+@pytest.mark.parametrize("gs,n", [(32, 288 * 37), (64, 4096 * 9), (64, 11008 * 3), (16, 1600), (128, 128 * 50)])
+def test_quantize_bitexact(env, gs, n):
+    torch, l2c, dec = env
+    x = _quant_inputs(n, gs, gs + n)
+    q_ref, s_ref = oracle.quantize(x, gs)
+    xd = torch.from_numpy(x).cuda()
+    q = torch.empty(n, dtype=torch.int8, device="cuda")
+    s = torch.empty(n // gs, dtype=torch.float32, device="cuda")
+    dec.quantize_q80(xd, gs, q, s)
+    dec.sync()
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+def test_quantize_weight_blob_bitexact(env):
+    # the 15M-shape embedding table: 9.2M seeded N(0, 0.02) weights, GS = 32
+    torch, l2c, dec = env
+    spec = synth.M15
+    E = np.empty(spec.vocab_size * spec.dim, np.float32)
+    synth.blob_into(spec, E)
+    q_ref, s_ref = oracle.quantize(E, 32)
+    q = torch.empty(E.size, dtype=torch.int8, device="cuda")
+    s = torch.empty(E.size // 32, dtype=torch.float32, device="cuda")
+    dec.quantize_q80(torch.from_numpy(E).cuda(), 32, q, s)
+    dec.sync()
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+
+
+@pytest.mark.parametrize("rows,K,gs", [(7, 288, 32), (33, 4096, 64), (5, 11008, 64), (3, 768, 64), (9, 256, 128)])
+def test_group_dots_bitexact(env, rows, K, gs):
+    torch, l2c, dec = env
+    rng = np.random.default_rng(rows * K)
+    qw = rng.integers(-127, 128, (rows, K)).astype(np.int8)
+    qx = rng.integers(-127, 128, K).astype(np.int8)
+    qw[0, :] = -127
+    qx[:gs] = -127   # extreme group: 64 * 127^2
+    ref = oracle.q80_group_dots(qw, qx, gs)
+    out = torch.empty((rows, K // gs), dtype=torch.int32, device="cuda")
+    dec.q80_group_dots(torch.from_numpy(qw).cuda(), torch.from_numpy(qx).cuda(), gs, out)
+    dec.sync()
+    assert np.array_equal(out.cpu().numpy(), ref)
+
+
+def test_argmax_first_index(env):
+    torch, l2c, dec = env
+    rng = np.random.default_rng(5)
+    for n in (1, 31, 32000, 100_003):
+        x = rng.standard_normal(n).astype(np.float32)
+        if n > 10:
+            x[n // 3] = x[n // 2] = x[-1] = x.max() + 1.0  # three-way tie
+        assert dec.argmax(torch.from_numpy(x).cuda()) == oracle.argmax(x)
+    neg = -np.abs(rng.standard_normal(500)).astype(np.float32) - 1
+    assert dec.argmax(torch.from_numpy(neg).cuda()) == oracle.argmax(neg)
+
+
+def test_argmax_nan_is_reported(env):
+    torch, l2c, dec = env
+    x = np.zeros(100, np.float32)
+    x[7] = np.nan
+    with pytest.raises(l2c.L2CError) as e:
+        dec.argmax(torch.from_numpy(x).cuda())
+    assert e.value.code == l2c.L2C_E_DEVICE
