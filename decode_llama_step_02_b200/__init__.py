@@ -21,7 +21,7 @@ L2C_OK, L2C_E_ARG, L2C_E_OOM, L2C_E_CUDA, L2C_E_DEVICE, L2C_E_STATE = 0, -1, -2,
 EXPORTS = (
     "l2c_blob_floats", "l2c_create", "l2c_enable_q80", "l2c_forward", "l2c_forward_q80", "l2c_argmax",
     "l2c_generate", "l2c_forward_batch", "l2c_quantize_q80", "l2c_q80_group_dots", "l2c_kv_load",
-    "l2c_kv_read", "l2c_kv_reset", "l2c_time_kernel", "l2c_sync", "l2c_stream", "l2c_last_status", "l2c_last_error",
+    "l2c_kv_read", "l2c_kv_reset", "l2c_attention", "l2c_time_kernel", "l2c_sync", "l2c_stream", "l2c_last_status", "l2c_last_error",
     "l2c_destroy",
 )
 
@@ -65,6 +65,7 @@ def lib():
             "l2c_kv_load": (i32, [vp, i32, i32, vp, vp]),
             "l2c_kv_read": (i32, [vp, i32, i32, vp, vp]),
             "l2c_kv_reset": (i32, [vp, i32]),
+            "l2c_attention": (i32, [vp, vp, vp, vp, i32, i32, vp]),
             "l2c_time_kernel": (i32, [vp, i32, i32, i32, ctypes.POINTER(ctypes.c_float)]),
             "l2c_sync": (i32, [vp]),
             "l2c_stream": (vp, [vp]),
@@ -186,6 +187,10 @@ class Decoder:
     # -- standalone kernels
     def quantize_q80(self, x, gs: int, q_out, s_out):
         self._check(lib().l2c_quantize_q80(self._h, _ptr(x), int(x.numel()), int(gs), _ptr(q_out), _ptr(s_out)))
+
+    def attention(self, q, k, v, pos: int, out, precision: int = 0):
+        """One layer's GQA attention for positions 0..pos (l2c_attention)."""
+        self._check(lib().l2c_attention(self._h, _ptr(q), _ptr(k), _ptr(v), int(pos), int(precision), _ptr(out)))
 
     def q80_group_dots(self, qw, qx, gs: int, out):
         rows, K = qw.shape

@@ -1,0 +1,333 @@
+// batched.cuh - the Q8_0 decode step for B independent sequences (sm_100a).
+//
+// With B sequences each matvec becomes a skinny GEMM Y[B][rows] = X[B][K] W^T.
+// At B = 32 the int8 work is 32 multiply-adds per weight byte, more than dp4a
+// sustains at HBM speed, so the group dot products run on the tensor cores:
+// mma.sync m16n8k32 s8*s8 -> s32 gives the exact int32 dot of every
+// (row, sequence, group), then ival * sw * sx is summed over groups in double,
+// as in the single-sequence kernel.  Per layer:
+//
+//   prep<QKV>   per sequence: embedding row (layer 0), RMSNorm, quantize -> xq, xs
+//   gemm<QKV>   q, RoPE, K/V cache write at each sequence's own position
+//   attention   k_attention over (chunk, KV head, sequence), ragged positions
+//   prep<Q>     quantize the attention output
+//   gemm<RESID> x += Wo att
+//   prep<QKV>   RMSNorm + quantize
+//   gemm<W13>   hb = silu(W1 x) * (W3 x)
+//   prep<Q>     quantize hb
+//   gemm<RESID> x += W2 hb
+// and prep + gemm<CLS> (logits and a per-sequence argmax) at the end.
+#pragma once
+#include "kernels.cuh"
+
+namespace l2c {
+
+constexpr int BMAX = 32;          // sequences per GEMM (n = 4 tiles of 8)
+constexpr int BG_WARPS = 2;       // consumer warps per CTA, 16 rows each
+constexpr int BG_ROWS = 16 * BG_WARPS;
+
+struct BPrepArgs {
+    const float* in;        // [B][K] fp32 input (x, attention output or hb)
+    size_t in_stride;       // floats between sequences
+    const float* norm_w;    // RMSNorm gain or nullptr
+    const uint8_t* emb;     // layer 0: embedding row records (codes | scales), else nullptr
+    size_t emb_rb;          // record bytes
+    float* x_resid;         // layer 0: receives the dequantized embedding rows [B][d]
+    int K, gs;
+    int8_t* xq;             // [B][kq_stride] codes
+    float* xs;              // [B][ks_stride] scales
+    size_t kq_stride, ks_stride;
+    const int* tp;          // [B][2] token, pos
+    int vocab, seq_len;
+    unsigned long long* amax;  // reset per sequence on layer 0
+    int* err;
+};
+
+// One CTA per sequence: input row, optional RMSNorm (double), Q8_0 codes.
+__global__ void __launch_bounds__(256) k_bprep(const BPrepArgs a) {
+    extern __shared__ float bp_xs[];
+    __shared__ double red[32];
+    const int b = blockIdx.x;
+    grid_dep_wait();
+    grid_dep_launch();
+    const int K = a.K, gs = a.gs;
+    const float* in = a.in + (size_t)b * a.in_stride;
+    if (a.emb) {
+        int token = a.tp[2 * b];
+        if (token < 0 || token >= a.vocab) {
+            if (threadIdx.x == 0) set_error(a.err, DERR_TOKEN);
+            token = 0;
+        }
+        const uint8_t* rec = a.emb + (size_t)token * a.emb_rb;
+        const int8_t* eq = reinterpret_cast<const int8_t*>(rec);
+        const float* es = reinterpret_cast<const float*>(rec + K);
+        for (int i = threadIdx.x; i < K; i += blockDim.x) {
+            float v = (float)eq[i] * es[i / gs];
+            bp_xs[i] = v;
+            a.x_resid[(size_t)b * K + i] = v;
+        }
+        if (a.amax && threadIdx.x == 0) a.amax[b] = 0ull;
+    } else {
+        for (int i = threadIdx.x; i < K; i += blockDim.x) bp_xs[i] = in[i];
+    }
+    __syncthreads();
+    if (a.norm_w) {
+        double ss = 0.0;
+        for (int i = threadIdx.x; i < K; i += blockDim.x) ss += (double)bp_xs[i] * (double)bp_xs[i];
+        ss = block_sum(ss, red);
+        double inv = 1.0 / sqrt(ss / (double)K + 1e-5);
+        for (int i = threadIdx.x; i < K; i += blockDim.x)
+            bp_xs[i] = (float)((double)a.norm_w[i] * (inv * (double)bp_xs[i]));
+        __syncthreads();
+    }
+    const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int8_t* q = a.xq + (size_t)b * a.kq_stride;
+    float* s = a.xs + (size_t)b * a.ks_stride;
+    for (int g = warp; g < K / gs; g += nw) quantize_group_warp(bp_xs + g * gs, gs, q + g * gs, s + g);
+}
+
+struct BGemmArgs {
+    const uint8_t* W;       // Q8_0 row records [rows][rb]
+    size_t rb;
+    int rows, K, gs, kc;    // kc: K bytes per stage (a multiple of 32 and of gs, dividing K)
+    int B;                  // live sequences (<= BMAX); codes of the others are zero
+    const int8_t* xq;       // [BMAX][kq_stride]
+    const float* xs;        // [BMAX][ks_stride]
+    size_t kq_stride, ks_stride;
+    float* out;             // QKV: q [B][d]; RESID: x [B][d]; W13: hb [B][h]; CLS: logits [B][V]
+    size_t out_stride;
+    float* kc_base;         // QKV: this layer's key cache of sequence 0
+    float* vc_base;
+    size_t seq_stride;      // floats between sequences' caches
+    const float* freq;
+    int d, kvd, hs, seq_len;
+    const int* tp;
+    unsigned long long* amax;
+    int* err;
+    size_t prefetch_bytes;
+};
+
+__device__ __forceinline__ void mma_s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Shared memory per stage: weights [BG_ROWS][kc+16], weight scales
+// [BG_ROWS][kc/gs], activations [BMAX][kc+16], activation scales [BMAX][kc/gs].
+struct BLayout {
+    int ns;
+    int kcp;          // kc + 16 (row pitch in shared memory; spreads rows over banks)
+    size_t w_off, ws_off, x_off, xs_off, stage_bytes;
+};
+
+__host__ __device__ inline BLayout make_blayout(int kc, int gs, int ns) {
+    BLayout L;
+    L.ns = ns;
+    L.kcp = kc + 16;
+    const size_t sc = ((size_t)(kc / gs) * 4 + 15) & ~size_t(15);
+    L.w_off = 0;
+    L.ws_off = L.w_off + (size_t)BG_ROWS * L.kcp;
+    L.x_off = L.ws_off + (size_t)BG_ROWS * sc;
+    L.xs_off = L.x_off + (size_t)BMAX * L.kcp;
+    L.stage_bytes = L.xs_off + (size_t)BMAX * sc;
+    L.stage_bytes = (L.stage_bytes + 127) & ~size_t(127);
+    return L;
+}
+
+// grid = ceil(rows / BG_ROWS) CTAs of (BG_WARPS + 1) warps; the last warp is
+// the producer (its 32 lanes issue the stage's bulk copies).
+template <int MODE>
+__global__ void __launch_bounds__(32 * (BG_WARPS + 1)) k_bgemm_q8(const BGemmArgs a, const BLayout L) {
+    extern __shared__ __align__(128) uint8_t bsm[];
+    __shared__ float stage_out[BG_ROWS][BMAX + 1];
+    __shared__ unsigned long long best_s[BMAX];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int r0 = blockIdx.x * BG_ROWS;
+    const int nrows = min(BG_ROWS, a.rows - r0);
+    const int nchunks = a.K / a.kc;
+    const int gpc = a.kc / a.gs;                 // groups per chunk
+    const size_t sc_bytes = (size_t)gpc * 4;     // scale bytes per row per chunk (multiple of 16 by construction)
+    uint64_t* full = reinterpret_cast<uint64_t*>(bsm + (size_t)L.ns * L.stage_bytes);
+    uint64_t* empty = full + L.ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < L.ns; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], BG_WARPS);
+        }
+        mbar_fence_init();
+    }
+    if (threadIdx.x < BMAX) best_s[threadIdx.x] = 0ull;
+    __syncthreads();
+
+    if (warp == BG_WARPS) {
+        // ---------------- producer
+        const uint64_t pol_w = policy_evict_first();
+        const uint64_t pol_x = policy_evict_last();
+        const uint8_t* Wb = a.W + (size_t)r0 * a.rb;
+        if (lane == 0 && a.prefetch_bytes) {
+            // the row block's records are contiguous: prefetch them into L2
+            size_t bytes = (size_t)nrows * a.rb;
+            if (bytes > a.prefetch_bytes) bytes = a.prefetch_bytes;
+            prefetch_l2_range(Wb, bytes & ~size_t(15), policy_evict_last());
+        }
+        // activations come from the prep kernel: wait for it before copying them
+        grid_dep_wait();
+        const uint32_t bytes_stage =
+            (uint32_t)((size_t)nrows * (a.kc + sc_bytes) + (size_t)BMAX * (a.kc + sc_bytes));
+        bool ok = true;
+        int issued = 0;
+        for (int c = 0; c < nchunks && ok; c++) {
+            const int s = c % L.ns;
+            if (c >= L.ns) {
+                bool w = true;
+                if (lane == 0) w = mbar_wait_bounded(&empty[s], ((c / L.ns) - 1) & 1, a.err);
+                w = __shfl_sync(0xffffffffu, w, 0);
+                if (!w) { ok = false; break; }
+            }
+            uint8_t* st = bsm + (size_t)s * L.stage_bytes;
+            if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes_stage);
+            __syncwarp();
+            for (int r = lane; r < nrows; r += 32) {
+                const uint8_t* rec = Wb + (size_t)r * a.rb;
+                bulk_g2s(st + L.w_off + (size_t)r * L.kcp, rec + (size_t)c * a.kc, a.kc, &full[s], pol_w);
+                bulk_g2s(st + L.ws_off + (size_t)r * ((sc_bytes + 15) & ~size_t(15)),
+                         rec + a.K + (size_t)c * sc_bytes, (uint32_t)sc_bytes, &full[s], pol_w);
+            }
+            for (int b = lane; b < BMAX; b += 32) {
+                bulk_g2s(st + L.x_off + (size_t)b * L.kcp, a.xq + (size_t)b * a.kq_stride + (size_t)c * a.kc, a.kc,
+                         &full[s], pol_x);
+                bulk_g2s(st + L.xs_off + (size_t)b * ((sc_bytes + 15) & ~size_t(15)),
+                         reinterpret_cast<const uint8_t*>(a.xs + (size_t)b * a.ks_stride) + (size_t)c * sc_bytes,
+                         (uint32_t)sc_bytes, &full[s], pol_x);
+            }
+            issued = c + 1;
+        }
+        if (!ok && lane == 0) {
+            for (int c = max(0, issued - L.ns); c < issued; c++)
+                mbar_wait_bounded(&full[c % L.ns], (c / L.ns) & 1, a.err);
+        }
+        return;
+    }
+
+    // ---------------- consumers: warp w owns rows r0 + 16w .. +15 of the block
+    grid_dep_wait();
+    grid_dep_launch();
+    const int gid = lane >> 2, tig = lane & 3;
+    const size_t scp = (sc_bytes + 15) & ~size_t(15);
+    double acc[4][4];
+#pragma unroll
+    for (int n = 0; n < 4; n++) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0;
+    const int wr0 = 16 * warp;   // first row of this warp in the block
+    bool ok = true;
+    for (int c = 0; c < nchunks; c++) {
+        const int s = c % L.ns;
+        if (!mbar_wait_bounded(&full[s], (c / L.ns) & 1, a.err)) { ok = false; break; }
+        const uint8_t* st = bsm + (size_t)s * L.stage_bytes;
+        const uint8_t* wt = st + L.w_off;
+        const float* wsc = reinterpret_cast<const float*>(st + L.ws_off);
+        const uint8_t* xt = st + L.x_off;
+        const float* xsc = reinterpret_cast<const float*>(st + L.xs_off);
+        if (wr0 < nrows) {
+            for (int g = 0; g < gpc; g++) {
+                int cc[4][4];
+#pragma unroll
+                for (int n = 0; n < 4; n++) cc[n][0] = cc[n][1] = cc[n][2] = cc[n][3] = 0;
+                for (int ks = 0; ks < a.gs; ks += 32) {
+                    const int k0 = g * a.gs + ks + 4 * tig;
+                    uint32_t af[4];
+                    af[0] = *reinterpret_cast<const uint32_t*>(wt + (size_t)(wr0 + gid) * L.kcp + k0);
+                    af[1] = *reinterpret_cast<const uint32_t*>(wt + (size_t)(wr0 + gid + 8) * L.kcp + k0);
+                    af[2] = *reinterpret_cast<const uint32_t*>(wt + (size_t)(wr0 + gid) * L.kcp + k0 + 16);
+                    af[3] = *reinterpret_cast<const uint32_t*>(wt + (size_t)(wr0 + gid + 8) * L.kcp + k0 + 16);
+#pragma unroll
+                    for (int n = 0; n < 4; n++) {
+                        const uint8_t* xr = xt + (size_t)(8 * n + gid) * L.kcp + k0;
+                        uint32_t b0 = *reinterpret_cast<const uint32_t*>(xr);
+                        uint32_t b1 = *reinterpret_cast<const uint32_t*>(xr + 16);
+                        mma_s8(cc[n], af, b0, b1);
+                    }
+                }
+                // scale the exact group dots: rows (gid, gid+8), sequences (2 tig, 2 tig + 1) of each tile
+                const double sw0 = (double)wsc[(size_t)(wr0 + gid) * (scp / 4) + g];
+                const double sw1 = (double)wsc[(size_t)(wr0 + gid + 8) * (scp / 4) + g];
+#pragma unroll
+                for (int n = 0; n < 4; n++) {
+                    const double sx0 = (double)xsc[(size_t)(8 * n + 2 * tig) * (scp / 4) + g];
+                    const double sx1 = (double)xsc[(size_t)(8 * n + 2 * tig + 1) * (scp / 4) + g];
+                    acc[n][0] += (double)cc[n][0] * sw0 * sx0;
+                    acc[n][1] += (double)cc[n][1] * sw0 * sx1;
+                    acc[n][2] += (double)cc[n][2] * sw1 * sx0;
+                    acc[n][3] += (double)cc[n][3] * sw1 * sx1;
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    if (!ok) return;
+    // results of this warp's rows -> shared staging (fp32, rounded once)
+#pragma unroll
+    for (int n = 0; n < 4; n++) {
+        stage_out[wr0 + gid][8 * n + 2 * tig] = (float)acc[n][0];
+        stage_out[wr0 + gid][8 * n + 2 * tig + 1] = (float)acc[n][1];
+        stage_out[wr0 + gid + 8][8 * n + 2 * tig] = (float)acc[n][2];
+        stage_out[wr0 + gid + 8][8 * n + 2 * tig + 1] = (float)acc[n][3];
+    }
+    asm volatile("bar.sync 1, %0;" :: "r"(32 * BG_WARPS) : "memory");
+    // epilogue: thread t takes (row unit, sequence) pairs
+    const int nt = 32 * BG_WARPS;
+    if (MODE == M_QKV || MODE == M_W13) {
+        for (int i = threadIdx.x; i < (nrows / 2) * a.B; i += nt) {
+            const int up = i / a.B, b = i % a.B;
+            const int r = r0 + 2 * up;
+            const float v0 = stage_out[2 * up][b], v1 = stage_out[2 * up + 1][b];
+            if (MODE == M_W13) {
+                a.out[(size_t)b * a.out_stride + r / 2] = (float)(silu_d((double)v0) * (double)v1);
+            } else {
+                int pos = a.tp[2 * b + 1];
+                if (pos < 0 || pos >= a.seq_len) pos = 0;  // flagged by the prep kernel
+                if (r < a.d) {
+                    float o0, o1;
+                    rope_pair(v0, v1, r % a.hs, pos, a.freq, o0, o1);
+                    a.out[(size_t)b * a.out_stride + r] = o0;
+                    a.out[(size_t)b * a.out_stride + r + 1] = o1;
+                } else if (r < a.d + a.kvd) {
+                    const int j = r - a.d;
+                    float o0, o1;
+                    rope_pair(v0, v1, j % a.hs, pos, a.freq, o0, o1);
+                    float* k = a.kc_base + (size_t)b * a.seq_stride + (size_t)pos * a.kvd;
+                    k[j] = o0;
+                    k[j + 1] = o1;
+                } else {
+                    const int j = r - a.d - a.kvd;
+                    float* v = a.vc_base + (size_t)b * a.seq_stride + (size_t)pos * a.kvd;
+                    v[j] = v0;
+                    v[j + 1] = v1;
+                }
+            }
+        }
+    } else {
+        for (int i = threadIdx.x; i < nrows * a.B; i += nt) {
+            const int rr = i / a.B, b = i % a.B;
+            const float v = stage_out[rr][b];
+            float* o = a.out + (size_t)b * a.out_stride + r0 + rr;
+            if (MODE == M_RESID) {
+                *o = *o + v;
+            } else {
+                *o = v;
+                if (v != v) set_error(a.err, DERR_NAN);
+                atomicMax(&best_s[b], argmax_key(v, r0 + rr));
+            }
+        }
+        if (MODE == M_CLS) {
+            asm volatile("bar.sync 1, %0;" :: "r"(32 * BG_WARPS) : "memory");
+            if (threadIdx.x < a.B && best_s[threadIdx.x]) atomicMax(&a.amax[threadIdx.x], best_s[threadIdx.x]);
+        }
+    }
+}
+
+}  // namespace l2c

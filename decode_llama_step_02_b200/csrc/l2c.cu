@@ -21,6 +21,7 @@
 #include <vector>
 
 #include "../../include/l2c.h"
+#include "batched.cuh"
 #include "kernels.cuh"
 
 using namespace l2c;
@@ -57,6 +58,11 @@ struct l2c_ctx {
     int attn_chunk = 64, attn_nchunks = 1;
     // graphs: [q80][gen]
     cudaGraphExec_t graph[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+    // batched Q8_0 step: quantized activations of every sequence, one graph per batch size
+    int8_t* bxq = nullptr;
+    float* bxs = nullptr;
+    size_t bkq = 0, bks = 0;  // strides (bytes of codes, floats of scales) per sequence
+    std::vector<cudaGraphExec_t> bgraph;  // index B (1..max_batch)
     // tuning
     size_t pf_f32 = 256 << 10, pf_q8 = 128 << 10;
     int f32_ctas_per_sm = 1;
@@ -217,6 +223,11 @@ static int set_smem_limits(l2c_ctx* h) {
     CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     CK(cudaFuncSetAttribute(k_gemv_q8<M_W13>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+    CK(cudaFuncSetAttribute(k_bgemm_q8<M_QKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
+    CK(cudaFuncSetAttribute(k_bgemm_q8<M_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
+    CK(cudaFuncSetAttribute(k_bgemm_q8<M_W13>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
+    CK(cudaFuncSetAttribute(k_bgemm_q8<M_CLS>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
+    CK(cudaFuncSetAttribute(k_bprep, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     return L2C_OK;
 }
 
@@ -224,16 +235,23 @@ static int set_smem_limits(l2c_ctx* h) {
 enum StepKernel : int { SK_QKV = 0, SK_ATTN = 1, SK_WO = 2, SK_W13 = 3, SK_W2 = 4, SK_CLS = 5 };
 
 // Enqueues kernel `kind` of layer l (sequence 0) on stream s.
-static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, int l) {
+static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, int l, int seq = 0) {
     g_pdl = h->pdl;
     const size_t d = h->d, kvd = h->kvd, hh = h->h, S = h->S;
-    float* kslot = h->kc + (size_t)l * S * kvd;
-    float* vslot = h->vc + (size_t)l * S * kvd;
+    const size_t cache_off = (size_t)seq * h->L * S * kvd;
+    float* kslot = h->kc + cache_off + (size_t)l * S * kvd;
+    float* vslot = h->vc + cache_off + (size_t)l * S * kvd;
+    float* x = h->x + (size_t)seq * d;
+    float* q = h->q + (size_t)seq * d;
+    float* att = h->att + (size_t)seq * d;
+    float* hb = h->hb + (size_t)seq * hh;
+    int* tp = h->tp + 2 * seq;
+    unsigned long long* amax = h->amax + seq;
     cudaStream_t saved = h->cap;
     h->cap = s;  // launch_gemv enqueues on h->cap
     cudaError_t e = cudaSuccess;
     GemvArgs a = {};
-    a.gs = h->gs; a.tp = h->tp; a.err = h->err; a.vocab = h->V; a.seq_len = h->S;
+    a.gs = h->gs; a.tp = tp; a.err = h->err; a.vocab = h->V; a.seq_len = h->S;
     a.d = (int)d; a.kvd = (int)kvd; a.hs = h->hs;
     switch (kind) {
     case SK_QKV:  // RMSNorm + q/k/v + RoPE + cache write
@@ -241,14 +259,14 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
         a.K = (int)d;
         if (q80) { a.W = h->qWqkv.p + (size_t)l * a.rows * h->qWqkv.rb; a.ld = h->qWqkv.rb; }
         else { a.W = h->Wqkv + (size_t)l * a.rows * d; a.ld = d; }
-        a.in = h->x;
+        a.in = x;
         a.norm_w = h->rms_att + (size_t)l * d;
         if (l == 0) {
             a.emb = q80 ? (const void*)h->qE.p : (const void*)h->E;
-            a.x_resid = h->x;
-            a.amax = h->amax;
+            a.x_resid = x;
+            a.amax = amax;
         }
-        a.out = h->q;
+        a.out = q;
         a.kslot = kslot;
         a.vslot = vslot;
         a.freq = h->freq;
@@ -256,8 +274,8 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
         break;
     case SK_ATTN: {
         AttnArgs t = {};
-        t.q = h->q; t.kc = kslot; t.vc = vslot; t.seq_stride = (size_t)h->L * S * kvd;
-        t.out = h->att; t.tp = h->tp; t.tp_stride = 2;
+        t.q = q; t.kc = kslot; t.vc = vslot; t.seq_stride = (size_t)h->L * S * kvd;
+        t.out = att; t.tp = tp; t.tp_stride = 2;
         t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = (int)kvd; t.seq_len = h->S;
         t.chunk = h->attn_chunk; t.nchunks = h->attn_nchunks;
         t.part = h->attn_part; t.count = h->attn_cnt; t.err = h->err;
@@ -269,28 +287,28 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
         a.rows = (int)d; a.K = (int)d;
         if (q80) { a.W = h->qWo.p + (size_t)l * d * h->qWo.rb; a.ld = h->qWo.rb; }
         else { a.W = h->Wo + (size_t)l * d * d; a.ld = d; }
-        a.in = h->att; a.out = h->x;
+        a.in = att; a.out = x;
         e = launch_gemv<M_RESID>(h, q80, a, 1);
         break;
     case SK_W13:  // RMSNorm + W1/W3 + SwiGLU
         a.rows = (int)(2 * hh); a.K = (int)d;
         if (q80) { a.W = h->qW13.p + (size_t)l * 2 * hh * h->qW13.rb; a.ld = h->qW13.rb; }
         else { a.W = h->W13 + (size_t)l * 2 * hh * d; a.ld = d; }
-        a.in = h->x; a.norm_w = h->rms_ffn + (size_t)l * d; a.out = h->hb;
+        a.in = x; a.norm_w = h->rms_ffn + (size_t)l * d; a.out = hb;
         e = launch_gemv<M_W13>(h, q80, a, 2);
         break;
     case SK_W2:  // W2 + residual
         a.rows = (int)d; a.K = (int)hh;
         if (q80) { a.W = h->qW2.p + (size_t)l * d * h->qW2.rb; a.ld = h->qW2.rb; }
         else { a.W = h->W2 + (size_t)l * d * hh; a.ld = hh; }
-        a.in = h->hb; a.out = h->x;
+        a.in = hb; a.out = x;
         e = launch_gemv<M_RESID>(h, q80, a, 1);
         break;
     default:  // final RMSNorm + classifier + argmax
         a.rows = h->V; a.K = (int)d;
         if (q80) { a.W = h->qWcls.p; a.ld = h->qWcls.rb; }
         else { a.W = h->Wcls; a.ld = d; }
-        a.in = h->x; a.norm_w = h->rms_final; a.out = h->logits; a.amax = h->amax;
+        a.in = x; a.norm_w = h->rms_final; a.out = h->logits + (size_t)seq * h->V; a.amax = amax;
         e = launch_gemv<M_CLS>(h, q80, a, 1);
         break;
     }
@@ -306,6 +324,106 @@ static int enqueue_step(l2c_ctx* h, bool q80) {
         for (int k = SK_QKV; k <= SK_W2; k++)
             if ((rc = launch_step_kernel(h, h->cap, k, q80, l)) != L2C_OK) return rc;
     return launch_step_kernel(h, h->cap, SK_CLS, q80, 0);
+}
+
+// ------------------------------------------------------------- batched step --
+
+// K bytes per GEMM stage: a multiple of 32 (the MMA k) and of 4*gs (16-byte
+// scale copies) that divides K, at most 512.
+static int batched_kc(int K, int gs) {
+    int unit = 4 * gs > 32 ? 4 * gs : 32;
+    for (int kc = 512 - 512 % unit; kc >= unit; kc -= unit)
+        if (K % kc == 0) return kc;
+    return 0;
+}
+
+static int ensure_batched(l2c_ctx* h) {
+    if (h->bxq) return L2C_OK;
+    const size_t kmax = (size_t)(h->d > h->h ? h->d : h->h);
+    h->bkq = (kmax + 15) & ~size_t(15);
+    h->bks = ((kmax / h->gs) + 3) & ~size_t(3);
+    int rc;
+    if ((rc = dalloc(h, (void**)&h->bxq, (size_t)BMAX * h->bkq)) != L2C_OK) return rc;
+    if ((rc = dalloc(h, (void**)&h->bxs, (size_t)BMAX * h->bks * 4)) != L2C_OK) return rc;
+    CK(cudaMemsetAsync(h->bxq, 0, (size_t)BMAX * h->bkq, h->stream));
+    CK(cudaMemsetAsync(h->bxs, 0, (size_t)BMAX * h->bks * 4, h->stream));
+    h->bgraph.assign((size_t)h->max_batch + 1, nullptr);
+    return L2C_OK;
+}
+
+static int bprep(l2c_ctx* h, cudaStream_t s, int B, const float* in, size_t in_stride, int K, const float* norm,
+                 bool emb, unsigned long long* amax) {
+    BPrepArgs p = {};
+    p.in = in; p.in_stride = in_stride; p.norm_w = norm;
+    p.emb = emb ? h->qE.p : nullptr; p.emb_rb = h->qE.rb; p.x_resid = h->x;
+    p.K = K; p.gs = h->gs; p.xq = h->bxq; p.xs = h->bxs; p.kq_stride = h->bkq; p.ks_stride = h->bks;
+    p.tp = h->tp; p.vocab = h->V; p.seq_len = h->S; p.amax = amax; p.err = h->err;
+    CK(launch(s, true, k_bprep, dim3(B), dim3(256), (size_t)K * 4, p));
+    return L2C_OK;
+}
+
+template <int MODE>
+static int bgemm(l2c_ctx* h, cudaStream_t s, int B, const Q8Mat& m, size_t row0, int rows, int K, float* out,
+                 size_t out_stride, int l) {
+    BGemmArgs g = {};
+    g.W = m.p + row0 * m.rb; g.rb = m.rb; g.rows = rows; g.K = K; g.gs = h->gs; g.kc = batched_kc(K, h->gs);
+    g.B = B; g.xq = h->bxq; g.xs = h->bxs; g.kq_stride = h->bkq; g.ks_stride = h->bks;
+    g.out = out; g.out_stride = out_stride;
+    g.kc_base = h->kc + (size_t)l * h->S * h->kvd; g.vc_base = h->vc + (size_t)l * h->S * h->kvd;
+    g.seq_stride = (size_t)h->L * h->S * h->kvd;
+    g.freq = h->freq; g.d = h->d; g.kvd = h->kvd; g.hs = h->hs; g.seq_len = h->S;
+    g.tp = h->tp; g.amax = h->amax; g.err = h->err; g.prefetch_bytes = h->pf_q8;
+    BLayout L = make_blayout(g.kc, h->gs, 3);
+    size_t smem = (size_t)L.ns * L.stage_bytes + 16 * (size_t)L.ns;
+    int grid = (rows + BG_ROWS - 1) / BG_ROWS;
+    CK(launch(s, true, k_bgemm_q8<MODE>, dim3(grid), dim3(32 * (BG_WARPS + 1)), smem, g, L));
+    return L2C_OK;
+}
+
+// One batched Q8_0 step of sequences 0..B-1 on stream s.
+static int enqueue_batch_step(l2c_ctx* h, cudaStream_t s, int B) {
+    g_pdl = h->pdl;
+    const size_t d = h->d, hh = h->h, kvd = h->kvd, S = h->S;
+    AttnKernel ak = attn_kernel_for<double>(h->hs, h->rep);
+    int rc;
+    for (int l = 0; l < h->L; l++) {
+        if ((rc = bprep(h, s, B, h->x, d, (int)d, h->rms_att + (size_t)l * d, l == 0, l == 0 ? h->amax : nullptr)))
+            return rc;
+        if ((rc = bgemm<M_QKV>(h, s, B, h->qWqkv, (size_t)l * (d + 2 * kvd), (int)(d + 2 * kvd), (int)d, h->q, d, l)))
+            return rc;
+        AttnArgs t = {};
+        t.q = h->q; t.kc = h->kc + (size_t)l * S * kvd; t.vc = h->vc + (size_t)l * S * kvd;
+        t.seq_stride = (size_t)h->L * S * kvd; t.out = h->att; t.tp = h->tp; t.tp_stride = 2;
+        t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = (int)kvd; t.seq_len = h->S;
+        t.chunk = h->attn_chunk; t.nchunks = h->attn_nchunks;
+        t.part = h->attn_part; t.count = h->attn_cnt; t.err = h->err;
+        CK(launch(s, true, ak, dim3(h->attn_nchunks, h->Hkv, B), dim3(128), 0, t));
+        if ((rc = bprep(h, s, B, h->att, d, (int)d, nullptr, false, nullptr))) return rc;
+        if ((rc = bgemm<M_RESID>(h, s, B, h->qWo, (size_t)l * d, (int)d, (int)d, h->x, d, l))) return rc;
+        if ((rc = bprep(h, s, B, h->x, d, (int)d, h->rms_ffn + (size_t)l * d, false, nullptr))) return rc;
+        if ((rc = bgemm<M_W13>(h, s, B, h->qW13, (size_t)l * 2 * hh, (int)(2 * hh), (int)d, h->hb, hh, l))) return rc;
+        if ((rc = bprep(h, s, B, h->hb, hh, (int)hh, nullptr, false, nullptr))) return rc;
+        if ((rc = bgemm<M_RESID>(h, s, B, h->qW2, (size_t)l * d, (int)d, (int)hh, h->x, d, l))) return rc;
+    }
+    if ((rc = bprep(h, s, B, h->x, d, (int)d, h->rms_final, false, nullptr))) return rc;
+    return bgemm<M_CLS>(h, s, B, h->qWcls, 0, h->V, (int)d, h->logits, (size_t)h->V, 0);
+}
+
+static int build_batch_graph(l2c_ctx* h, int B) {
+    if (h->bgraph[B]) return L2C_OK;
+    CK(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
+    int rc = enqueue_batch_step(h, h->cap, B);
+    cudaGraph_t g = nullptr;
+    cudaError_t e = cudaStreamEndCapture(h->cap, &g);
+    if (rc != L2C_OK) {
+        if (g) cudaGraphDestroy(g);
+        return rc;
+    }
+    if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "batched capture failed: %s", cudaGetErrorString(e));
+    e = cudaGraphInstantiate(&h->bgraph[B], g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "batched graph instantiate: %s", cudaGetErrorString(e));
+    return L2C_OK;
 }
 
 static int build_graph(l2c_ctx* h, bool q80, bool gen) {
@@ -576,8 +694,61 @@ extern "C" int l2c_generate(l2c_ctx* h, int token0, int pos0, int steps, int q80
 
 extern "C" int l2c_forward_batch(l2c_ctx* h, int B, const int32_t* tokens, const int32_t* pos, int q80,
                                  float* logits_out) {
-    (void)B; (void)tokens; (void)pos; (void)q80; (void)logits_out;
-    return fail(h, L2C_E_STATE, "batched step not available in this build");
+    if (!h || !tokens || !pos || !logits_out || B < 1 || B > h->max_batch)
+        return fail(h, L2C_E_ARG, "forward_batch: need 1 <= B <= max_batch and non-null arrays");
+    if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
+    if (q80 && B > BMAX) return fail(h, L2C_E_ARG, "forward_batch: the Q8_0 batched step takes at most %d sequences", BMAX);
+    const bool tok_dev = is_device_ptr(tokens), pos_dev = is_device_ptr(pos);
+    if (!tok_dev && !pos_dev) {
+        for (int b = 0; b < B; b++) {
+            if (tokens[b] < 0 || tokens[b] >= h->V) return fail(h, L2C_E_ARG, "token[%d]=%d out of range", b, tokens[b]);
+            if (pos[b] < 0 || pos[b] >= h->S) return fail(h, L2C_E_ARG, "pos[%d]=%d out of range", b, pos[b]);
+        }
+    }
+    // (token, pos) pairs into the device words the kernels read; device-side
+    // checks flag out-of-range values passed in device memory
+    CK(cudaMemcpy2DAsync(h->tp, 8, tokens, 4, 4, (size_t)B,
+                         tok_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice, h->stream));
+    CK(cudaMemcpy2DAsync(h->tp + 1, 8, pos, 4, 4, (size_t)B,
+                         pos_dev ? cudaMemcpyDeviceToDevice : cudaMemcpyHostToDevice, h->stream));
+    int rc;
+    if (q80) {
+        if (batched_kc(h->d, h->gs) == 0 || batched_kc(h->h, h->gs) == 0 || h->gs % 32)
+            return fail(h, L2C_E_ARG, "batched Q8_0 step needs gs a multiple of 32 and widths it tiles");
+        if ((rc = ensure_batched(h))) return rc;
+        if (h->graphs) {
+            if ((rc = build_batch_graph(h, B))) return rc;
+            CK(cudaGraphLaunch(h->bgraph[B], h->stream));
+        } else if ((rc = enqueue_batch_step(h, h->stream, B))) {
+            return rc;
+        }
+    } else {
+        // fp32: the single-sequence kernels, one sequence after another
+        for (int b = 0; b < B; b++) {
+            for (int l = 0; l < h->L; l++)
+                for (int k = SK_QKV; k <= SK_W2; k++)
+                    if ((rc = launch_step_kernel(h, h->stream, k, false, l, b))) return rc;
+            if ((rc = launch_step_kernel(h, h->stream, SK_CLS, false, 0, b))) return rc;
+        }
+    }
+    CK(cudaMemcpyAsync(logits_out, h->logits, (size_t)B * h->V * 4, cudaMemcpyDeviceToDevice, h->stream));
+    return L2C_OK;
+}
+
+extern "C" int l2c_attention(l2c_ctx* h, const float* q, const float* k, const float* v, int pos, int precision,
+                             float* out) {
+    if (!h || !q || !k || !v || !out || pos < 0 || pos >= h->S || (precision != 0 && precision != 1))
+        return fail(h, L2C_E_ARG, "attention: need pos in [0, seq_len) and precision 0 or 1");
+    k_set_tp<<<1, 1, 0, h->stream>>>(h->tp, 0, pos);
+    AttnArgs t = {};
+    t.q = q; t.kc = k; t.vc = v; t.seq_stride = 0;
+    t.out = out; t.tp = h->tp; t.tp_stride = 2;
+    t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = h->kvd; t.seq_len = h->S;
+    t.chunk = h->attn_chunk; t.nchunks = h->attn_nchunks;
+    t.part = h->attn_part; t.count = h->attn_cnt; t.err = h->err;
+    AttnKernel ak = precision ? attn_kernel_for<double>(h->hs, h->rep) : attn_kernel_for<float>(h->hs, h->rep);
+    CK(launch(h->stream, false, ak, dim3(h->attn_nchunks, h->Hkv, 1), dim3(128), 0, t));
+    return L2C_OK;
 }
 
 extern "C" int l2c_time_kernel(l2c_ctx* h, int kind, int q80, int iters, float* avg_ms) {
@@ -717,6 +888,8 @@ extern "C" void l2c_destroy(l2c_ctx* h) {
     for (int a = 0; a < 2; a++)
         for (int b = 0; b < 2; b++)
             if (h->graph[a][b]) cudaGraphExecDestroy(h->graph[a][b]);
+    for (cudaGraphExec_t g : h->bgraph)
+        if (g) cudaGraphExecDestroy(g);
     for (void* p : h->allocs) cudaFree(p);
     if (h->cap) cudaStreamDestroy(h->cap);
     delete h;

@@ -182,6 +182,20 @@ L2C_API int l2c_kv_read(l2c_ctx* h, int seq, int n_pos, float* k_host, float* v_
 L2C_API int l2c_kv_reset(l2c_ctx* h, int seq);
 
 /*
+ * l2c_attention - the grouped-query attention of one layer ([qa] GQA and KV
+ * Cache) run alone with the handle's head layout: for query head i, with KV
+ * head g = i / (n_heads / n_kv_heads), scores q_i . k_t / sqrt(head_size)
+ * over t = 0..pos, softmax, and out_i = sum_t a_t v_t.  q_dev [n_heads *
+ * head_size] (already rotated), k_dev and v_dev [>= pos+1][kv_dim] (one
+ * layer's caches), out_dev [n_heads * head_size]; all device fp32.
+ * precision: 0 accumulates in fp32 (as the fp32 step does), 1 in double (as
+ * the Q8_0 step does).  pos must be in [0, seq_len).  Uses the handle's
+ * scratch; asynchronous on the handle's stream.
+ */
+L2C_API int l2c_attention(l2c_ctx* h, const float* q_dev, const float* k_dev, const float* v_dev, int pos,
+                          int precision, float* out_dev);
+
+/*
  * l2c_time_kernel - measurement hook: runs kernel `kind` of the fp32 (q80 = 0)
  * or Q8_0 step alone, iters times back to back on the handle's stream, and
  * stores the average time per launch in ms (two CUDA events around the

@@ -92,3 +92,34 @@ def test_argmax_nan_is_reported(env):
     with pytest.raises(l2c.L2CError) as e:
         dec.argmax(torch.from_numpy(x).cuda())
     assert e.value.code == l2c.L2C_E_DEVICE
+
+
+ATTN_SHAPES = [  # (n_heads, n_kv_heads, head_size, seq_len, positions)
+    (32, 32, 128, 4096, (0, 63, 64, 1000, 4095)),   # 7B shape
+    (32, 8, 128, 2048, (0, 130, 2047)),             # GQA-7B shape
+    (8, 4, 8, 512, (0, 5, 511)),                     # tiny shape
+    (6, 6, 48, 256, (0, 200, 255)),                  # 15M shape
+]
+
+
+@pytest.mark.parametrize("H,Hkv,hs,S,positions", ATTN_SHAPES, ids=["7B", "GQA-7B", "tiny", "15M"])
+def test_attention_matches_oracle(H, Hkv, hs, S, positions):
+    torch, l2c = need_gpu()
+    d = H * hs
+    spec = synth.ModelSpec("attn", d, 4 * d, 1, H, Hkv, 64, S, 1, seed=3)
+    dec = l2c.Decoder(spec.cfg, synth.blob(spec), 1)
+    rng = np.random.default_rng(H * S)
+    kvd = Hkv * hs
+    kc, vc = synth.kv_prefill(spec, seq=0, n_pos=S)
+    kc, vc = kc[0], vc[0]
+    kd, vd = torch.from_numpy(kc).cuda(), torch.from_numpy(vc).cuda()
+    for pos in positions:
+        q = rng.standard_normal(d).astype(np.float32)
+        ref = oracle.attention(q, kc, vc, pos, H, Hkv)
+        for precision, tol in ((0, 2e-6), (1, 1e-7)):
+            out = torch.empty(d, dtype=torch.float32, device="cuda")
+            dec.attention(torch.from_numpy(q).cuda(), kd, vd, pos, out, precision)
+            dec.sync()
+            got = out.cpu().numpy()
+            assert np.abs(got - ref).max() <= tol * np.abs(ref).max(), (pos, precision)
+    dec.close()
