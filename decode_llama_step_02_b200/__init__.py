@@ -15,13 +15,13 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libl2c.so")
 
-L2C_OK, L2C_E_ARG, L2C_E_OOM, L2C_E_CUDA, L2C_E_DEVICE, L2C_E_STATE = 0, -1, -2, -3, -4, -5
+L2C_OK, L2C_E_ARG, L2C_E_OOM, L2C_E_CUDA, L2C_E_DEVICE, L2C_E_STATE, L2C_E_SCRATCH = 0, -1, -2, -3, -4, -5, -6
 
 # every symbol declared in include/l2c.h
 EXPORTS = (
     "l2c_blob_floats", "l2c_create", "l2c_enable_q80", "l2c_forward", "l2c_forward_q80", "l2c_argmax",
     "l2c_generate", "l2c_forward_batch", "l2c_quantize_q80", "l2c_q80_group_dots", "l2c_kv_load",
-    "l2c_kv_read", "l2c_kv_reset", "l2c_attention", "l2c_time_kernel", "l2c_sync", "l2c_stream", "l2c_last_status", "l2c_last_error",
+    "l2c_kv_read", "l2c_kv_reset", "l2c_attention", "l2c_attention_noalloc", "l2c_time_kernel", "l2c_sync", "l2c_stream", "l2c_last_status", "l2c_last_error",
     "l2c_destroy",
 )
 
@@ -66,6 +66,7 @@ def lib():
             "l2c_kv_read": (i32, [vp, i32, i32, vp, vp]),
             "l2c_kv_reset": (i32, [vp, i32]),
             "l2c_attention": (i32, [vp, vp, vp, vp, i32, i32, vp]),
+            "l2c_attention_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
             "l2c_time_kernel": (i32, [vp, i32, i32, i32, ctypes.POINTER(ctypes.c_float)]),
             "l2c_sync": (i32, [vp]),
             "l2c_stream": (vp, [vp]),

@@ -9,7 +9,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libl2c.so")
-SOURCES = [os.path.join(HERE, "csrc", "l2c.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "l2c.cu"), os.path.join(HERE, "csrc", "attention_noalloc.cu")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -1,0 +1,99 @@
+// attention_noalloc.cu - grouped-query attention that allocates no memory.
+//
+// Some callers cannot allocate device memory: their process has handed the
+// GPU's memory to another allocator up front (a framework's pool or a serving
+// engine that reserves HBM at start-up, where a stray cudaMalloc would fail
+// or break the owner's accounting), or they run on a latency-critical path
+// where cudaMalloc and cudaFree may synchronize the device.  Such callers also
+// cannot create an l2c handle, which owns weights, caches and scratch.  For
+// them, l2c_attention_noalloc runs the same attention kernel as
+// l2c_attention on buffers the caller owns.  The kernel's scratch (partial
+// softmax state per KV head and position chunk, arrival counters and the
+// position word) lives in a file-scope __device__ array of fixed size instead
+// of a handle's allocation.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "../../include/l2c.h"
+#include "attention.cuh"
+
+using namespace l2c;
+
+namespace {
+
+// The fixed scratch: 4 MiB, held by every GPU that loads the library until
+// the process exits.  Layout: [0, 256) position word and error word,
+// [256, 256 + 4*n_kv_heads) arrival counters (rounded up to 256 B), then the
+// partial (m, l, o) records of every (KV head, chunk, query head).
+constexpr size_t kScratchBytes = size_t(4) << 20;
+constexpr int kChunk = 64;      // positions per CTA, as in the decode step
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_attn_scratch[kScratchBytes];
+
+std::mutex g_setup_mutex;
+void* g_scratch_addr[kMaxDevices] = {nullptr};
+
+// The device address of g_attn_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is queried
+// once per device with that device current.
+int scratch_on_current_device(unsigned char** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return L2C_E_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return L2C_E_ARG;
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess || !p) return L2C_E_CUDA;
+        g_scratch_addr[dev] = p;
+    }
+    *out = static_cast<unsigned char*>(g_scratch_addr[dev]);
+    return L2C_OK;
+}
+
+// Writes the position word and clears the arrival counters (they must start
+// at zero; the array keeps whatever the previous call left).
+__global__ void k_noalloc_prepare(int* tp, int pos, int* counters, int n) {
+    if (threadIdx.x == 0) {
+        tp[0] = 0;
+        tp[1] = pos;
+        tp[2] = 0;  // error word
+    }
+    for (int i = threadIdx.x; i < n; i += blockDim.x) counters[i] = 0;
+}
+
+}  // namespace
+
+extern "C" int l2c_attention_noalloc(const float* q_dev, const float* k_dev, const float* v_dev, int n_heads,
+                                     int n_kv_heads, int head_size, int pos, int precision, float* out_dev,
+                                     void* cuda_stream) {
+    if (!q_dev || !k_dev || !v_dev || !out_dev || n_heads <= 0 || n_kv_heads <= 0 || head_size <= 0 || pos < 0 ||
+        n_heads % n_kv_heads || (precision != 0 && precision != 1))
+        return L2C_E_ARG;
+    const int rep = n_heads / n_kv_heads;
+    AttnKernel ak = precision ? attn_kernel_for<double>(head_size, rep) : attn_kernel_for<float>(head_size, rep);
+    if (!ak) return L2C_E_ARG;
+    const int nchunks = pos / kChunk + 1;
+    const size_t acc = precision ? sizeof(double) : sizeof(float);
+    const size_t cnt_bytes = ((size_t)n_kv_heads * sizeof(int) + 255) & ~size_t(255);
+    const size_t part_bytes = (size_t)n_kv_heads * nchunks * rep * (head_size + 2) * acc;
+    if (256 + cnt_bytes + part_bytes > kScratchBytes) return L2C_E_SCRATCH;
+    unsigned char* scratch = nullptr;
+    int rc = scratch_on_current_device(&scratch);
+    if (rc != L2C_OK) return rc;
+    int* tp = reinterpret_cast<int*>(scratch);
+    int* counters = reinterpret_cast<int*>(scratch + 256);
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    k_noalloc_prepare<<<1, 256, 0, s>>>(tp, pos, counters, n_kv_heads);
+    if (cudaGetLastError() != cudaSuccess) return L2C_E_CUDA;
+    AttnArgs t = {};
+    t.q = q_dev; t.kc = k_dev; t.vc = v_dev; t.seq_stride = 0;
+    t.out = out_dev; t.tp = tp; t.tp_stride = 2;
+    t.H = n_heads; t.Hkv = n_kv_heads; t.hs = head_size; t.kvd = n_kv_heads * head_size; t.seq_len = pos + 1;
+    t.chunk = kChunk; t.nchunks = nchunks;
+    t.part = scratch + 256 + cnt_bytes; t.count = counters; t.err = tp + 2;
+    ak<<<dim3(nchunks, n_kv_heads, 1), 128, 0, s>>>(t);
+    if (cudaGetLastError() != cudaSuccess) return L2C_E_CUDA;
+    return L2C_OK;
+}

@@ -145,25 +145,6 @@ extern "C" size_t l2c_blob_floats(const l2c_config* c, int shared_weights) {
     return shared_weights ? n : n + V * d;
 }
 
-// ------------------------------------------------------------ attention table --
-
-typedef void (*AttnKernel)(const AttnArgs);
-
-template <typename Acc>
-static AttnKernel attn_kernel_for(int hs, int rep) {
-#define L2C_ATTN(HS_, REP_) \
-    if (hs == HS_ && rep == REP_) return k_attention<Acc, HS_, REP_>;
-    L2C_ATTN(8, 1) L2C_ATTN(8, 2) L2C_ATTN(8, 3) L2C_ATTN(8, 4)
-    L2C_ATTN(16, 1) L2C_ATTN(16, 2) L2C_ATTN(16, 4)
-    L2C_ATTN(32, 1) L2C_ATTN(32, 2) L2C_ATTN(32, 4)
-    L2C_ATTN(48, 1) L2C_ATTN(48, 2) L2C_ATTN(48, 4)
-    L2C_ATTN(64, 1) L2C_ATTN(64, 2) L2C_ATTN(64, 4) L2C_ATTN(64, 8)
-    L2C_ATTN(96, 1) L2C_ATTN(96, 2) L2C_ATTN(96, 4)
-    L2C_ATTN(128, 1) L2C_ATTN(128, 2) L2C_ATTN(128, 4) L2C_ATTN(128, 8)
-#undef L2C_ATTN
-    return nullptr;
-}
-
 // ------------------------------------------------------------- step building --
 
 struct GemvShape {

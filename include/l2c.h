@@ -53,6 +53,7 @@ extern "C" {
 #define L2C_E_CUDA (-3)   /* a CUDA runtime call failed */
 #define L2C_E_DEVICE (-4) /* a kernel recorded an error (see l2c_last_error) */
 #define L2C_E_STATE (-5)  /* call not valid in the handle's state (e.g. Q8_0 not enabled) */
+#define L2C_E_SCRATCH (-6) /* the problem needs more than l2c_attention_noalloc's fixed scratch */
 
 /* The model shape: the seven integers of llama2.c's checkpoint header
  * ([hub] 数据格式: "layers, dimensions, heads ..."; [qa] GQA: kv heads).
@@ -194,6 +195,49 @@ L2C_API int l2c_kv_reset(l2c_ctx* h, int seq);
  */
 L2C_API int l2c_attention(l2c_ctx* h, const float* q_dev, const float* k_dev, const float* v_dev, int pos,
                           int precision, float* out_dev);
+
+/*
+ * l2c_attention_noalloc - l2c_attention for callers that cannot allocate
+ * device memory, with no handle.  (The pages have no counterpart: this is an
+ * interface of this library, not a step of llama2.c.)
+ *
+ * Who needs it: a process whose device memory belongs to another allocator
+ * (a framework's pool or a serving engine that reserves HBM up front, where a
+ * stray cudaMalloc fails or breaks the owner's accounting), or code on a
+ * latency-critical path where cudaMalloc/cudaFree may synchronize the device.
+ * Such callers cannot create an l2c handle either (it owns weights, caches and
+ * scratch), so this entry point takes every shape argument explicitly and
+ * calls no cudaMalloc, cudaFree or allocating library routine.
+ *
+ * Computes exactly what l2c_attention computes, with the same kernel: for
+ * query head i and KV head g = i / (n_heads / n_kv_heads), scores
+ * q_i . k_t / sqrt(head_size) over t = 0..pos, softmax, out_i = sum a_t v_t.
+ * q_dev [n_heads * head_size], k_dev and v_dev [>= pos+1][n_kv_heads *
+ * head_size], out_dev [n_heads * head_size]: device fp32, owned by the
+ * caller.  precision: 0 = fp32 accumulation, 1 = double.  Supported head
+ * sizes and GQA ratios are those of l2c_create.  Enqueued on cuda_stream
+ * (NULL = the legacy stream); returns before the kernels finish.
+ *
+ * Scratch: a fixed 4 MiB device array in the library (every GPU that loads
+ * the library holds it until the process exits).  A call needs
+ * 256 + 4*n_kv_heads (rounded up to 256) + n_kv_heads * (pos/64 + 1) *
+ * (n_heads/n_kv_heads) * (head_size + 2) * (4 or 8 for precision 0 or 1)
+ * bytes; a larger problem is rejected with L2C_E_SCRATCH before anything is
+ * enqueued.  (For 32 heads of 128 that is about 8000 positions in double.)
+ * All calls share the array, so calls that overlap on the GPU (different
+ * streams, or different host threads, without ordering between them) race
+ * and may corrupt each other's results; order them on one stream.  Each call
+ * clears the counters it uses before its kernel runs.
+ *
+ * Set-up: the first call on a device, with that device current, looks up the
+ * array's device address (cudaGetSymbolAddress) and caches it; make that
+ * first call before capturing work on the device's streams.
+ * Errors: L2C_E_ARG (null pointer, bad shape, unsupported head size or ratio),
+ * L2C_E_SCRATCH, L2C_E_CUDA.
+ */
+L2C_API int l2c_attention_noalloc(const float* q_dev, const float* k_dev, const float* v_dev, int n_heads,
+                                  int n_kv_heads, int head_size, int pos, int precision, float* out_dev,
+                                  void* cuda_stream);
 
 /*
  * l2c_time_kernel - measurement hook: runs kernel `kind` of the fp32 (q80 = 0)
