@@ -116,36 +116,70 @@ __device__ __forceinline__ void read_tp(const GemvArgs& a, int& token, int& pos)
 }
 
 // fp32 input into shared memory: RMSNorm (double) when norm_w is set.
-// On layer 0 the input is the embedding row E[token] (fp32 or dequantized
-// Q8_0: code * scale in fp32) and CTA 0 also stores it as the residual x.
-template <bool Q8>
-__device__ void load_input(const GemvArgs& a, int token, float* xs, double* red) {
-    const int K = a.K;
-    const float* in = a.in;
-    const int8_t* eq = nullptr;
-    const float* es = nullptr;
-    if (a.emb) {
-        if (Q8) {
-            const uint8_t* rec = static_cast<const uint8_t*>(a.emb) + (size_t)token * a.ld;
-            eq = reinterpret_cast<const int8_t*>(rec);
-            es = reinterpret_cast<const float*>(rec + K);
-        } else {
-            in = static_cast<const float*>(a.emb) + (size_t)token * a.K;
+// On layer 0 the input is the embedding row E[token] (fp32) and CTA 0 also
+// stores it as the residual x.  Requires K % 4 == 0.  Every thread issues its
+// (at most 8) float4 loads of the input and the gain at once, so the
+// prologue costs one round trip to L2.
+template <bool NORM>
+__device__ void load_input_f32(const GemvArgs& a, int token, float* xs, double* red) {
+    const int K4 = a.K >> 2;
+    const float4* in = reinterpret_cast<const float4*>(
+        a.emb ? static_cast<const float*>(a.emb) + (size_t)token * a.K : a.in);
+    const float4* nw = NORM ? reinterpret_cast<const float4*>(a.norm_w) : nullptr;
+    float4* xs4 = reinterpret_cast<float4*>(xs);
+    constexpr int PER = NORM ? 4 : 8;
+    float4 v[PER], w[NORM ? PER : 1];
+    const int nt = blockDim.x;
+    if (K4 <= PER * nt) {
+#pragma unroll
+        for (int j = 0; j < PER; j++) {
+            const int i = threadIdx.x + j * nt;
+            v[j] = i < K4 ? in[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (NORM) w[NORM ? j : 0] = i < K4 ? nw[i] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        if (a.emb && blockIdx.x == 0) {
+#pragma unroll
+            for (int j = 0; j < PER; j++) {
+                const int i = threadIdx.x + j * nt;
+                if (i < K4) reinterpret_cast<float4*>(a.x_resid)[i] = v[j];
+            }
+        }
+        if (NORM) {
+            double ss = 0.0;
+#pragma unroll
+            for (int j = 0; j < PER; j++)
+                ss += (double)v[j].x * v[j].x + (double)v[j].y * v[j].y + (double)v[j].z * v[j].z +
+                      (double)v[j].w * v[j].w;
+            ss = block_sum(ss, red);
+            const double inv = 1.0 / sqrt(ss / (double)a.K + 1e-5);
+#pragma unroll
+            for (int j = 0; j < PER; j++) {
+                const float4 g = w[NORM ? j : 0];
+                v[j].x = (float)((double)g.x * (inv * (double)v[j].x));
+                v[j].y = (float)((double)g.y * (inv * (double)v[j].y));
+                v[j].z = (float)((double)g.z * (inv * (double)v[j].z));
+                v[j].w = (float)((double)g.w * (inv * (double)v[j].w));
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < PER; j++) {
+            const int i = threadIdx.x + j * nt;
+            if (i < K4) xs4[i] = v[j];
+        }
+        return;
     }
-    for (int i = threadIdx.x; i < K; i += blockDim.x) {
-        float v = eq ? (float)eq[i] * es[i / a.gs] : in[i];
-        xs[i] = v;
-        if (a.emb && blockIdx.x == 0) a.x_resid[i] = v;
+    // wide inputs: a plain strided loop
+    for (int i = threadIdx.x; i < K4; i += nt) {
+        xs4[i] = in[i];
+        if (a.emb && blockIdx.x == 0) reinterpret_cast<float4*>(a.x_resid)[i] = in[i];
     }
-    if (a.norm_w) {
+    if (NORM) {
         __syncthreads();
         double ss = 0.0;
-        for (int i = threadIdx.x; i < K; i += blockDim.x) ss += (double)xs[i] * (double)xs[i];
+        for (int i = threadIdx.x; i < a.K; i += nt) ss += (double)xs[i] * (double)xs[i];
         ss = block_sum(ss, red);
-        double inv = 1.0 / sqrt(ss / (double)K + 1e-5);
-        for (int i = threadIdx.x; i < K; i += blockDim.x)
-            xs[i] = (float)((double)a.norm_w[i] * (inv * (double)xs[i]));
+        const double inv = 1.0 / sqrt(ss / (double)a.K + 1e-5);
+        for (int i = threadIdx.x; i < a.K; i += nt) xs[i] = (float)((double)a.norm_w[i] * (inv * (double)xs[i]));
     }
 }
 
@@ -222,7 +256,7 @@ __global__ void __launch_bounds__(F32_THREADS, 2) k_gemv_f32(const GemvArgs a) {
     int token = 0, pos = 0;
     if (MODE == M_QKV) read_tp(a, token, pos);
     if (MODE == M_QKV && a.amax && blockIdx.x == 0 && threadIdx.x == 0) *a.amax = 0ull;
-    load_input<false>(a, token, xs, red);
+    load_input_f32<MODE != M_RESID>(a, token, xs, red);
     __syncthreads();
     const int K4 = a.K >> 2;
     unsigned long long best = 0ull;
@@ -275,192 +309,361 @@ __device__ __forceinline__ void quantize_group_warp(const float* x, int gs, int8
     if (lane == 0) *s = scale;
 }
 
+// The value of input element i of a Q8_0 GEMV: the embedding row on layer 0
+// (code * scale in fp32), else the input vector; RMSNorm'd (double, rounded
+// once to fp32) when norm_w is set.
+__device__ __forceinline__ float q8_input_value(const GemvArgs& a, const int8_t* eq, const float* es, double inv,
+                                                int i) {
+    float v = eq ? (float)eq[i] * es[i / a.gs] : a.in[i];
+    if (a.norm_w) v = (float)((double)a.norm_w[i] * (inv * (double)v));
+    return v;
+}
+
+// Quantizes the GEMV input (embedding row or input vector, RMSNorm'd when
+// norm_w is set) into shared codes and scales; all threads of the CTA call it.
+// Warp w owns groups w, w + Q8_WARPS, ...; a lane holds elements
+// g*gs + lane + 32e of each of them in registers, so the loads of the whole
+// vector are in flight at once (one round trip to L2) instead of a chain of
+// dependent loads.  Falls back to a plain loop when a lane would need more
+// than Q8_VPL values.
+// Slow path: one group at a time straight from global memory.
+__device__ __noinline__ void q8_quantize_input_loop(const GemvArgs& a, const int8_t* eq, const float* es, int8_t* xq,
+                                                    float* xsc, double* red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int K = a.K, gs = a.gs;
+    double inv = 1.0;
+    if (a.norm_w) {
+        double ss = 0.0;
+        for (int i = threadIdx.x; i < K; i += blockDim.x) {
+            const float v = eq ? (float)eq[i] * es[i / gs] : a.in[i];
+            ss += (double)v * (double)v;
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) red[warp] = ss;
+        __syncthreads();
+        double tot = 0.0;
+        for (int i = 0; i < nw; i++) tot += red[i];
+        inv = 1.0 / sqrt(tot / (double)K + 1e-5);
+    }
+    if (a.emb && blockIdx.x == 0)
+        for (int i = threadIdx.x; i < K; i += blockDim.x) a.x_resid[i] = (float)eq[i] * es[i / gs];
+    for (int g = warp; g < K / gs; g += nw) {
+        float m = 0.f;
+        for (int i = lane; i < gs; i += 32) m = fmaxf(m, fabsf(q8_input_value(a, eq, es, inv, g * gs + i)));
+        m = warp_max(m);
+        const float scale = m / 127.0f;
+        for (int i = lane; i < gs; i += 32) {
+            const float v = q8_input_value(a, eq, es, inv, g * gs + i);
+            xq[g * gs + i] = (int8_t)(int)(scale == 0.f ? 0.f : roundf(v / scale));
+        }
+        if (lane == 0) xsc[g] = scale;
+    }
+}
+
+// Fast path: warp w owns groups w + jg*nw (jg < GMAX); a lane holds elements
+// lane + 32e (e < EPL = gs/32) of each in registers, all loaded at once.
+template <int GMAX, int EPL, bool NORM>
+__device__ __forceinline__ bool q8_quantize_input_regs(const GemvArgs& a, const int8_t* eq, const float* es,
+                                                       int8_t* xq, float* xsc, double* red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int K = a.K, gs = 32 * EPL;
+    const int ng = K / gs;
+    if ((ng + nw - 1) / nw > GMAX) return false;  // uniform across the CTA
+    float v[GMAX][EPL];
+    float w[NORM ? GMAX : 1][EPL];
+#pragma unroll
+    for (int jg = 0; jg < GMAX; jg++) {
+        const int g = warp + jg * nw;
+#pragma unroll
+        for (int e = 0; e < EPL; e++) {
+            const int i = g * gs + lane + 32 * e;
+            v[jg][e] = g < ng ? (eq ? (float)eq[i] * es[g] : a.in[i]) : 0.f;
+            if (NORM) w[NORM ? jg : 0][e] = g < ng ? a.norm_w[i] : 0.f;
+        }
+    }
+    if (a.emb && blockIdx.x == 0) {
+#pragma unroll
+        for (int jg = 0; jg < GMAX; jg++) {
+            const int g = warp + jg * nw;
+#pragma unroll
+            for (int e = 0; e < EPL; e++)
+                if (g < ng) a.x_resid[g * gs + lane + 32 * e] = v[jg][e];
+        }
+    }
+    if (NORM) {
+        double ss = 0.0;
+#pragma unroll
+        for (int jg = 0; jg < GMAX; jg++)
+#pragma unroll
+            for (int e = 0; e < EPL; e++) ss += (double)v[jg][e] * (double)v[jg][e];
+        ss = warp_sum(ss);
+        if (lane == 0) red[warp] = ss;
+        __syncthreads();
+        double tot = 0.0;
+        for (int i = 0; i < nw; i++) tot += red[i];
+        const double inv = 1.0 / sqrt(tot / (double)K + 1e-5);
+#pragma unroll
+        for (int jg = 0; jg < GMAX; jg++)
+#pragma unroll
+            for (int e = 0; e < EPL; e++)
+                v[jg][e] = (float)((double)w[NORM ? jg : 0][e] * (inv * (double)v[jg][e]));
+    }
+#pragma unroll
+    for (int jg = 0; jg < GMAX; jg++) {
+        const int g = warp + jg * nw;
+        if (g < ng) {  // warp-uniform
+            float m = 0.f;
+#pragma unroll
+            for (int e = 0; e < EPL; e++) m = fmaxf(m, fabsf(v[jg][e]));
+            m = warp_max(m);
+            const float scale = m / 127.0f;
+#pragma unroll
+            for (int e = 0; e < EPL; e++) {
+                const float q = scale == 0.f ? 0.f : roundf(v[jg][e] / scale);
+                xq[g * gs + lane + 32 * e] = (int8_t)(int)q;
+            }
+            if (lane == 0) xsc[g] = scale;
+        }
+    }
+    return true;
+}
+
+// Quantizes the GEMV input (embedding row or input vector, RMSNorm'd when
+// norm_w is set) into shared codes and scales; every thread of the CTA calls
+// it.  Register fast paths for gs = 32/64/128 load the whole vector at once
+// (one round trip to L2 instead of a chain of dependent loads).
+template <bool NORM>
+__device__ __forceinline__ void q8_quantize_input(const GemvArgs& a, const int8_t* eq, const float* es, int8_t* xq,
+                                                  float* xsc, double* red) {
+    constexpr int BUDGET = NORM ? 16 : 48;  // values per lane kept in registers
+    bool done = false;
+    if (a.gs == 32) done = q8_quantize_input_regs<BUDGET, 1, NORM>(a, eq, es, xq, xsc, red);
+    else if (a.gs == 64) done = q8_quantize_input_regs<BUDGET / 2, 2, NORM>(a, eq, es, xq, xsc, red);
+    else if (a.gs == 128) done = q8_quantize_input_regs<BUDGET / 4, 4, NORM>(a, eq, es, xq, xsc, red);
+    if (!done) q8_quantize_input_loop(a, eq, es, xq, xsc, red);
+}
+
+// Exact-int32 group dots of UNIT rows (records at rec, stride rb) with the
+// input codes xq, scaled and summed per lane in double.  Lane t covers the 64
+// contiguous bytes [64t, 64t+64) of a row: one group at GS = 64, two at
+// GS = 32, half of one at GS = 128 (a lane pair).  The four 16-byte reads of a
+// lane are rotated by (lane >> 1) & 3 so that a quarter-warp touches eight
+// distinct 16-byte bank groups.  Requires K % 64 == 0.
+template <int GS, int UNIT>
+__device__ __forceinline__ void q8_rows_dot64(const uint8_t* rec, size_t rb, const int8_t* xq, const double* sxd,
+                                              int K, double (&acc)[UNIT]) {
+    const int lane = threadIdx.x & 31;
+    const int n64 = K >> 6;
+    const int rot = (lane >> 1) & 3;
+#pragma unroll
+    for (int r = 0; r < UNIT; r++) acc[r] = 0.0;
+    for (int t0 = 0; t0 < n64; t0 += 32) {
+        const int t = t0 + lane;
+        const bool in = t < n64;
+        int4 xv[4];
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const int f = (j + rot) & 3;
+            xv[j] = in ? *reinterpret_cast<const int4*>(xq + 64 * t + 16 * f) : make_int4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int r = 0; r < UNIT; r++) {
+            const uint8_t* row = rec + r * rb;
+            int c[4];
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const int f = (j + rot) & 3;
+                const int4 wv = in ? *reinterpret_cast<const int4*>(row + 64 * t + 16 * f) : make_int4(0, 0, 0, 0);
+                int dd = __dp4a(wv.x, xv[j].x, 0);
+                dd = __dp4a(wv.y, xv[j].y, dd);
+                dd = __dp4a(wv.z, xv[j].z, dd);
+                c[j] = __dp4a(wv.w, xv[j].w, dd);
+            }
+            const float* sw = reinterpret_cast<const float*>(row + K);
+            if (GS == 64) {
+                const int d = (c[0] + c[1]) + (c[2] + c[3]);
+                if (in) acc[r] += (double)d * (double)sw[t] * sxd[t];
+            } else if (GS == 32) {
+                // chunk f of step j: the group of the lane's first 32 bytes is f < 2
+                int lo = 0, hi = 0;
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const int f = (j + rot) & 3;
+                    lo += f < 2 ? c[j] : 0;
+                    hi += f < 2 ? 0 : c[j];
+                }
+                if (in) {
+                    acc[r] += (double)lo * (double)sw[2 * t] * sxd[2 * t];
+                    acc[r] += (double)hi * (double)sw[2 * t + 1] * sxd[2 * t + 1];
+                }
+            } else {  // GS == 128: lanes 2m and 2m+1 hold the two halves of group t/2
+                int d = (c[0] + c[1]) + (c[2] + c[3]);
+                d += __shfl_xor_sync(0xffffffffu, d, 1);
+                if (in && (t & 1) == 0) acc[r] += (double)d * (double)sw[t >> 1] * sxd[t >> 1];
+            }
+        }
+    }
+}
+
 struct Q8Layout {
-    // shared memory carve-up of k_gemv_q8
-    int ns;            // ring stages
-    int units_per_stage;
-    size_t stage_bytes;
-    int stage_fp32;    // 1: the input is normalised (or dequantized) into shared fp32 first
+    int nslot;          // ring slots per warp, one unit (UNIT row records) each
+    size_t unit_bytes;  // UNIT * record bytes
 };
 
-// One warp per unit (row or row pair) of each stage.  Warp `nwc` is the
-// producer: lane 0 issues the bulk copies.  Dynamic shared memory:
-//   ring [ns][stage_bytes] | x fp32 [K] (only with stage_fp32) | x codes [K]
-//   | x scales [K/gs] | barriers
-template <int MODE>
-__global__ void __launch_bounds__(288, 1) k_gemv_q8(const GemvArgs a, const Q8Layout L) {
+constexpr int Q8_WARPS = 8;
+
+// Every warp streams its own units (round-robin over the CTA's contiguous
+// range) through its own ring of `nslot` shared-memory slots filled by 1-D bulk
+// copies; lane 0 issues a copy as soon as the warp has finished with a slot,
+// so nslot-1 units per warp stay in flight.  GS is the group size of the
+// 64-byte-per-lane dot (32, 64 or 128, K % 64 == 0), or 0 for the generic
+// 16-byte-per-lane loop.  Dynamic shared memory:
+//   slots [Q8_WARPS][nslot][unit_bytes] | x codes [K, padded to 16] |
+//   x scales [K/gs] fp32 | x scales [K/gs] double | barriers [Q8_WARPS][nslot]
+template <int MODE, int GS>
+__global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, const Q8Layout L) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int UNIT = (MODE == M_QKV || MODE == M_W13) ? 2 : 1;
-    __shared__ double red[32];
-    __shared__ unsigned long long best_s[32];
+    __shared__ double red[Q8_WARPS];
+    __shared__ unsigned long long best_s[Q8_WARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int nwc = (blockDim.x >> 5) - 1;  // consumer warps
     const int K = a.K, gs = a.gs;
     const size_t rb = a.ld;
-    uint8_t* ring = smem;
-    float* xs = reinterpret_cast<float*>(smem + (size_t)L.ns * L.stage_bytes);
-    int8_t* xq = reinterpret_cast<int8_t*>(xs + (L.stage_fp32 ? K : 0));
+    const int ns = L.nslot;
+    uint8_t* slots = smem + (size_t)warp * ns * L.unit_bytes;
+    int8_t* xq = reinterpret_cast<int8_t*>(smem + (size_t)Q8_WARPS * ns * L.unit_bytes);
     float* xsc = reinterpret_cast<float*>(xq + ((K + 15) & ~15));
-    uint64_t* full = reinterpret_cast<uint64_t*>(
-        (reinterpret_cast<uintptr_t>(xsc + K / gs) + 15) & ~uintptr_t(15));
-    uint64_t* empty = full + L.ns;
+    double* sxd = reinterpret_cast<double*>((reinterpret_cast<uintptr_t>(xsc + K / gs) + 15) & ~uintptr_t(15));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sxd + ((K / gs + 1) & ~1));
+    uint64_t* full = bars + warp * ns;
 
     const int units = a.rows / UNIT;
     const int u0 = (int)((long long)units * blockIdx.x / gridDim.x);
     const int u1 = (int)((long long)units * (blockIdx.x + 1) / gridDim.x);
-    const int nunits = u1 - u0;
-    const int ups = L.units_per_stage;
-    const int nstages = (nunits + ups - 1) / ups;
-    const uint8_t* Wb = static_cast<const uint8_t*>(a.W) + (size_t)u0 * UNIT * rb;
+    const int nmine = (u1 - u0 - warp + Q8_WARPS - 1) / Q8_WARPS;  // units of this warp
+    const uint8_t* Wb = static_cast<const uint8_t*>(a.W);
+    const uint64_t pol = policy_evict_first();
+    auto unit_src = [&](int k) { return Wb + (size_t)(u0 + warp + k * Q8_WARPS) * UNIT * rb; };
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < L.ns; s++) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], nwc);
-        }
+    // weights do not depend on earlier kernels: start streaming before the wait
+    if (lane == 0) {
+        for (int s = 0; s < ns; s++) mbar_init(&full[s], 1);
         mbar_fence_init();
-    }
-    __syncthreads();
-
-    if (warp == nwc) {
-        // ---------------- producer: weights do not depend on earlier kernels
-        if (lane == 0 && nstages > 0) {
-            const uint64_t pol = policy_evict_first();
-            size_t total = (size_t)nunits * UNIT * rb;
-            size_t ring_bytes = (size_t)L.ns * L.stage_bytes;
-            if (a.prefetch_bytes && total > ring_bytes) {
-                size_t pf = total - ring_bytes;
-                if (pf > a.prefetch_bytes) pf = a.prefetch_bytes;
-                prefetch_l2_range(Wb + ring_bytes, pf, policy_evict_last());
-            }
-            int issued = 0;
-            bool ok = true;
-            for (int i = 0; i < nstages; i++) {
-                int s = i % L.ns;
-                if (i >= L.ns && !mbar_wait_bounded(&empty[s], ((i / L.ns) - 1) & 1, a.err)) {
-                    ok = false;
-                    break;
-                }
-                int nu = min(ups, nunits - i * ups);
-                uint32_t bytes = (uint32_t)((size_t)nu * UNIT * rb);
-                mbar_arrive_expect_tx(&full[s], bytes);
-                bulk_g2s(ring + (size_t)s * L.stage_bytes, Wb + (size_t)i * ups * UNIT * rb, bytes, &full[s], pol);
-                issued = i + 1;
-            }
-            if (!ok) {
-                // drain the copies still in flight before leaving (bounded)
-                for (int i = max(0, issued - L.ns); i < issued; i++)
-                    mbar_wait_bounded(&full[i % L.ns], (i / L.ns) & 1, a.err);
+        for (int k = 0; k < ns && k < nmine; k++) {
+            mbar_arrive_expect_tx(&full[k], (uint32_t)L.unit_bytes);
+            bulk_g2s(slots + (size_t)k * L.unit_bytes, unit_src(k), (uint32_t)L.unit_bytes, &full[k], pol);
+        }
+        if (warp == 0 && a.prefetch_bytes) {
+            // the CTA's rows beyond the first slots of every warp, into L2
+            const size_t first = (size_t)(u0 + Q8_WARPS * ns) * UNIT * rb;
+            const size_t last = (size_t)u1 * UNIT * rb;
+            if (last > first) {
+                size_t bytes = last - first;
+                if (bytes > a.prefetch_bytes) bytes = a.prefetch_bytes;
+                prefetch_l2_range(Wb + first, bytes, policy_evict_last());
             }
         }
-        return;
     }
-
-    // ---------------- consumers
     grid_dep_wait();
     grid_dep_launch();
+
+    // ---- input: token/pos, optional RMSNorm, Q8_0 codes of every group
     int token = 0, pos = 0;
     if (MODE == M_QKV) read_tp(a, token, pos);
     if (MODE == M_QKV && a.amax && blockIdx.x == 0 && threadIdx.x == 0) *a.amax = 0ull;
-    // input (RMSNorm in double) then Q8_0 quantization, one warp per group.
-    {
-        // load_input uses blockDim-strided loops; restrict to consumer threads
-        const int nct = nwc * 32;
-        const int8_t* eq = nullptr;
-        const float* es = nullptr;
-        if (a.emb) {
-            const uint8_t* rec = static_cast<const uint8_t*>(a.emb) + (size_t)token * a.ld;
-            eq = reinterpret_cast<const int8_t*>(rec);
-            es = reinterpret_cast<const float*>(rec + K);
-        }
-        if (L.stage_fp32) {
-            for (int i = threadIdx.x; i < K; i += nct) {
-                float v = eq ? (float)eq[i] * es[i / gs] : a.in[i];
-                xs[i] = v;
-                if (eq && blockIdx.x == 0) a.x_resid[i] = v;
-            }
-            asm volatile("bar.sync 1, %0;" :: "r"(nct) : "memory");
-        }
-        if (L.stage_fp32 && a.norm_w) {
-            double ss = 0.0;
-            for (int i = threadIdx.x; i < K; i += nct) ss += (double)xs[i] * (double)xs[i];
-            ss = warp_sum(ss);
-            if (lane == 0) red[warp] = ss;
-            asm volatile("bar.sync 1, %0;" :: "r"(nct) : "memory");
-            double tot = 0.0;
-            for (int i = 0; i < nwc; i++) tot += red[i];
-            double inv = 1.0 / sqrt(tot / (double)K + 1e-5);
-            for (int i = threadIdx.x; i < K; i += nct)
-                xs[i] = (float)((double)a.norm_w[i] * (inv * (double)xs[i]));
-            asm volatile("bar.sync 1, %0;" :: "r"(nct) : "memory");
-        }
-        const float* src = L.stage_fp32 ? xs : a.in;
-        for (int g = warp; g < K / gs; g += nwc) quantize_group_warp(src + g * gs, gs, xq + g * gs, xsc + g);
-        asm volatile("bar.sync 1, %0;" :: "r"(nct) : "memory");
+    const int8_t* eq = nullptr;
+    const float* es = nullptr;
+    if (a.emb) {
+        const uint8_t* rec = static_cast<const uint8_t*>(a.emb) + (size_t)token * a.ld;
+        eq = reinterpret_cast<const int8_t*>(rec);
+        es = reinterpret_cast<const float*>(rec + K);
     }
+    q8_quantize_input<MODE != M_RESID>(a, eq, es, xq, xsc, red);
+    __syncthreads();
+    for (int g = threadIdx.x; g < K / gs; g += blockDim.x) sxd[g] = (double)xsc[g];
+    __syncthreads();
 
-    const int nchunk = K >> 4;              // 16-byte chunks per row
-    const int cpg = gs >> 4;                // chunks per group
+    // ---- stream this warp's units
+    const int nchunk = K >> 4;   // 16-byte chunks per row
+    const int cpg = gs >> 4;     // chunks per group
     const int iters = (nchunk + 31) >> 5;
     unsigned long long best = 0ull;
-    bool ok = true;
-    for (int i = 0; i < nstages && ok; i++) {
-        const int s = i % L.ns;
-        if (!mbar_wait_bounded(&full[s], (i / L.ns) & 1, a.err)) { ok = false; break; }
-        const int nu = min(ups, nunits - i * ups);
-        if (warp < nu) {
-            const int u = u0 + i * ups + warp;
-            const uint8_t* base = ring + (size_t)s * L.stage_bytes + (size_t)warp * UNIT * rb;
-            double accd[UNIT];
+    for (int k = 0; k < nmine; k++) {
+        const int s = k % ns;
+        if (!mbar_wait_bounded(&full[s], (k / ns) & 1, a.err)) {
+            // give up: let the copies already issued land before the CTA leaves
+            for (int j = k + 1; j < nmine && j < k + ns; j++) mbar_wait_bounded(&full[j % ns], (j / ns) & 1, a.err);
+            return;
+        }
+        const uint8_t* base = slots + (size_t)s * L.unit_bytes;
+        double acc[UNIT];
+        if (GS != 0) {
+            q8_rows_dot64<GS == 0 ? 64 : GS, UNIT>(base, rb, xq, sxd, K, acc);
+        } else {
 #pragma unroll
-            for (int r = 0; r < UNIT; r++) {
-                const uint8_t* rec = base + r * rb;
-                const float* sw = reinterpret_cast<const float*>(rec + K);
-                double acc = 0.0;
-                for (int it = 0; it < iters; it++) {
-                    const int c = lane + 32 * it;
-                    int dsum = 0;
-                    if (c < nchunk) {
-                        int4 wv = *reinterpret_cast<const int4*>(rec + 16 * c);
-                        int4 xv = *reinterpret_cast<const int4*>(xq + 16 * c);
-                        dsum = __dp4a(wv.x, xv.x, dsum);
-                        dsum = __dp4a(wv.y, xv.y, dsum);
-                        dsum = __dp4a(wv.z, xv.z, dsum);
-                        dsum = __dp4a(wv.w, xv.w, dsum);
-                    }
-                    for (int o = 1; o < cpg; o <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
-                    if (c < nchunk && (c & (cpg - 1)) == 0) {
-                        const int g = c / cpg;
-                        acc += (double)dsum * (double)sw[g] * (double)xsc[g];
+            for (int r = 0; r < UNIT; r++) acc[r] = 0.0;
+            for (int it = 0; it < iters; it++) {
+                const int c = lane + 32 * it;
+                const bool in = c < nchunk;
+                int dsum[UNIT];
+                int4 xv = in ? *reinterpret_cast<const int4*>(xq + 16 * c) : make_int4(0, 0, 0, 0);
+#pragma unroll
+                for (int r = 0; r < UNIT; r++) {
+                    dsum[r] = 0;
+                    if (in) {
+                        const int4 wv = *reinterpret_cast<const int4*>(base + r * rb + 16 * c);
+                        dsum[r] = __dp4a(wv.x, xv.x, dsum[r]);
+                        dsum[r] = __dp4a(wv.y, xv.y, dsum[r]);
+                        dsum[r] = __dp4a(wv.z, xv.z, dsum[r]);
+                        dsum[r] = __dp4a(wv.w, xv.w, dsum[r]);
                     }
                 }
-                accd[r] = warp_sum(acc);
-            }
-            if (lane == 0) {
-                if (MODE == M_QKV) {
-                    epi_qkv(a, u, (float)accd[0], (float)accd[UNIT - 1], pos);
-                } else if (MODE == M_W13) {
-                    epi_w13(a, u, (float)accd[0], (float)accd[UNIT - 1]);
-                } else if (MODE == M_RESID) {
-                    a.out[u] = a.out[u] + (float)accd[0];
-                } else {
-                    float v = (float)accd[0];
-                    a.out[u] = v;
-                    if (v != v) set_error(a.err, DERR_NAN);
-                    unsigned long long k = argmax_key(v, u);
-                    best = k > best ? k : best;
+                for (int o = 1; o < cpg; o <<= 1) {
+#pragma unroll
+                    for (int r = 0; r < UNIT; r++) dsum[r] += __shfl_xor_sync(0xffffffffu, dsum[r], o);
+                }
+                if (in && (c & (cpg - 1)) == 0) {
+                    const int g = c / cpg;
+#pragma unroll
+                    for (int r = 0; r < UNIT; r++) {
+                        const float* sw = reinterpret_cast<const float*>(base + r * rb + K);
+                        acc[r] += (double)dsum[r] * (double)sw[g] * sxd[g];
+                    }
                 }
             }
         }
+        // refill the slot with the unit ns ahead once every lane is done with it
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        if (lane == 0 && k + ns < nmine) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive_expect_tx(&full[s], (uint32_t)L.unit_bytes);
+            bulk_g2s(slots + (size_t)s * L.unit_bytes, unit_src(k + ns), (uint32_t)L.unit_bytes, &full[s], pol);
+        }
+#pragma unroll
+        for (int r = 0; r < UNIT; r++) acc[r] = warp_sum(acc[r]);
+        const int u = u0 + warp + k * Q8_WARPS;
+        if (lane == 0) {
+            if (MODE == M_QKV) {
+                epi_qkv(a, u, (float)acc[0], (float)acc[UNIT - 1], pos);
+            } else if (MODE == M_W13) {
+                epi_w13(a, u, (float)acc[0], (float)acc[UNIT - 1]);
+            } else if (MODE == M_RESID) {
+                a.out[u] = a.out[u] + (float)acc[0];
+            } else {
+                const float v = (float)acc[0];
+                a.out[u] = v;
+                if (v != v) set_error(a.err, DERR_NAN);
+                const unsigned long long key = argmax_key(v, u);
+                best = key > best ? key : best;
+            }
+        }
     }
     if (MODE == M_CLS) {
         if (lane == 0) best_s[warp] = best;
-        asm volatile("bar.sync 1, %0;" :: "r"(nwc * 32) : "memory");
+        __syncthreads();
         if (threadIdx.x == 0) {
             unsigned long long b = 0ull;
-            for (int i = 0; i < nwc; i++) b = best_s[i] > b ? best_s[i] : b;
+            for (int i = 0; i < Q8_WARPS; i++) b = best_s[i] > b ? best_s[i] : b;
             if (b) atomicMax(a.amax, b);
         }
     }

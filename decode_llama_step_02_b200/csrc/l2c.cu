@@ -66,6 +66,7 @@ struct l2c_ctx {
     // tuning
     size_t pf_f32 = 256 << 10, pf_q8 = 128 << 10;
     int f32_ctas_per_sm = 1;
+    size_t q8_smem_budget = 220 << 10;  // dynamic shared memory of one Q8_0 GEMV CTA
     bool pdl = true;     // programmatic dependent launch between the step's kernels
     bool graphs = true;  // replay the step as a CUDA graph (off: plain launches)
     std::vector<void*> allocs;
@@ -151,27 +152,19 @@ struct GemvShape {
     int rows, K, unit;
 };
 
-static Q8Layout q8_layout(const l2c_ctx* h, int K, size_t rb, int unit, int* nwc_out) {
-    (void)h;
-    int nwc = (unit == 2) ? 4 : (K > 4096 ? 4 : 8);
+// Ring slots per warp: as many as fit next to the input codes, 2..8.
+static Q8Layout q8_layout(const l2c_ctx* h, int K, int gs, size_t rb, int unit, size_t* smem_out) {
     Q8Layout L = {};
-    L.units_per_stage = nwc;
-    L.stage_bytes = (size_t)nwc * unit * rb;
-    size_t budget = 96 << 10;
-    int ns = (int)(budget / L.stage_bytes);
-    L.ns = ns < 2 ? 2 : (ns > 4 ? 4 : ns);
-    *nwc_out = nwc;
-    return L;
-}
-
-static size_t q8_smem(int K, int gs, const Q8Layout& L, bool stage_fp32) {
-    size_t b = (size_t)L.ns * L.stage_bytes;
-    if (stage_fp32) b += (size_t)K * 4;
-    b += ((size_t)K + 15) & ~size_t(15);
-    b += (size_t)(K / gs) * 4;
+    L.unit_bytes = (size_t)unit * rb;
+    size_t fixed = (((size_t)K + 15) & ~size_t(15)) + (size_t)(K / gs) * 4 + 16 + (size_t)((K / gs + 1) & ~1) * 8;
+    size_t budget = h->q8_smem_budget;
+    int ns = (int)((budget - fixed - 16 * 8 * Q8_WARPS) / ((size_t)Q8_WARPS * L.unit_bytes));
+    L.nslot = ns < 2 ? 2 : (ns > 8 ? 8 : ns);
+    size_t b = (size_t)Q8_WARPS * L.nslot * L.unit_bytes + fixed;
     b = (b + 15) & ~size_t(15);
-    b += 16 * (size_t)L.ns;
-    return b;
+    b += 8 * (size_t)Q8_WARPS * L.nslot;
+    *smem_out = b;
+    return L;
 }
 
 template <int MODE>
@@ -183,14 +176,16 @@ static cudaError_t launch_gemv(l2c_ctx* h, bool q80, GemvArgs a, int unit) {
         a.prefetch_bytes = h->pf_f32;
         return launch(h->cap, true, k_gemv_f32<MODE>, dim3(grid), dim3(F32_THREADS), (size_t)a.K * 4, a);
     }
-    int nwc = 8;
-    Q8Layout L = q8_layout(h, a.K, a.ld, unit, &nwc);
-    L.stage_fp32 = (a.norm_w != nullptr || a.emb != nullptr) ? 1 : 0;
-    size_t smem = q8_smem(a.K, a.gs, L, L.stage_fp32 != 0);
+    size_t smem = 0;
+    Q8Layout L = q8_layout(h, a.K, a.gs, a.ld, unit, &smem);
     int grid = h->sms;
     if (grid > units) grid = units;
     a.prefetch_bytes = h->pf_q8;
-    return launch(h->cap, true, k_gemv_q8<MODE>, dim3(grid), dim3(32 * (nwc + 1)), smem, a, L);
+    const bool k64 = a.K % 64 == 0;
+    if (k64 && a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64>, dim3(grid), dim3(32 * Q8_WARPS), smem, a, L);
+    if (k64 && a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32>, dim3(grid), dim3(32 * Q8_WARPS), smem, a, L);
+    if (k64 && a.gs == 128) return launch(h->cap, true, k_gemv_q8<MODE, 128>, dim3(grid), dim3(32 * Q8_WARPS), smem, a, L);
+    return launch(h->cap, true, k_gemv_q8<MODE, 0>, dim3(grid), dim3(32 * Q8_WARPS), smem, a, L);
 }
 
 static int set_smem_limits(l2c_ctx* h) {
@@ -200,10 +195,13 @@ static int set_smem_limits(l2c_ctx* h) {
     CK(cudaFuncSetAttribute(k_gemv_f32<M_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     CK(cudaFuncSetAttribute(k_gemv_f32<M_W13>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     CK(cudaFuncSetAttribute(k_gemv_f32<M_CLS>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_QKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_W13>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+#define L2C_Q8_ATTR(GS_)                                                                                           \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_QKV, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096)); \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_W13, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+    L2C_Q8_ATTR(0) L2C_Q8_ATTR(32) L2C_Q8_ATTR(64) L2C_Q8_ATTR(128)
+#undef L2C_Q8_ATTR
     CK(cudaFuncSetAttribute(k_bgemm_q8<M_QKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
     CK(cudaFuncSetAttribute(k_bgemm_q8<M_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
     CK(cudaFuncSetAttribute(k_bgemm_q8<M_W13>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
@@ -484,6 +482,7 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
     h->S = cfg->seq_len; h->rep = h->H / h->Hkv;
     h->pf_f32 = env_size("L2C_PREFETCH_F32", h->pf_f32);
     h->pf_q8 = env_size("L2C_PREFETCH_Q8", h->pf_q8);
+    h->q8_smem_budget = env_size("L2C_Q8_SMEM", h->q8_smem_budget);
     h->f32_ctas_per_sm = (int)env_size("L2C_F32_CTAS_PER_SM", 1);
     h->attn_chunk = (int)env_size("L2C_ATTN_CHUNK", 64);
     h->pdl = env_size("L2C_NO_PDL", 0) == 0;

@@ -17,6 +17,8 @@ pytestmark = pytest.mark.gpu
 ODD = synth.ModelSpec("odd", 48, 100, 2, 6, 2, 50, 160, 0, seed=10, wsigma=0.2, nsigma=0.1)
 ODDQ = synth.ModelSpec("oddq", 96, 160, 3, 6, 3, 300, 200, 0, seed=11, wsigma=0.1, nsigma=0.1)
 GQA_SMALL = synth.ModelSpec("gqa-small", 256, 688, 2, 8, 2, 1000, 300, 0, seed=12)
+# widths that are multiples of 64: the Q8_0 GEMV's 64-bytes-per-lane path
+Q64 = synth.ModelSpec("q64", 256, 768, 2, 4, 2, 700, 200, 0, seed=14)
 
 
 @pytest.fixture(scope="module")
@@ -56,8 +58,9 @@ def test_fp32_teacher_forced(gpu, spec, steps):
     assert errs.max() <= TOL_F32, errs
 
 
-@pytest.mark.parametrize("spec,gs,steps", [(synth.M15, 32, 40), (ODDQ, 32, 70), (GQA_SMALL, 16, 70)],
-                         ids=["15M-gs32", "oddq-gs32", "gqa-small-gs16"])
+@pytest.mark.parametrize("spec,gs,steps", [(synth.M15, 32, 40), (ODDQ, 32, 70), (GQA_SMALL, 16, 70),
+                                           (Q64, 32, 70), (Q64, 64, 70), (Q64, 128, 70)],
+                         ids=["15M-gs32", "oddq-gs32", "gqa-small-gs16", "q64-gs32", "q64-gs64", "q64-gs128"])
 def test_q80_teacher_forced(gpu, spec, gs, steps):
     errs = _forced(gpu, spec, steps, gs)
     assert errs.max() <= TOL_Q80, errs
