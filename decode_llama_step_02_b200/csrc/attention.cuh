@@ -19,29 +19,33 @@ struct AttnArgs {
     const int* tp;       // {token, pos} per sequence, stride tp_stride ints
     int tp_stride;
     int H, Hkv, hs, kvd, seq_len;
-    int chunk;           // positions per CTA
-    int nchunks;         // gridDim.x
+    int nchunks;         // gridDim.x: the positions 0..pos are split into this many chunks
     void* part;          // partials [B][Hkv][nchunks][rep][hs+2] (Acc)
     int* count;          // [B][Hkv] arrival counters (zero between launches)
     int* err;
 };
 
-// grid (nchunks, Hkv, B), 128 threads.  CTA (c, g, b) handles positions
-// [c*chunk, min((c+1)*chunk, pos+1)) of sequence b for the rep = H/Hkv query
-// heads sharing KV head g (heads g*rep .. g*rep+rep-1: contiguous groups).
-// Each active CTA writes (m, l, o) per head: the running max of the scaled
-// scores, the sum of exp(s - m) and the unnormalised weighted V sum.  The
-// last CTA to arrive for (b, g) merges the partials and writes the output.
+// grid (nchunks, Hkv, B), 128 threads.  The positions 0..pos of sequence b
+// are split into nchunks equal chunks (ceil((pos+1)/nchunks) each); CTA
+// (c, g, b) handles chunk c for the rep = H/Hkv query heads sharing KV head g
+// (heads g*rep .. g*rep+rep-1: contiguous groups), so every K/V row is read
+// once per group.  Within a CTA, sub-chunks of TC positions go through three
+// passes: scores (one warp per position: the row slice is one coalesced
+// 16-byte-per-lane load, the dot a warp reduction), the sub-chunk max and
+// exp(s - m), and the weighted V sum (one warp per position again).  Each
+// active CTA writes (m, l, o) per head: the running max of the scaled scores,
+// the sum of exp(s - m) and the unnormalised weighted V sum.  The last CTA to
+// arrive for (b, g) merges the partials and writes the output.
 template <typename Acc, int HS, int REP>
 __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
-    constexpr int NT = 128;
+    static_assert(HS % 4 == 0 && HS <= 128, "head size");
+    constexpr int NT = 128, NW = 4;
     constexpr int TC = 64;                 // positions per sub-chunk held in shared memory
-    constexpr int V4 = HS / 4;             // float4 per K/V row slice
-    constexpr int PVL = (V4 + 31) / 32;    // float4 per lane in the weighted V sum
-    __shared__ Acc qs[REP][HS];
+    constexpr int V4 = HS / 4;             // float4 per K/V row slice (<= 32: one per lane)
+    constexpr int PB = 8;                  // positions a warp loads before reducing
     __shared__ Acc sc[TC][REP];
-    __shared__ Acc red[4][REP];
-    __shared__ Acc ostage[4][REP][HS];
+    __shared__ Acc red[NW][REP];
+    __shared__ Acc ostage[NW][REP][HS];
     __shared__ int last_s;
     const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -51,44 +55,53 @@ __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
     int pos = a.tp[b * a.tp_stride + 1];
     if (pos < 0 || pos >= a.seq_len) pos = 0;  // the GEMV kernel has flagged it
     const int T = pos + 1;
-    const int nact = (T + a.chunk - 1) / a.chunk;  // active chunks for this sequence
+    const int chunk = (T + a.nchunks - 1) / a.nchunks;
+    const int nact = (T + chunk - 1) / chunk;  // active chunks for this sequence
     if (c >= nact) return;
-    const int t0 = c * a.chunk, t1 = min(T, t0 + a.chunk);
+    const int t0 = c * chunk, t1 = min(T, t0 + chunk);
     const float* kc = a.kc + (size_t)b * a.seq_stride + (size_t)g * HS;
     const float* vc = a.vc + (size_t)b * a.seq_stride + (size_t)g * HS;
     const float* q = a.q + (size_t)b * a.H * HS + (size_t)g * REP * HS;
-    for (int i = tid; i < REP * HS; i += NT) qs[i / HS][i % HS] = (Acc)q[i];
+    const bool lane_on = lane < V4;
+    // this lane's four q values of every head, converted once
+    Acc qr[REP][4];
+#pragma unroll
+    for (int h = 0; h < REP; h++) {
+        float4 qv = lane_on ? *reinterpret_cast<const float4*>(q + (size_t)h * HS + 4 * lane)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        qr[h][0] = (Acc)qv.x; qr[h][1] = (Acc)qv.y; qr[h][2] = (Acc)qv.z; qr[h][3] = (Acc)qv.w;
+    }
     const Acc scale = (Acc)1 / sqrt((Acc)HS);
 
-    Acc m[REP], l[REP], o[REP][PVL][4];
+    Acc m[REP], l[REP], o[REP][4];
 #pragma unroll
     for (int h = 0; h < REP; h++) {
         m[h] = -INFINITY;
         l[h] = 0;
-#pragma unroll
-        for (int p = 0; p < PVL; p++) o[h][p][0] = o[h][p][1] = o[h][p][2] = o[h][p][3] = 0;
+        o[h][0] = o[h][1] = o[h][2] = o[h][3] = 0;
     }
-    __syncthreads();
 
     for (int tb = t0; tb < t1; tb += TC) {
         const int n = min(TC, t1 - tb);
-        // scores: one thread per position
-        for (int t = tid; t < n; t += NT) {
-            const float4* kr = reinterpret_cast<const float4*>(kc + (size_t)(tb + t) * a.kvd);
-            Acc s[REP];
+        // scores: warp per position, lanes across the head's row slice; each
+        // warp loads PB positions' rows before reducing, to keep loads in flight
+        for (int tq = warp * PB; tq < n; tq += NW * PB) {
+            float4 kv[PB];
 #pragma unroll
-            for (int h = 0; h < REP; h++) s[h] = 0;
-#pragma unroll 4
-            for (int j = 0; j < V4; j++) {
-                float4 kv = __ldg(kr + j);
+            for (int i = 0; i < PB; i++)
+                kv[i] = (lane_on && tq + i < n)
+                            ? __ldg(reinterpret_cast<const float4*>(kc + (size_t)(tb + tq + i) * a.kvd) + lane)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < PB; i++) {
 #pragma unroll
                 for (int h = 0; h < REP; h++) {
-                    s[h] += (Acc)kv.x * qs[h][4 * j] + (Acc)kv.y * qs[h][4 * j + 1] +
-                            (Acc)kv.z * qs[h][4 * j + 2] + (Acc)kv.w * qs[h][4 * j + 3];
+                    Acc s = (Acc)kv[i].x * qr[h][0] + (Acc)kv[i].y * qr[h][1] + (Acc)kv[i].z * qr[h][2] +
+                            (Acc)kv[i].w * qr[h][3];
+                    s = warp_sum(s);
+                    if (lane == 0 && tq + i < n) sc[tq + i][h] = s * scale;
                 }
             }
-#pragma unroll
-            for (int h = 0; h < REP; h++) sc[t][h] = s[h] * scale;
         }
         __syncthreads();
         // max over the sub-chunk, new running max, weights p = exp(s - m_new)
@@ -124,25 +137,24 @@ __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
         for (int h = 0; h < REP; h++) {
             l[h] = l[h] * alpha[h] + (red[0][h] + red[1][h]) + (red[2][h] + red[3][h]);
             m[h] = mnew[h];
-#pragma unroll
-            for (int p = 0; p < PVL; p++) {
-                o[h][p][0] *= alpha[h]; o[h][p][1] *= alpha[h];
-                o[h][p][2] *= alpha[h]; o[h][p][3] *= alpha[h];
-            }
+            o[h][0] *= alpha[h]; o[h][1] *= alpha[h]; o[h][2] *= alpha[h]; o[h][3] *= alpha[h];
         }
-        // weighted V sum: warp per position, lane owns float4 slices of the row
-        for (int t = warp; t < n; t += 4) {
-            const float4* vr = reinterpret_cast<const float4*>(vc + (size_t)(tb + t) * a.kvd);
+        // weighted V sum: warp per position, lane owns one float4 slice of the row
+        for (int tq = warp * PB; tq < n; tq += NW * PB) {
+            float4 vv[PB];
 #pragma unroll
-            for (int p = 0; p < PVL; p++) {
-                const int j = lane + 32 * p;
-                if (j < V4) {
-                    float4 vv = __ldg(vr + j);
+            for (int i = 0; i < PB; i++)
+                vv[i] = (lane_on && tq + i < n)
+                            ? __ldg(reinterpret_cast<const float4*>(vc + (size_t)(tb + tq + i) * a.kvd) + lane)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < PB; i++) {
+                if (tq + i < n) {
 #pragma unroll
                     for (int h = 0; h < REP; h++) {
-                        Acc w = sc[t][h];
-                        o[h][p][0] += w * (Acc)vv.x; o[h][p][1] += w * (Acc)vv.y;
-                        o[h][p][2] += w * (Acc)vv.z; o[h][p][3] += w * (Acc)vv.w;
+                        const Acc w = sc[tq + i][h];
+                        o[h][0] += w * (Acc)vv[i].x; o[h][1] += w * (Acc)vv[i].y;
+                        o[h][2] += w * (Acc)vv[i].z; o[h][3] += w * (Acc)vv[i].w;
                     }
                 }
             }
@@ -150,15 +162,11 @@ __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
         __syncthreads();
     }
     // combine the four warps' weighted sums (same running max)
+    if (lane_on) {
 #pragma unroll
-    for (int p = 0; p < PVL; p++) {
-        const int j = lane + 32 * p;
-        if (j < V4) {
-#pragma unroll
-            for (int h = 0; h < REP; h++) {
-                ostage[warp][h][4 * j] = o[h][p][0]; ostage[warp][h][4 * j + 1] = o[h][p][1];
-                ostage[warp][h][4 * j + 2] = o[h][p][2]; ostage[warp][h][4 * j + 3] = o[h][p][3];
-            }
+        for (int h = 0; h < REP; h++) {
+            ostage[warp][h][4 * lane] = o[h][0]; ostage[warp][h][4 * lane + 1] = o[h][1];
+            ostage[warp][h][4 * lane + 2] = o[h][2]; ostage[warp][h][4 * lane + 3] = o[h][3];
         }
     }
     __syncthreads();

@@ -91,7 +91,7 @@ extern "C" int l2c_attention_noalloc(const float* q_dev, const float* k_dev, con
     t.q = q_dev; t.kc = k_dev; t.vc = v_dev; t.seq_stride = 0;
     t.out = out_dev; t.tp = tp; t.tp_stride = 2;
     t.H = n_heads; t.Hkv = n_kv_heads; t.hs = head_size; t.kvd = n_kv_heads * head_size; t.seq_len = pos + 1;
-    t.chunk = kChunk; t.nchunks = nchunks;
+    t.nchunks = nchunks;
     t.part = scratch + 256 + cnt_bytes; t.count = counters; t.err = tp + 2;
     ak<<<dim3(nchunks, n_kv_heads, 1), 128, 0, s>>>(t);
     if (cudaGetLastError() != cudaSuccess) return L2C_E_CUDA;

@@ -100,6 +100,21 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// Phase timestamps for development builds that define L2C_PHASE_STAMPS
+// (a single translation unit): g_l2c_stamps[CTA][16]; compiled out otherwise.
+#ifdef L2C_PHASE_STAMPS
+__device__ unsigned long long g_l2c_stamps[1024 * 16];
+#define L2C_STAMP(slot)                                                                              \
+    do {                                                                                             \
+        if ((threadIdx.x & 31) == 0 && blockIdx.y == 0 && blockIdx.z == 0 && blockIdx.x < 1024)     \
+            g_l2c_stamps[blockIdx.x * 16 + (slot)] = global_timer_ns();                              \
+    } while (0)
+#else
+#define L2C_STAMP(slot) \
+    do {                \
+    } while (0)
+#endif
+
 // Waits for the barrier phase with the given parity.  Gives up after
 // `limit_ns` of wall time, records DERR_TIMEOUT and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err,

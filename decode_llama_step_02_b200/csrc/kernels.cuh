@@ -53,6 +53,7 @@ struct GemvArgs {
     unsigned long long* amax;  // argmax key (classifier); reset by layer 0
     int* err;
     size_t prefetch_bytes;   // L2 prefetch issued before the dependency wait
+    int late_trigger;        // 1: let the next kernel launch only after this CTA's last weight loads
 };
 
 // ----------------------------------------------------------------- epilogues --
@@ -70,18 +71,36 @@ __device__ __forceinline__ void rope_pair(float a, float b, int j, int pos, cons
     o1 = (float)((double)a * s + (double)b * c);
 }
 
+// The same rotation from a table cs[j/2] = (cos, sin) of the pair's angle.
+__device__ __forceinline__ void rope_pair_tab(float a, float b, int j, const double2* cs, float& o0, float& o1) {
+    const double2 t = cs[j >> 1];
+    o0 = (float)((double)a * t.x - (double)b * t.y);
+    o1 = (float)((double)a * t.y + (double)b * t.x);
+}
+
+// Fills cs[i] = (cos, sin)(pos * freq[i]) for the hs/2 pair frequencies: one
+// sincos per pair index per CTA instead of one per output pair.
+__device__ __forceinline__ void rope_table(const GemvArgs& a, int pos, double2* cs) {
+    for (int i = threadIdx.x; i < a.hs / 2; i += blockDim.x) {
+        const float theta = (float)pos * a.freq[i];
+        double sn, c;
+        sincos((double)theta, &sn, &c);
+        cs[i] = make_double2(c, sn);
+    }
+}
+
 // Unit u of the QKV matrix is the row pair (2u, 2u+1); v0/v1 its two outputs.
-__device__ __forceinline__ void epi_qkv(const GemvArgs& a, int u, float v0, float v1, int pos) {
+__device__ __forceinline__ void epi_qkv(const GemvArgs& a, int u, float v0, float v1, int pos, const double2* cs) {
     int r = 2 * u;
     if (r < a.d) {
         float o0, o1;
-        rope_pair(v0, v1, r % a.hs, pos, a.freq, o0, o1);
+        rope_pair_tab(v0, v1, r % a.hs, cs, o0, o1);
         a.out[r] = o0;
         a.out[r + 1] = o1;
     } else if (r < a.d + a.kvd) {
         int i = r - a.d;
         float o0, o1;
-        rope_pair(v0, v1, i % a.hs, pos, a.freq, o0, o1);
+        rope_pair_tab(v0, v1, i % a.hs, cs, o0, o1);
         float* k = a.kslot + (size_t)pos * a.kvd;
         k[i] = o0;
         k[i + 1] = o1;
@@ -115,65 +134,86 @@ __device__ __forceinline__ void read_tp(const GemvArgs& a, int& token, int& pos)
     }
 }
 
-// fp32 input into shared memory: RMSNorm (double) when norm_w is set.
-// On layer 0 the input is the embedding row E[token] (fp32) and CTA 0 also
-// stores it as the residual x.  Requires K % 4 == 0.  Every thread issues its
-// (at most 8) float4 loads of the input and the gain at once, so the
-// prologue costs one round trip to L2.
-template <bool NORM>
-__device__ void load_input_f32(const GemvArgs& a, int token, float* xs, double* red) {
-    const int K4 = a.K >> 2;
+// fp32 GEMV input, in two halves around the dependency wait.  Thread t owns
+// the float4 elements t + j*blockDim (j < F32_PER).  pre: the RMSNorm gain and,
+// on layer 0, the embedding row E[token] (neither is written by the step's
+// kernels).  post: the input vector written by the previous kernel, then
+// RMSNorm in double into shared memory; CTA 0 also stores the embedding row as
+// the residual x.  Requires K % 4 == 0 and K/4 <= F32_PER * blockDim.
+constexpr int F32_PER = 4;
+
+struct F32Pre {
+    float4 v[F32_PER];
+    float4 w[F32_PER];
+};
+
+__device__ __forceinline__ bool f32_pre_fits(const GemvArgs& a) { return (a.K >> 2) <= F32_PER * (int)blockDim.x; }
+
+__device__ __forceinline__ void f32_pre_load(const GemvArgs& a, int token, F32Pre& r) {
+    const int K4 = a.K >> 2, nt = blockDim.x;
+    const float4* nw = reinterpret_cast<const float4*>(a.norm_w);
+    const float4* emb = a.emb ? reinterpret_cast<const float4*>(static_cast<const float*>(a.emb) + (size_t)token * a.K)
+                              : nullptr;
+#pragma unroll
+    for (int j = 0; j < F32_PER; j++) {
+        const int i = threadIdx.x + j * nt;
+        r.w[j] = (nw && i < K4) ? nw[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        r.v[j] = (emb && i < K4) ? emb[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+}
+
+__device__ __forceinline__ void f32_post_load(const GemvArgs& a, F32Pre& r, float* xs, double* red) {
+    const int K4 = a.K >> 2, nt = blockDim.x;
+    float4* xs4 = reinterpret_cast<float4*>(xs);
+    if (!a.emb) {
+        const float4* in = reinterpret_cast<const float4*>(a.in);
+#pragma unroll
+        for (int j = 0; j < F32_PER; j++) {
+            const int i = threadIdx.x + j * nt;
+            r.v[j] = i < K4 ? in[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    } else if (blockIdx.x == 0) {
+#pragma unroll
+        for (int j = 0; j < F32_PER; j++) {
+            const int i = threadIdx.x + j * nt;
+            if (i < K4) reinterpret_cast<float4*>(a.x_resid)[i] = r.v[j];
+        }
+    }
+    if (a.norm_w) {
+        double ss = 0.0;
+#pragma unroll
+        for (int j = 0; j < F32_PER; j++)
+            ss += (double)r.v[j].x * r.v[j].x + (double)r.v[j].y * r.v[j].y + (double)r.v[j].z * r.v[j].z +
+                  (double)r.v[j].w * r.v[j].w;
+        ss = block_sum(ss, red);
+        const double inv = 1.0 / sqrt(ss / (double)a.K + 1e-5);
+#pragma unroll
+        for (int j = 0; j < F32_PER; j++) {
+            const float4 g = r.w[j];
+            r.v[j].x = (float)((double)g.x * (inv * (double)r.v[j].x));
+            r.v[j].y = (float)((double)g.y * (inv * (double)r.v[j].y));
+            r.v[j].z = (float)((double)g.z * (inv * (double)r.v[j].z));
+            r.v[j].w = (float)((double)g.w * (inv * (double)r.v[j].w));
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < F32_PER; j++) {
+        const int i = threadIdx.x + j * nt;
+        if (i < K4) xs4[i] = r.v[j];
+    }
+}
+
+// Wide inputs (K/4 > F32_PER * blockDim): a plain strided loop after the wait.
+__device__ void load_input_f32_wide(const GemvArgs& a, int token, float* xs, double* red) {
+    const int K4 = a.K >> 2, nt = blockDim.x;
     const float4* in = reinterpret_cast<const float4*>(
         a.emb ? static_cast<const float*>(a.emb) + (size_t)token * a.K : a.in);
-    const float4* nw = NORM ? reinterpret_cast<const float4*>(a.norm_w) : nullptr;
     float4* xs4 = reinterpret_cast<float4*>(xs);
-    constexpr int PER = NORM ? 4 : 8;
-    float4 v[PER], w[NORM ? PER : 1];
-    const int nt = blockDim.x;
-    if (K4 <= PER * nt) {
-#pragma unroll
-        for (int j = 0; j < PER; j++) {
-            const int i = threadIdx.x + j * nt;
-            v[j] = i < K4 ? in[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-            if (NORM) w[NORM ? j : 0] = i < K4 ? nw[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        if (a.emb && blockIdx.x == 0) {
-#pragma unroll
-            for (int j = 0; j < PER; j++) {
-                const int i = threadIdx.x + j * nt;
-                if (i < K4) reinterpret_cast<float4*>(a.x_resid)[i] = v[j];
-            }
-        }
-        if (NORM) {
-            double ss = 0.0;
-#pragma unroll
-            for (int j = 0; j < PER; j++)
-                ss += (double)v[j].x * v[j].x + (double)v[j].y * v[j].y + (double)v[j].z * v[j].z +
-                      (double)v[j].w * v[j].w;
-            ss = block_sum(ss, red);
-            const double inv = 1.0 / sqrt(ss / (double)a.K + 1e-5);
-#pragma unroll
-            for (int j = 0; j < PER; j++) {
-                const float4 g = w[NORM ? j : 0];
-                v[j].x = (float)((double)g.x * (inv * (double)v[j].x));
-                v[j].y = (float)((double)g.y * (inv * (double)v[j].y));
-                v[j].z = (float)((double)g.z * (inv * (double)v[j].z));
-                v[j].w = (float)((double)g.w * (inv * (double)v[j].w));
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < PER; j++) {
-            const int i = threadIdx.x + j * nt;
-            if (i < K4) xs4[i] = v[j];
-        }
-        return;
-    }
-    // wide inputs: a plain strided loop
     for (int i = threadIdx.x; i < K4; i += nt) {
         xs4[i] = in[i];
         if (a.emb && blockIdx.x == 0) reinterpret_cast<float4*>(a.x_resid)[i] = in[i];
     }
-    if (NORM) {
+    if (a.norm_w) {
         __syncthreads();
         double ss = 0.0;
         for (int i = threadIdx.x; i < a.K; i += nt) ss += (double)xs[i] * (double)xs[i];
@@ -212,15 +252,25 @@ __device__ __forceinline__ void dot_rows_f32(const float* __restrict__ w, size_t
             }
         }
     }
-    for (; j < K4; j += 32) {
-        float4 xv = xs[j];
+    if (j < K4) {  // tail: one predicated batch, all loads in flight together
+        float4 wv[R][U];
 #pragma unroll
-        for (int r = 0; r < R; r++) {
-            float4 wv = ld_stream_f4(reinterpret_cast<const float4*>(w + r * ldw) + j, pol);
-            acc[r] = fmaf(wv.x, xv.x, acc[r]);
-            acc[r] = fmaf(wv.y, xv.y, acc[r]);
-            acc[r] = fmaf(wv.z, xv.z, acc[r]);
-            acc[r] = fmaf(wv.w, xv.w, acc[r]);
+        for (int u = 0; u < U; u++)
+#pragma unroll
+            for (int r = 0; r < R; r++)
+                wv[r][u] = j + 32 * u < K4
+                               ? ld_stream_f4(reinterpret_cast<const float4*>(w + r * ldw) + j + 32 * u, pol)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const float4 xv = j + 32 * u < K4 ? xs[j + 32 * u] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int r = 0; r < R; r++) {
+                acc[r] = fmaf(wv[r][u].x, xv.x, acc[r]);
+                acc[r] = fmaf(wv[r][u].y, xv.y, acc[r]);
+                acc[r] = fmaf(wv[r][u].z, xv.z, acc[r]);
+                acc[r] = fmaf(wv[r][u].w, xv.w, acc[r]);
+            }
         }
     }
 #pragma unroll
@@ -229,57 +279,86 @@ __device__ __forceinline__ void dot_rows_f32(const float* __restrict__ w, size_t
 
 constexpr int F32_THREADS = 512;
 
-// Requires K % 4 == 0 (rows are 16-byte aligned).  Dynamic shared memory:
-// K floats.  Each CTA owns a contiguous range of units (1 row, or a row pair
-// for QKV/W13); its warps take the units round-robin.
+// Requires K % (4*ks) == 0 (rows are 16-byte aligned).  Dynamic shared
+// memory: K floats of input, then the partial sums [rows of the CTA][ks].
+// Each CTA owns a contiguous range of rows (an even start for the row-pair
+// epilogues); a warp's unit is one K/ks slice of one row, taken round-robin,
+// so the CTA's ks*rows slices spread evenly over its 16 warps.  After a
+// barrier the CTA sums the slices of each row in a fixed order and runs the
+// epilogue (RoPE and the cache write, SwiGLU, the residual, or argmax).
 template <int MODE>
-__global__ void __launch_bounds__(F32_THREADS, 2) k_gemv_f32(const GemvArgs a) {
+__global__ void __launch_bounds__(F32_THREADS, 2) k_gemv_f32(const GemvArgs a, const int ks) {
     extern __shared__ float4 smem_f4[];
     float* xs = reinterpret_cast<float*>(smem_f4);
+    float* part = xs + a.K;
     __shared__ double red[32];
     __shared__ unsigned long long best_s[32];
-    constexpr int UNIT = (MODE == M_QKV || MODE == M_W13) ? 2 : 1;
-    constexpr int U = (UNIT == 2) ? 4 : 8;
+    __shared__ double2 rope_cs[MODE == M_QKV ? 128 : 1];
+    constexpr int PAIR = (MODE == M_QKV || MODE == M_W13) ? 2 : 1;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    const int units = a.rows / UNIT;
-    const int u0 = (int)((long long)units * blockIdx.x / gridDim.x);
-    const int u1 = (int)((long long)units * (blockIdx.x + 1) / gridDim.x);
+    const int npair = a.rows / PAIR;
+    const int r0 = PAIR * (int)((long long)npair * blockIdx.x / gridDim.x);
+    const int r1 = PAIR * (int)((long long)npair * (blockIdx.x + 1) / gridDim.x);
     const float* W = static_cast<const float*>(a.W);
     const uint64_t pol = policy_evict_first();
-    if (threadIdx.x == 0 && u1 > u0 && a.prefetch_bytes) {
-        size_t bytes = (size_t)(u1 - u0) * UNIT * a.ld * sizeof(float);
-        if (bytes > a.prefetch_bytes) bytes = a.prefetch_bytes;
-        prefetch_l2_range(W + (size_t)u0 * UNIT * a.ld, bytes, policy_evict_last());
-    }
-    grid_dep_wait();
-    grid_dep_launch();
+    // before the wait: token/position (written before the step), RMSNorm gain,
+    // embedding row, RoPE table; then the L2 prefetch of this CTA's weights
     int token = 0, pos = 0;
     if (MODE == M_QKV) read_tp(a, token, pos);
+    F32Pre pre;
+    const bool fits = f32_pre_fits(a);
+    if (fits) f32_pre_load(a, token, pre);
+    if (MODE == M_QKV) rope_table(a, pos, rope_cs);
+    if (threadIdx.x == 0 && r1 > r0 && a.prefetch_bytes) {
+        size_t bytes = (size_t)(r1 - r0) * a.ld * sizeof(float);
+        if (bytes > a.prefetch_bytes) bytes = a.prefetch_bytes;
+        prefetch_l2_range(W + (size_t)r0 * a.ld, bytes, policy_evict_last());
+    }
+    grid_dep_wait();
+    if (!a.late_trigger) grid_dep_launch();
     if (MODE == M_QKV && a.amax && blockIdx.x == 0 && threadIdx.x == 0) *a.amax = 0ull;
-    load_input_f32<MODE != M_RESID>(a, token, xs, red);
+    if (fits) f32_post_load(a, pre, xs, red);
+    else load_input_f32_wide(a, token, xs, red);
     __syncthreads();
-    const int K4 = a.K >> 2;
+    const int kp4 = (a.K >> 2) / ks;  // float4 per slice
+    const int nunits = (r1 - r0) * ks;
+    for (int u = warp; u < nunits; u += nwarps) {
+        const int rr = u / ks, p = u - rr * ks;
+        float acc[1];
+        dot_rows_f32<1, 8>(W + (size_t)(r0 + rr) * a.ld + (size_t)p * kp4 * 4, a.ld, kp4,
+                           reinterpret_cast<const float4*>(xs) + (size_t)p * kp4, pol, acc);
+        if (lane == 0) part[u] = acc[0];
+    }
+    if (a.late_trigger) grid_dep_launch();
+    __syncthreads();
     unsigned long long best = 0ull;
-    for (int u = u0 + warp; u < u1; u += nwarps) {
-        const float* wr = W + (size_t)u * UNIT * a.ld;
-        float acc[UNIT];
-        dot_rows_f32<UNIT, U>(wr, a.ld, K4, reinterpret_cast<const float4*>(xs), pol, acc);
-        if (lane == 0) {
-            if (MODE == M_QKV) {
-                epi_qkv(a, u, acc[0], acc[UNIT - 1], pos);
-            } else if (MODE == M_W13) {
-                epi_w13(a, u, acc[0], acc[UNIT - 1]);
-            } else if (MODE == M_RESID) {
-                a.out[u] = a.out[u] + acc[0];
-            } else {
-                a.out[u] = acc[0];
-                if (acc[0] != acc[0]) set_error(a.err, DERR_NAN);
-                unsigned long long k = argmax_key(acc[0], u);
-                best = k > best ? k : best;
-            }
+    for (int j = threadIdx.x; j < (r1 - r0) / PAIR; j += blockDim.x) {
+        float v[PAIR];
+#pragma unroll
+        for (int q = 0; q < PAIR; q++) {
+            float t = 0.f;
+            for (int p = 0; p < ks; p++) t += part[(PAIR * j + q) * ks + p];
+            v[q] = t;
+        }
+        const int r = r0 + PAIR * j;
+        if (MODE == M_QKV) {
+            epi_qkv(a, r / 2, v[0], v[PAIR - 1], pos, rope_cs);
+        } else if (MODE == M_W13) {
+            epi_w13(a, r / 2, v[0], v[PAIR - 1]);
+        } else if (MODE == M_RESID) {
+            a.out[r] = a.out[r] + v[0];
+        } else {
+            a.out[r] = v[0];
+            if (v[0] != v[0]) set_error(a.err, DERR_NAN);
+            unsigned long long k = argmax_key(v[0], r);
+            best = k > best ? k : best;
         }
     }
     if (MODE == M_CLS) {
+        for (int o = 16; o > 0; o >>= 1) {
+            unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+            best = other > best ? other : best;
+        }
         if (lane == 0) best_s[warp] = best;
         __syncthreads();
         if (threadIdx.x == 0) {
@@ -360,87 +439,145 @@ __device__ __noinline__ void q8_quantize_input_loop(const GemvArgs& a, const int
     }
 }
 
-// Fast path: warp w owns groups w + jg*nw (jg < GMAX); a lane holds elements
-// lane + 32e (e < EPL = gs/32) of each in registers, all loaded at once.
-template <int GMAX, int EPL, bool NORM>
-__device__ __forceinline__ bool q8_quantize_input_regs(const GemvArgs& a, const int8_t* eq, const float* es,
-                                                       int8_t* xq, float* xsc, double* red) {
+// Fast path for gs = 32 * EPL.  Pass 1 (RMSNorm only): the sum of squares
+// from 16-byte loads, four in flight per thread.  Pass 2: warp w quantizes its
+// groups w, w + nw, ... in batches of QB, issuing the loads of a whole batch
+// before using them.  A few round trips to L2 in all, with little code.
+template <int EPL, bool NORM>
+__device__ __forceinline__ void q8_quantize_input_batched(const GemvArgs& a, const int8_t* eq, const float* es,
+                                                          int8_t* xq, float* xsc, double* red) {
+    constexpr int QB = 8;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int K = a.K, gs = 32 * EPL;
     const int ng = K / gs;
-    if ((ng + nw - 1) / nw > GMAX) return false;  // uniform across the CTA
-    float v[GMAX][EPL];
-    float w[NORM ? GMAX : 1][EPL];
+    if (NORM) {
+        // the whole vector and gain in registers (one round trip): the sum of
+        // squares and the codes both come from the same loaded values
+        constexpr int GM = 16 / EPL;
+        if ((ng + nw - 1) / nw <= GM) {
+            float v[GM][EPL], w[GM][EPL];
 #pragma unroll
-    for (int jg = 0; jg < GMAX; jg++) {
-        const int g = warp + jg * nw;
+            for (int j = 0; j < GM; j++) {
+                const int g = warp + j * nw;
 #pragma unroll
-        for (int e = 0; e < EPL; e++) {
-            const int i = g * gs + lane + 32 * e;
-            v[jg][e] = g < ng ? (eq ? (float)eq[i] * es[g] : a.in[i]) : 0.f;
-            if (NORM) w[NORM ? jg : 0][e] = g < ng ? a.norm_w[i] : 0.f;
+                for (int e = 0; e < EPL; e++) {
+                    const int i = g * gs + lane + 32 * e;
+                    v[j][e] = g < ng ? (eq ? (float)eq[i] * es[g] : a.in[i]) : 0.f;
+                    w[j][e] = g < ng ? a.norm_w[i] : 0.f;
+                }
+            }
+            double ss = 0.0;
+#pragma unroll
+            for (int j = 0; j < GM; j++)
+#pragma unroll
+                for (int e = 0; e < EPL; e++) ss += (double)v[j][e] * (double)v[j][e];
+            ss = warp_sum(ss);
+            if (lane == 0) red[warp] = ss;
+            __syncthreads();
+            if (warp == 0) L2C_STAMP(5);
+            double tot = 0.0;
+            for (int i = 0; i < nw; i++) tot += red[i];
+            const double inv = 1.0 / sqrt(tot / (double)K + 1e-5);
+#pragma unroll
+            for (int j = 0; j < GM; j++) {
+                const int g = warp + j * nw;
+                if (g < ng) {  // warp-uniform
+                    if (a.emb && blockIdx.x == 0) {
+#pragma unroll
+                        for (int e = 0; e < EPL; e++) a.x_resid[g * gs + lane + 32 * e] = v[j][e];
+                    }
+                    float m = 0.f;
+#pragma unroll
+                    for (int e = 0; e < EPL; e++) {
+                        v[j][e] = (float)((double)w[j][e] * (inv * (double)v[j][e]));
+                        m = fmaxf(m, fabsf(v[j][e]));
+                    }
+                    m = warp_max(m);
+                    const float scale = m / 127.0f;
+#pragma unroll
+                    for (int e = 0; e < EPL; e++) {
+                        const float q = scale == 0.f ? 0.f : roundf(v[j][e] / scale);
+                        xq[g * gs + lane + 32 * e] = (int8_t)(int)q;
+                    }
+                    if (lane == 0) xsc[g] = scale;
+                }
+            }
+            return;
         }
     }
-    if (a.emb && blockIdx.x == 0) {
-#pragma unroll
-        for (int jg = 0; jg < GMAX; jg++) {
-            const int g = warp + jg * nw;
-#pragma unroll
-            for (int e = 0; e < EPL; e++)
-                if (g < ng) a.x_resid[g * gs + lane + 32 * e] = v[jg][e];
-        }
-    }
+    double inv = 1.0;
     if (NORM) {
         double ss = 0.0;
-#pragma unroll
-        for (int jg = 0; jg < GMAX; jg++)
-#pragma unroll
-            for (int e = 0; e < EPL; e++) ss += (double)v[jg][e] * (double)v[jg][e];
+        const int K4 = K >> 2;
+#pragma unroll 4
+        for (int i4 = threadIdx.x; i4 < K4; i4 += blockDim.x) {
+            float4 v;
+            if (eq) {
+                const char4 c4 = reinterpret_cast<const char4*>(eq)[i4];
+                const float sc = es[(4 * i4) / gs];
+                v = make_float4((float)c4.x * sc, (float)c4.y * sc, (float)c4.z * sc, (float)c4.w * sc);
+            } else {
+                v = reinterpret_cast<const float4*>(a.in)[i4];
+            }
+            ss += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
+        }
         ss = warp_sum(ss);
         if (lane == 0) red[warp] = ss;
         __syncthreads();
         double tot = 0.0;
         for (int i = 0; i < nw; i++) tot += red[i];
-        const double inv = 1.0 / sqrt(tot / (double)K + 1e-5);
-#pragma unroll
-        for (int jg = 0; jg < GMAX; jg++)
-#pragma unroll
-            for (int e = 0; e < EPL; e++)
-                v[jg][e] = (float)((double)w[NORM ? jg : 0][e] * (inv * (double)v[jg][e]));
+        inv = 1.0 / sqrt(tot / (double)K + 1e-5);
     }
+    for (int g0 = warp; g0 < ng; g0 += QB * nw) {
+        float v[QB][EPL];
+        float w[NORM ? QB : 1][EPL];
 #pragma unroll
-    for (int jg = 0; jg < GMAX; jg++) {
-        const int g = warp + jg * nw;
-        if (g < ng) {  // warp-uniform
-            float m = 0.f;
-#pragma unroll
-            for (int e = 0; e < EPL; e++) m = fmaxf(m, fabsf(v[jg][e]));
-            m = warp_max(m);
-            const float scale = m / 127.0f;
+        for (int j = 0; j < QB; j++) {
+            const int g = g0 + j * nw;
 #pragma unroll
             for (int e = 0; e < EPL; e++) {
-                const float q = scale == 0.f ? 0.f : roundf(v[jg][e] / scale);
-                xq[g * gs + lane + 32 * e] = (int8_t)(int)q;
+                const int i = g * gs + lane + 32 * e;
+                v[j][e] = g < ng ? (eq ? (float)eq[i] * es[g] : a.in[i]) : 0.f;
+                if (NORM) w[NORM ? j : 0][e] = g < ng ? a.norm_w[i] : 0.f;
             }
-            if (lane == 0) xsc[g] = scale;
+        }
+#pragma unroll
+        for (int j = 0; j < QB; j++) {
+            const int g = g0 + j * nw;
+            if (g < ng) {  // warp-uniform
+                if (a.emb && blockIdx.x == 0) {
+#pragma unroll
+                    for (int e = 0; e < EPL; e++) a.x_resid[g * gs + lane + 32 * e] = v[j][e];
+                }
+                float m = 0.f;
+#pragma unroll
+                for (int e = 0; e < EPL; e++) {
+                    if (NORM) v[j][e] = (float)((double)w[NORM ? j : 0][e] * (inv * (double)v[j][e]));
+                    m = fmaxf(m, fabsf(v[j][e]));
+                }
+                m = warp_max(m);
+                const float scale = m / 127.0f;
+#pragma unroll
+                for (int e = 0; e < EPL; e++) {
+                    const float q = scale == 0.f ? 0.f : roundf(v[j][e] / scale);
+                    xq[g * gs + lane + 32 * e] = (int8_t)(int)q;
+                }
+                if (lane == 0) xsc[g] = scale;
+            }
         }
     }
-    return true;
 }
 
 // Quantizes the GEMV input (embedding row or input vector, RMSNorm'd when
 // norm_w is set) into shared codes and scales; every thread of the CTA calls
-// it.  Register fast paths for gs = 32/64/128 load the whole vector at once
-// (one round trip to L2 instead of a chain of dependent loads).
+// it.
 template <bool NORM>
 __device__ __forceinline__ void q8_quantize_input(const GemvArgs& a, const int8_t* eq, const float* es, int8_t* xq,
                                                   float* xsc, double* red) {
-    constexpr int BUDGET = NORM ? 16 : 48;  // values per lane kept in registers
-    bool done = false;
-    if (a.gs == 32) done = q8_quantize_input_regs<BUDGET, 1, NORM>(a, eq, es, xq, xsc, red);
-    else if (a.gs == 64) done = q8_quantize_input_regs<BUDGET / 2, 2, NORM>(a, eq, es, xq, xsc, red);
-    else if (a.gs == 128) done = q8_quantize_input_regs<BUDGET / 4, 4, NORM>(a, eq, es, xq, xsc, red);
-    if (!done) q8_quantize_input_loop(a, eq, es, xq, xsc, red);
+    if (a.gs == 32) q8_quantize_input_batched<1, NORM>(a, eq, es, xq, xsc, red);
+    else if (a.gs == 64) q8_quantize_input_batched<2, NORM>(a, eq, es, xq, xsc, red);
+    else if (a.gs == 128) q8_quantize_input_batched<4, NORM>(a, eq, es, xq, xsc, red);
+    else q8_quantize_input_loop(a, eq, es, xq, xsc, red);
 }
 
 // Exact-int32 group dots of UNIT rows (records at rec, stride rb) with the
@@ -457,6 +594,7 @@ __device__ __forceinline__ void q8_rows_dot64(const uint8_t* rec, size_t rb, con
     const int rot = (lane >> 1) & 3;
 #pragma unroll
     for (int r = 0; r < UNIT; r++) acc[r] = 0.0;
+#pragma unroll 2
     for (int t0 = 0; t0 < n64; t0 += 32) {
         const int t = t0 + lane;
         const bool in = t < n64;
@@ -505,6 +643,120 @@ __device__ __forceinline__ void q8_rows_dot64(const uint8_t* rec, size_t rb, con
     }
 }
 
+// Registers of the split prologue (gs = 32 * EPL): warp w holds groups
+// w + j*nw (j < GM), a lane elements lane + 32e of each; w holds the RMSNorm
+// gain when NORM.
+template <int EPL, int GM, bool NORM>
+struct Q8Pre {
+    float v[GM][EPL];
+    float w[NORM ? GM : 1][EPL];
+};
+
+// Group slots per warp of the register prologue: 16 values per lane with an
+// RMSNorm gain, 48 without.
+template <int EPL, bool NORM>
+struct Q8PreGM {
+    static constexpr int value = (NORM ? 16 : 48) / EPL;
+};
+
+template <int EPL, int GM>
+__device__ __forceinline__ bool q8_pre_fits(const GemvArgs& a) {
+    const int ng = a.K / (32 * EPL), nw = blockDim.x >> 5;
+    return a.gs == 32 * EPL && (ng + nw - 1) / nw <= GM;
+}
+
+// Loads the gain (gain = true) or the values (from src, or the embedding
+// codes eq * scale es) of the warp's groups.
+template <int EPL, int GM, bool NORM>
+__device__ __forceinline__ void q8_pre_load(const GemvArgs& a, const float* src, const int8_t* eq, const float* es,
+                                            bool gain, Q8Pre<EPL, GM, NORM>& r) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int gs = 32 * EPL, ng = a.K / gs;
+#pragma unroll
+    for (int j = 0; j < GM; j++) {
+        const int g = warp + j * nw;
+#pragma unroll
+        for (int e = 0; e < EPL; e++) {
+            const int i = g * gs + lane + 32 * e;
+            if (gain) {
+                if (NORM) r.w[NORM ? j : 0][e] = g < ng ? a.norm_w[i] : 0.f;
+            } else {
+                r.v[j][e] = g < ng ? (eq ? (float)eq[i] * es[g] : src[i]) : 0.f;
+            }
+        }
+    }
+}
+
+// RMSNorm (double, when NORM) and Q8_0 codes of the values in r.  The
+// reductions of all groups run interleaved so their latencies overlap.
+template <int EPL, int GM, bool NORM, typename AfterLoads>
+__device__ __forceinline__ void q8_pre_finish(const GemvArgs& a, Q8Pre<EPL, GM, NORM>& r, int8_t* xq, float* xsc,
+                                              double* red, AfterLoads after_loads) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int gs = 32 * EPL, ng = a.K / gs;
+    if (a.emb && blockIdx.x == 0) {
+#pragma unroll
+        for (int j = 0; j < GM; j++) {
+            const int g = warp + j * nw;
+            if (g < ng) {
+#pragma unroll
+                for (int e = 0; e < EPL; e++) a.x_resid[g * gs + lane + 32 * e] = r.v[j][e];
+            }
+        }
+    }
+    if (NORM) {
+        double part[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+        for (int j = 0; j < GM; j++)
+#pragma unroll
+            for (int e = 0; e < EPL; e++) part[(j * EPL + e) & 3] += (double)r.v[j][e] * (double)r.v[j][e];
+        double ss = (part[0] + part[1]) + (part[2] + part[3]);
+        after_loads();  // every value has arrived by now
+        ss = warp_sum(ss);
+        if (lane == 0) red[warp] = ss;
+        __syncthreads();
+        double tot = 0.0;
+        for (int i = 0; i < nw; i++) tot += red[i];
+        const double inv = 1.0 / sqrt(tot / (double)a.K + 1e-5);
+#pragma unroll
+        for (int j = 0; j < GM; j++)
+#pragma unroll
+            for (int e = 0; e < EPL; e++)
+                r.v[j][e] = (float)((double)r.w[NORM ? j : 0][e] * (inv * (double)r.v[j][e]));
+    }
+    float m[GM];
+#pragma unroll
+    for (int j = 0; j < GM; j++) {
+        m[j] = fabsf(r.v[j][0]);
+#pragma unroll
+        for (int e = 1; e < EPL; e++) m[j] = fmaxf(m[j], fabsf(r.v[j][e]));
+    }
+    if (!NORM) {
+        float all = 0.f;
+#pragma unroll
+        for (int j = 0; j < GM; j++) all = fmaxf(all, m[j]);
+        asm volatile("" ::"f"(all));  // every value has arrived by now
+        after_loads();
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int j = 0; j < GM; j++) m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], o));
+#pragma unroll
+    for (int j = 0; j < GM; j++) {
+        const int g = warp + j * nw;
+        const float scale = m[j] / 127.0f;
+        if (g < ng) {
+#pragma unroll
+            for (int e = 0; e < EPL; e++) {
+                const float q = scale == 0.f ? 0.f : roundf(r.v[j][e] / scale);
+                xq[g * gs + lane + 32 * e] = (int8_t)(int)q;
+            }
+            if (lane == 0) xsc[g] = scale;
+        }
+    }
+}
+
 struct Q8Layout {
     int nslot;          // ring slots per warp, one unit (UNIT row records) each
     size_t unit_bytes;  // UNIT * record bytes
@@ -526,6 +778,7 @@ __global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, 
     constexpr int UNIT = (MODE == M_QKV || MODE == M_W13) ? 2 : 1;
     __shared__ double red[Q8_WARPS];
     __shared__ unsigned long long best_s[Q8_WARPS];
+    __shared__ double2 rope_cs[MODE == M_QKV ? 128 : 1];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int K = a.K, gs = a.gs;
     const size_t rb = a.ld;
@@ -545,32 +798,22 @@ __global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, 
     const uint64_t pol = policy_evict_first();
     auto unit_src = [&](int k) { return Wb + (size_t)(u0 + warp + k * Q8_WARPS) * UNIT * rb; };
 
-    // weights do not depend on earlier kernels: start streaming before the wait
+    if (warp == 0) L2C_STAMP(0);
+    // ---- before the dependency wait: everything that earlier kernels of the
+    // step do not write.  The small loads (token/position, RMSNorm gain,
+    // embedding row, RoPE frequencies) go first, then the L2 prefetch of this
+    // CTA's weights, so that those loads do not queue behind it in HBM.
     if (lane == 0) {
         for (int s = 0; s < ns; s++) mbar_init(&full[s], 1);
         mbar_fence_init();
-        for (int k = 0; k < ns && k < nmine; k++) {
-            mbar_arrive_expect_tx(&full[k], (uint32_t)L.unit_bytes);
-            bulk_g2s(slots + (size_t)k * L.unit_bytes, unit_src(k), (uint32_t)L.unit_bytes, &full[k], pol);
-        }
-        if (warp == 0 && a.prefetch_bytes) {
-            // the CTA's rows beyond the first slots of every warp, into L2
-            const size_t first = (size_t)(u0 + Q8_WARPS * ns) * UNIT * rb;
-            const size_t last = (size_t)u1 * UNIT * rb;
-            if (last > first) {
-                size_t bytes = last - first;
-                if (bytes > a.prefetch_bytes) bytes = a.prefetch_bytes;
-                prefetch_l2_range(Wb + first, bytes, policy_evict_last());
-            }
-        }
     }
-    grid_dep_wait();
-    grid_dep_launch();
-
-    // ---- input: token/pos, optional RMSNorm, Q8_0 codes of every group
+    constexpr int EPL = GS > 0 ? GS / 32 : 1;
+    constexpr bool NORM = MODE != M_RESID;
+    constexpr int GM = Q8PreGM<EPL, NORM>::value;
+    Q8Pre<EPL, GM, NORM> pre;
+    const bool split = GS > 0 && (NORM == (a.norm_w != nullptr)) && q8_pre_fits<EPL, GM>(a);  // CTA-uniform
     int token = 0, pos = 0;
-    if (MODE == M_QKV) read_tp(a, token, pos);
-    if (MODE == M_QKV && a.amax && blockIdx.x == 0 && threadIdx.x == 0) *a.amax = 0ull;
+    if (MODE == M_QKV) read_tp(a, token, pos);  // written before the step's first kernel
     const int8_t* eq = nullptr;
     const float* es = nullptr;
     if (a.emb) {
@@ -578,10 +821,50 @@ __global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, 
         eq = reinterpret_cast<const int8_t*>(rec);
         es = reinterpret_cast<const float*>(rec + K);
     }
-    q8_quantize_input<MODE != M_RESID>(a, eq, es, xq, xsc, red);
+    if (split) {
+        if (NORM) q8_pre_load<EPL, GM, NORM>(a, nullptr, nullptr, nullptr, true, pre);
+        if (eq) q8_pre_load<EPL, GM, NORM>(a, nullptr, eq, es, false, pre);
+    }
+    if (MODE == M_QKV) rope_table(a, pos, rope_cs);
+    if (warp == 0 && lane == 0 && a.prefetch_bytes) {
+        const size_t first = (size_t)u0 * UNIT * rb;
+        const size_t last = (size_t)u1 * UNIT * rb;
+        if (last > first) {
+            size_t bytes = last - first;
+            if (bytes > a.prefetch_bytes) bytes = a.prefetch_bytes;
+            prefetch_l2_range(Wb + first, bytes, policy_evict_last());
+        }
+    }
+    if (warp == 0) L2C_STAMP(3);
+    grid_dep_wait();
+    if (!a.late_trigger) grid_dep_launch();
+    if (warp == 0) L2C_STAMP(1);
+
+    // ---- after the wait: the input written by the previous kernel, then the
+    // ring fill (its copies land while the codes are computed)
+    if (MODE == M_QKV && a.amax && blockIdx.x == 0 && threadIdx.x == 0) *a.amax = 0ull;
+    if (split && !eq) q8_pre_load<EPL, GM, NORM>(a, a.in, nullptr, nullptr, false, pre);
+    if (warp == 0) L2C_STAMP(4);
+    auto fill_ring = [&]() {
+        if (lane == 0) {
+            for (int k = 0; k < ns && k < nmine; k++) {
+                mbar_arrive_expect_tx(&full[k], (uint32_t)L.unit_bytes);
+                bulk_g2s(slots + (size_t)k * L.unit_bytes, unit_src(k), (uint32_t)L.unit_bytes, &full[k], pol);
+            }
+        }
+    };
+    if (split) {
+        q8_pre_finish<EPL, GM, NORM>(a, pre, xq, xsc, red, fill_ring);
+    } else {
+        q8_quantize_input<NORM>(a, eq, es, xq, xsc, red);
+        fill_ring();
+    }
+    if (warp == 0) L2C_STAMP(6);
     __syncthreads();
+    if (warp == 0) L2C_STAMP(7);
     for (int g = threadIdx.x; g < K / gs; g += blockDim.x) sxd[g] = (double)xsc[g];
     __syncthreads();
+    if (warp == 0) L2C_STAMP(2);
 
     // ---- stream this warp's units
     const int nchunk = K >> 4;   // 16-byte chunks per row
@@ -634,6 +917,7 @@ __global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, 
         }
         // refill the slot with the unit ns ahead once every lane is done with it
         __syncwarp();
+        if (a.late_trigger && k + ns == nmine) grid_dep_launch();  // this warp's last copy is in
         if (lane == 0 && k + ns < nmine) {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             mbar_arrive_expect_tx(&full[s], (uint32_t)L.unit_bytes);
@@ -644,7 +928,7 @@ __global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, 
         const int u = u0 + warp + k * Q8_WARPS;
         if (lane == 0) {
             if (MODE == M_QKV) {
-                epi_qkv(a, u, (float)acc[0], (float)acc[UNIT - 1], pos);
+                epi_qkv(a, u, (float)acc[0], (float)acc[UNIT - 1], pos, rope_cs);
             } else if (MODE == M_W13) {
                 epi_w13(a, u, (float)acc[0], (float)acc[UNIT - 1]);
             } else if (MODE == M_RESID) {
@@ -658,6 +942,8 @@ __global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, 
             }
         }
     }
+    if (a.late_trigger) grid_dep_launch();  // (repeat triggers are harmless)
+    L2C_STAMP(8 + warp);
     if (MODE == M_CLS) {
         if (lane == 0) best_s[warp] = best;
         __syncthreads();

@@ -55,7 +55,7 @@ struct l2c_ctx {
     unsigned long long* key_scratch = nullptr;
     void* attn_part = nullptr;
     int* attn_cnt = nullptr;
-    int attn_chunk = 64, attn_nchunks = 1;
+    int attn_nchunks = 16;  // CTAs per (sequence, KV head) in attention
     // graphs: [q80][gen]
     cudaGraphExec_t graph[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
     // batched Q8_0 step: quantized activations of every sequence, one graph per batch size
@@ -64,10 +64,11 @@ struct l2c_ctx {
     size_t bkq = 0, bks = 0;  // strides (bytes of codes, floats of scales) per sequence
     std::vector<cudaGraphExec_t> bgraph;  // index B (1..max_batch)
     // tuning
-    size_t pf_f32 = 256 << 10, pf_q8 = 128 << 10;
+    size_t pf_f32 = 256 << 10, pf_q8 = 256 << 10;
     int f32_ctas_per_sm = 1;
     size_t q8_smem_budget = 220 << 10;  // dynamic shared memory of one Q8_0 GEMV CTA
     bool pdl = true;     // programmatic dependent launch between the step's kernels
+    int late_trigger = 0;  // GEMVs let the next kernel launch only near their end
     bool graphs = true;  // replay the step as a CUDA graph (off: plain launches)
     std::vector<void*> allocs;
     char msg[512] = {0};
@@ -170,11 +171,26 @@ static Q8Layout q8_layout(const l2c_ctx* h, int K, int gs, size_t rb, int unit, 
 template <int MODE>
 static cudaError_t launch_gemv(l2c_ctx* h, bool q80, GemvArgs a, int unit) {
     const int units = a.rows / unit;
+    a.late_trigger = h->late_trigger;
     if (!q80) {
         int grid = h->sms * h->f32_ctas_per_sm;
         if (grid > units) grid = units;
         a.prefetch_bytes = h->pf_f32;
-        return launch(h->cap, true, k_gemv_f32<MODE>, dim3(grid), dim3(F32_THREADS), (size_t)a.K * 4, a);
+        // K slices per row: the split that spreads the CTA's slices most evenly
+        // over its 16 warps (slices of at least 512 floats)
+        const int warps = F32_THREADS / 32;
+        const int rows_max = unit * ((units + grid - 1) / grid);
+        const double rows_avg = (double)a.rows / grid;
+        int ks = 1;
+        double best = 0.0;
+        for (int k = 1; k <= 4; k *= 2) {
+            if (a.K % (4 * k) || a.K / k < 1024) break;  // slices of at least one full load batch
+            const int per_warp = (rows_max * k + warps - 1) / warps;
+            const double eff = rows_avg * k / warps / per_warp;
+            if (eff > best * 1.03) { best = eff; ks = k; }
+        }
+        const size_t smem = (size_t)a.K * 4 + (size_t)rows_max * ks * 4;
+        return launch(h->cap, true, k_gemv_f32<MODE>, dim3(grid), dim3(F32_THREADS), smem, a, ks);
     }
     size_t smem = 0;
     Q8Layout L = q8_layout(h, a.K, a.gs, a.ld, unit, &smem);
@@ -256,7 +272,7 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
         t.q = q; t.kc = kslot; t.vc = vslot; t.seq_stride = (size_t)h->L * S * kvd;
         t.out = att; t.tp = tp; t.tp_stride = 2;
         t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = (int)kvd; t.seq_len = h->S;
-        t.chunk = h->attn_chunk; t.nchunks = h->attn_nchunks;
+        t.nchunks = h->attn_nchunks;
         t.part = h->attn_part; t.count = h->attn_cnt; t.err = h->err;
         AttnKernel ak = q80 ? attn_kernel_for<double>(h->hs, h->rep) : attn_kernel_for<float>(h->hs, h->rep);
         e = launch(s, true, ak, dim3(h->attn_nchunks, h->Hkv, 1), dim3(128), 0, t);
@@ -374,7 +390,7 @@ static int enqueue_batch_step(l2c_ctx* h, cudaStream_t s, int B) {
         t.q = h->q; t.kc = h->kc + (size_t)l * S * kvd; t.vc = h->vc + (size_t)l * S * kvd;
         t.seq_stride = (size_t)h->L * S * kvd; t.out = h->att; t.tp = h->tp; t.tp_stride = 2;
         t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = (int)kvd; t.seq_len = h->S;
-        t.chunk = h->attn_chunk; t.nchunks = h->attn_nchunks;
+        t.nchunks = h->attn_nchunks;
         t.part = h->attn_part; t.count = h->attn_cnt; t.err = h->err;
         CK(launch(s, true, ak, dim3(h->attn_nchunks, h->Hkv, B), dim3(128), 0, t));
         if ((rc = bprep(h, s, B, h->att, d, (int)d, nullptr, false, nullptr))) return rc;
@@ -484,11 +500,12 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
     h->pf_q8 = env_size("L2C_PREFETCH_Q8", h->pf_q8);
     h->q8_smem_budget = env_size("L2C_Q8_SMEM", h->q8_smem_budget);
     h->f32_ctas_per_sm = (int)env_size("L2C_F32_CTAS_PER_SM", 1);
-    h->attn_chunk = (int)env_size("L2C_ATTN_CHUNK", 64);
     h->pdl = env_size("L2C_NO_PDL", 0) == 0;
+    h->late_trigger = (int)env_size("L2C_LATE_TRIGGER", 0);
     h->graphs = env_size("L2C_NO_GRAPH", 0) == 0;
-    if (h->attn_chunk < 1) h->attn_chunk = 64;
-    h->attn_nchunks = (h->S + h->attn_chunk - 1) / h->attn_chunk;
+    h->attn_nchunks = (int)env_size("L2C_ATTN_SPLIT", 16);
+    if (h->attn_nchunks < 1) h->attn_nchunks = 16;
+    if (h->attn_nchunks > h->S) h->attn_nchunks = h->S;
     auto bail = [&](int code) { l2c_destroy(h); return code; };
     if (cudaGetDevice(&h->dev) != cudaSuccess) return bail(fail(h, L2C_E_CUDA, "no CUDA device"));
     if (cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->dev) != cudaSuccess)
@@ -724,7 +741,7 @@ extern "C" int l2c_attention(l2c_ctx* h, const float* q, const float* k, const f
     t.q = q; t.kc = k; t.vc = v; t.seq_stride = 0;
     t.out = out; t.tp = h->tp; t.tp_stride = 2;
     t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = h->kvd; t.seq_len = h->S;
-    t.chunk = h->attn_chunk; t.nchunks = h->attn_nchunks;
+    t.nchunks = h->attn_nchunks;
     t.part = h->attn_part; t.count = h->attn_cnt; t.err = h->err;
     AttnKernel ak = precision ? attn_kernel_for<double>(h->hs, h->rep) : attn_kernel_for<float>(h->hs, h->rep);
     CK(launch(h->stream, false, ak, dim3(h->attn_nchunks, h->Hkv, 1), dim3(128), 0, t));
