@@ -9,13 +9,12 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libl2c.so")
-SOURCES = [os.path.join(HERE, "csrc", "l2c.cu"), os.path.join(HERE, "csrc", "attention_noalloc.cu")]
+SOURCES = [os.path.join(HERE, "csrc", n) for n in ("l2c.cu", "attention_noalloc.cu", "persistent.cu")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17",
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
-    "-shared",
 ]
 
 
@@ -36,14 +35,29 @@ def stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+    """Compiles every source to an object (in parallel), then links the library."""
     if not force and not stale():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-o", tmp, *SOURCES, "-lcudart"]
-    if verbose:
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
+    tag = f".tmp{os.getpid()}"
+    objs, procs = [], []
+    for src in SOURCES:
+        obj = os.path.join(HERE, os.path.basename(src) + tag + ".o")
+        cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-c", "-o", obj, src]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        objs.append(obj)
+        procs.append(subprocess.Popen(cmd))
+    try:
+        failed = [src for src, p in zip(SOURCES, procs) if p.wait() != 0]
+        if failed:
+            raise subprocess.CalledProcessError(1, f"nvcc {' '.join(failed)}")
+        tmp = LIB + tag
+        subprocess.check_call([_nvcc(), *NVCC_FLAGS, "-shared", "-o", tmp, *objs, "-lcudart"])
+        os.replace(tmp, LIB)
+    finally:
+        for o in objs:
+            if os.path.exists(o):
+                os.remove(o)
     return LIB
 
 

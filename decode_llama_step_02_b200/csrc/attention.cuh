@@ -25,33 +25,42 @@ struct AttnArgs {
     int* err;
 };
 
-// grid (nchunks, Hkv, B), 128 threads.  The positions 0..pos of sequence b
-// are split into nchunks equal chunks (ceil((pos+1)/nchunks) each); CTA
-// (c, g, b) handles chunk c for the rep = H/Hkv query heads sharing KV head g
-// (heads g*rep .. g*rep+rep-1: contiguous groups), so every K/V row is read
-// once per group.  Within a CTA, sub-chunks of TC positions go through three
-// passes: scores (one warp per position: the row slice is one coalesced
-// 16-byte-per-lane load, the dot a warp reduction), the sub-chunk max and
-// exp(s - m), and the weighted V sum (one warp per position again).  Each
-// active CTA writes (m, l, o) per head: the running max of the scaled scores,
-// the sum of exp(s - m) and the unnormalised weighted V sum.  The last CTA to
-// arrive for (b, g) merges the partials and writes the output.
+// Shared memory of one attention work item (four warps).
 template <typename Acc, int HS, int REP>
-__global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
+struct AttnSmem {
+    static constexpr int TC = 64;  // positions per sub-chunk held in shared memory
+    Acc sc[TC][REP];
+    Acc red[4][REP];
+    Acc ostage[4][REP][HS];
+    int last;
+};
+
+// One work item: chunk c of sequence b for the rep = H/Hkv query heads that
+// share KV head g (heads g*rep .. g*rep+rep-1: contiguous groups), run by 128
+// threads (tid 0..127) that synchronise through `sy`.  The positions 0..pos
+// of sequence b are split into nchunks equal chunks (ceil((pos+1)/nchunks)
+// each), so every K/V row is read once per group.  Within an item, sub-chunks
+// of TC positions go through three passes: scores (one warp per position: the
+// row slice is one coalesced 16-byte-per-lane load, the dot a warp
+// reduction), the sub-chunk max and exp(s - m), and the weighted V sum (one
+// warp per position again).  Each active item writes (m, l, o) per head: the
+// running max of the scaled scores, the sum of exp(s - m) and the unnormalised
+// weighted V sum.  The last item to arrive for (b, g) merges the partials and
+// writes the output.  q, K and V are read through L2 (ld.global.cg), so an
+// item may follow, in the same launch, the kernel phase that wrote them.
+template <typename Acc, int HS, int REP, typename SY>
+__device__ __forceinline__ void attn_item(const AttnArgs& a, int c, int g, int b, int tid, const SY& sy,
+                                          AttnSmem<Acc, HS, REP>& sm) {
     static_assert(HS % 4 == 0 && HS <= 128, "head size");
     constexpr int NT = 128, NW = 4;
-    constexpr int TC = 64;                 // positions per sub-chunk held in shared memory
+    constexpr int TC = AttnSmem<Acc, HS, REP>::TC;
     constexpr int V4 = HS / 4;             // float4 per K/V row slice (<= 32: one per lane)
     constexpr int PB = 8;                  // positions a warp loads before reducing
-    __shared__ Acc sc[TC][REP];
-    __shared__ Acc red[NW][REP];
-    __shared__ Acc ostage[NW][REP][HS];
-    __shared__ int last_s;
-    const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    auto& sc = sm.sc;
+    auto& red = sm.red;
+    auto& ostage = sm.ostage;
+    const int lane = tid & 31, warp = tid >> 5;
 
-    grid_dep_wait();
-    grid_dep_launch();
     int pos = a.tp[b * a.tp_stride + 1];
     if (pos < 0 || pos >= a.seq_len) pos = 0;  // the GEMV kernel has flagged it
     const int T = pos + 1;
@@ -67,7 +76,7 @@ __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
     Acc qr[REP][4];
 #pragma unroll
     for (int h = 0; h < REP; h++) {
-        float4 qv = lane_on ? *reinterpret_cast<const float4*>(q + (size_t)h * HS + 4 * lane)
+        float4 qv = lane_on ? __ldcg(reinterpret_cast<const float4*>(q + (size_t)h * HS + 4 * lane))
                             : make_float4(0.f, 0.f, 0.f, 0.f);
         qr[h][0] = (Acc)qv.x; qr[h][1] = (Acc)qv.y; qr[h][2] = (Acc)qv.z; qr[h][3] = (Acc)qv.w;
     }
@@ -90,7 +99,7 @@ __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
 #pragma unroll
             for (int i = 0; i < PB; i++)
                 kv[i] = (lane_on && tq + i < n)
-                            ? __ldg(reinterpret_cast<const float4*>(kc + (size_t)(tb + tq + i) * a.kvd) + lane)
+                            ? __ldcg(reinterpret_cast<const float4*>(kc + (size_t)(tb + tq + i) * a.kvd) + lane)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < PB; i++) {
@@ -103,7 +112,7 @@ __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
                 }
             }
         }
-        __syncthreads();
+        sy.sync();
         // max over the sub-chunk, new running max, weights p = exp(s - m_new)
         Acc mnew[REP], alpha[REP];
 #pragma unroll
@@ -113,14 +122,14 @@ __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
             mx = warp_max(mx);
             if (lane == 0) red[warp][h] = mx;
         }
-        __syncthreads();
+        sy.sync();
 #pragma unroll
         for (int h = 0; h < REP; h++) {
             Acc mx = max(max(red[0][h], red[1][h]), max(red[2][h], red[3][h]));
             mnew[h] = max(m[h], mx);
             alpha[h] = exp(m[h] - mnew[h]);  // exp(-inf) = 0 on the first sub-chunk
         }
-        __syncthreads();
+        sy.sync();
 #pragma unroll
         for (int h = 0; h < REP; h++) {
             Acc ps = 0;
@@ -132,7 +141,7 @@ __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
             ps = warp_sum(ps);
             if (lane == 0) red[warp][h] = ps;
         }
-        __syncthreads();
+        sy.sync();
 #pragma unroll
         for (int h = 0; h < REP; h++) {
             l[h] = l[h] * alpha[h] + (red[0][h] + red[1][h]) + (red[2][h] + red[3][h]);
@@ -145,7 +154,7 @@ __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
 #pragma unroll
             for (int i = 0; i < PB; i++)
                 vv[i] = (lane_on && tq + i < n)
-                            ? __ldg(reinterpret_cast<const float4*>(vc + (size_t)(tb + tq + i) * a.kvd) + lane)
+                            ? __ldcg(reinterpret_cast<const float4*>(vc + (size_t)(tb + tq + i) * a.kvd) + lane)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int i = 0; i < PB; i++) {
@@ -159,7 +168,7 @@ __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
                 }
             }
         }
-        __syncthreads();
+        sy.sync();
     }
     // combine the four warps' weighted sums (same running max)
     if (lane_on) {
@@ -169,7 +178,15 @@ __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
             ostage[warp][h][4 * lane + 2] = o[h][2]; ostage[warp][h][4 * lane + 3] = o[h][3];
         }
     }
-    __syncthreads();
+    sy.sync();
+    if (nact == 1) {  // the whole range in one item: O / L directly (the merge would scale by e^0 = 1)
+        for (int i = tid; i < REP * HS; i += NT) {
+            const int h = i / HS, e = i % HS;
+            const Acc o_sum = (ostage[0][h][e] + ostage[1][h][e]) + (ostage[2][h][e] + ostage[3][h][e]);
+            a.out[(size_t)b * a.H * HS + ((size_t)g * REP + h) * HS + e] = (float)(o_sum / l[h]);
+        }
+        return;
+    }
     Acc* part = static_cast<Acc*>(a.part) +
                 ((((size_t)b * a.Hkv + g) * a.nchunks + c) * REP) * (HS + 2);
     for (int i = tid; i < REP * HS; i += NT) {
@@ -181,11 +198,11 @@ __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
         part[(size_t)tid * (HS + 2) + HS + 1] = l[tid];
     }
     __threadfence();
-    __syncthreads();
+    sy.sync();
     int* cnt = a.count + (size_t)b * a.Hkv + g;
-    if (tid == 0) last_s = (atomicAdd(cnt, 1) == nact - 1);
-    __syncthreads();
-    if (!last_s) return;
+    if (tid == 0) sm.last = (atomicAdd(cnt, 1) == nact - 1);
+    sy.sync();
+    if (!sm.last) return;
     __threadfence();
     // merge the nact partials of (b, g): M = max m_c, L = sum l_c e^{m_c - M},
     // O = sum o_c e^{m_c - M}; output O / L.
@@ -204,6 +221,15 @@ __global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
         a.out[(size_t)b * a.H * HS + ((size_t)g * REP + h) * HS + e] = (float)(Os / Ls);
     }
     if (tid == 0) *cnt = 0;
+}
+
+// grid (nchunks, Hkv, B), 128 threads: CTA (c, g, b) runs work item (c, g, b).
+template <typename Acc, int HS, int REP>
+__global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
+    __shared__ AttnSmem<Acc, HS, REP> sm;
+    grid_dep_wait();
+    grid_dep_launch();
+    attn_item<Acc, HS, REP>(a, blockIdx.x, blockIdx.y, blockIdx.z, threadIdx.x, SyncCTA(), sm);
 }
 
 typedef void (*AttnKernel)(const AttnArgs);

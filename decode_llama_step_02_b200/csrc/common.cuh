@@ -140,6 +140,20 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src, uint32
         : "memory");
 }
 
+// ---- CTA-wide synchronisation policies ------------------------------------------
+// Helpers that a whole group of threads runs together take one of these: the
+// full CTA (barrier 0), or the first n threads of the CTA on a named barrier
+// (a persistent kernel whose producer warp does not take part).
+struct SyncCTA {
+    __device__ __forceinline__ void sync() const { __syncthreads(); }
+    __device__ __forceinline__ int nthreads() const { return blockDim.x; }
+};
+struct SyncNamed {
+    int id, n;  // barrier 1..15, thread count (a multiple of 32)
+    __device__ __forceinline__ void sync() const { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+    __device__ __forceinline__ int nthreads() const { return n; }
+};
+
 // ---- reductions --------------------------------------------------------------
 template <typename T>
 __device__ __forceinline__ T warp_sum(T v) {

@@ -204,7 +204,7 @@ __device__ __forceinline__ void f32_post_load(const GemvArgs& a, F32Pre& r, floa
 }
 
 // Wide inputs (K/4 > F32_PER * blockDim): a plain strided loop after the wait.
-__device__ void load_input_f32_wide(const GemvArgs& a, int token, float* xs, double* red) {
+static __device__ void load_input_f32_wide(const GemvArgs& a, int token, float* xs, double* red) {
     const int K4 = a.K >> 2, nt = blockDim.x;
     const float4* in = reinterpret_cast<const float4*>(
         a.emb ? static_cast<const float*>(a.emb) + (size_t)token * a.K : a.in);
@@ -393,7 +393,7 @@ __device__ __forceinline__ void quantize_group_warp(const float* x, int gs, int8
 // once to fp32) when norm_w is set.
 __device__ __forceinline__ float q8_input_value(const GemvArgs& a, const int8_t* eq, const float* es, double inv,
                                                 int i) {
-    float v = eq ? (float)eq[i] * es[i / a.gs] : a.in[i];
+    float v = eq ? (float)eq[i] * es[i / a.gs] : __ldcg(a.in + i);
     if (a.norm_w) v = (float)((double)a.norm_w[i] * (inv * (double)v));
     return v;
 }
@@ -406,26 +406,27 @@ __device__ __forceinline__ float q8_input_value(const GemvArgs& a, const int8_t*
 // dependent loads.  Falls back to a plain loop when a lane would need more
 // than Q8_VPL values.
 // Slow path: one group at a time straight from global memory.
+template <typename SY>
 __device__ __noinline__ void q8_quantize_input_loop(const GemvArgs& a, const int8_t* eq, const float* es, int8_t* xq,
-                                                    float* xsc, double* red) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+                                                    float* xsc, double* red, const SY sy) {
+    const int nt = sy.nthreads(), lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = nt >> 5;
     const int K = a.K, gs = a.gs;
     double inv = 1.0;
     if (a.norm_w) {
         double ss = 0.0;
-        for (int i = threadIdx.x; i < K; i += blockDim.x) {
-            const float v = eq ? (float)eq[i] * es[i / gs] : a.in[i];
+        for (int i = threadIdx.x; i < K; i += nt) {
+            const float v = eq ? (float)eq[i] * es[i / gs] : __ldcg(a.in + i);
             ss += (double)v * (double)v;
         }
         ss = warp_sum(ss);
         if (lane == 0) red[warp] = ss;
-        __syncthreads();
+        sy.sync();
         double tot = 0.0;
         for (int i = 0; i < nw; i++) tot += red[i];
         inv = 1.0 / sqrt(tot / (double)K + 1e-5);
     }
     if (a.emb && blockIdx.x == 0)
-        for (int i = threadIdx.x; i < K; i += blockDim.x) a.x_resid[i] = (float)eq[i] * es[i / gs];
+        for (int i = threadIdx.x; i < K; i += nt) a.x_resid[i] = (float)eq[i] * es[i / gs];
     for (int g = warp; g < K / gs; g += nw) {
         float m = 0.f;
         for (int i = lane; i < gs; i += 32) m = fmaxf(m, fabsf(q8_input_value(a, eq, es, inv, g * gs + i)));
@@ -443,11 +444,11 @@ __device__ __noinline__ void q8_quantize_input_loop(const GemvArgs& a, const int
 // from 16-byte loads, four in flight per thread.  Pass 2: warp w quantizes its
 // groups w, w + nw, ... in batches of QB, issuing the loads of a whole batch
 // before using them.  A few round trips to L2 in all, with little code.
-template <int EPL, bool NORM>
+template <int EPL, bool NORM, typename SY>
 __device__ __forceinline__ void q8_quantize_input_batched(const GemvArgs& a, const int8_t* eq, const float* es,
-                                                          int8_t* xq, float* xsc, double* red) {
+                                                          int8_t* xq, float* xsc, double* red, const SY& sy) {
     constexpr int QB = 8;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int nt = sy.nthreads(), lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = nt >> 5;
     const int K = a.K, gs = 32 * EPL;
     const int ng = K / gs;
     if (NORM) {
@@ -462,7 +463,7 @@ __device__ __forceinline__ void q8_quantize_input_batched(const GemvArgs& a, con
 #pragma unroll
                 for (int e = 0; e < EPL; e++) {
                     const int i = g * gs + lane + 32 * e;
-                    v[j][e] = g < ng ? (eq ? (float)eq[i] * es[g] : a.in[i]) : 0.f;
+                    v[j][e] = g < ng ? (eq ? (float)eq[i] * es[g] : __ldcg(a.in + i)) : 0.f;
                     w[j][e] = g < ng ? a.norm_w[i] : 0.f;
                 }
             }
@@ -473,7 +474,7 @@ __device__ __forceinline__ void q8_quantize_input_batched(const GemvArgs& a, con
                 for (int e = 0; e < EPL; e++) ss += (double)v[j][e] * (double)v[j][e];
             ss = warp_sum(ss);
             if (lane == 0) red[warp] = ss;
-            __syncthreads();
+            sy.sync();
             if (warp == 0) L2C_STAMP(5);
             double tot = 0.0;
             for (int i = 0; i < nw; i++) tot += red[i];
@@ -510,20 +511,20 @@ __device__ __forceinline__ void q8_quantize_input_batched(const GemvArgs& a, con
         double ss = 0.0;
         const int K4 = K >> 2;
 #pragma unroll 4
-        for (int i4 = threadIdx.x; i4 < K4; i4 += blockDim.x) {
+        for (int i4 = threadIdx.x; i4 < K4; i4 += nt) {
             float4 v;
             if (eq) {
                 const char4 c4 = reinterpret_cast<const char4*>(eq)[i4];
                 const float sc = es[(4 * i4) / gs];
                 v = make_float4((float)c4.x * sc, (float)c4.y * sc, (float)c4.z * sc, (float)c4.w * sc);
             } else {
-                v = reinterpret_cast<const float4*>(a.in)[i4];
+                v = __ldcg(reinterpret_cast<const float4*>(a.in) + i4);
             }
             ss += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
         }
         ss = warp_sum(ss);
         if (lane == 0) red[warp] = ss;
-        __syncthreads();
+        sy.sync();
         double tot = 0.0;
         for (int i = 0; i < nw; i++) tot += red[i];
         inv = 1.0 / sqrt(tot / (double)K + 1e-5);
@@ -537,7 +538,7 @@ __device__ __forceinline__ void q8_quantize_input_batched(const GemvArgs& a, con
 #pragma unroll
             for (int e = 0; e < EPL; e++) {
                 const int i = g * gs + lane + 32 * e;
-                v[j][e] = g < ng ? (eq ? (float)eq[i] * es[g] : a.in[i]) : 0.f;
+                v[j][e] = g < ng ? (eq ? (float)eq[i] * es[g] : __ldcg(a.in + i)) : 0.f;
                 if (NORM) w[NORM ? j : 0][e] = g < ng ? a.norm_w[i] : 0.f;
             }
         }
@@ -571,13 +572,13 @@ __device__ __forceinline__ void q8_quantize_input_batched(const GemvArgs& a, con
 // Quantizes the GEMV input (embedding row or input vector, RMSNorm'd when
 // norm_w is set) into shared codes and scales; every thread of the CTA calls
 // it.
-template <bool NORM>
+template <bool NORM, typename SY = SyncCTA>
 __device__ __forceinline__ void q8_quantize_input(const GemvArgs& a, const int8_t* eq, const float* es, int8_t* xq,
-                                                  float* xsc, double* red) {
-    if (a.gs == 32) q8_quantize_input_batched<1, NORM>(a, eq, es, xq, xsc, red);
-    else if (a.gs == 64) q8_quantize_input_batched<2, NORM>(a, eq, es, xq, xsc, red);
-    else if (a.gs == 128) q8_quantize_input_batched<4, NORM>(a, eq, es, xq, xsc, red);
-    else q8_quantize_input_loop(a, eq, es, xq, xsc, red);
+                                                  float* xsc, double* red, const SY sy = SY()) {
+    if (a.gs == 32) q8_quantize_input_batched<1, NORM>(a, eq, es, xq, xsc, red, sy);
+    else if (a.gs == 64) q8_quantize_input_batched<2, NORM>(a, eq, es, xq, xsc, red, sy);
+    else if (a.gs == 128) q8_quantize_input_batched<4, NORM>(a, eq, es, xq, xsc, red, sy);
+    else q8_quantize_input_loop(a, eq, es, xq, xsc, red, sy);
 }
 
 // Exact-int32 group dots of UNIT rows (records at rec, stride rb) with the
@@ -660,8 +661,8 @@ struct Q8PreGM {
 };
 
 template <int EPL, int GM>
-__device__ __forceinline__ bool q8_pre_fits(const GemvArgs& a) {
-    const int ng = a.K / (32 * EPL), nw = blockDim.x >> 5;
+__device__ __forceinline__ bool q8_pre_fits(const GemvArgs& a, int nw) {
+    const int ng = a.K / (32 * EPL);
     return a.gs == 32 * EPL && (ng + nw - 1) / nw <= GM;
 }
 
@@ -669,8 +670,8 @@ __device__ __forceinline__ bool q8_pre_fits(const GemvArgs& a) {
 // codes eq * scale es) of the warp's groups.
 template <int EPL, int GM, bool NORM>
 __device__ __forceinline__ void q8_pre_load(const GemvArgs& a, const float* src, const int8_t* eq, const float* es,
-                                            bool gain, Q8Pre<EPL, GM, NORM>& r) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+                                            bool gain, Q8Pre<EPL, GM, NORM>& r, int nw) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gs = 32 * EPL, ng = a.K / gs;
 #pragma unroll
     for (int j = 0; j < GM; j++) {
@@ -681,7 +682,7 @@ __device__ __forceinline__ void q8_pre_load(const GemvArgs& a, const float* src,
             if (gain) {
                 if (NORM) r.w[NORM ? j : 0][e] = g < ng ? a.norm_w[i] : 0.f;
             } else {
-                r.v[j][e] = g < ng ? (eq ? (float)eq[i] * es[g] : src[i]) : 0.f;
+                r.v[j][e] = g < ng ? (eq ? (float)eq[i] * es[g] : __ldcg(src + i)) : 0.f;
             }
         }
     }
@@ -689,10 +690,10 @@ __device__ __forceinline__ void q8_pre_load(const GemvArgs& a, const float* src,
 
 // RMSNorm (double, when NORM) and Q8_0 codes of the values in r.  The
 // reductions of all groups run interleaved so their latencies overlap.
-template <int EPL, int GM, bool NORM, typename AfterLoads>
+template <int EPL, int GM, bool NORM, typename AfterLoads, typename SY = SyncCTA>
 __device__ __forceinline__ void q8_pre_finish(const GemvArgs& a, Q8Pre<EPL, GM, NORM>& r, int8_t* xq, float* xsc,
-                                              double* red, AfterLoads after_loads) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+                                              double* red, AfterLoads after_loads, const SY sy = SY()) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = sy.nthreads() >> 5;
     const int gs = 32 * EPL, ng = a.K / gs;
     if (a.emb && blockIdx.x == 0) {
 #pragma unroll
@@ -714,7 +715,7 @@ __device__ __forceinline__ void q8_pre_finish(const GemvArgs& a, Q8Pre<EPL, GM, 
         after_loads();  // every value has arrived by now
         ss = warp_sum(ss);
         if (lane == 0) red[warp] = ss;
-        __syncthreads();
+        sy.sync();
         double tot = 0.0;
         for (int i = 0; i < nw; i++) tot += red[i];
         const double inv = 1.0 / sqrt(tot / (double)a.K + 1e-5);
@@ -811,7 +812,7 @@ __global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, 
     constexpr bool NORM = MODE != M_RESID;
     constexpr int GM = Q8PreGM<EPL, NORM>::value;
     Q8Pre<EPL, GM, NORM> pre;
-    const bool split = GS > 0 && (NORM == (a.norm_w != nullptr)) && q8_pre_fits<EPL, GM>(a);  // CTA-uniform
+    const bool split = GS > 0 && (NORM == (a.norm_w != nullptr)) && q8_pre_fits<EPL, GM>(a, Q8_WARPS);  // CTA-uniform
     int token = 0, pos = 0;
     if (MODE == M_QKV) read_tp(a, token, pos);  // written before the step's first kernel
     const int8_t* eq = nullptr;
@@ -822,8 +823,8 @@ __global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, 
         es = reinterpret_cast<const float*>(rec + K);
     }
     if (split) {
-        if (NORM) q8_pre_load<EPL, GM, NORM>(a, nullptr, nullptr, nullptr, true, pre);
-        if (eq) q8_pre_load<EPL, GM, NORM>(a, nullptr, eq, es, false, pre);
+        if (NORM) q8_pre_load<EPL, GM, NORM>(a, nullptr, nullptr, nullptr, true, pre, Q8_WARPS);
+        if (eq) q8_pre_load<EPL, GM, NORM>(a, nullptr, eq, es, false, pre, Q8_WARPS);
     }
     if (MODE == M_QKV) rope_table(a, pos, rope_cs);
     if (warp == 0 && lane == 0 && a.prefetch_bytes) {
@@ -843,7 +844,7 @@ __global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, 
     // ---- after the wait: the input written by the previous kernel, then the
     // ring fill (its copies land while the codes are computed)
     if (MODE == M_QKV && a.amax && blockIdx.x == 0 && threadIdx.x == 0) *a.amax = 0ull;
-    if (split && !eq) q8_pre_load<EPL, GM, NORM>(a, a.in, nullptr, nullptr, false, pre);
+    if (split && !eq) q8_pre_load<EPL, GM, NORM>(a, a.in, nullptr, nullptr, false, pre, Q8_WARPS);
     if (warp == 0) L2C_STAMP(4);
     auto fill_ring = [&]() {
         if (lane == 0) {
@@ -957,14 +958,14 @@ __global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, 
 
 // ------------------------------------------------------------- small kernels --
 
-__global__ void k_set_tp(int* tp, int token, int pos) {
+static __global__ void k_set_tp(int* tp, int token, int pos) {
     tp[0] = token;
     tp[1] = pos;
 }
 
 // Greedy feedback between steps: token <- argmax of the step, pos += 1, and
 // the token is appended to the output ring.
-__global__ void k_advance(int* tp, const unsigned long long* amax, int* out_tokens, int* counter) {
+static __global__ void k_advance(int* tp, const unsigned long long* amax, int* out_tokens, int* counter) {
     int tok = argmax_key_index(*amax);
     tp[0] = tok;
     tp[1] += 1;
@@ -973,11 +974,11 @@ __global__ void k_advance(int* tp, const unsigned long long* amax, int* out_toke
     *counter = i + 1;
 }
 
-__global__ void k_argmax_index(const unsigned long long* amax, int* out) { *out = argmax_key_index(*amax); }
+static __global__ void k_argmax_index(const unsigned long long* amax, int* out) { *out = argmax_key_index(*amax); }
 
 // Block-reduced argmax over n values: per-thread best key, then one 64-bit
 // atomicMax per block (first index among equal maxima).
-__global__ void k_argmax(const float* x, int n, unsigned long long* key, int* err) {
+static __global__ void k_argmax(const float* x, int n, unsigned long long* key, int* err) {
     unsigned long long best = 0ull;
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
         float v = x[i];
@@ -1000,14 +1001,14 @@ __global__ void k_argmax(const float* x, int n, unsigned long long* key, int* er
 
 // Standalone Q8_0 quantization: one warp per group (bit-exact with the rule
 // of the quantize() listing).
-__global__ void k_quantize(const float* x, long long ngroups, int gs, int8_t* q, float* s) {
+static __global__ void k_quantize(const float* x, long long ngroups, int gs, int8_t* q, float* s) {
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
     for (long long g = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < ngroups; g += warps)
         quantize_group_warp(x + g * gs, gs, q + g * gs, s + g);
 }
 
 // Re-lays an fp32 matrix [rows][K] as Q8_0 row records [codes | scales | pad].
-__global__ void k_quantize_rows(const float* W, long long rows, int K, int gs, uint8_t* out, size_t rb) {
+static __global__ void k_quantize_rows(const float* W, long long rows, int K, int gs, uint8_t* out, size_t rb) {
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
     const int ng = K / gs;
     const long long total = rows * ng;
@@ -1022,7 +1023,7 @@ __global__ void k_quantize_rows(const float* W, long long rows, int K, int gs, u
 
 // Exact int32 group dot products through the same dp4a chunk loop as the Q8_0
 // GEMV: out[r][g] = sum_k qw[r][g*gs+k] * qx[g*gs+k].  One warp per row.
-__global__ void k_group_dots(const int8_t* qw, const int8_t* qx, int rows, int K, int gs, int* out) {
+static __global__ void k_group_dots(const int8_t* qw, const int8_t* qx, int rows, int K, int gs, int* out) {
     const int lane = threadIdx.x & 31;
     const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (r >= rows) return;

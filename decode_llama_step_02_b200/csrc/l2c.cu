@@ -22,6 +22,7 @@
 
 #include "../../include/l2c.h"
 #include "batched.cuh"
+#include "persistent.h"
 #include "kernels.cuh"
 
 using namespace l2c;
@@ -64,12 +65,22 @@ struct l2c_ctx {
     size_t bkq = 0, bks = 0;  // strides (bytes of codes, floats of scales) per sequence
     std::vector<cudaGraphExec_t> bgraph;  // index B (1..max_batch)
     // tuning
-    size_t pf_f32 = 256 << 10, pf_q8 = 256 << 10;
+    size_t pf_f32 = 32 << 10, pf_q8 = 64 << 10;  // per CTA; larger leads measured slower in the step graph
     int f32_ctas_per_sm = 1;
     size_t q8_smem_budget = 220 << 10;  // dynamic shared memory of one Q8_0 GEMV CTA
     bool pdl = true;     // programmatic dependent launch between the step's kernels
-    int late_trigger = 0;  // GEMVs let the next kernel launch only near their end
+    int late_trigger = 2;  // bit 0 fp32, bit 1 Q8_0: GEMVs let the next kernel launch only near their end
     bool graphs = true;  // replay the step as a CUDA graph (off: plain launches)
+    // persistent Q8_0 step (one launch per token), set up on first use
+    bool use_pstep = false;  // L2C_PERSISTENT=1 turns it on
+    bool pk_tried = false;
+    const void* pk = nullptr;  // nullptr: the per-layer kernels run instead
+    PLayout pl{};
+    int pk_grid = 0, pk_nchunks = 0;
+    size_t pk_pf = 0;  // L2 prefetch lead of the persistent step, bytes per CTA (0: off; measured no gain)
+    void* pk_part = nullptr;
+    unsigned* pk_sync = nullptr;  // {barrier arrivals, CTAs finished, abort flag, pad}
+    char pk_note[512] = {0};      // why the persistent step was dropped, if it was
     std::vector<void*> allocs;
     char msg[512] = {0};
     int status = L2C_OK;  // code of the last failure
@@ -171,7 +182,7 @@ static Q8Layout q8_layout(const l2c_ctx* h, int K, int gs, size_t rb, int unit, 
 template <int MODE>
 static cudaError_t launch_gemv(l2c_ctx* h, bool q80, GemvArgs a, int unit) {
     const int units = a.rows / unit;
-    a.late_trigger = h->late_trigger;
+    a.late_trigger = (h->late_trigger >> (q80 ? 1 : 0)) & 1;
     if (!q80) {
         int grid = h->sms * h->f32_ctas_per_sm;
         if (grid > units) grid = units;
@@ -227,7 +238,7 @@ static int set_smem_limits(l2c_ctx* h) {
 }
 
 // Kernels of the step, in order within a layer.
-enum StepKernel : int { SK_QKV = 0, SK_ATTN = 1, SK_WO = 2, SK_W13 = 3, SK_W2 = 4, SK_CLS = 5 };
+enum StepKernel : int { SK_QKV = 0, SK_ATTN = 1, SK_WO = 2, SK_W13 = 3, SK_W2 = 4, SK_CLS = 5, SK_STEP = 6 };
 
 // Enqueues kernel `kind` of layer l (sequence 0) on stream s.
 static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, int l, int seq = 0) {
@@ -312,9 +323,77 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
     return L2C_OK;
 }
 
+// Sets up the persistent Q8_0 step on first use; leaves h->pk null (the
+// per-layer kernels run) when the shapes or the device do not allow it: a
+// head size / GQA ratio without an instantiation, a width not a multiple of
+// 64, a group size other than 32, 64 or 128, no cooperative launch, or a ring
+// smaller than two of the largest row units.
+static int ensure_pstep(l2c_ctx* h) {
+    if (h->pk_tried) return L2C_OK;
+    h->pk_tried = true;
+    if (!h->use_pstep) return L2C_OK;
+    const void* k = pstep_kernel(h->hs, h->rep);
+    if (!k || h->d % 64 || h->h % 64 || (h->gs != 32 && h->gs != 64 && h->gs != 128)) return L2C_OK;
+    int coop = 0, maxopt = 0;
+    CK(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, h->dev));
+    CK(cudaDeviceGetAttribute(&maxopt, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->dev));
+    if (!coop) return L2C_OK;
+    size_t st = 0;
+    CK(pstep_static_smem(k, &st));
+    const int kmax = h->d > h->h ? h->d : h->h;
+    const PLayout L0 = pstep_layout(0, kmax, h->gs, h->hs, h->rep);
+    const size_t used = st + L0.total + 1024;
+    if ((size_t)maxopt <= used) return L2C_OK;
+    size_t ring = ((size_t)maxopt - used) & ~size_t(127);
+    const size_t cap = env_size("L2C_PSTEP_RING", 0);
+    if (cap && cap < ring) ring = cap & ~size_t(127);
+    const size_t umax = PS_UNIT * h->qWqkv.rb > h->qW2.rb ? PS_UNIT * h->qWqkv.rb : h->qW2.rb;
+    if (((ring / PS_PRODUCERS) & ~size_t(127)) < 2 * umax) return L2C_OK;  // two units per producer slice
+    const PLayout L = pstep_layout((uint32_t)ring, kmax, h->gs, h->hs, h->rep);
+    CK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total));
+    int occ = 0;
+    CK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, PS_THREADS, L.total));
+    if (occ < 1) return L2C_OK;
+    int nch = 2 * h->sms / h->Hkv;
+    nch = nch < 1 ? 1 : (nch > 64 ? 64 : nch);
+    int rc;
+    if ((rc = dalloc(h, &h->pk_part, (size_t)h->Hkv * nch * h->rep * (h->hs + 2) * sizeof(double))) ||
+        (rc = dalloc(h, (void**)&h->pk_sync, 16)))
+        return rc;
+    CK(cudaMemsetAsync(h->pk_sync, 0, 16, h->stream));
+    h->pk = k;
+    h->pl = L;
+    h->pk_grid = h->sms;
+    h->pk_nchunks = nch;
+    return L2C_OK;
+}
+
+static int launch_pstep(l2c_ctx* h) {
+    PStepArgs a = {};
+    a.Wqkv = h->qWqkv.p; a.Wo = h->qWo.p; a.W13 = h->qW13.p; a.W2 = h->qW2.p; a.Wcls = h->qWcls.p; a.E = h->qE.p;
+    a.rb_d = h->qWqkv.rb; a.rb_h = h->qW2.rb;
+    a.rms_att = h->rms_att; a.rms_ffn = h->rms_ffn; a.rms_final = h->rms_final; a.freq = h->freq;
+    a.x = h->x; a.q = h->q; a.att = h->att; a.hb = h->hb; a.logits = h->logits;
+    a.kc = h->kc; a.vc = h->vc;
+    a.d = h->d; a.hdim = h->h; a.L = h->L; a.H = h->H; a.Hkv = h->Hkv; a.hs = h->hs; a.kvd = h->kvd;
+    a.V = h->V; a.S = h->S; a.gs = h->gs;
+    a.tp = h->tp; a.amax = h->amax; a.err = h->err;
+    a.bar = h->pk_sync; a.abort_flag = reinterpret_cast<int*>(h->pk_sync + 2);
+    a.part = h->pk_part; a.count = h->attn_cnt; a.nchunks = h->pk_nchunks;
+    a.ring_bytes = h->pl.xq - h->pl.ring;  // the ring is a multiple of 128 bytes
+    a.pf_bytes = h->pk_pf;
+    cudaError_t e = pstep_launch(h->pk, h->pk_grid, a, h->pl, h->cap);
+    if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "persistent step launch: %s", cudaGetErrorString(e));
+    return L2C_OK;
+}
+
 // Enqueues one decode step of sequence 0 on h->cap (being captured).
 static int enqueue_step(l2c_ctx* h, bool q80) {
     int rc;
+    if (q80 && h->use_pstep) {
+        if ((rc = ensure_pstep(h)) != L2C_OK) return rc;
+        if (h->pk) return launch_pstep(h);
+    }
     for (int l = 0; l < h->L; l++)
         for (int k = SK_QKV; k <= SK_W2; k++)
             if ((rc = launch_step_kernel(h, h->cap, k, q80, l)) != L2C_OK) return rc;
@@ -421,7 +500,25 @@ static int build_batch_graph(l2c_ctx* h, int B) {
     return L2C_OK;
 }
 
+static int build_graph_once(l2c_ctx* h, bool q80, bool gen);
+
+// Captures the step graph.  If the persistent Q8_0 step cannot be captured
+// (cooperative launches in graphs), the per-layer kernels take its place.
 static int build_graph(l2c_ctx* h, bool q80, bool gen) {
+    if (h->graph[q80][gen]) return L2C_OK;
+    int rc = q80 ? ensure_pstep(h) : L2C_OK;  // allocates: not while capturing
+    if (rc != L2C_OK) return rc;
+    rc = build_graph_once(h, q80, gen);
+    if (rc != L2C_OK && q80 && h->pk) {
+        snprintf(h->pk_note, sizeof(h->pk_note), "persistent step not capturable: %.400s", h->msg);
+        snprintf(h->msg, sizeof(h->msg), "%s", h->pk_note);  // readable through l2c_last_error
+        h->pk = nullptr;
+        rc = build_graph_once(h, q80, gen);
+    }
+    return rc;
+}
+
+static int build_graph_once(l2c_ctx* h, bool q80, bool gen) {
     if (h->graph[q80][gen]) return L2C_OK;
     CK(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
     int rc = enqueue_step(h, q80);
@@ -501,9 +598,11 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
     h->q8_smem_budget = env_size("L2C_Q8_SMEM", h->q8_smem_budget);
     h->f32_ctas_per_sm = (int)env_size("L2C_F32_CTAS_PER_SM", 1);
     h->pdl = env_size("L2C_NO_PDL", 0) == 0;
-    h->late_trigger = (int)env_size("L2C_LATE_TRIGGER", 0);
+    h->late_trigger = (int)env_size("L2C_LATE_TRIGGER", (size_t)h->late_trigger);
     h->graphs = env_size("L2C_NO_GRAPH", 0) == 0;
     h->attn_nchunks = (int)env_size("L2C_ATTN_SPLIT", 16);
+    h->use_pstep = env_size("L2C_PERSISTENT", 0) != 0;
+    h->pk_pf = env_size("L2C_PSTEP_PF", h->pk_pf);
     if (h->attn_nchunks < 1) h->attn_nchunks = 16;
     if (h->attn_nchunks > h->S) h->attn_nchunks = h->S;
     auto bail = [&](int code) { l2c_destroy(h); return code; };
@@ -749,15 +848,28 @@ extern "C" int l2c_attention(l2c_ctx* h, const float* q, const float* k, const f
 }
 
 extern "C" int l2c_time_kernel(l2c_ctx* h, int kind, int q80, int iters, float* avg_ms) {
-    if (!h || kind < SK_QKV || kind > SK_CLS || iters < 1 || !avg_ms) return fail(h, L2C_E_ARG, "time_kernel: bad arguments");
+    if (!h || kind < SK_QKV || kind > SK_STEP || iters < 1 || !avg_ms) return fail(h, L2C_E_ARG, "time_kernel: bad arguments");
     if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
+    if (kind == SK_STEP) {
+        int rc = q80 ? ensure_pstep(h) : L2C_OK;
+        if (rc) return rc;
+        if (!q80 || !h->pk) return fail(h, L2C_E_STATE, "time_kernel: the step does not run as one kernel here");
+    }
     cudaEvent_t e0, e1;
     CK(cudaEventCreate(&e0));
     CK(cudaEventCreate(&e1));
     int rc = L2C_OK;
     cudaError_t er = cudaEventRecord(e0, h->stream);
-    for (int i = 0; i < iters && rc == L2C_OK && er == cudaSuccess; i++)
-        rc = launch_step_kernel(h, h->stream, kind, q80 != 0, kind == SK_CLS ? 0 : i % h->L);
+    for (int i = 0; i < iters && rc == L2C_OK && er == cudaSuccess; i++) {
+        if (kind == SK_STEP) {
+            cudaStream_t saved = h->cap;
+            h->cap = h->stream;
+            rc = launch_pstep(h);
+            h->cap = saved;
+        } else {
+            rc = launch_step_kernel(h, h->stream, kind, q80 != 0, kind == SK_CLS ? 0 : i % h->L);
+        }
+    }
     if (er == cudaSuccess) er = cudaEventRecord(e1, h->stream);
     if (er == cudaSuccess) er = cudaEventSynchronize(e1);
     float ms = 0.f;
@@ -858,11 +970,23 @@ extern "C" int l2c_sync(l2c_ctx* h) {
     CK(cudaMemcpy(&e, h->err, 4, cudaMemcpyDeviceToHost));
     if (e) {
         CK(cudaMemset(h->err, 0, 4));
+        if (e & DERR_TIMEOUT) {  // an abandoned step can leave barriers and counters mid-way
+            if (h->pk_sync) CK(cudaMemset(h->pk_sync, 0, 16));
+            CK(cudaMemset(h->attn_cnt, 0, (size_t)h->max_batch * h->Hkv * 4));
+        }
         return fail(h, L2C_E_DEVICE, "device error word 0x%x:%s%s%s%s", e, (e & DERR_TOKEN) ? " token" : "",
                     (e & DERR_POS) ? " pos" : "", (e & DERR_TIMEOUT) ? " wait-timeout" : "",
                     (e & DERR_NAN) ? " nan" : "");
     }
     return L2C_OK;
+}
+
+extern "C" int l2c_persistent(l2c_ctx* h) {
+    if (!h) return L2C_E_ARG;
+    if (!h->gs) return 0;
+    int rc = ensure_pstep(h);
+    if (rc) return rc;
+    return h->pk ? 1 : 0;
 }
 
 extern "C" void* l2c_stream(l2c_ctx* h) { return h ? (void*)h->stream : nullptr; }

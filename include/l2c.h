@@ -245,11 +245,28 @@ L2C_API int l2c_attention_noalloc(const float* q_dev, const float* k_dev, const 
  * stores the average time per launch in ms (two CUDA events around the
  * loop).  Launch i uses layer i % n_layers, so consecutive launches stream
  * different weights.  kind: 0 = RMSNorm+QKV+RoPE, 1 = attention, 2 = wo,
- * 3 = RMSNorm+W1/W3+SwiGLU, 4 = W2, 5 = final RMSNorm+classifier.  The
- * kernels use the handle's current token/position and update its state
- * (KV slot, activations) as in a step.  Blocks.
+ * 3 = RMSNorm+W1/W3+SwiGLU, 4 = W2, 5 = final RMSNorm+classifier,
+ * 6 = the whole Q8_0 step as one persistent kernel (q80 = 1 only; L2C_E_STATE
+ * where l2c_persistent() is 0).  The kernels use the handle's current
+ * token/position and update its state (KV slot, activations) as in a step.
+ * Blocks.
  */
 L2C_API int l2c_time_kernel(l2c_ctx* h, int kind, int q80, int iters, float* avg_ms);
+
+/*
+ * l2c_persistent - whether the single-sequence Q8_0 step (l2c_forward_q80,
+ * l2c_generate with q80) runs as ONE persistent kernel: one CTA per SM that
+ * streams every weight row of the step through a shared-memory ring while
+ * grid barriers order the layer phases.  The arithmetic and the results are
+ * those of the per-layer kernels.  It does where the Q8_0 group size is 32, 64
+ * or 128, dim and hidden_dim are multiples of 64, (head_size, n_heads /
+ * n_kv_heads) has an instantiation, the device supports cooperative launches,
+ * the ring fits, and the environment variable L2C_PERSISTENT=1 was set at
+ * l2c_create (off by default: on the 7B shape the per-layer kernels are
+ * faster).  Sets it up on first call.
+ * Returns 1 or 0 (0 too before l2c_enable_q80), or a negative error code.
+ */
+L2C_API int l2c_persistent(l2c_ctx* h);
 
 /* l2c_sync - waits for the handle's stream, then reads and clears the
  * device error word: L2C_E_DEVICE if a kernel recorded an error since the
