@@ -105,9 +105,15 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            # nvidia-smi takes a moment to start: let its first sample arrive before
+            # the timed region opens, then keep only samples taken inside it
+            t_end = time.time() + 5.0
+            while not self.rows and time.time() < t_end and self.proc.poll() is None:
+                time.sleep(0.02)
+            self.rows.clear()
         except Exception:
             self.proc = None
         return self

@@ -101,15 +101,18 @@ __device__ __forceinline__ void attn_item(const AttnArgs& a, int c, int g, int b
                 kv[i] = (lane_on && tq + i < n)
                             ? __ldcg(reinterpret_cast<const float4*>(kc + (size_t)(tb + tq + i) * a.kvd) + lane)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
+            // the PB scores of each head in one reduce-scatter: lane 4i ends with
+            // position tq + i's total
 #pragma unroll
-            for (int i = 0; i < PB; i++) {
+            for (int h = 0; h < REP; h++) {
+                Acc sp[PB];
 #pragma unroll
-                for (int h = 0; h < REP; h++) {
-                    Acc s = (Acc)kv[i].x * qr[h][0] + (Acc)kv[i].y * qr[h][1] + (Acc)kv[i].z * qr[h][2] +
+                for (int i = 0; i < PB; i++)
+                    sp[i] = (Acc)kv[i].x * qr[h][0] + (Acc)kv[i].y * qr[h][1] + (Acc)kv[i].z * qr[h][2] +
                             (Acc)kv[i].w * qr[h][3];
-                    s = warp_sum(s);
-                    if (lane == 0 && tq + i < n) sc[tq + i][h] = s * scale;
-                }
+                const Acc s = warp_sum_scatter<PB>(sp);
+                const int i = lane >> 2;
+                if ((lane & 3) == 0 && tq + i < n) sc[tq + i][h] = s * scale;
             }
         }
         sy.sync();

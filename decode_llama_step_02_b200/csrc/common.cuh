@@ -169,6 +169,36 @@ __device__ __forceinline__ T warp_max(T v) {
     return v;
 }
 
+// Sums each of v[0..N-1] over the warp (N = 1, 2, 4 or 8); lane l ends with
+// the total of v[(l / (32 / N)) % N].  A reduce-scatter: at each of the first
+// log2(N) steps (offsets 16, 8, ...) a lane keeps half of its values and adds
+// its partner's copies of them, then a butterfly finishes; each total comes
+// from the same additions in the same order as warp_sum applied to that value
+// alone, in 5 shuffle rounds of one value instead of 5 of N.
+template <int N, typename T>
+__device__ __forceinline__ T warp_sum_scatter(const T (&v)[N]) {
+    static_assert(N == 1 || N == 2 || N == 4 || N == 8, "N");
+    const int lane = threadIdx.x & 31;
+    T w[N];
+#pragma unroll
+    for (int j = 0; j < N; j++) w[j] = v[j];
+    int o = 16;
+#pragma unroll
+    for (int m = N; m > 1; m >>= 1, o >>= 1) {
+        const bool up = lane & o;
+#pragma unroll
+        for (int j = 0; j < m / 2; j++) {
+            const T keep = up ? w[j + m / 2] : w[j];
+            const T send = up ? w[j] : w[j + m / 2];
+            w[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    T t = w[0];
+#pragma unroll
+    for (; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    return t;
+}
+
 // Block-wide sum; `red` must hold one T per warp.  All threads get the result.
 template <typename T>
 __device__ __forceinline__ T block_sum(T v, T* red) {

@@ -317,6 +317,9 @@ __global__ void __launch_bounds__(F32_THREADS, 2) k_gemv_f32(const GemvArgs a, c
     grid_dep_wait();
     if (!a.late_trigger) grid_dep_launch();
     if (MODE == M_QKV && a.amax && blockIdx.x == 0 && threadIdx.x == 0) *a.amax = 0ull;
+    // residual: thread j fetches x of row r0 + j now, for the epilogue
+    float xres = 0.f;
+    if (MODE == M_RESID && (int)threadIdx.x < r1 - r0) xres = __ldcg(a.out + r0 + threadIdx.x);
     if (fits) f32_post_load(a, pre, xs, red);
     else load_input_f32_wide(a, token, xs, red);
     __syncthreads();
@@ -346,7 +349,7 @@ __global__ void __launch_bounds__(F32_THREADS, 2) k_gemv_f32(const GemvArgs a, c
         } else if (MODE == M_W13) {
             epi_w13(a, r / 2, v[0], v[PAIR - 1]);
         } else if (MODE == M_RESID) {
-            a.out[r] = a.out[r] + v[0];
+            a.out[r] = (j == (int)threadIdx.x ? xres : __ldcg(a.out + r)) + v[0];
         } else {
             a.out[r] = v[0];
             if (v[0] != v[0]) set_error(a.err, DERR_NAN);
@@ -845,6 +848,9 @@ __global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, 
     // ring fill (its copies land while the codes are computed)
     if (MODE == M_QKV && a.amax && blockIdx.x == 0 && threadIdx.x == 0) *a.amax = 0ull;
     if (split && !eq) q8_pre_load<EPL, GM, NORM>(a, a.in, nullptr, nullptr, false, pre, Q8_WARPS);
+    // residual: lane k fetches now the x of this warp's k-th row, for the epilogue
+    float xres = 0.f;
+    if (MODE == M_RESID && lane < nmine) xres = __ldcg(a.out + u0 + warp + lane * Q8_WARPS);
     if (warp == 0) L2C_STAMP(4);
     auto fill_ring = [&]() {
         if (lane == 0) {
@@ -927,13 +933,14 @@ __global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, 
 #pragma unroll
         for (int r = 0; r < UNIT; r++) acc[r] = warp_sum(acc[r]);
         const int u = u0 + warp + k * Q8_WARPS;
+        const float xo = MODE == M_RESID ? __shfl_sync(0xffffffffu, xres, k & 31) : 0.f;
         if (lane == 0) {
             if (MODE == M_QKV) {
                 epi_qkv(a, u, (float)acc[0], (float)acc[UNIT - 1], pos, rope_cs);
             } else if (MODE == M_W13) {
                 epi_w13(a, u, (float)acc[0], (float)acc[UNIT - 1]);
             } else if (MODE == M_RESID) {
-                a.out[u] = a.out[u] + (float)acc[0];
+                a.out[u] = (k < 32 ? xo : __ldcg(a.out + u)) + (float)acc[0];
             } else {
                 const float v = (float)acc[0];
                 a.out[u] = v;

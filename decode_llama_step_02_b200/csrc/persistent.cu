@@ -319,37 +319,6 @@ __device__ __forceinline__ bool p_prologue_gs(const GemvArgs& a, const int8_t* e
     return p_prologue<4, NORM>(a, eq, es, bar_idx, s, sy, flag, xq, xsc, sxd, red, wp);
 }
 
-// Sums each of v[0..U-1] over the warp; lane l ends with the total of
-// v[l / (32 / U)].  A reduce-scatter: the lanes first trade the values they
-// do not keep, then finish with a butterfly, so every total comes from the
-// same additions in the same order as warp_sum applied to that value alone.
-template <int U>
-__device__ __forceinline__ double warp_sum_scatter(const double (&v)[U]) {
-    static_assert(U == 1 || U == 2 || U == 4, "unit");
-    const int lane = threadIdx.x & 31;
-    if constexpr (U == 1) {
-        return warp_sum(v[0]);
-    } else if constexpr (U == 2) {
-        const bool h = lane & 16;
-        double keep = h ? v[1] : v[0];
-        keep += __shfl_xor_sync(0xffffffffu, h ? v[0] : v[1], 16);
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
-        return keep;
-    } else {
-        const bool h = lane & 16;
-        double k0 = h ? v[2] : v[0], k1 = h ? v[3] : v[1];
-        k0 += __shfl_xor_sync(0xffffffffu, h ? v[0] : v[2], 16);
-        k1 += __shfl_xor_sync(0xffffffffu, h ? v[1] : v[3], 16);
-        const bool g = lane & 8;
-        double keep = g ? k1 : k0;
-        keep += __shfl_xor_sync(0xffffffffu, g ? k0 : k1, 8);
-#pragma unroll
-        for (int o = 4; o > 0; o >>= 1) keep += __shfl_xor_sync(0xffffffffu, keep, o);
-        return keep;
-    }
-}
-
 template <int UNIT>
 __device__ __forceinline__ void pdot(const uint8_t* base, size_t rb, const int8_t* xq, const double* sxd, int K, int gs,
                                      double (&acc)[UNIT]) {
