@@ -387,6 +387,110 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+# ------------------------------------------------- supplementary configs ----
+
+def run_extra(args):
+    """The other workloads of the measurement plan, one JSON line each (not bench
+    lines): tiny, 15M and 110M decoded with forced uniform tokens over all their
+    positions, timed in buckets of 64 positions; the GQA-7B batch of 32 ragged
+    sequences (Q8_0 GS=64) as one batched step."""
+    import torch
+
+    import __graft_entry__
+    __graft_entry__.build()
+    import decode_llama_step_02_b200 as l2c
+
+    peak, peak_kind = measured_peak()
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    stream = torch.cuda.current_stream()
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    small = ((synth.TINY, 0, (False,)), (synth.M15, 32, (False, True)), (synth.M110, 64, (False, True)))
+    for spec, gs, variants in (small if args.extra in ("all", "small") else ()):
+        dec = l2c.Decoder(spec.cfg, torch.from_numpy(synth.blob(spec)).cuda(), spec.shared_weights)
+        if gs:
+            dec.enable_q80(gs)
+        S = spec.seq_len
+        toks = synth.tokens(spec.seed, 2, S, spec.vocab_size)
+        for q80 in variants:
+            for p in range(8):  # warm-up, captures the step graph
+                dec.forward_ptr(int(toks[p]), p, q80)
+            dec.sync()
+            buckets = []
+            for b0 in range(0, S, 64):
+                a, b = ev(), ev()
+                a.record(stream)
+                for p in range(b0, min(S, b0 + 64)):
+                    dec.forward_ptr(int(toks[p]), p, q80)
+                b.record(stream)
+                torch.cuda.synchronize()
+                n = min(S, b0 + 64) - b0
+                us = 1e3 * a.elapsed_time(b) / n
+                by = bytes_per_token(q80, b0 + n // 2, spec, gs or GS)
+                buckets.append({"pos": [b0, b0 + n - 1], "us_per_token": us, "tokens_per_s": 1e6 / us,
+                                "bytes_per_token_mid": by, "gbs": by / us / 1e3})
+            dec.sync()
+            weights = bytes_per_token(q80, 0, spec, gs or GS)
+            resident = weights < l2
+            for bk in buckets:
+                bk["frac_of_measured_hbm"] = None if resident else bk["gbs"] / peak
+            print(json.dumps({
+                "extra": True, "config": spec.name, "variant": f"q8_0 gs={gs}" if q80 else "fp32",
+                "shape": dict(zip(("dim", "hidden", "layers", "heads", "kv_heads", "vocab", "seq_len"), spec.cfg)),
+                "inputs": "forced tokens uniform in [0, vocab) (stream 2), positions 0..seq_len-1 in order",
+                "timing": "CUDA events around 64 consecutive decode steps through the C ABI, host launch included",
+                "l2_resident": bool(resident), "l2_bytes": l2, "peak_gbs": peak, "peak_kind": peak_kind,
+                "buckets": buckets}), flush=True)
+        dec.close()
+
+    if args.extra not in ("all", "batch"):
+        return 0
+    # GQA-7B, 32 sequences, one batched Q8_0 step
+    spec, B = synth.GQA7B, 32
+    blob = device_blob(torch, spec)
+    dec = l2c.Decoder(spec.cfg, blob, spec.shared_weights, max_batch=B)
+    del blob
+    torch.cuda.empty_cache()
+    dec.enable_q80(GS)
+    toks = synth.tokens(spec.seed, 0, B, spec.vocab_size)
+    pos = synth.positions(spec.seed, 0, B, spec.seq_len)
+    for sq in range(B):
+        if pos[sq]:
+            k, v = synth.kv_prefill(spec, seq=sq, n_pos=int(pos[sq]))
+            dec.kv_load(k, v, seq=sq)
+            del k, v
+    tk = torch.from_numpy(toks.astype(np.int32)).cuda()
+    ps = torch.from_numpy(pos.astype(np.int32)).cuda()
+    out = torch.empty((B, spec.vocab_size), dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        dec.forward_batch(tk, ps, out, q80=True)
+    dec.sync()
+    reps = 10
+    a, b = ev(), ev()
+    a.record(stream)
+    for _ in range(reps):
+        dec.forward_batch(tk, ps, out, q80=True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    dec.sync()
+    ms = a.elapsed_time(b) / reps
+    d, h, L, H, Hkv, V, S = spec.cfg
+    kvd = Hkv * (d // H)
+    wbytes = bytes_per_token(True, -1, spec, GS)  # weights only (pos -1: no KV)
+    kvbytes = float(sum(8.0 * L * (int(p) + 1) * kvd for p in pos))
+    by = wbytes + kvbytes
+    print(json.dumps({
+        "extra": True, "config": spec.name + " batch 32", "variant": f"q8_0 gs={GS}", "ms_per_step": ms,
+        "tokens_per_s": B / ms * 1e3, "bytes_per_step": by, "weight_bytes": wbytes, "kv_bytes": kvbytes,
+        "gbs": by / ms / 1e6, "frac_of_measured_hbm": by / ms / 1e6 / peak, "frac_of_8tbs": by / ms / 1e6 / NOMINAL_HBM_GBS,
+        "inputs": "tokens uniform (stream 2), positions uniform in [0, 2047] (stream 3), caches prefilled N(0,1)",
+        "timing": f"CUDA events around {reps} batched steps (l2c_forward_batch), device-resident inputs"}), flush=True)
+    dec.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -394,6 +498,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extra", nargs="?", const="all", choices=("all", "small", "batch"),
+                    help="the other workloads (small: tiny, 15M, 110M position curves; batch: GQA-7B batch 32), "
+                         "not bench lines")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling case: the 7B widths with this many layers (not a bench line)")
     args = ap.parse_args()
@@ -408,6 +515,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         return run_reference(args, rank)
+    if args.extra:
+        return run_extra(args)
     if world > 1:
         import datetime
 

@@ -41,14 +41,14 @@ struct AttnSmem {
 // of sequence b are split into nchunks equal chunks (ceil((pos+1)/nchunks)
 // each), so every K/V row is read once per group.  Within an item, sub-chunks
 // of TC positions go through three passes: scores (one warp per position: the
-// row slice is one coalesced 16-byte-per-lane load, the dot a warp
-// reduction), the sub-chunk max and exp(s - m), and the weighted V sum (one
-// warp per position again).  Each active item writes (m, l, o) per head: the
+// row slice is one coalesced 16-byte-per-lane load, the dots of a batch of
+// positions one reduce-scatter), the sub-chunk max and exp(s - m), and the
+// weighted V sum (one warp per position again).  Each active item writes (m, l, o) per head: the
 // running max of the scaled scores, the sum of exp(s - m) and the unnormalised
 // weighted V sum.  The last item to arrive for (b, g) merges the partials and
 // writes the output.  q, K and V are read through L2 (ld.global.cg), so an
 // item may follow, in the same launch, the kernel phase that wrote them.
-template <typename Acc, int HS, int REP, typename SY>
+template <typename Acc, int HS, int REP, typename SY, bool PRE = false>
 __device__ __forceinline__ void attn_item(const AttnArgs& a, int c, int g, int b, int tid, const SY& sy,
                                           AttnSmem<Acc, HS, REP>& sm) {
     static_assert(HS % 4 == 0 && HS <= 128, "head size");
@@ -90,29 +90,59 @@ __device__ __forceinline__ void attn_item(const AttnArgs& a, int c, int g, int b
         o[h][0] = o[h][1] = o[h][2] = o[h][3] = 0;
     }
 
+    // Sub-chunks of TC positions: warp w takes the NB batches of PB positions
+    // starting at w*PB + j*NW*PB.
+    constexpr int NB = TC / (NW * PB);
+    // PRE = true requests a sub-chunk's rows at once; it costs registers, and at
+    // 168 a thread only 3 CTAs fit an SM, so the 16-chunk grid needs two waves:
+    // measured slower, hence one batch at a time by default
+    constexpr bool VPRE = PRE && sizeof(Acc) == 4 && REP <= 2;
+    constexpr bool KPRE = PRE && (sizeof(Acc) == 4 || REP <= 2);
+    const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int tb = t0; tb < t1; tb += TC) {
         const int n = min(TC, t1 - tb);
-        // scores: warp per position, lanes across the head's row slice; each
-        // warp loads PB positions' rows before reducing, to keep loads in flight
-        for (int tq = warp * PB; tq < n; tq += NW * PB) {
-            float4 kv[PB];
+        float4 kv[KPRE ? NB : 1][PB];
+        float4 vv[VPRE ? NB : 1][PB];
+        auto load_k = [&](int j, float4 (&dst)[PB]) {
+            const int tq = warp * PB + j * NW * PB;
 #pragma unroll
-            for (int i = 0; i < PB; i++)
-                kv[i] = (lane_on && tq + i < n)
-                            ? __ldcg(reinterpret_cast<const float4*>(kc + (size_t)(tb + tq + i) * a.kvd) + lane)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-            // the PB scores of each head in one reduce-scatter: lane 4i ends with
-            // position tq + i's total
+            for (int i = 0; i < PB; i++) {
+                const bool on = lane_on && tq + i < n;
+                dst[i] = on ? __ldcg(reinterpret_cast<const float4*>(kc + (size_t)(tb + tq + i) * a.kvd) + lane)
+                            : zero4;
+            }
+        };
 #pragma unroll
-            for (int h = 0; h < REP; h++) {
-                Acc sp[PB];
+        for (int j = 0; j < NB; j++) {
+            const int tq = warp * PB + j * NW * PB;
+            if (KPRE) load_k(j, kv[KPRE ? j : 0]);
 #pragma unroll
-                for (int i = 0; i < PB; i++)
-                    sp[i] = (Acc)kv[i].x * qr[h][0] + (Acc)kv[i].y * qr[h][1] + (Acc)kv[i].z * qr[h][2] +
-                            (Acc)kv[i].w * qr[h][3];
-                const Acc s = warp_sum_scatter<PB>(sp);
-                const int i = lane >> 2;
-                if ((lane & 3) == 0 && tq + i < n) sc[tq + i][h] = s * scale;
+            for (int i = 0; i < PB; i++) {
+                const bool on = lane_on && tq + i < n;
+                if (VPRE)
+                    vv[VPRE ? j : 0][i] =
+                        on ? __ldcg(reinterpret_cast<const float4*>(vc + (size_t)(tb + tq + i) * a.kvd) + lane) : zero4;
+            }
+        }
+        // scores: the PB sums of each head in one reduce-scatter (lane 4i ends
+        // with position tq + i's total)
+#pragma unroll
+        for (int j = 0; j < NB; j++) {
+            const int tq = warp * PB + j * NW * PB;
+            if (tq < n) {  // warp-uniform
+                if (!KPRE) load_k(j, kv[0]);
+                const float4 (&kj)[PB] = kv[KPRE ? j : 0];
+#pragma unroll
+                for (int h = 0; h < REP; h++) {
+                    Acc sp[PB];
+#pragma unroll
+                    for (int i = 0; i < PB; i++)
+                        sp[i] = (Acc)kj[i].x * qr[h][0] + (Acc)kj[i].y * qr[h][1] +
+                                (Acc)kj[i].z * qr[h][2] + (Acc)kj[i].w * qr[h][3];
+                    const Acc s = warp_sum_scatter<PB>(sp);
+                    const int i = lane >> 2;
+                    if ((lane & 3) == 0 && tq + i < n) sc[tq + i][h] = s * scale;
+                }
             }
         }
         sy.sync();
@@ -152,21 +182,30 @@ __device__ __forceinline__ void attn_item(const AttnArgs& a, int c, int g, int b
             o[h][0] *= alpha[h]; o[h][1] *= alpha[h]; o[h][2] *= alpha[h]; o[h][3] *= alpha[h];
         }
         // weighted V sum: warp per position, lane owns one float4 slice of the row
-        for (int tq = warp * PB; tq < n; tq += NW * PB) {
-            float4 vv[PB];
 #pragma unroll
-            for (int i = 0; i < PB; i++)
-                vv[i] = (lane_on && tq + i < n)
-                            ? __ldcg(reinterpret_cast<const float4*>(vc + (size_t)(tb + tq + i) * a.kvd) + lane)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < NB; j++) {
+            const int tq = warp * PB + j * NW * PB;
+            if (tq < n) {  // warp-uniform
+                float4 vl[PB];
 #pragma unroll
-            for (int i = 0; i < PB; i++) {
-                if (tq + i < n) {
+                for (int i = 0; i < PB; i++) {
+                    if (VPRE) {
+                        vl[i] = vv[VPRE ? j : 0][i];
+                    } else {
+                        const bool on = lane_on && tq + i < n;
+                        vl[i] = on ? __ldcg(reinterpret_cast<const float4*>(vc + (size_t)(tb + tq + i) * a.kvd) + lane)
+                                   : zero4;
+                    }
+                }
 #pragma unroll
-                    for (int h = 0; h < REP; h++) {
-                        const Acc w = sc[tq + i][h];
-                        o[h][0] += w * (Acc)vv[i].x; o[h][1] += w * (Acc)vv[i].y;
-                        o[h][2] += w * (Acc)vv[i].z; o[h][3] += w * (Acc)vv[i].w;
+                for (int i = 0; i < PB; i++) {
+                    if (tq + i < n) {
+#pragma unroll
+                        for (int h = 0; h < REP; h++) {
+                            const Acc w = sc[tq + i][h];
+                            o[h][0] += w * (Acc)vl[i].x; o[h][1] += w * (Acc)vl[i].y;
+                            o[h][2] += w * (Acc)vl[i].z; o[h][3] += w * (Acc)vl[i].w;
+                        }
                     }
                 }
             }

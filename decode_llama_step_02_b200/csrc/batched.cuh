@@ -25,6 +25,7 @@ namespace l2c {
 constexpr int BMAX = 32;          // sequences per GEMM (n = 4 tiles of 8)
 constexpr int BG_WARPS = 2;       // consumer warps per CTA, 16 rows each
 constexpr int BG_ROWS = 16 * BG_WARPS;
+constexpr int BPREP_SPLIT = 8;    // CTAs per sequence of the prep kernel (ranges of groups)
 
 struct BPrepArgs {
     const float* in;        // [B][K] fp32 input (x, attention output or hb)
@@ -35,7 +36,7 @@ struct BPrepArgs {
     float* x_resid;         // layer 0: receives the dequantized embedding rows [B][d]
     int K, gs;
     int8_t* xq;             // [B][kq_stride] codes
-    float* xs;              // [B][ks_stride] scales
+    double* xs;             // [B][ks_stride] scales, in double (exact copies of the fp32 scales)
     size_t kq_stride, ks_stride;
     const int* tp;          // [B][2] token, pos
     int vocab, seq_len;
@@ -43,11 +44,17 @@ struct BPrepArgs {
     int* err;
 };
 
-// One CTA per sequence: input row, optional RMSNorm (double), Q8_0 codes.
+// CTA (b, y) of a (B, Y) grid: sequence b's input row and its RMSNorm sum (the
+// whole row, in every CTA of the sequence), then the RMSNorm (double) and the
+// Q8_0 codes of the y-th of Y equal ranges of the row's groups.
 __global__ void __launch_bounds__(256) k_bprep(const BPrepArgs a) {
     extern __shared__ float bp_xs[];
     __shared__ double red[32];
     const int b = blockIdx.x;
+    const int ngr = a.K / a.gs;
+    const int g0 = (int)((long long)ngr * blockIdx.y / gridDim.y);
+    const int g1 = (int)((long long)ngr * (blockIdx.y + 1) / gridDim.y);
+    const int i0 = g0 * a.gs, i1 = g1 * a.gs;  // this CTA's elements
     grid_dep_wait();
     grid_dep_launch();
     const int K = a.K, gs = a.gs;
@@ -64,11 +71,13 @@ __global__ void __launch_bounds__(256) k_bprep(const BPrepArgs a) {
         for (int i = threadIdx.x; i < K; i += blockDim.x) {
             float v = (float)eq[i] * es[i / gs];
             bp_xs[i] = v;
-            a.x_resid[(size_t)b * K + i] = v;
+            if (i >= i0 && i < i1) a.x_resid[(size_t)b * K + i] = v;
         }
-        if (a.amax && threadIdx.x == 0) a.amax[b] = 0ull;
+        if (a.amax && threadIdx.x == 0 && blockIdx.y == 0) a.amax[b] = 0ull;
+    } else if (a.norm_w) {
+        for (int i = threadIdx.x; i < K; i += blockDim.x) bp_xs[i] = in[i];  // the whole row for the norm
     } else {
-        for (int i = threadIdx.x; i < K; i += blockDim.x) bp_xs[i] = in[i];
+        for (int i = i0 + (int)threadIdx.x; i < i1; i += blockDim.x) bp_xs[i] = in[i];
     }
     __syncthreads();
     if (a.norm_w) {
@@ -76,14 +85,17 @@ __global__ void __launch_bounds__(256) k_bprep(const BPrepArgs a) {
         for (int i = threadIdx.x; i < K; i += blockDim.x) ss += (double)bp_xs[i] * (double)bp_xs[i];
         ss = block_sum(ss, red);
         double inv = 1.0 / sqrt(ss / (double)K + 1e-5);
-        for (int i = threadIdx.x; i < K; i += blockDim.x)
+        for (int i = i0 + (int)threadIdx.x; i < i1; i += blockDim.x)
             bp_xs[i] = (float)((double)a.norm_w[i] * (inv * (double)bp_xs[i]));
         __syncthreads();
     }
     const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     int8_t* q = a.xq + (size_t)b * a.kq_stride;
-    float* s = a.xs + (size_t)b * a.ks_stride;
-    for (int g = warp; g < K / gs; g += nw) quantize_group_warp(bp_xs + g * gs, gs, q + g * gs, s + g);
+    double* s = a.xs + (size_t)b * a.ks_stride;
+    for (int g = g0 + warp; g < g1; g += nw) {
+        const float scale = quantize_group_warp(bp_xs + g * gs, gs, q + g * gs, nullptr);
+        if ((threadIdx.x & 31) == 0) s[g] = (double)scale;
+    }
 }
 
 struct BGemmArgs {
@@ -92,7 +104,7 @@ struct BGemmArgs {
     int rows, K, gs, kc;    // kc: K bytes per stage (a multiple of 32 and of gs, dividing K)
     int B;                  // live sequences (<= BMAX); codes of the others are zero
     const int8_t* xq;       // [BMAX][kq_stride]
-    const float* xs;        // [BMAX][ks_stride]
+    const double* xs;       // [BMAX][ks_stride] activation scales in double
     size_t kq_stride, ks_stride;
     float* out;             // QKV: q [B][d]; RESID: x [B][d]; W13: hb [B][h]; CLS: logits [B][V]
     size_t out_stride;
@@ -116,7 +128,8 @@ __device__ __forceinline__ void mma_s8(int (&c)[4], const uint32_t (&a)[4], uint
 }
 
 // Shared memory per stage: weights [BG_ROWS][kc+16], weight scales
-// [BG_ROWS][kc/gs], activations [BMAX][kc+16], activation scales [BMAX][kc/gs].
+// [BG_ROWS][kc/gs] fp32, activations [BMAX][kc+16], activation scales
+// [BMAX][kc/gs] double.
 struct BLayout {
     int ns;
     int kcp;          // kc + 16 (row pitch in shared memory; spreads rows over banks)
@@ -128,11 +141,12 @@ __host__ __device__ inline BLayout make_blayout(int kc, int gs, int ns) {
     L.ns = ns;
     L.kcp = kc + 16;
     const size_t sc = ((size_t)(kc / gs) * 4 + 15) & ~size_t(15);
+    const size_t scx = ((size_t)(kc / gs) * 8 + 15) & ~size_t(15);
     L.w_off = 0;
     L.ws_off = L.w_off + (size_t)BG_ROWS * L.kcp;
     L.x_off = L.ws_off + (size_t)BG_ROWS * sc;
     L.xs_off = L.x_off + (size_t)BMAX * L.kcp;
-    L.stage_bytes = L.xs_off + (size_t)BMAX * sc;
+    L.stage_bytes = L.xs_off + (size_t)BMAX * scx;
     L.stage_bytes = (L.stage_bytes + 127) & ~size_t(127);
     return L;
 }
@@ -177,7 +191,7 @@ __global__ void __launch_bounds__(32 * (BG_WARPS + 1)) k_bgemm_q8(const BGemmArg
         // activations come from the prep kernel: wait for it before copying them
         grid_dep_wait();
         const uint32_t bytes_stage =
-            (uint32_t)((size_t)nrows * (a.kc + sc_bytes) + (size_t)BMAX * (a.kc + sc_bytes));
+            (uint32_t)((size_t)nrows * (a.kc + sc_bytes) + (size_t)BMAX * (a.kc + 2 * sc_bytes));
         bool ok = true;
         int issued = 0;
         for (int c = 0; c < nchunks && ok; c++) {
@@ -200,9 +214,9 @@ __global__ void __launch_bounds__(32 * (BG_WARPS + 1)) k_bgemm_q8(const BGemmArg
             for (int b = lane; b < BMAX; b += 32) {
                 bulk_g2s(st + L.x_off + (size_t)b * L.kcp, a.xq + (size_t)b * a.kq_stride + (size_t)c * a.kc, a.kc,
                          &full[s], pol_x);
-                bulk_g2s(st + L.xs_off + (size_t)b * ((sc_bytes + 15) & ~size_t(15)),
-                         reinterpret_cast<const uint8_t*>(a.xs + (size_t)b * a.ks_stride) + (size_t)c * sc_bytes,
-                         (uint32_t)sc_bytes, &full[s], pol_x);
+                bulk_g2s(st + L.xs_off + (size_t)b * ((2 * sc_bytes + 15) & ~size_t(15)),
+                         reinterpret_cast<const uint8_t*>(a.xs + (size_t)b * a.ks_stride) + (size_t)c * 2 * sc_bytes,
+                         (uint32_t)(2 * sc_bytes), &full[s], pol_x);
             }
             issued = c + 1;
         }
@@ -230,7 +244,8 @@ __global__ void __launch_bounds__(32 * (BG_WARPS + 1)) k_bgemm_q8(const BGemmArg
         const uint8_t* wt = st + L.w_off;
         const float* wsc = reinterpret_cast<const float*>(st + L.ws_off);
         const uint8_t* xt = st + L.x_off;
-        const float* xsc = reinterpret_cast<const float*>(st + L.xs_off);
+        const double* xsc = reinterpret_cast<const double*>(st + L.xs_off);
+        const size_t scxp = ((2 * sc_bytes + 15) & ~size_t(15)) / 8;  // doubles per sequence
         if (wr0 < nrows) {
             for (int g = 0; g < gpc; g++) {
                 int cc[4][4];
@@ -256,12 +271,12 @@ __global__ void __launch_bounds__(32 * (BG_WARPS + 1)) k_bgemm_q8(const BGemmArg
                 const double sw1 = (double)wsc[(size_t)(wr0 + gid + 8) * (scp / 4) + g];
 #pragma unroll
                 for (int n = 0; n < 4; n++) {
-                    const double sx0 = (double)xsc[(size_t)(8 * n + 2 * tig) * (scp / 4) + g];
-                    const double sx1 = (double)xsc[(size_t)(8 * n + 2 * tig + 1) * (scp / 4) + g];
-                    acc[n][0] += (double)cc[n][0] * sw0 * sx0;
-                    acc[n][1] += (double)cc[n][1] * sw0 * sx1;
-                    acc[n][2] += (double)cc[n][2] * sw1 * sx0;
-                    acc[n][3] += (double)cc[n][3] * sw1 * sx1;
+                    const double sx0 = xsc[(size_t)(8 * n + 2 * tig) * scxp + g];
+                    const double sx1 = xsc[(size_t)(8 * n + 2 * tig + 1) * scxp + g];
+                    acc[n][0] += i2d_exact(cc[n][0]) * sw0 * sx0;
+                    acc[n][1] += i2d_exact(cc[n][1]) * sw0 * sx1;
+                    acc[n][2] += i2d_exact(cc[n][2]) * sw1 * sx0;
+                    acc[n][3] += i2d_exact(cc[n][3]) * sw1 * sx1;
                 }
             }
         }

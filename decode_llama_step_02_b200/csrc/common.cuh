@@ -154,6 +154,14 @@ struct SyncNamed {
     __device__ __forceinline__ int nthreads() const { return n; }
 };
 
+// ---- exact int32 -> double on the FP64 pipe ------------------------------------
+// 2^52 + 2^31 + v is a double whose low word is the bits of v + 2^31: build it
+// and subtract 2^52 + 2^31 (one DADD, exact).  Same value as the conversion
+// instruction, which issues on a narrow unit on this part.
+__device__ __forceinline__ double i2d_exact(int v) {
+    return __hiloint2double(0x43300000, (int)((unsigned)v ^ 0x80000000u)) - 4503601774854144.0;
+}
+
 // ---- reductions --------------------------------------------------------------
 template <typename T>
 __device__ __forceinline__ T warp_sum(T v) {

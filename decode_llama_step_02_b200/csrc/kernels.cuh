@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(F32_THREADS, 2) k_gemv_f32(const GemvArgs a, c
 // codes and scales in shared memory, one warp per group, with the rule of the
 // quantize() listing: scale = max|x| / 127 in fp32, code = round(x / scale)
 // (fp32 quotient, half away from zero); a zero group gets scale 0, codes 0.
-__device__ __forceinline__ void quantize_group_warp(const float* x, int gs, int8_t* q, float* s) {
+__device__ __forceinline__ float quantize_group_warp(const float* x, int gs, int8_t* q, float* s) {
     const int lane = threadIdx.x & 31;
     float m = 0.f;
     for (int i = lane; i < gs; i += 32) m = fmaxf(m, fabsf(x[i]));
@@ -388,7 +388,8 @@ __device__ __forceinline__ void quantize_group_warp(const float* x, int gs, int8
         float v = scale == 0.f ? 0.f : roundf(x[i] / scale);
         q[i] = (int8_t)(int)v;
     }
-    if (lane == 0) *s = scale;
+    if (lane == 0 && s) *s = scale;
+    return scale;
 }
 
 // The value of input element i of a Q8_0 GEMV: the embedding row on layer 0
@@ -624,7 +625,7 @@ __device__ __forceinline__ void q8_rows_dot64(const uint8_t* rec, size_t rb, con
             const float* sw = reinterpret_cast<const float*>(row + K);
             if (GS == 64) {
                 const int d = (c[0] + c[1]) + (c[2] + c[3]);
-                if (in) acc[r] += (double)d * (double)sw[t] * sxd[t];
+                if (in) acc[r] += i2d_exact(d) * (double)sw[t] * sxd[t];
             } else if (GS == 32) {
                 // chunk f of step j: the group of the lane's first 32 bytes is f < 2
                 int lo = 0, hi = 0;
@@ -635,13 +636,13 @@ __device__ __forceinline__ void q8_rows_dot64(const uint8_t* rec, size_t rb, con
                     hi += f < 2 ? 0 : c[j];
                 }
                 if (in) {
-                    acc[r] += (double)lo * (double)sw[2 * t] * sxd[2 * t];
-                    acc[r] += (double)hi * (double)sw[2 * t + 1] * sxd[2 * t + 1];
+                    acc[r] += i2d_exact(lo) * (double)sw[2 * t] * sxd[2 * t];
+                    acc[r] += i2d_exact(hi) * (double)sw[2 * t + 1] * sxd[2 * t + 1];
                 }
             } else {  // GS == 128: lanes 2m and 2m+1 hold the two halves of group t/2
                 int d = (c[0] + c[1]) + (c[2] + c[3]);
                 d += __shfl_xor_sync(0xffffffffu, d, 1);
-                if (in && (t & 1) == 0) acc[r] += (double)d * (double)sw[t >> 1] * sxd[t >> 1];
+                if (in && (t & 1) == 0) acc[r] += i2d_exact(d) * (double)sw[t >> 1] * sxd[t >> 1];
             }
         }
     }

@@ -61,9 +61,11 @@ struct l2c_ctx {
     cudaGraphExec_t graph[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
     // batched Q8_0 step: quantized activations of every sequence, one graph per batch size
     int8_t* bxq = nullptr;
-    float* bxs = nullptr;
+    double* bxs = nullptr;
     size_t bkq = 0, bks = 0;  // strides (bytes of codes, floats of scales) per sequence
     std::vector<cudaGraphExec_t> bgraph;  // index B (1..max_batch)
+    size_t bgemm_smem = 64 << 10;         // dynamic shared memory a batched GEMM CTA may take
+    int bgemm_stages = 3;                 // ring stages (deeper rings cost the second CTA per SM)
     // tuning
     size_t pf_f32 = 32 << 10, pf_q8 = 64 << 10;  // per CTA; larger leads measured slower in the step graph
     int f32_ctas_per_sm = 1;
@@ -229,6 +231,7 @@ static int set_smem_limits(l2c_ctx* h) {
     CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     L2C_Q8_ATTR(0) L2C_Q8_ATTR(32) L2C_Q8_ATTR(64) L2C_Q8_ATTR(128)
 #undef L2C_Q8_ATTR
+    h->bgemm_smem = (size_t)maxopt - 8192;
     CK(cudaFuncSetAttribute(k_bgemm_q8<M_QKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
     CK(cudaFuncSetAttribute(k_bgemm_q8<M_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
     CK(cudaFuncSetAttribute(k_bgemm_q8<M_W13>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
@@ -418,9 +421,9 @@ static int ensure_batched(l2c_ctx* h) {
     h->bks = ((kmax / h->gs) + 3) & ~size_t(3);
     int rc;
     if ((rc = dalloc(h, (void**)&h->bxq, (size_t)BMAX * h->bkq)) != L2C_OK) return rc;
-    if ((rc = dalloc(h, (void**)&h->bxs, (size_t)BMAX * h->bks * 4)) != L2C_OK) return rc;
+    if ((rc = dalloc(h, (void**)&h->bxs, (size_t)BMAX * h->bks * 8)) != L2C_OK) return rc;
     CK(cudaMemsetAsync(h->bxq, 0, (size_t)BMAX * h->bkq, h->stream));
-    CK(cudaMemsetAsync(h->bxs, 0, (size_t)BMAX * h->bks * 4, h->stream));
+    CK(cudaMemsetAsync(h->bxs, 0, (size_t)BMAX * h->bks * 8, h->stream));
     h->bgraph.assign((size_t)h->max_batch + 1, nullptr);
     return L2C_OK;
 }
@@ -432,7 +435,7 @@ static int bprep(l2c_ctx* h, cudaStream_t s, int B, const float* in, size_t in_s
     p.emb = emb ? h->qE.p : nullptr; p.emb_rb = h->qE.rb; p.x_resid = h->x;
     p.K = K; p.gs = h->gs; p.xq = h->bxq; p.xs = h->bxs; p.kq_stride = h->bkq; p.ks_stride = h->bks;
     p.tp = h->tp; p.vocab = h->V; p.seq_len = h->S; p.amax = amax; p.err = h->err;
-    CK(launch(s, true, k_bprep, dim3(B), dim3(256), (size_t)K * 4, p));
+    CK(launch(s, true, k_bprep, dim3(B, BPREP_SPLIT), dim3(256), (size_t)K * 4, p));
     return L2C_OK;
 }
 
@@ -447,7 +450,12 @@ static int bgemm(l2c_ctx* h, cudaStream_t s, int B, const Q8Mat& m, size_t row0,
     g.seq_stride = (size_t)h->L * h->S * h->kvd;
     g.freq = h->freq; g.d = h->d; g.kvd = h->kvd; g.hs = h->hs; g.seq_len = h->S;
     g.tp = h->tp; g.amax = h->amax; g.err = h->err; g.prefetch_bytes = h->pf_q8;
-    BLayout L = make_blayout(g.kc, h->gs, 3);
+    // as many ring stages as the shared memory holds (2..16): the weight slices
+    // of one stage are small, so the depth sets the bytes in flight
+    BLayout L = make_blayout(g.kc, h->gs, 1);
+    int ns = (int)(h->bgemm_smem / (L.stage_bytes + 16));
+    ns = ns < 2 ? 2 : (ns > h->bgemm_stages ? h->bgemm_stages : ns);
+    L = make_blayout(g.kc, h->gs, ns);
     size_t smem = (size_t)L.ns * L.stage_bytes + 16 * (size_t)L.ns;
     int grid = (rows + BG_ROWS - 1) / BG_ROWS;
     CK(launch(s, true, k_bgemm_q8<MODE>, dim3(grid), dim3(32 * (BG_WARPS + 1)), smem, g, L));
@@ -602,6 +610,7 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
     h->graphs = env_size("L2C_NO_GRAPH", 0) == 0;
     h->attn_nchunks = (int)env_size("L2C_ATTN_SPLIT", 16);
     h->use_pstep = env_size("L2C_PERSISTENT", 0) != 0;
+    h->bgemm_stages = (int)env_size("L2C_BGEMM_STAGES", (size_t)h->bgemm_stages);
     h->pk_pf = env_size("L2C_PSTEP_PF", h->pk_pf);
     if (h->attn_nchunks < 1) h->attn_nchunks = 16;
     if (h->attn_nchunks > h->S) h->attn_nchunks = h->S;
