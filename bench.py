@@ -203,6 +203,24 @@ def oracle_sample(q80_also=True, pos=512):
     return ntok, dt, setup
 
 
+# ---------------------------------------------------------- ranks (N > 1) ----
+
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The largest of every rank's x (all ranks call it; one all-reduce)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, seconds_max: float) -> float:
+    """Units per second of the whole job: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / seconds_max
+
+
 def host_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -276,12 +294,6 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # warm-up (captures both step graphs)
     for _ in range(max(args.warmup, 1)):
@@ -301,9 +313,9 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
     barrier()
     dec.sync()
-    ms = max_over_ranks(e0.elapsed_time(e1))
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
     tokens = 2 * len(POSITIONS) * args.steps * world
-    value = tokens / (ms / 1e3)
+    value = whole_job_rate(2 * len(POSITIONS) * args.steps, world, ms / 1e3)
 
     # ---- per (variant, position) breakdown
     peak, peak_kind = measured_peak()
@@ -356,7 +368,7 @@ def run_ours(args, rank, world, local_rank):
                 lg = dec.forward(TOKEN, p, q80)
                 host.copy_(lg, non_blocking=True)
         torch.cuda.synchronize()
-    e2e_s = max_over_ranks(time.perf_counter() - t0)
+    e2e_s = max_over_ranks(time.perf_counter() - t0, world)
     barrier()
     e2e = {"value": tokens / e2e_s, "unit": UNIT,
            "h2d_bytes_per_step": 2 * len(POSITIONS) * 8,          # token + position per decode step
