@@ -46,11 +46,15 @@ struct AttnSmem {
 // weighted V sum (one warp per position again).  Each active item writes (m, l, o) per head: the
 // running max of the scaled scores, the sum of exp(s - m) and the unnormalised
 // weighted V sum.  The last item to arrive for (b, g) merges the partials and
-// writes the output.  q, K and V are read through L2 (ld.global.cg), so an
-// item may follow, in the same launch, the kernel phase that wrote them.
-template <typename Acc, int HS, int REP, typename SY, bool PRE = false>
+// writes the output.  With COH, q, K and V are read through L2 (ld.global.cg),
+// so an item may follow, in the same launch, the kernel phase that wrote them;
+// otherwise through the read-only path.
+template <typename Acc, int HS, int REP, typename SY, bool PRE = false, bool COH = false>
 __device__ __forceinline__ void attn_item(const AttnArgs& a, int c, int g, int b, int tid, const SY& sy,
                                           AttnSmem<Acc, HS, REP>& sm) {
+    // q, K and V: read-only for this launch unless COH (then through L2, coherent
+    // with writes of other CTAs earlier in the same launch)
+    auto ld4 = [](const float4* p) { return COH ? __ldcg(p) : __ldg(p); };
     static_assert(HS % 4 == 0 && HS <= 128, "head size");
     constexpr int NT = 128, NW = 4;
     constexpr int TC = AttnSmem<Acc, HS, REP>::TC;
@@ -76,7 +80,7 @@ __device__ __forceinline__ void attn_item(const AttnArgs& a, int c, int g, int b
     Acc qr[REP][4];
 #pragma unroll
     for (int h = 0; h < REP; h++) {
-        float4 qv = lane_on ? __ldcg(reinterpret_cast<const float4*>(q + (size_t)h * HS + 4 * lane))
+        float4 qv = lane_on ? ld4(reinterpret_cast<const float4*>(q + (size_t)h * HS + 4 * lane))
                             : make_float4(0.f, 0.f, 0.f, 0.f);
         qr[h][0] = (Acc)qv.x; qr[h][1] = (Acc)qv.y; qr[h][2] = (Acc)qv.z; qr[h][3] = (Acc)qv.w;
     }
@@ -108,7 +112,7 @@ __device__ __forceinline__ void attn_item(const AttnArgs& a, int c, int g, int b
 #pragma unroll
             for (int i = 0; i < PB; i++) {
                 const bool on = lane_on && tq + i < n;
-                dst[i] = on ? __ldcg(reinterpret_cast<const float4*>(kc + (size_t)(tb + tq + i) * a.kvd) + lane)
+                dst[i] = on ? ld4(reinterpret_cast<const float4*>(kc + (size_t)(tb + tq + i) * a.kvd) + lane)
                             : zero4;
             }
         };
@@ -121,7 +125,7 @@ __device__ __forceinline__ void attn_item(const AttnArgs& a, int c, int g, int b
                 const bool on = lane_on && tq + i < n;
                 if (VPRE)
                     vv[VPRE ? j : 0][i] =
-                        on ? __ldcg(reinterpret_cast<const float4*>(vc + (size_t)(tb + tq + i) * a.kvd) + lane) : zero4;
+                        on ? ld4(reinterpret_cast<const float4*>(vc + (size_t)(tb + tq + i) * a.kvd) + lane) : zero4;
             }
         }
         // scores: the PB sums of each head in one reduce-scatter (lane 4i ends
@@ -193,7 +197,7 @@ __device__ __forceinline__ void attn_item(const AttnArgs& a, int c, int g, int b
                         vl[i] = vv[VPRE ? j : 0][i];
                     } else {
                         const bool on = lane_on && tq + i < n;
-                        vl[i] = on ? __ldcg(reinterpret_cast<const float4*>(vc + (size_t)(tb + tq + i) * a.kvd) + lane)
+                        vl[i] = on ? ld4(reinterpret_cast<const float4*>(vc + (size_t)(tb + tq + i) * a.kvd) + lane)
                                    : zero4;
                     }
                 }

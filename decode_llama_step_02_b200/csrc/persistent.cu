@@ -515,8 +515,8 @@ __global__ void __launch_bounds__(PS_THREADS, 1) k_step_q8(const PStepArgs s, co
             const SyncNamed hsy{2 + half, 128};
             const int items = nch * s.Hkv;
             for (int it = (int)blockIdx.x * 2 + half; it < items; it += 2 * (int)gridDim.x)
-                attn_item<double, HS, REP, SyncNamed, false>(t, it % nch, it / nch, 0, threadIdx.x & 127, hsy,
-                                                             asm2[half]);
+                attn_item<double, HS, REP, SyncNamed, false, true>(t, it % nch, it / nch, 0, threadIdx.x & 127,
+                                                                   hsy, asm2[half]);
             if (threadIdx.x == 0) PSTAMP(wp, 4);
         }
     }
