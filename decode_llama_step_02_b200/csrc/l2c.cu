@@ -56,7 +56,8 @@ struct l2c_ctx {
     unsigned long long* key_scratch = nullptr;
     void* attn_part = nullptr;
     int* attn_cnt = nullptr;
-    int attn_nchunks = 16;  // CTAs per (sequence, KV head) in attention
+    int attn_nchunks = 16;      // CTAs per (sequence, KV head) in the fp32 attention
+    int attn_nchunks_f64 = 24;  // ... in the double attention (compute-bound: more CTAs pay)
     // graphs: [q80][gen]
     cudaGraphExec_t graph[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
     // batched Q8_0 step: quantized activations of every sequence, one graph per batch size
@@ -286,10 +287,10 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
         t.q = q; t.kc = kslot; t.vc = vslot; t.seq_stride = (size_t)h->L * S * kvd;
         t.out = att; t.tp = tp; t.tp_stride = 2;
         t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = (int)kvd; t.seq_len = h->S;
-        t.nchunks = h->attn_nchunks;
+        t.nchunks = q80 ? h->attn_nchunks_f64 : h->attn_nchunks;
         t.part = h->attn_part; t.count = h->attn_cnt; t.err = h->err;
         AttnKernel ak = q80 ? attn_kernel_for<double>(h->hs, h->rep) : attn_kernel_for<float>(h->hs, h->rep);
-        e = launch(s, true, ak, dim3(h->attn_nchunks, h->Hkv, 1), dim3(128), 0, t);
+        e = launch(s, true, ak, dim3(t.nchunks, h->Hkv, 1), dim3(128), 0, t);
         break;
     }
     case SK_WO:  // wo + residual
@@ -477,9 +478,9 @@ static int enqueue_batch_step(l2c_ctx* h, cudaStream_t s, int B) {
         t.q = h->q; t.kc = h->kc + (size_t)l * S * kvd; t.vc = h->vc + (size_t)l * S * kvd;
         t.seq_stride = (size_t)h->L * S * kvd; t.out = h->att; t.tp = h->tp; t.tp_stride = 2;
         t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = (int)kvd; t.seq_len = h->S;
-        t.nchunks = h->attn_nchunks;
+        t.nchunks = h->attn_nchunks_f64;
         t.part = h->attn_part; t.count = h->attn_cnt; t.err = h->err;
-        CK(launch(s, true, ak, dim3(h->attn_nchunks, h->Hkv, B), dim3(128), 0, t));
+        CK(launch(s, true, ak, dim3(t.nchunks, h->Hkv, B), dim3(128), 0, t));
         if ((rc = bprep(h, s, B, h->att, d, (int)d, nullptr, false, nullptr))) return rc;
         if ((rc = bgemm<M_RESID>(h, s, B, h->qWo, (size_t)l * d, (int)d, (int)d, h->x, d, l))) return rc;
         if ((rc = bprep(h, s, B, h->x, d, (int)d, h->rms_ffn + (size_t)l * d, false, nullptr))) return rc;
@@ -614,6 +615,9 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
     h->pk_pf = env_size("L2C_PSTEP_PF", h->pk_pf);
     if (h->attn_nchunks < 1) h->attn_nchunks = 16;
     if (h->attn_nchunks > h->S) h->attn_nchunks = h->S;
+    h->attn_nchunks_f64 = (int)env_size("L2C_ATTN_SPLIT_F64", (size_t)h->attn_nchunks_f64);
+    if (h->attn_nchunks_f64 < 1) h->attn_nchunks_f64 = 24;
+    if (h->attn_nchunks_f64 > h->S) h->attn_nchunks_f64 = h->S;
     auto bail = [&](int code) { l2c_destroy(h); return code; };
     if (cudaGetDevice(&h->dev) != cudaSuccess) return bail(fail(h, L2C_E_CUDA, "no CUDA device"));
     if (cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->dev) != cudaSuccess)
@@ -655,7 +659,8 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
     ALLOC(h->gen_count, 4);
     ALLOC(h->idx_out, 4);
     ALLOC(h->key_scratch, 8);
-    ALLOC(h->attn_part, B * (size_t)h->Hkv * h->attn_nchunks * h->rep * (h->hs + 2) * sizeof(double));
+    ALLOC(h->attn_part, B * (size_t)h->Hkv * (h->attn_nchunks > h->attn_nchunks_f64 ? h->attn_nchunks : h->attn_nchunks_f64) *
+                            h->rep * (h->hs + 2) * sizeof(double));
     ALLOC(h->attn_cnt, B * (size_t)h->Hkv * 4);
 #undef ALLOC
     // zero state
@@ -849,10 +854,10 @@ extern "C" int l2c_attention(l2c_ctx* h, const float* q, const float* k, const f
     t.q = q; t.kc = k; t.vc = v; t.seq_stride = 0;
     t.out = out; t.tp = h->tp; t.tp_stride = 2;
     t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = h->kvd; t.seq_len = h->S;
-    t.nchunks = h->attn_nchunks;
+    t.nchunks = precision ? h->attn_nchunks_f64 : h->attn_nchunks;
     t.part = h->attn_part; t.count = h->attn_cnt; t.err = h->err;
     AttnKernel ak = precision ? attn_kernel_for<double>(h->hs, h->rep) : attn_kernel_for<float>(h->hs, h->rep);
-    CK(launch(h->stream, false, ak, dim3(h->attn_nchunks, h->Hkv, 1), dim3(128), 0, t));
+    CK(launch(h->stream, false, ak, dim3(t.nchunks, h->Hkv, 1), dim3(128), 0, t));
     return L2C_OK;
 }
 
