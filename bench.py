@@ -55,6 +55,40 @@ def bytes_per_token(q80: bool, pos: int, spec=None, gs=GS) -> float:
     return (1 + 4.0 / gs) * (mats + d) + 4.0 * (2 * L * d + d) + kv
 
 
+def kernel_bytes(kind: int, q80: bool, pos: int, spec=None, gs=GS) -> float:
+    """Algorithmic bytes of one launch of step kernel `kind` (the numbering of
+    l2c_time_kernel: 0 RMSNorm+QKV+RoPE, 1 attention, 2 wo, 3 RMSNorm+W1/W3+SwiGLU,
+    4 W2, 5 final RMSNorm+classifier): its weights once (Q8_0: codes plus fp32
+    group scales), plus the vectors it reads and writes; attention: K and V of
+    positions 0..pos, q and the output."""
+    spec = spec or SPEC
+    d, h, L, H, Hkv, V, S = spec.cfg
+    kvd = Hkv * (d // H)
+    bpw = (1 + 4.0 / gs) if q80 else 4.0
+    if kind == 0:
+        return (d + 2 * kvd) * d * bpw + 4.0 * (2 * d + d + 2 * kvd)
+    if kind == 1:
+        return 8.0 * (pos + 1) * kvd + 4.0 * 2 * d
+    if kind == 2:
+        return d * d * bpw + 4.0 * 3 * d
+    if kind == 3:
+        return 2 * h * d * bpw + 4.0 * (2 * d + h)
+    if kind == 4:
+        return d * h * bpw + 4.0 * (h + 2 * d)
+    return V * d * bpw + 4.0 * (2 * d + V)
+
+
+KERNEL_NAMES = ("rmsnorm_qkv_rope", "attention", "wo_residual", "rmsnorm_w13_swiglu", "w2_residual",
+                "final_norm_classifier")
+
+
+def pct(xs, q):
+    xs = sorted(xs)
+    i = (len(xs) - 1) * q
+    lo, hi = int(i), min(int(i) + 1, len(xs) - 1)
+    return xs[lo] + (xs[hi] - xs[lo]) * (i - lo)
+
+
 def w13_bytes(q80: bool, spec=None, gs=GS) -> float:
     """Algorithmic bytes of one W1/W3 launch: both weight matrices, the RMSNorm
     gain, the input x and the output hb."""
@@ -179,9 +213,10 @@ def one_step(dec):
 
 # ----------------------------------------------------------- CPU oracle ------
 
-def oracle_sample(q80_also=True, pos=512):
-    """Seconds per token of the CPU oracle on the 7B-shape model at `pos`:
-    one fp32 step and (optionally) one Q8_0 step.  Returns (tokens, seconds, setup_s)."""
+def oracle_sample(steps_per_variant=3, pos=512):
+    """The CPU oracle on the 7B-shape model at `pos`: `steps_per_variant` fp32
+    steps, then as many Q8_0 steps.  Returns (tokens, seconds, setup seconds,
+    seconds per fp32 step, seconds per Q8_0 step)."""
     import oracle
     t0 = time.perf_counter()
     blob = synth.blob(SPEC)
@@ -189,18 +224,16 @@ def oracle_sample(q80_also=True, pos=512):
     k, v = synth.kv_prefill(SPEC, seq=0, n_pos=pos)
     m.kv_load(k, v)
     del k, v
-    if q80_also:
-        m.enable_q80(GS)
+    m.enable_q80(GS)
     setup = time.perf_counter() - t0
-    t1 = time.perf_counter()
-    m.forward(TOKEN, pos, q80=False)
-    ntok = 1
-    if q80_also:
-        m.forward(TOKEN, pos, q80=True)
-        ntok += 1
-    dt = time.perf_counter() - t1
+    per = []
+    for q80 in (False, True):
+        t1 = time.perf_counter()
+        for _ in range(steps_per_variant):
+            m.forward(TOKEN, pos, q80=q80)
+        per.append((time.perf_counter() - t1) / steps_per_variant)
     m.close()
-    return ntok, dt, setup
+    return 2 * steps_per_variant, steps_per_variant * (per[0] + per[1]), setup, per[0], per[1]
 
 
 # ---------------------------------------------------------- ranks (N > 1) ----
@@ -317,37 +350,56 @@ def run_ours(args, rank, world, local_rank):
     tokens = 2 * len(POSITIONS) * args.steps * world
     value = whole_job_rate(2 * len(POSITIONS) * args.steps, world, ms / 1e3)
 
-    # ---- per (variant, position) breakdown
+    # ---- per (variant, position) breakdown: every replay timed on its own
     peak, peak_kind = measured_peak()
-    reps = max(3, args.steps)
+    reps = max(50, args.steps)
     variants = {}
     for q80 in (False, True):
         for p in POSITIONS:
-            for _ in range(2):
+            for _ in range(3):
                 dec.forward_ptr(TOKEN, p, q80)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
             torch.cuda.synchronize()
-            a.record(stream)
-            for _ in range(reps):
+            for a, b in evs:
+                a.record(stream)
                 dec.forward_ptr(TOKEN, p, q80)
-            b.record(stream)
+                b.record(stream)
             torch.cuda.synchronize()
-            t = a.elapsed_time(b) / reps
+            ts = [a.elapsed_time(b) for a, b in evs]
+            t = statistics.median(ts)
             by = bytes_per_token(q80, p)
             variants[f"{'q8_0' if q80 else 'fp32'}@pos{p}"] = {
-                "ms_per_token": t, "tokens_per_s": 1e3 / t, "bytes_per_token": by,
+                "ms_per_token_median": t, "ms_p10": pct(ts, 0.1), "ms_p90": pct(ts, 0.9), "replays": reps,
+                "tokens_per_s": 1e3 / t, "bytes_per_token": by,
                 "gbs": by / t / 1e6, "frac_of_measured_hbm": by / t / 1e6 / peak,
                 "frac_of_8tbs_roofline": by / t / 1e6 / NOMINAL_HBM_GBS,
                 "roofline_tokens_per_s_8tbs": NOMINAL_HBM_GBS * 1e9 / by,
             }
     dec.sync()
 
+    # ---- every kernel of the step, run alone back to back (l2c_time_kernel:
+    # 2 * n_layers launches on the handle's stream, launch i on layer i % n_layers,
+    # programmatic dependent launch between them as in the step graph)
+    kpos = POSITIONS[-1]
+    kernels = {}
+    for q80 in (False, True):
+        dec.forward_ptr(TOKEN, kpos, q80)  # the handle's state: position kpos
+        rows = {}
+        for kind, name in enumerate(KERNEL_NAMES):
+            iters = 2 * SPEC.n_layers if kind != 5 else 8
+            dec.time_kernel(kind, q80, max(4, iters // 4))  # warm
+            ms = dec.time_kernel(kind, q80, iters)
+            by = kernel_bytes(kind, q80, kpos)
+            rows[name] = {"avg_launch_us": 1e3 * ms, "bytes_per_launch": by, "gbs": by / ms / 1e6,
+                          "frac_of_measured_hbm": by / ms / 1e6 / peak, "launches_timed": iters}
+        kernels["q8_0" if q80 else "fp32"] = rows
+    kernels["note"] = (f"each kernel alone, back to back over the layers' weights, at pos {kpos} "
+                       f"(attention reads K/V of positions 0..{kpos})")
+
     # ---- dominant kernel: RMSNorm + W1/W3 + SwiGLU (44% of the fp32 step's bytes)
     def kernel_roofline(q80: bool):
-        dec.forward_ptr(TOKEN, 512, q80)
-        iters = 2 * SPEC.n_layers
-        dec.time_kernel(l2c.K_W13, q80, SPEC.n_layers)  # warm
-        avg_ms = dec.time_kernel(l2c.K_W13, q80, iters)
+        row = kernels["q8_0" if q80 else "fp32"]["rmsnorm_w13_swiglu"]
+        avg_ms = row["avg_launch_us"] / 1e3
         ach = w13_bytes(q80) / avg_ms / 1e6
         key = "k_gemv_q8<W13>" if q80 else "k_gemv_f32<W13>"
         return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
@@ -377,11 +429,12 @@ def run_ours(args, rank, world, local_rank):
     # ---- CPU oracle beside it (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ntok, dt, setup = oracle_sample()
+        ntok, dt, setup, s32, s8 = oracle_sample()
         cpu = {"value": ntok / dt, "unit": UNIT, "cores": host_cores(), "kind": "oracle",
-               "sample": f"one fp32 and one Q8_0 decode step of the 7B-shape model at pos 512 "
-                         f"({dt:.1f} s of compute; {setup:.0f} s to generate the weights, prefill the cache "
-                         f"and quantize, not counted)"}
+               "sample": f"3 fp32 and 3 Q8_0 decode steps of the 7B-shape model at pos 512 "
+                         f"({dt:.1f} s of compute: {s32:.2f} s per fp32 step, {s8:.2f} s per Q8_0 step; "
+                         f"{setup:.0f} s to generate the weights, prefill the cache and quantize, not counted)",
+               "s_per_step_fp32": s32, "s_per_step_q8_0": s8}
 
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -389,7 +442,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": "f32 | i8*i8->i32 with f64 group sums", "data": "synthetic",
         "config": workload_config(), "roofline": roof, "roofline_q8_0": roof_q8,
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_token * 2 * len(POSITIONS) * args.steps,
-        "clocks": clk.summary(), "variants": variants,
+        "clocks": clk.summary(), "variants": variants, "kernels": kernels,
         "context": "pages' CPU figures: ~110 tok/s 15M int8 on an M1 MacBook Air; ~0.8 tok/s 7B fp32 on a "
                    "16-core Ryzen 9 7950X; ~4 tok/s 7B on a 96-thread server",
     }
@@ -444,6 +497,24 @@ def run_extra(args):
                 buckets.append({"pos": [b0, b0 + n - 1], "us_per_token": us, "tokens_per_s": 1e6 / us,
                                 "bytes_per_token_mid": by, "gbs": by / us / 1e3})
             dec.sync()
+            # secondary datum: the same positions with L2 flushed before each
+            # timed step (a write of twice the L2 size outside the events)
+            flush = torch.empty(2 * l2 // 4, dtype=torch.float32, device="cuda")
+            flushed = []
+            for b0 in range(0, S, 64):
+                ts = []
+                for p in range(b0, min(S, b0 + 64), 8):
+                    flush.fill_(1.0)
+                    a, b = ev(), ev()
+                    a.record(stream)
+                    dec.forward_ptr(int(toks[p]), p, q80)
+                    b.record(stream)
+                    torch.cuda.synchronize()
+                    ts.append(1e3 * a.elapsed_time(b))
+                flushed.append({"pos": [b0, min(S, b0 + 64) - 1], "us_per_token_median": statistics.median(ts),
+                                "steps": len(ts)})
+            del flush
+            dec.sync()
             weights = bytes_per_token(q80, 0, spec, gs or GS)
             resident = weights < l2
             for bk in buckets:
@@ -454,7 +525,9 @@ def run_extra(args):
                 "inputs": "forced tokens uniform in [0, vocab) (stream 2), positions 0..seq_len-1 in order",
                 "timing": "CUDA events around 64 consecutive decode steps through the C ABI, host launch included",
                 "l2_resident": bool(resident), "l2_bytes": l2, "peak_gbs": peak, "peak_kind": peak_kind,
-                "buckets": buckets}), flush=True)
+                "buckets": buckets,
+                "l2_flushed": {"how": "2x L2 bytes written before each timed step; events around the step only",
+                               "buckets": flushed}}), flush=True)
         dec.close()
 
     if args.extra not in ("all", "batch"):

@@ -21,12 +21,12 @@ L2C_OK, L2C_E_ARG, L2C_E_OOM, L2C_E_CUDA, L2C_E_DEVICE, L2C_E_STATE, L2C_E_SCRAT
 EXPORTS = (
     "l2c_blob_floats", "l2c_create", "l2c_enable_q80", "l2c_forward", "l2c_forward_q80", "l2c_argmax",
     "l2c_generate", "l2c_forward_batch", "l2c_quantize_q80", "l2c_q80_group_dots", "l2c_kv_load",
-    "l2c_kv_read", "l2c_kv_reset", "l2c_attention", "l2c_attention_noalloc", "l2c_time_kernel", "l2c_persistent", "l2c_sync", "l2c_stream", "l2c_last_status", "l2c_last_error",
+    "l2c_kv_read", "l2c_kv_reset", "l2c_attention", "l2c_attention_noalloc", "l2c_time_kernel", "l2c_sync", "l2c_stream", "l2c_last_status", "l2c_last_error",
     "l2c_destroy",
 )
 
 # kernels of the step, as numbered by l2c_time_kernel
-K_QKV, K_ATTN, K_WO, K_W13, K_W2, K_CLS, K_STEP = range(7)
+K_QKV, K_ATTN, K_WO, K_W13, K_W2, K_CLS = range(6)
 
 
 class L2CError(RuntimeError):
@@ -68,7 +68,6 @@ def lib():
             "l2c_attention": (i32, [vp, vp, vp, vp, i32, i32, vp]),
             "l2c_attention_noalloc": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
             "l2c_time_kernel": (i32, [vp, i32, i32, i32, ctypes.POINTER(ctypes.c_float)]),
-            "l2c_persistent": (i32, [vp]),
             "l2c_sync": (i32, [vp]),
             "l2c_stream": (vp, [vp]),
             "l2c_last_status": (i32, [vp]),
@@ -197,13 +196,6 @@ class Decoder:
     def q80_group_dots(self, qw, qx, gs: int, out):
         rows, K = qw.shape
         self._check(lib().l2c_q80_group_dots(self._h, _ptr(qw), _ptr(qx), int(rows), int(K), int(gs), _ptr(out)))
-
-    def persistent(self) -> bool:
-        """True when the Q8_0 step runs as one persistent kernel (l2c_persistent)."""
-        rc = lib().l2c_persistent(self._h)
-        if rc < 0:
-            self._check(rc)
-        return rc == 1
 
     def time_kernel(self, kind: int, q80: bool, iters: int) -> float:
         """Average ms per launch of one kernel of the step run alone (l2c_time_kernel)."""

@@ -9,7 +9,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libl2c.so")
-SOURCES = [os.path.join(HERE, "csrc", n) for n in ("l2c.cu", "attention_noalloc.cu", "persistent.cu")]
+SOURCES = [os.path.join(HERE, "csrc", n) for n in ("l2c.cu", "attention_noalloc.cu")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -2,6 +2,35 @@
 //
 // Shared by the step kernels and by standalone entry points: it holds only
 // templates and inline functions, so any translation unit may include it.
+//
+// Work item (chunk c, KV head g, sequence b): the positions [t0, t1) of the
+// chunk, for the rep = H/Hkv query heads that share KV head g (heads
+// g*rep .. g*rep+rep-1: contiguous groups), so every K/V row is read once per
+// group.  One CTA of four warps per item.  Each warp takes batches of
+// positions in turn and runs an online softmax over them (scores from one
+// reduce-scatter per head, running max, rescaled weighted V sum) while the
+// next two batches stream into shared memory (cp.async, per lane); then the
+// warps merge their states.  Rows before the current position do not depend
+// on the kernel that precedes attention in the step, so a warp's first
+// batches are copied before the dependency wait when they do not contain the
+// current position's row.
+//
+// Each active chunk writes its (o, m, l) per head; the last CTA to arrive for
+// (b, g) (an atomic counter, no spin-wait) merges them:
+// M = max m_c, L = sum l_c e^{m_c - M}, O = sum o_c e^{m_c - M}; out = O / L.
+// A single active chunk writes O / L directly.
+//
+// Precision.  Acc = float accumulates in fp32 (the fp32 step).  Acc = double
+// accumulates in double (the Q8_0 step, whose attention output is quantized,
+// so it must round to the same fp32 values as a double reference): K and V
+// elements are widened to double with integer operations instead of the
+// conversion instruction, which issues on a narrow unit.  The widening keeps
+// the float's bits and leaves its exponent unbiased, i.e. it yields x * 2^-896
+// exactly, for every finite x including zeros and subnormals; scores and the
+// weighted V sums are scaled back by 2^896 (exact) once per position / once
+// at the end.  Products below 2^-126 in magnitude flush to zero there, far
+// below the last bit of any sum they join.  A non-finite K or V element makes
+// the output NaN.
 #pragma once
 #include "common.cuh"
 
@@ -19,248 +48,129 @@ struct AttnArgs {
     const int* tp;       // {token, pos} per sequence, stride tp_stride ints
     int tp_stride;
     int H, Hkv, hs, kvd, seq_len;
-    int nchunks;         // gridDim.x: the positions 0..pos are split into this many chunks
+    int nchunks;         // gridDim.x: the positions 0..pos are split into at most this many chunks
+    int min_chunk;       // ... of at least this many positions each
     void* part;          // partials [B][Hkv][nchunks][rep][hs+2] (Acc)
     int* count;          // [B][Hkv] arrival counters (zero between launches)
-    int* err;
 };
 
-// Shared memory of one attention work item (four warps).
+// x * 2^-896 as a double, exactly, for every finite float x (see above).
+__device__ __forceinline__ double widen_scaled(float x) {
+    const uint32_t b = __float_as_uint(x);
+    const uint32_t hi = ((b & 0x7fffffffu) >> 3) | (b & 0x80000000u);
+    return __hiloint2double((int)hi, (int)(b << 29));
+}
+constexpr double kTwo896 = 0x1p896;
+
+__device__ __forceinline__ bool nonfinite4(const float4 v) {
+    return ((__float_as_uint(v.x) & 0x7f800000u) == 0x7f800000u) |
+           ((__float_as_uint(v.y) & 0x7f800000u) == 0x7f800000u) |
+           ((__float_as_uint(v.z) & 0x7f800000u) == 0x7f800000u) |
+           ((__float_as_uint(v.w) & 0x7f800000u) == 0x7f800000u);
+}
+
+template <typename Acc>
+__device__ __forceinline__ void widen4(const float4 v, Acc (&w)[4]) {
+    if (sizeof(Acc) == 8) {
+        w[0] = (Acc)widen_scaled(v.x); w[1] = (Acc)widen_scaled(v.y);
+        w[2] = (Acc)widen_scaled(v.z); w[3] = (Acc)widen_scaled(v.w);
+    } else {
+        w[0] = (Acc)v.x; w[1] = (Acc)v.y; w[2] = (Acc)v.z; w[3] = (Acc)v.w;
+    }
+}
+
+constexpr int ATTN_WARPS = 4;
+constexpr int ATTN_THREADS = 32 * ATTN_WARPS;
+constexpr int ATTN_NB = 3;  // batches in each lane's shared-memory ring
+
+// Positions a warp loads at once (one batch): fewer in double or when the
+// query group is large, to bound the registers of the batch being computed.
+template <typename Acc, int REP>
+struct AttnPB {
+    static constexpr int value = sizeof(Acc) == 8 ? (REP >= 4 ? 2 : 4) : (REP >= 3 ? 4 : 8);
+};
+
+// Dynamic shared memory of an attention CTA: per warp ATTN_NB batches of PB
+// positions, K and V, one float4 per lane.
+template <typename Acc, int REP>
+constexpr int attn_ring_bytes() {
+    return ATTN_WARPS * ATTN_NB * AttnPB<Acc, REP>::value * 2 * 32 * 16;
+}
+
+// 16-byte global -> shared asynchronous copy (cp.async, L2 evict-first); with
+// on == false nothing is read and the destination is zero-filled.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool on, uint64_t pol) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;"
+                 :: "r"(smem_u32(dst)), "l"(src), "r"(on ? 16 : 0), "l"(pol) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
+
+// The merge of a work item's four warps and of the chunks of (b, g); every
+// thread of the CTA calls it after its warp's online softmax is done.
 template <typename Acc, int HS, int REP>
-struct AttnSmem {
-    static constexpr int TC = 64;  // positions per sub-chunk held in shared memory
-    Acc sc[TC][REP];
-    Acc red[4][REP];
-    Acc ostage[4][REP][HS];
-    int last;
-};
-
-// One work item: chunk c of sequence b for the rep = H/Hkv query heads that
-// share KV head g (heads g*rep .. g*rep+rep-1: contiguous groups), run by 128
-// threads (tid 0..127) that synchronise through `sy`.  The positions 0..pos
-// of sequence b are split into nchunks equal chunks (ceil((pos+1)/nchunks)
-// each), so every K/V row is read once per group.  Within an item, sub-chunks
-// of TC positions go through three passes: scores (one warp per position: the
-// row slice is one coalesced 16-byte-per-lane load, the dots of a batch of
-// positions one reduce-scatter), the sub-chunk max and exp(s - m), and the
-// weighted V sum (one warp per position again).  Each active item writes (m, l, o) per head: the
-// running max of the scaled scores, the sum of exp(s - m) and the unnormalised
-// weighted V sum.  The last item to arrive for (b, g) merges the partials and
-// writes the output.  With COH, q, K and V are read through L2 (ld.global.cg),
-// so an item may follow, in the same launch, the kernel phase that wrote them;
-// otherwise through the read-only path.
-template <typename Acc, int HS, int REP, typename SY, bool PRE = false, bool COH = false>
-__device__ __forceinline__ void attn_item(const AttnArgs& a, int c, int g, int b, int tid, const SY& sy,
-                                          AttnSmem<Acc, HS, REP>& sm) {
-    // q, K and V: read-only for this launch unless COH (then through L2, coherent
-    // with writes of other CTAs earlier in the same launch)
-    auto ld4 = [](const float4* p) { return COH ? __ldcg(p) : __ldg(p); };
-    static_assert(HS % 4 == 0 && HS <= 128, "head size");
-    constexpr int NT = 128, NW = 4;
-    constexpr int TC = AttnSmem<Acc, HS, REP>::TC;
-    constexpr int V4 = HS / 4;             // float4 per K/V row slice (<= 32: one per lane)
-    constexpr int PB = 8;                  // positions a warp loads before reducing
-    auto& sc = sm.sc;
-    auto& red = sm.red;
-    auto& ostage = sm.ostage;
-    const int lane = tid & 31, warp = tid >> 5;
-
-    int pos = a.tp[b * a.tp_stride + 1];
-    if (pos < 0 || pos >= a.seq_len) pos = 0;  // the GEMV kernel has flagged it
-    const int T = pos + 1;
-    const int chunk = (T + a.nchunks - 1) / a.nchunks;
-    const int nact = (T + chunk - 1) / chunk;  // active chunks for this sequence
-    if (c >= nact) return;
-    const int t0 = c * chunk, t1 = min(T, t0 + chunk);
-    const float* kc = a.kc + (size_t)b * a.seq_stride + (size_t)g * HS;
-    const float* vc = a.vc + (size_t)b * a.seq_stride + (size_t)g * HS;
-    const float* q = a.q + (size_t)b * a.H * HS + (size_t)g * REP * HS;
-    const bool lane_on = lane < V4;
-    // this lane's four q values of every head, converted once
-    Acc qr[REP][4];
+__device__ __forceinline__ void attn_finish(const AttnArgs& a, int c, int g, int b, int nact, const Acc (&m)[REP],
+                                            const Acc (&l)[REP], const Acc (&o)[REP][4], Acc (*sm_m)[REP],
+                                            Acc (*sm_l)[REP], Acc (*sm_o)[REP][HS], int* last_s) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool lane_on = lane < HS / 4;
+    // merge the four warps' states (a warp without positions has m = -inf, l = 0)
+    if (lane == 0) {
 #pragma unroll
-    for (int h = 0; h < REP; h++) {
-        float4 qv = lane_on ? ld4(reinterpret_cast<const float4*>(q + (size_t)h * HS + 4 * lane))
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
-        qr[h][0] = (Acc)qv.x; qr[h][1] = (Acc)qv.y; qr[h][2] = (Acc)qv.z; qr[h][3] = (Acc)qv.w;
+        for (int h = 0; h < REP; h++) {
+            sm_m[warp][h] = m[h];
+            sm_l[warp][h] = l[h];
+        }
     }
-    const Acc scale = (Acc)1 / sqrt((Acc)HS);
-
-    Acc m[REP], l[REP], o[REP][4];
-#pragma unroll
-    for (int h = 0; h < REP; h++) {
-        m[h] = -INFINITY;
-        l[h] = 0;
-        o[h][0] = o[h][1] = o[h][2] = o[h][3] = 0;
-    }
-
-    // Sub-chunks of TC positions: warp w takes the NB batches of PB positions
-    // starting at w*PB + j*NW*PB.
-    constexpr int NB = TC / (NW * PB);
-    // PRE = true requests a sub-chunk's rows at once; it costs registers, and at
-    // 168 a thread only 3 CTAs fit an SM, so the 16-chunk grid needs two waves:
-    // measured slower, hence one batch at a time by default
-    constexpr bool VPRE = PRE && sizeof(Acc) == 4 && REP <= 2;
-    constexpr bool KPRE = PRE && (sizeof(Acc) == 4 || REP <= 2);
-    const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int tb = t0; tb < t1; tb += TC) {
-        const int n = min(TC, t1 - tb);
-        float4 kv[KPRE ? NB : 1][PB];
-        float4 vv[VPRE ? NB : 1][PB];
-        auto load_k = [&](int j, float4 (&dst)[PB]) {
-            const int tq = warp * PB + j * NW * PB;
-#pragma unroll
-            for (int i = 0; i < PB; i++) {
-                const bool on = lane_on && tq + i < n;
-                dst[i] = on ? ld4(reinterpret_cast<const float4*>(kc + (size_t)(tb + tq + i) * a.kvd) + lane)
-                            : zero4;
-            }
-        };
-#pragma unroll
-        for (int j = 0; j < NB; j++) {
-            const int tq = warp * PB + j * NW * PB;
-            if (KPRE) load_k(j, kv[KPRE ? j : 0]);
-#pragma unroll
-            for (int i = 0; i < PB; i++) {
-                const bool on = lane_on && tq + i < n;
-                if (VPRE)
-                    vv[VPRE ? j : 0][i] =
-                        on ? ld4(reinterpret_cast<const float4*>(vc + (size_t)(tb + tq + i) * a.kvd) + lane) : zero4;
-            }
-        }
-        // scores: the PB sums of each head in one reduce-scatter (lane 4i ends
-        // with position tq + i's total)
-#pragma unroll
-        for (int j = 0; j < NB; j++) {
-            const int tq = warp * PB + j * NW * PB;
-            if (tq < n) {  // warp-uniform
-                if (!KPRE) load_k(j, kv[0]);
-                const float4 (&kj)[PB] = kv[KPRE ? j : 0];
-#pragma unroll
-                for (int h = 0; h < REP; h++) {
-                    Acc sp[PB];
-#pragma unroll
-                    for (int i = 0; i < PB; i++)
-                        sp[i] = (Acc)kj[i].x * qr[h][0] + (Acc)kj[i].y * qr[h][1] +
-                                (Acc)kj[i].z * qr[h][2] + (Acc)kj[i].w * qr[h][3];
-                    const Acc s = warp_sum_scatter<PB>(sp);
-                    const int i = lane >> 2;
-                    if ((lane & 3) == 0 && tq + i < n) sc[tq + i][h] = s * scale;
-                }
-            }
-        }
-        sy.sync();
-        // max over the sub-chunk, new running max, weights p = exp(s - m_new)
-        Acc mnew[REP], alpha[REP];
-#pragma unroll
-        for (int h = 0; h < REP; h++) {
-            Acc mx = -INFINITY;
-            for (int t = tid; t < n; t += NT) mx = max(mx, sc[t][h]);
-            mx = warp_max(mx);
-            if (lane == 0) red[warp][h] = mx;
-        }
-        sy.sync();
-#pragma unroll
-        for (int h = 0; h < REP; h++) {
-            Acc mx = max(max(red[0][h], red[1][h]), max(red[2][h], red[3][h]));
-            mnew[h] = max(m[h], mx);
-            alpha[h] = exp(m[h] - mnew[h]);  // exp(-inf) = 0 on the first sub-chunk
-        }
-        sy.sync();
-#pragma unroll
-        for (int h = 0; h < REP; h++) {
-            Acc ps = 0;
-            for (int t = tid; t < n; t += NT) {
-                Acc p = exp(sc[t][h] - mnew[h]);
-                sc[t][h] = p;
-                ps += p;
-            }
-            ps = warp_sum(ps);
-            if (lane == 0) red[warp][h] = ps;
-        }
-        sy.sync();
-#pragma unroll
-        for (int h = 0; h < REP; h++) {
-            l[h] = l[h] * alpha[h] + (red[0][h] + red[1][h]) + (red[2][h] + red[3][h]);
-            m[h] = mnew[h];
-            o[h][0] *= alpha[h]; o[h][1] *= alpha[h]; o[h][2] *= alpha[h]; o[h][3] *= alpha[h];
-        }
-        // weighted V sum: warp per position, lane owns one float4 slice of the row
-#pragma unroll
-        for (int j = 0; j < NB; j++) {
-            const int tq = warp * PB + j * NW * PB;
-            if (tq < n) {  // warp-uniform
-                float4 vl[PB];
-#pragma unroll
-                for (int i = 0; i < PB; i++) {
-                    if (VPRE) {
-                        vl[i] = vv[VPRE ? j : 0][i];
-                    } else {
-                        const bool on = lane_on && tq + i < n;
-                        vl[i] = on ? ld4(reinterpret_cast<const float4*>(vc + (size_t)(tb + tq + i) * a.kvd) + lane)
-                                   : zero4;
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < PB; i++) {
-                    if (tq + i < n) {
-#pragma unroll
-                        for (int h = 0; h < REP; h++) {
-                            const Acc w = sc[tq + i][h];
-                            o[h][0] += w * (Acc)vl[i].x; o[h][1] += w * (Acc)vl[i].y;
-                            o[h][2] += w * (Acc)vl[i].z; o[h][3] += w * (Acc)vl[i].w;
-                        }
-                    }
-                }
-            }
-        }
-        sy.sync();
-    }
-    // combine the four warps' weighted sums (same running max)
     if (lane_on) {
 #pragma unroll
-        for (int h = 0; h < REP; h++) {
-            ostage[warp][h][4 * lane] = o[h][0]; ostage[warp][h][4 * lane + 1] = o[h][1];
-            ostage[warp][h][4 * lane + 2] = o[h][2]; ostage[warp][h][4 * lane + 3] = o[h][3];
-        }
+        for (int h = 0; h < REP; h++)
+#pragma unroll
+            for (int e = 0; e < 4; e++) sm_o[warp][h][4 * lane + e] = o[h][e];
     }
-    sy.sync();
-    if (nact == 1) {  // the whole range in one item: O / L directly (the merge would scale by e^0 = 1)
-        for (int i = tid; i < REP * HS; i += NT) {
-            const int h = i / HS, e = i % HS;
-            const Acc o_sum = (ostage[0][h][e] + ostage[1][h][e]) + (ostage[2][h][e] + ostage[3][h][e]);
-            a.out[(size_t)b * a.H * HS + ((size_t)g * REP + h) * HS + e] = (float)(o_sum / l[h]);
-        }
-        return;
-    }
-    Acc* part = static_cast<Acc*>(a.part) +
-                ((((size_t)b * a.Hkv + g) * a.nchunks + c) * REP) * (HS + 2);
-    for (int i = tid; i < REP * HS; i += NT) {
+    __syncthreads();
+    Acc* part = static_cast<Acc*>(a.part) + ((((size_t)b * a.Hkv + g) * a.nchunks + c) * REP) * (HS + 2);
+    for (int i = tid; i < REP * HS; i += ATTN_THREADS) {
         const int h = i / HS, e = i % HS;
-        part[(size_t)h * (HS + 2) + e] = (ostage[0][h][e] + ostage[1][h][e]) + (ostage[2][h][e] + ostage[3][h][e]);
+        Acc M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < ATTN_WARPS; w++) M = max(M, sm_m[w][h]);
+        Acc L = 0, O = 0;
+#pragma unroll
+        for (int w = 0; w < ATTN_WARPS; w++) {
+            const Acc f = sm_m[w][h] == -INFINITY ? (Acc)0 : exp(sm_m[w][h] - M);
+            L += sm_l[w][h] * f;
+            O += sm_o[w][h][e] * f;
+        }
+        if (nact == 1) {
+            a.out[(size_t)b * a.H * HS + ((size_t)g * REP + h) * HS + e] = (float)(O / L);
+        } else {
+            part[(size_t)h * (HS + 2) + e] = O;
+            if (e == 0) {
+                part[(size_t)h * (HS + 2) + HS] = M;
+                part[(size_t)h * (HS + 2) + HS + 1] = L;
+            }
+        }
     }
-    if (tid < REP) {
-        part[(size_t)tid * (HS + 2) + HS] = m[tid];
-        part[(size_t)tid * (HS + 2) + HS + 1] = l[tid];
-    }
+    if (nact == 1) return;
+    // the last CTA of (b, g) to arrive merges the chunks
     __threadfence();
-    sy.sync();
+    __syncthreads();
     int* cnt = a.count + (size_t)b * a.Hkv + g;
-    if (tid == 0) sm.last = (atomicAdd(cnt, 1) == nact - 1);
-    sy.sync();
-    if (!sm.last) return;
+    if (tid == 0) *last_s = (atomicAdd(cnt, 1) == nact - 1);
+    __syncthreads();
+    if (!*last_s) return;
     __threadfence();
-    // merge the nact partials of (b, g): M = max m_c, L = sum l_c e^{m_c - M},
-    // O = sum o_c e^{m_c - M}; output O / L.
     const Acc* p0 = static_cast<const Acc*>(a.part) + (((size_t)b * a.Hkv + g) * a.nchunks * REP) * (HS + 2);
-    for (int i = tid; i < REP * HS; i += NT) {
+    for (int i = tid; i < REP * HS; i += ATTN_THREADS) {
         const int h = i / HS, e = i % HS;
         Acc M = -INFINITY;
         for (int k = 0; k < nact; k++) M = max(M, __ldcg(p0 + ((size_t)k * REP + h) * (HS + 2) + HS));
         Acc Ls = 0, Os = 0;
         for (int k = 0; k < nact; k++) {
             const Acc* pk = p0 + ((size_t)k * REP + h) * (HS + 2);
-            Acc f = exp(__ldcg(pk + HS) - M);
+            const Acc f = exp(__ldcg(pk + HS) - M);
             Ls += __ldcg(pk + HS + 1) * f;
             Os += __ldcg(pk + e) * f;
         }
@@ -269,31 +179,295 @@ __device__ __forceinline__ void attn_item(const AttnArgs& a, int c, int g, int b
     if (tid == 0) *cnt = 0;
 }
 
-// grid (nchunks, Hkv, B), 128 threads: CTA (c, g, b) runs work item (c, g, b).
-template <typename Acc, int HS, int REP>
-__global__ void __launch_bounds__(128) k_attention(const AttnArgs a) {
-    __shared__ AttnSmem<Acc, HS, REP> sm;
+// The online-softmax update of one warp with a batch of PB positions (n of
+// them valid): K and V row slices of this lane (one float4 each).
+template <typename Acc, int REP, int PB, typename KV>
+__device__ __forceinline__ void attn_batch(int n, KV kv, const Acc (&qr)[REP][4], Acc scale, Acc (&m)[REP],
+                                           Acc (&l)[REP], Acc (&o)[REP][4]) {
+    float4 kr[PB];
+#pragma unroll
+    for (int i = 0; i < PB; i++) kr[i] = kv(i, 0);
+#pragma unroll
+    for (int h = 0; h < REP; h++) {
+        Acc sp[PB];
+#pragma unroll
+        for (int i = 0; i < PB; i++) {
+            Acc kw[4];
+            widen4<Acc>(kr[i], kw);
+            sp[i] = kw[0] * qr[h][0] + kw[1] * qr[h][1] + kw[2] * qr[h][2] + kw[3] * qr[h][3];
+        }
+        const Acc tot = warp_sum_scatter<PB>(sp);  // lane l: position (l / (32/PB)) % PB
+        Acc sc[PB];
+        Acc mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < PB; i++) {
+            const Acc si = __shfl_sync(0xffffffffu, tot, i * (32 / PB));
+            sc[i] = i < n ? si * scale : (Acc)-INFINITY;
+            mx = max(mx, sc[i]);
+        }
+        const Acc mnew = max(m[h], mx);
+        const Acc alpha = exp(m[h] - mnew);  // exp(-inf) = 0 on the warp's first batch
+        Acc ps = 0, w4[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int i = 0; i < PB; i++) {
+            const Acc p = exp(sc[i] - mnew);  // masked positions: exp(-inf) = 0
+            Acc vw[4];
+            widen4<Acc>(kv(i, 1), vw);
+            ps += p;
+            w4[0] += p * vw[0]; w4[1] += p * vw[1]; w4[2] += p * vw[2]; w4[3] += p * vw[3];
+        }
+        l[h] = l[h] * alpha + ps;
+        o[h][0] = o[h][0] * alpha + w4[0]; o[h][1] = o[h][1] * alpha + w4[1];
+        o[h][2] = o[h][2] * alpha + w4[2]; o[h][3] = o[h][3] * alpha + w4[3];
+        m[h] = mnew;
+    }
+}
+
+// The work item of CTA (c, g, b): its chunk [t0, t1) and the number of
+// active chunks of sequence b; false when this CTA has no positions.
+__device__ __forceinline__ bool attn_item(const AttnArgs& a, int c, int b, int& t0, int& t1, int& nact, int& pos) {
+    pos = a.tp[b * a.tp_stride + 1];  // written before the step: readable before the wait
+    if (pos < 0 || pos >= a.seq_len) pos = 0;  // the q/k/v kernel has flagged it
+    const int T = pos + 1;
+    nact = (T + a.min_chunk - 1) / a.min_chunk;
+    if (nact > a.nchunks) nact = a.nchunks;
+    const int chunk = (T + nact - 1) / nact;
+    nact = (T + chunk - 1) / chunk;
+    if (c >= nact) return false;
+    t0 = c * chunk;
+    t1 = min(T, t0 + chunk);
+    return true;
+}
+
+template <int REP>
+struct AttnPBF {  // fp32 kernel: positions per batch
+    static constexpr int value = REP >= 3 ? 4 : 8;
+};
+
+// fp32 attention, grid (nchunks, Hkv, B), ATTN_THREADS threads, no dynamic
+// shared memory (the fp32 step's kernels keep the default L1 / shared split).
+// The chunk's positions go in batches of PB to the four warps in turn; a lane
+// holds one float4 of each K and V row slice (hs <= 128) in registers, and
+// every warp keeps the next batch's 128-bit loads in flight while it computes
+// the current one.
+template <int HS, int REP>
+__global__ void __launch_bounds__(ATTN_THREADS) k_attention_f32(const AttnArgs a) {
+    constexpr int V4 = HS / 4;
+    constexpr int PB = AttnPBF<REP>::value;
+    static_assert(HS % 4 == 0 && HS <= 128, "head size");
+    __shared__ float sm_m[ATTN_WARPS][REP], sm_l[ATTN_WARPS][REP];
+    __shared__ float sm_o[ATTN_WARPS][REP][HS];
+    __shared__ int last_s;
+    const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const bool lane_on = lane < V4;
+    int t0, t1, nact, pos;
+    if (!attn_item(a, c, b, t0, t1, nact, pos)) return;
+    const int nb = (t1 - t0 + PB - 1) / PB;
+    const float* kc = a.kc + (size_t)b * a.seq_stride + (size_t)g * HS + 4 * lane;
+    const float* vc = a.vc + (size_t)b * a.seq_stride + (size_t)g * HS + 4 * lane;
+    const uint64_t pol = policy_evict_first();
+    auto load = [&](int bi, float4 (&kr)[PB], float4 (&vr)[PB]) {
+#pragma unroll
+        for (int i = 0; i < PB; i++) {
+            const int t = t0 + bi * PB + i;
+            const bool on = lane_on && t < t1;
+            kr[i] = on ? ld_stream_f4(reinterpret_cast<const float4*>(kc + (size_t)t * a.kvd), pol)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+            vr[i] = on ? ld_stream_f4(reinterpret_cast<const float4*>(vc + (size_t)t * a.kvd), pol)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    };
+    float4 ka[PB], va[PB], kb[PB], vb[PB];
+    int bi = warp;
+    // the warp's first batch, if all its rows precede the current position,
+    // is read before the wait (only row pos comes from the kernel before)
+    const bool early = bi < nb && t0 + (bi + 1) * PB <= pos;
+    if (early) load(bi, ka, va);
     grid_dep_wait();
     grid_dep_launch();
-    attn_item<Acc, HS, REP>(a, blockIdx.x, blockIdx.y, blockIdx.z, threadIdx.x, SyncCTA(), sm);
+    if (!early && bi < nb) load(bi, ka, va);
+    const float* q = a.q + (size_t)b * a.H * HS + (size_t)g * REP * HS;
+    float qr[REP][4];
+#pragma unroll
+    for (int h = 0; h < REP; h++) {
+        const float4 qv = lane_on ? __ldg(reinterpret_cast<const float4*>(q + (size_t)h * HS) + lane)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        qr[h][0] = qv.x; qr[h][1] = qv.y; qr[h][2] = qv.z; qr[h][3] = qv.w;
+    }
+    const float scale = 1.0f / sqrtf((float)HS);
+    float m[REP], l[REP], o[REP][4];
+#pragma unroll
+    for (int h = 0; h < REP; h++) {
+        m[h] = -INFINITY;
+        l[h] = 0.f;
+        o[h][0] = o[h][1] = o[h][2] = o[h][3] = 0.f;
+    }
+    // two register buffers: batch bi in (ka, va), the next one loading into (kb, vb)
+    while (bi < nb) {
+        if (bi + ATTN_WARPS < nb) load(bi + ATTN_WARPS, kb, vb);
+        attn_batch<float, REP, PB>(min(PB, t1 - (t0 + bi * PB)),
+                                   [&](int i, int kv) { return kv ? va[i] : ka[i]; }, qr, scale, m, l, o);
+        bi += ATTN_WARPS;
+        if (bi >= nb) break;
+        if (bi + ATTN_WARPS < nb) load(bi + ATTN_WARPS, ka, va);
+        attn_batch<float, REP, PB>(min(PB, t1 - (t0 + bi * PB)),
+                                   [&](int i, int kv) { return kv ? vb[i] : kb[i]; }, qr, scale, m, l, o);
+        bi += ATTN_WARPS;
+    }
+    attn_finish<float, HS, REP>(a, c, g, b, nact, m, l, o, sm_m, sm_l, sm_o, &last_s);
+}
+
+// grid (nchunks, Hkv, B), ATTN_THREADS threads, attn_ring_bytes<Acc, REP>()
+// bytes of dynamic shared memory: CTA (c, g, b) runs work item (c, g, b).
+// The chunk's positions go in batches of PB to the four warps in turn; a lane
+// owns one float4 of each K and V row slice (hs <= 128) and streams it into
+// its own ring of ATTN_NB batches in shared memory with cp.async, so two
+// batches are in flight while it computes a third, without holding them in
+// registers (each lane reads back only what it copied: no synchronisation).
+template <typename Acc, int HS, int REP>
+__global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
+    constexpr bool DBL = sizeof(Acc) == 8;
+    constexpr int V4 = HS / 4;  // float4 per row slice (<= 32: one per lane)
+    constexpr int PB = AttnPB<Acc, REP>::value;
+    static_assert(HS % 4 == 0 && HS <= 128, "head size");
+    extern __shared__ __align__(16) float4 aring[];
+    __shared__ Acc sm_m[ATTN_WARPS][REP], sm_l[ATTN_WARPS][REP];
+    __shared__ Acc sm_o[ATTN_WARPS][REP][HS];
+    __shared__ int last_s;
+    const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const bool lane_on = lane < V4;
+    int t0, t1, nact, pos;
+    if (!attn_item(a, c, b, t0, t1, nact, pos)) return;
+    const int nb = (t1 - t0 + PB - 1) / PB;   // batches of the chunk; warp w takes w, w+4, ...
+    const float* kc = a.kc + (size_t)b * a.seq_stride + (size_t)g * HS + 4 * (lane_on ? lane : 0);
+    const float* vc = a.vc + (size_t)b * a.seq_stride + (size_t)g * HS + 4 * (lane_on ? lane : 0);
+    const uint64_t pol = policy_evict_first();
+    float4* ring = aring + (size_t)warp * ATTN_NB * PB * 2 * 32;
+    // ring entry of (slot, position i, K or V) for this lane
+    auto ent = [&](int slot, int i, int kv) -> float4* { return ring + ((slot * PB + i) * 2 + kv) * 32 + lane; };
+    // copies of the warp's jj-th batch into slot jj % ATTN_NB; always one commit group
+    auto issue = [&](int jj) {
+        const int bi = warp + ATTN_WARPS * jj;
+        const int slot = jj % ATTN_NB;
+#pragma unroll
+        for (int i = 0; i < PB; i++) {
+            const int t = t0 + bi * PB + i;
+            const bool on = lane_on && bi < nb && t < t1;
+            const size_t off = on ? (size_t)t * a.kvd : 0;
+            cp_async16(ent(slot, i, 0), kc + off, on, pol);
+            cp_async16(ent(slot, i, 1), vc + off, on, pol);
+        }
+        cp_async_commit();
+    };
+    // a batch whose rows all precede the current position (only row pos comes
+    // from the kernel before) may be copied before the dependency wait
+    auto before_wait_ok = [&](int jj) { return t0 + (warp + ATTN_WARPS * jj + 1) * PB <= pos; };
+    int nissued = 0;
+    while (nissued < ATTN_NB - 1 && before_wait_ok(nissued)) issue(nissued++);
+    grid_dep_wait();
+    grid_dep_launch();
+    while (nissued < ATTN_NB - 1) issue(nissued++);
+
+    const float* q = a.q + (size_t)b * a.H * HS + (size_t)g * REP * HS;
+    Acc qr[REP][4];
+#pragma unroll
+    for (int h = 0; h < REP; h++) {
+        const float4 qv = lane_on ? __ldg(reinterpret_cast<const float4*>(q + (size_t)h * HS) + lane)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        qr[h][0] = (Acc)qv.x; qr[h][1] = (Acc)qv.y; qr[h][2] = (Acc)qv.z; qr[h][3] = (Acc)qv.w;
+    }
+    // score scale (the 2^896 of the widened K elements folded in)
+    const Acc scale = DBL ? (Acc)(kTwo896 / sqrt((double)HS)) : (Acc)1 / sqrt((Acc)HS);
+    Acc m[REP], l[REP], o[REP][4];
+#pragma unroll
+    for (int h = 0; h < REP; h++) {
+        m[h] = -INFINITY;
+        l[h] = 0;
+        o[h][0] = o[h][1] = o[h][2] = o[h][3] = 0;
+    }
+    bool bad = false;  // a non-finite K/V element (double path)
+    for (int jj = 0;; jj++) {
+        const int bi = warp + ATTN_WARPS * jj;
+        if (bi >= nb) break;
+        cp_async_wait<ATTN_NB - 2>();  // batch jj has landed (this lane's copies)
+        issue(jj + ATTN_NB - 1);       // into the slot read in the previous round
+        const int slot = jj % ATTN_NB;
+        if (DBL) {
+#pragma unroll
+            for (int i = 0; i < PB; i++) bad |= nonfinite4(*ent(slot, i, 0)) | nonfinite4(*ent(slot, i, 1));
+        }
+        attn_batch<Acc, REP, PB>(min(PB, t1 - (t0 + bi * PB)), [&](int i, int kv) { return *ent(slot, i, kv); }, qr,
+                                 scale, m, l, o);
+    }
+    cp_async_wait<0>();  // no copy of this lane may land after the CTA leaves
+    if (DBL) {
+#pragma unroll
+        for (int h = 0; h < REP; h++) {
+            o[h][0] *= (Acc)kTwo896; o[h][1] *= (Acc)kTwo896; o[h][2] *= (Acc)kTwo896; o[h][3] *= (Acc)kTwo896;
+        }
+        if (__any_sync(0xffffffffu, bad))
+#pragma unroll
+            for (int h = 0; h < REP; h++) o[h][0] = o[h][1] = o[h][2] = o[h][3] = (Acc)NAN;
+    }
+    attn_finish<Acc, HS, REP>(a, c, g, b, nact, m, l, o, sm_m, sm_l, sm_o, &last_s);
 }
 
 typedef void (*AttnKernel)(const AttnArgs);
 
-// The attention instantiation for a head size and GQA ratio (nullptr if none).
+// The attention instantiation for a head size and GQA ratio (nullptr if none):
+// k_attention_f32 for Acc = float, k_attention<double> for Acc = double.
+#define L2C_ATTN_SHAPES(X)                                                                  \
+    X(8, 1) X(8, 2) X(8, 3) X(8, 4) X(16, 1) X(16, 2) X(16, 4) X(32, 1) X(32, 2) X(32, 4) \
+    X(48, 1) X(48, 2) X(48, 4) X(64, 1) X(64, 2) X(64, 4) X(64, 8) X(96, 1) X(96, 2)      \
+    X(96, 4) X(128, 1) X(128, 2) X(128, 4) X(128, 8)
+
 template <typename Acc>
 inline AttnKernel attn_kernel_for(int hs, int rep) {
-#define L2C_ATTN(HS_, REP_) \
-    if (hs == HS_ && rep == REP_) return k_attention<Acc, HS_, REP_>;
-    L2C_ATTN(8, 1) L2C_ATTN(8, 2) L2C_ATTN(8, 3) L2C_ATTN(8, 4)
-    L2C_ATTN(16, 1) L2C_ATTN(16, 2) L2C_ATTN(16, 4)
-    L2C_ATTN(32, 1) L2C_ATTN(32, 2) L2C_ATTN(32, 4)
-    L2C_ATTN(48, 1) L2C_ATTN(48, 2) L2C_ATTN(48, 4)
-    L2C_ATTN(64, 1) L2C_ATTN(64, 2) L2C_ATTN(64, 4) L2C_ATTN(64, 8)
-    L2C_ATTN(96, 1) L2C_ATTN(96, 2) L2C_ATTN(96, 4)
-    L2C_ATTN(128, 1) L2C_ATTN(128, 2) L2C_ATTN(128, 4) L2C_ATTN(128, 8)
-#undef L2C_ATTN
+#define L2C_ATTN_F(HS_, REP_) \
+    if (hs == HS_ && rep == REP_) return k_attention_f32<HS_, REP_>;
+#define L2C_ATTN_D(HS_, REP_) \
+    if (hs == HS_ && rep == REP_) return k_attention<double, HS_, REP_>;
+    if (sizeof(Acc) == 4) {
+        L2C_ATTN_SHAPES(L2C_ATTN_F)
+    } else {
+        L2C_ATTN_SHAPES(L2C_ATTN_D)
+    }
+#undef L2C_ATTN_F
+#undef L2C_ATTN_D
     return nullptr;
+}
+
+// Dynamic shared memory of the attention instantiation for a GQA ratio (the
+// fp32 kernel has none).
+template <typename Acc>
+inline int attn_smem_for(int rep) {
+    if (sizeof(Acc) == 4) return 0;
+    switch (rep) {
+    case 1: return attn_ring_bytes<double, 1>();
+    case 2: return attn_ring_bytes<double, 2>();
+    case 3: return attn_ring_bytes<double, 3>();
+    case 4: return attn_ring_bytes<double, 4>();
+    default: return attn_ring_bytes<double, 8>();
+    }
+}
+
+// The double attention kernels: their ring's shared-memory limit (above the
+// default 48 KB for some), and all of the shared memory as carveout, as the
+// Q8_0 kernels they run between ask for.
+inline cudaError_t attn_set_smem_limits() {
+    cudaError_t e = cudaSuccess;
+#define L2C_ATTN_ATTR(HS_, REP_)                                                                                  \
+    if ((e = cudaFuncSetAttribute(k_attention<double, HS_, REP_>, cudaFuncAttributeMaxDynamicSharedMemorySize,    \
+                                  attn_ring_bytes<double, REP_>())) != cudaSuccess)                               \
+        return e;                                                                                                 \
+    if ((e = cudaFuncSetAttribute(k_attention<double, HS_, REP_>, cudaFuncAttributePreferredSharedMemoryCarveout, \
+                                  (int)cudaSharedmemCarveoutMaxShared)) != cudaSuccess)                           \
+        return e;
+    L2C_ATTN_SHAPES(L2C_ATTN_ATTR)
+#undef L2C_ATTN_ATTR
+    return e;
 }
 
 }  // namespace l2c

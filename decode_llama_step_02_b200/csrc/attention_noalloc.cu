@@ -6,11 +6,11 @@
 // or break the owner's accounting), or they run on a latency-critical path
 // where cudaMalloc and cudaFree may synchronize the device.  Such callers also
 // cannot create an l2c handle, which owns weights, caches and scratch.  For
-// them, l2c_attention_noalloc runs the same attention kernel as
-// l2c_attention on buffers the caller owns.  The kernel's scratch (partial
-// softmax state per KV head and position chunk, arrival counters and the
-// position word) lives in a file-scope __device__ array of fixed size instead
-// of a handle's allocation.
+// them, l2c_attention_noalloc runs the attention kernel of l2c_attention on
+// buffers the caller owns.  The kernel's scratch (partial softmax state per
+// KV head and position chunk, arrival counters and the position word) lives
+// in a file-scope __device__ array of fixed size instead of a handle's
+// allocation.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -23,32 +23,69 @@ using namespace l2c;
 namespace {
 
 // The fixed scratch: 4 MiB, held by every GPU that loads the library until
-// the process exits.  Layout: [0, 256) position word and error word,
-// [256, 256 + 4*n_kv_heads) arrival counters (rounded up to 256 B), then the
-// partial (m, l, o) records of every (KV head, chunk, query head).
+// the process exits.  Layout: [0, 256) the position word, [256, 256 +
+// 4*n_kv_heads) arrival counters (rounded up to 256 B), then the partial
+// (o, m, l) records of every (KV head, chunk, query head).
 constexpr size_t kScratchBytes = size_t(4) << 20;
-constexpr int kChunk = 64;      // positions per CTA, as in the decode step
+constexpr int kChunk = 64;      // positions per chunk (the handle picks its own split)
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_attn_scratch[kScratchBytes];
 
-std::mutex g_setup_mutex;
-void* g_scratch_addr[kMaxDevices] = {nullptr};
+// cuCtxGetCurrent / cuCtxGetId, reached through the runtime's driver entry
+// points (the library links no driver library).
+typedef int (*CtxGetCurrentFn)(void** ctx);
+typedef int (*CtxGetIdFn)(void* ctx, unsigned long long* id);
 
-// The device address of g_attn_scratch on the current device.  In host code
-// the array's name is only a host-side stand-in, so the address is queried
-// once per device with that device current.
+struct Slot {
+    void* addr = nullptr;
+    unsigned long long ctx_id = 0;
+};
+
+std::mutex g_setup_mutex;
+Slot g_slot[kMaxDevices];
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
+
+int current_context_id(unsigned long long* id) {
+    if (!g_ctx_current || !g_ctx_id) {
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess || !f1 || !f2)
+            return L2C_E_CUDA;
+        g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+        g_ctx_id = reinterpret_cast<CtxGetIdFn>(f2);
+    }
+    void* ctx = nullptr;
+    if (g_ctx_current(&ctx) != 0 || !ctx || g_ctx_id(ctx, id) != 0) return L2C_E_CUDA;
+    return L2C_OK;
+}
+
+// The device address of g_attn_scratch in the current context.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// (cudaGetSymbolAddress) with the device current, once per device and
+// context: a context ID is never reused, so after a device reset (which
+// loads the module again, at a new address) the lookup runs again.  The
+// attention kernels' shared-memory limit is set at the same time.
 int scratch_on_current_device(unsigned char** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return L2C_E_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return L2C_E_ARG;
+    if (dev < 0 || dev >= kMaxDevices) return L2C_E_CUDA;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_addr[dev]) {
+    unsigned long long id = 0;
+    if (current_context_id(&id) != L2C_OK) return L2C_E_CUDA;
+    Slot& s = g_slot[dev];
+    if (!s.addr || s.ctx_id != id) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess || !p) return L2C_E_CUDA;
-        g_scratch_addr[dev] = p;
+        if (attn_set_smem_limits() != cudaSuccess) return L2C_E_CUDA;
+        s.addr = p;
+        s.ctx_id = id;
     }
-    *out = static_cast<unsigned char*>(g_scratch_addr[dev]);
+    *out = static_cast<unsigned char*>(s.addr);
     return L2C_OK;
 }
 
@@ -58,7 +95,6 @@ __global__ void k_noalloc_prepare(int* tp, int pos, int* counters, int n) {
     if (threadIdx.x == 0) {
         tp[0] = 0;
         tp[1] = pos;
-        tp[2] = 0;  // error word
     }
     for (int i = threadIdx.x; i < n; i += blockDim.x) counters[i] = 0;
 }
@@ -71,6 +107,7 @@ extern "C" int l2c_attention_noalloc(const float* q_dev, const float* k_dev, con
     if (!q_dev || !k_dev || !v_dev || !out_dev || n_heads <= 0 || n_kv_heads <= 0 || head_size <= 0 || pos < 0 ||
         n_heads % n_kv_heads || (precision != 0 && precision != 1))
         return L2C_E_ARG;
+    if (((uintptr_t)q_dev | (uintptr_t)k_dev | (uintptr_t)v_dev | (uintptr_t)out_dev) & 15) return L2C_E_ARG;
     const int rep = n_heads / n_kv_heads;
     AttnKernel ak = precision ? attn_kernel_for<double>(head_size, rep) : attn_kernel_for<float>(head_size, rep);
     if (!ak) return L2C_E_ARG;
@@ -92,8 +129,10 @@ extern "C" int l2c_attention_noalloc(const float* q_dev, const float* k_dev, con
     t.out = out_dev; t.tp = tp; t.tp_stride = 2;
     t.H = n_heads; t.Hkv = n_kv_heads; t.hs = head_size; t.kvd = n_kv_heads * head_size; t.seq_len = pos + 1;
     t.nchunks = nchunks;
-    t.part = scratch + 256 + cnt_bytes; t.count = counters; t.err = tp + 2;
-    ak<<<dim3(nchunks, n_kv_heads, 1), 128, 0, s>>>(t);
+    t.min_chunk = kChunk;
+    t.part = scratch + 256 + cnt_bytes; t.count = counters;
+    const int smem = precision ? attn_smem_for<double>(rep) : attn_smem_for<float>(rep);
+    ak<<<dim3(nchunks, n_kv_heads, 1), ATTN_THREADS, smem, s>>>(t);
     if (cudaGetLastError() != cudaSuccess) return L2C_E_CUDA;
     return L2C_OK;
 }

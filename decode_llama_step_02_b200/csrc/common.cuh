@@ -100,29 +100,30 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
-// Phase timestamps for development builds that define L2C_PHASE_STAMPS
-// (a single translation unit): g_l2c_stamps[CTA][16]; compiled out otherwise.
-#ifdef L2C_PHASE_STAMPS
-__device__ unsigned long long g_l2c_stamps[1024 * 16];
-#define L2C_STAMP(slot)                                                                              \
-    do {                                                                                             \
-        if ((threadIdx.x & 31) == 0 && blockIdx.y == 0 && blockIdx.z == 0 && blockIdx.x < 1024)     \
-            g_l2c_stamps[blockIdx.x * 16 + (slot)] = global_timer_ns();                              \
-    } while (0)
-#else
-#define L2C_STAMP(slot) \
-    do {                \
-    } while (0)
-#endif
+// Shared-memory counters handed between warps of a CTA (release / acquire).
+__device__ __forceinline__ void st_release_cta(int* p, int v) {
+    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_cta(const int* p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+
+// Default limit of every barrier wait (2 s of %globaltimer).
+constexpr unsigned long long kWaitNs = 2000000000ull;
 
 // Waits for the barrier phase with the given parity.  Gives up after
-// `limit_ns` of wall time, records DERR_TIMEOUT and returns false.
+// `limit_ns` of wall time (records DERR_TIMEOUT) or, without recording, as
+// soon as *abort (a CTA-shared flag, may be null) is set; returns false then.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err,
-                                                  uint64_t limit_ns = 2000000000ull) {
+                                                  unsigned long long limit_ns = kWaitNs,
+                                                  volatile int* abort = nullptr) {
     if (mbar_try_wait(bar, parity)) return true;
-    uint64_t t0 = global_timer_ns();
+    const uint64_t t0 = global_timer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
+        if (abort && *abort) return false;
         if (global_timer_ns() - t0 > limit_ns) {
             set_error(err, DERR_TIMEOUT);
             return false;
@@ -143,7 +144,7 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src, uint32
 // ---- CTA-wide synchronisation policies ------------------------------------------
 // Helpers that a whole group of threads runs together take one of these: the
 // full CTA (barrier 0), or the first n threads of the CTA on a named barrier
-// (a persistent kernel whose producer warp does not take part).
+// (a kernel whose producer warp does not take part).
 struct SyncCTA {
     __device__ __forceinline__ void sync() const { __syncthreads(); }
     __device__ __forceinline__ int nthreads() const { return blockDim.x; }
@@ -152,6 +153,17 @@ struct SyncNamed {
     int id, n;  // barrier 1..15, thread count (a multiple of 32)
     __device__ __forceinline__ void sync() const { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
     __device__ __forceinline__ int nthreads() const { return n; }
+    // A barrier that also returns whether any participating thread passed true.
+    __device__ __forceinline__ bool sync_or(bool v) const {
+        uint32_t r;
+        asm volatile(
+            "{\n\t.reg .pred p, q;\n\t"
+            "setp.ne.u32 p, %1, 0;\n\t"
+            "bar.red.or.pred q, %2, %3, p;\n\t"
+            "selp.u32 %0, 1, 0, q;\n\t}"
+            : "=r"(r) : "r"((uint32_t)v), "r"(id), "r"(n) : "memory");
+        return r != 0;
+    }
 };
 
 // ---- exact int32 -> double on the FP64 pipe ------------------------------------

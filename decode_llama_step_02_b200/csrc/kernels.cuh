@@ -52,8 +52,11 @@ struct GemvArgs {
     const int* tp;           // {token, pos}
     unsigned long long* amax;  // argmax key (classifier); reset by layer 0
     int* err;
-    size_t prefetch_bytes;   // L2 prefetch issued before the dependency wait
-    int late_trigger;        // 1: let the next kernel launch only after this CTA's last weight loads
+    size_t prefetch_bytes;   // fp32: L2 prefetch issued before the dependency wait
+    int late_trigger;        // fp32: 1 = let the next kernel launch only after this CTA's last weight loads
+    int early;               // Q8_0: 1 = let the next kernel launch as soon as this one starts
+    unsigned long long wait_ns;  // limit of every barrier wait
+    int* stall;              // test switch (Q8_0): CTA 0 withholds one ring copy once if *stall != 0
 };
 
 // ----------------------------------------------------------------- epilogues --
@@ -403,13 +406,8 @@ __device__ __forceinline__ float q8_input_value(const GemvArgs& a, const int8_t*
 }
 
 // Quantizes the GEMV input (embedding row or input vector, RMSNorm'd when
-// norm_w is set) into shared codes and scales; all threads of the CTA call it.
-// Warp w owns groups w, w + Q8_WARPS, ...; a lane holds elements
-// g*gs + lane + 32e of each of them in registers, so the loads of the whole
-// vector are in flight at once (one round trip to L2) instead of a chain of
-// dependent loads.  Falls back to a plain loop when a lane would need more
-// than Q8_VPL values.
-// Slow path: one group at a time straight from global memory.
+// norm_w is set) into shared codes and scales, for any group size: one group
+// at a time straight from global memory.  Every thread of `sy` calls it.
 template <typename SY>
 __device__ __noinline__ void q8_quantize_input_loop(const GemvArgs& a, const int8_t* eq, const float* es, int8_t* xq,
                                                     float* xsc, double* red, const SY sy) {
@@ -479,7 +477,6 @@ __device__ __forceinline__ void q8_quantize_input_batched(const GemvArgs& a, con
             ss = warp_sum(ss);
             if (lane == 0) red[warp] = ss;
             sy.sync();
-            if (warp == 0) L2C_STAMP(5);
             double tot = 0.0;
             for (int i = 0; i < nw; i++) tot += red[i];
             const double inv = 1.0 / sqrt(tot / (double)K + 1e-5);
@@ -585,238 +582,332 @@ __device__ __forceinline__ void q8_quantize_input(const GemvArgs& a, const int8_
     else q8_quantize_input_loop(a, eq, es, xq, xsc, red, sy);
 }
 
-// Exact-int32 group dots of UNIT rows (records at rec, stride rb) with the
-// input codes xq, scaled and summed per lane in double.  Lane t covers the 64
-// contiguous bytes [64t, 64t+64) of a row: one group at GS = 64, two at
-// GS = 32, half of one at GS = 128 (a lane pair).  The four 16-byte reads of a
-// lane are rotated by (lane >> 1) & 3 so that a quarter-warp touches eight
-// distinct 16-byte bank groups.  Requires K % 64 == 0.
-template <int GS, int UNIT>
-__device__ __forceinline__ void q8_rows_dot64(const uint8_t* rec, size_t rb, const int8_t* xq, const double* sxd,
-                                              int K, double (&acc)[UNIT]) {
+// The exact int32 group dots of one 64-byte chunk of a row.  Lane chunk t
+// covers bytes [64t, 64t+64) of the row and of the input codes: one group at
+// GS = 64 (g[0]), two at GS = 32 (g[0], g[1]), half of one at GS = 128 (the
+// lane pair 2m, 2m+1 adds its halves with one shuffle, so every lane of the
+// warp must call it; both lanes of a pair hold the group's dot in g[0]).  The
+// four 16-byte reads are rotated by rot = (lane >> 1) & 3 so that a
+// quarter-warp touches eight distinct 16-byte bank groups; xv holds the input
+// chunks in that rotated order.  Out-of-range lanes (in = false) read nothing.
+template <int GS>
+__device__ __forceinline__ void q8_chunk_dots(const uint8_t* row, const int4 (&xv)[4], int t, bool in, int rot,
+                                              int (&g)[GS == 32 ? 2 : 1]) {
+    int c[4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const int f = (j + rot) & 3;
+        const int4 wv = in ? *reinterpret_cast<const int4*>(row + 64 * t + 16 * f) : make_int4(0, 0, 0, 0);
+        int dd = __dp4a(wv.x, xv[j].x, 0);
+        dd = __dp4a(wv.y, xv[j].y, dd);
+        dd = __dp4a(wv.z, xv[j].z, dd);
+        c[j] = __dp4a(wv.w, xv[j].w, dd);
+    }
+    if (GS == 32) {
+        // chunk f: the lane's first group is made of chunks f < 2
+        int lo = 0, hi = 0;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const int f = (j + rot) & 3;
+            lo += f < 2 ? c[j] : 0;
+            hi += f < 2 ? 0 : c[j];
+        }
+        g[0] = lo;
+        g[GS == 32 ? 1 : 0] = hi;
+    } else {
+        int d = (c[0] + c[1]) + (c[2] + c[3]);
+        if (GS == 128) d += __shfl_xor_sync(0xffffffffu, d, 1);
+        g[0] = d;
+    }
+}
+
+// The input codes of lane chunk t, in the rotated order of q8_chunk_dots.
+__device__ __forceinline__ void q8_chunk_x(const int8_t* xq, int t, bool in, int rot, int4 (&xv)[4]) {
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const int f = (j + rot) & 3;
+        xv[j] = in ? *reinterpret_cast<const int4*>(xq + 64 * t + 16 * f) : make_int4(0, 0, 0, 0);
+    }
+}
+
+// x * 2^-896 as a double, exactly, for every finite float x: the float's bits
+// with the exponent left unbiased (integer operations only; the conversion
+// instruction issues on a narrow unit).
+__device__ __forceinline__ double widen_f32_scaled(float x) {
+    const uint32_t b = __float_as_uint(x);
+    const uint32_t hi = ((b & 0x7fffffffu) >> 3) | (b & 0x80000000u);
+    return __hiloint2double((int)hi, (int)(b << 29));
+}
+
+// UR rows (records at rec, stride rb) against the input codes xq: the exact
+// group dots of q8_chunk_dots, each times the row's group scale and the
+// input's group scale, summed per lane in double.  sxs holds the input scales
+// times 2^896 and the row scales are widened as sw * 2^-896, so each term is
+// the double product (ival * sw) * sx.  Requires K % 64 == 0.
+template <int GS, int UR>
+__device__ __forceinline__ void q8_rows_dot64(const uint8_t* rec, size_t rb, const int8_t* xq, const double* sxs,
+                                              int K, double (&acc)[UR]) {
     const int lane = threadIdx.x & 31;
     const int n64 = K >> 6;
     const int rot = (lane >> 1) & 3;
 #pragma unroll
-    for (int r = 0; r < UNIT; r++) acc[r] = 0.0;
+    for (int r = 0; r < UR; r++) acc[r] = 0.0;
 #pragma unroll 2
     for (int t0 = 0; t0 < n64; t0 += 32) {
         const int t = t0 + lane;
         const bool in = t < n64;
         int4 xv[4];
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const int f = (j + rot) & 3;
-            xv[j] = in ? *reinterpret_cast<const int4*>(xq + 64 * t + 16 * f) : make_int4(0, 0, 0, 0);
+        q8_chunk_x(xq, t, in, rot, xv);
+        double sx0 = 0.0, sx1 = 0.0;
+        if (in) {
+            if (GS == 64) sx0 = sxs[t];
+            else if (GS == 32) { sx0 = sxs[2 * t]; sx1 = sxs[2 * t + 1]; }
+            else sx0 = sxs[t >> 1];
         }
 #pragma unroll
-        for (int r = 0; r < UNIT; r++) {
+        for (int r = 0; r < UR; r++) {
             const uint8_t* row = rec + r * rb;
-            int c[4];
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int f = (j + rot) & 3;
-                const int4 wv = in ? *reinterpret_cast<const int4*>(row + 64 * t + 16 * f) : make_int4(0, 0, 0, 0);
-                int dd = __dp4a(wv.x, xv[j].x, 0);
-                dd = __dp4a(wv.y, xv[j].y, dd);
-                dd = __dp4a(wv.z, xv[j].z, dd);
-                c[j] = __dp4a(wv.w, xv[j].w, dd);
-            }
+            int gd[GS == 32 ? 2 : 1];
+            q8_chunk_dots<GS>(row, xv, t, in, rot, gd);
             const float* sw = reinterpret_cast<const float*>(row + K);
+            if (!in) continue;
             if (GS == 64) {
-                const int d = (c[0] + c[1]) + (c[2] + c[3]);
-                if (in) acc[r] += i2d_exact(d) * (double)sw[t] * sxd[t];
+                acc[r] = fma(i2d_exact(gd[0]) * widen_f32_scaled(sw[t]), sx0, acc[r]);
             } else if (GS == 32) {
-                // chunk f of step j: the group of the lane's first 32 bytes is f < 2
-                int lo = 0, hi = 0;
-#pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    const int f = (j + rot) & 3;
-                    lo += f < 2 ? c[j] : 0;
-                    hi += f < 2 ? 0 : c[j];
-                }
-                if (in) {
-                    acc[r] += i2d_exact(lo) * (double)sw[2 * t] * sxd[2 * t];
-                    acc[r] += i2d_exact(hi) * (double)sw[2 * t + 1] * sxd[2 * t + 1];
-                }
-            } else {  // GS == 128: lanes 2m and 2m+1 hold the two halves of group t/2
-                int d = (c[0] + c[1]) + (c[2] + c[3]);
-                d += __shfl_xor_sync(0xffffffffu, d, 1);
-                if (in && (t & 1) == 0) acc[r] += i2d_exact(d) * (double)sw[t >> 1] * sxd[t >> 1];
+                acc[r] = fma(i2d_exact(gd[0]) * widen_f32_scaled(sw[2 * t]), sx0, acc[r]);
+                acc[r] = fma(i2d_exact(gd[GS == 32 ? 1 : 0]) * widen_f32_scaled(sw[2 * t + 1]), sx1, acc[r]);
+            } else if ((t & 1) == 0) {  // GS == 128: the even lane of the pair
+                acc[r] = fma(i2d_exact(gd[0]) * widen_f32_scaled(sw[t >> 1]), sx0, acc[r]);
             }
         }
     }
 }
 
-// Registers of the split prologue (gs = 32 * EPL): warp w holds groups
-// w + j*nw (j < GM), a lane elements lane + 32e of each; w holds the RMSNorm
-// gain when NORM.
-template <int EPL, int GM, bool NORM>
-struct Q8Pre {
-    float v[GM][EPL];
-    float w[NORM ? GM : 1][EPL];
-};
+// Input quantization of the 64-byte-per-lane Q8_0 path (K % 64 == 0, GS 32,
+// 64 or 128), split around the dependency wait.  The input is taken in chunks
+// of 64 values, two per warp step: half-warp h of warp w takes chunk
+// 2*(w + NW*it) + h, its lane i the values 4i..4i+3 (one 16-byte load).  A
+// group is 8, 16 or 32 lanes, so its max is 3, 4 or 5 shuffles, and a lane
+// packs its four codes into one 32-bit store.  With an RMSNorm the values
+// stay in registers (at most MAXIT steps) between the sum of squares and the
+// codes; the gain, and on layer 0 the embedding row, are loaded before the
+// wait (no kernel of the step writes them).  Arithmetic as the listing's rule
+// and RMSNorm elsewhere: sums of squares in double, w * (inv * x) in double
+// rounded once to fp32, scale = max|x| / 127 in fp32, code = round(x / scale).
+template <int GS, bool NORM, int NW, int MAXIT>
+struct Q8Prologue {
+    static constexpr int IT = NORM ? MAXIT : 1;
+    float4 v[IT], w[IT];
+    int steps;
 
-// Group slots per warp of the register prologue: 16 values per lane with an
-// RMSNorm gain, 48 without.
-template <int EPL, bool NORM>
-struct Q8PreGM {
-    static constexpr int value = (NORM ? 16 : 48) / EPL;
-};
-
-template <int EPL, int GM>
-__device__ __forceinline__ bool q8_pre_fits(const GemvArgs& a, int nw) {
-    const int ng = a.K / (32 * EPL);
-    return a.gs == 32 * EPL && (ng + nw - 1) / nw <= GM;
-}
-
-// Loads the gain (gain = true) or the values (from src, or the embedding
-// codes eq * scale es) of the warp's groups.
-template <int EPL, int GM, bool NORM>
-__device__ __forceinline__ void q8_pre_load(const GemvArgs& a, const float* src, const int8_t* eq, const float* es,
-                                            bool gain, Q8Pre<EPL, GM, NORM>& r, int nw) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int gs = 32 * EPL, ng = a.K / gs;
+    // whether the input fits this path
+    static __device__ __forceinline__ bool fits(const GemvArgs& a) {
+        if (a.K % 64 || a.gs != GS) return false;
+        const int npair = (a.K / 64 + 1) / 2;
+        return !NORM || (npair + NW - 1) / NW <= MAXIT;
+    }
+    __device__ __forceinline__ int chunk(int it) const {
+        return 2 * ((threadIdx.x >> 5) + NW * it) + ((threadIdx.x >> 4) & 1);
+    }
+    __device__ __forceinline__ float4 load_value(const GemvArgs& a, const int8_t* eq, const float* es, int it) const {
+        const int c = chunk(it), i = threadIdx.x & 15;
+        if (c >= a.K / 64) return make_float4(0.f, 0.f, 0.f, 0.f);
+        const int idx = c * 64 + 4 * i;
+        if (eq) {
+            const char4 q = *reinterpret_cast<const char4*>(eq + idx);
+            const float sc = es[idx / a.gs];
+            return make_float4((float)q.x * sc, (float)q.y * sc, (float)q.z * sc, (float)q.w * sc);
+        }
+        return __ldcg(reinterpret_cast<const float4*>(a.in + idx));
+    }
+    // before the wait: the gain and the embedding row
+    __device__ __forceinline__ void pre(const GemvArgs& a, const int8_t* eq, const float* es) {
+        const int npair = (a.K / 64 + 1) / 2;
+        steps = (npair - (int)(threadIdx.x >> 5) + NW - 1) / NW;
+        if (NORM) {
 #pragma unroll
-    for (int j = 0; j < GM; j++) {
-        const int g = warp + j * nw;
-#pragma unroll
-        for (int e = 0; e < EPL; e++) {
-            const int i = g * gs + lane + 32 * e;
-            if (gain) {
-                if (NORM) r.w[NORM ? j : 0][e] = g < ng ? a.norm_w[i] : 0.f;
-            } else {
-                r.v[j][e] = g < ng ? (eq ? (float)eq[i] * es[g] : __ldcg(src + i)) : 0.f;
+            for (int it = 0; it < IT; it++) {
+                const int c = chunk(it);
+                const bool on = it < steps && c < a.K / 64;
+                w[it] = on ? *reinterpret_cast<const float4*>(a.norm_w + c * 64 + 4 * (threadIdx.x & 15))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                if (eq) v[it] = on ? load_value(a, eq, es, it) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
         }
     }
-}
-
-// RMSNorm (double, when NORM) and Q8_0 codes of the values in r.  The
-// reductions of all groups run interleaved so their latencies overlap.
-template <int EPL, int GM, bool NORM, typename AfterLoads, typename SY = SyncCTA>
-__device__ __forceinline__ void q8_pre_finish(const GemvArgs& a, Q8Pre<EPL, GM, NORM>& r, int8_t* xq, float* xsc,
-                                              double* red, AfterLoads after_loads, const SY sy = SY()) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = sy.nthreads() >> 5;
-    const int gs = 32 * EPL, ng = a.K / gs;
-    if (a.emb && blockIdx.x == 0) {
+    // the group max, scale and codes of the four values of step `it`
+    __device__ __forceinline__ void quantize(const GemvArgs& a, float4 x, int it, int8_t* xq, float* xsc) const {
+        const int c = chunk(it), i = threadIdx.x & 15;
+        float m = fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(x.z), fabsf(x.w)));
+        constexpr int LANES = GS / 4;  // lanes of one group
 #pragma unroll
-        for (int j = 0; j < GM; j++) {
-            const int g = warp + j * nw;
-            if (g < ng) {
-#pragma unroll
-                for (int e = 0; e < EPL; e++) a.x_resid[g * gs + lane + 32 * e] = r.v[j][e];
-            }
+        for (int o = 1; o < LANES; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (c >= a.K / 64) return;
+        const float scale = m / 127.0f;
+        int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+        if (scale != 0.f) {
+            q0 = (int)roundf(x.x / scale); q1 = (int)roundf(x.y / scale);
+            q2 = (int)roundf(x.z / scale); q3 = (int)roundf(x.w / scale);
         }
+        *reinterpret_cast<uint32_t*>(xq + c * 64 + 4 * i) =
+            (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) | ((uint32_t)(q2 & 0xff) << 16) |
+            ((uint32_t)(q3 & 0xff) << 24);
+        if ((threadIdx.x & (LANES - 1)) == 0) xsc[(c * 64 + 4 * i) / GS] = scale;
     }
-    if (NORM) {
-        double part[4] = {0.0, 0.0, 0.0, 0.0};
+    // after the wait: the input, the RMSNorm, the codes
+    __device__ __forceinline__ void post(const GemvArgs& a, const int8_t* eq, const float* es, int8_t* xq, float* xsc,
+                                         double* red) {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const bool resid = a.emb && blockIdx.x == 0;  // layer 0: CTA 0 stores the embedding row as x
+        if (!NORM) {
+            for (int it = 0; it < steps; it++) {
+                const float4 x = load_value(a, eq, es, it);
+                if (resid && chunk(it) < a.K / 64)
+                    reinterpret_cast<float4*>(a.x_resid)[(chunk(it) * 64 + 4 * (threadIdx.x & 15)) / 4] = x;
+                quantize(a, x, it, xq, xsc);
+            }
+            return;
+        }
+        if (!eq) {
 #pragma unroll
-        for (int j = 0; j < GM; j++)
+            for (int it = 0; it < IT; it++)
+                v[it] = it < steps ? load_value(a, eq, es, it) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        double ss = 0.0;
 #pragma unroll
-            for (int e = 0; e < EPL; e++) part[(j * EPL + e) & 3] += (double)r.v[j][e] * (double)r.v[j][e];
-        double ss = (part[0] + part[1]) + (part[2] + part[3]);
-        after_loads();  // every value has arrived by now
+        for (int it = 0; it < IT; it++) {
+            ss += (double)v[it].x * (double)v[it].x + (double)v[it].y * (double)v[it].y;
+            ss += (double)v[it].z * (double)v[it].z + (double)v[it].w * (double)v[it].w;
+            if (resid && it < steps && chunk(it) < a.K / 64)
+                reinterpret_cast<float4*>(a.x_resid)[(chunk(it) * 64 + 4 * (threadIdx.x & 15)) / 4] = v[it];
+        }
         ss = warp_sum(ss);
         if (lane == 0) red[warp] = ss;
-        sy.sync();
+        __syncthreads();
         double tot = 0.0;
-        for (int i = 0; i < nw; i++) tot += red[i];
+#pragma unroll
+        for (int k = 0; k < NW; k++) tot += red[k];
         const double inv = 1.0 / sqrt(tot / (double)a.K + 1e-5);
 #pragma unroll
-        for (int j = 0; j < GM; j++)
-#pragma unroll
-            for (int e = 0; e < EPL; e++)
-                r.v[j][e] = (float)((double)r.w[NORM ? j : 0][e] * (inv * (double)r.v[j][e]));
-    }
-    float m[GM];
-#pragma unroll
-    for (int j = 0; j < GM; j++) {
-        m[j] = fabsf(r.v[j][0]);
-#pragma unroll
-        for (int e = 1; e < EPL; e++) m[j] = fmaxf(m[j], fabsf(r.v[j][e]));
-    }
-    if (!NORM) {
-        float all = 0.f;
-#pragma unroll
-        for (int j = 0; j < GM; j++) all = fmaxf(all, m[j]);
-        asm volatile("" ::"f"(all));  // every value has arrived by now
-        after_loads();
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-        for (int j = 0; j < GM; j++) m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], o));
-#pragma unroll
-    for (int j = 0; j < GM; j++) {
-        const int g = warp + j * nw;
-        const float scale = m[j] / 127.0f;
-        if (g < ng) {
-#pragma unroll
-            for (int e = 0; e < EPL; e++) {
-                const float q = scale == 0.f ? 0.f : roundf(r.v[j][e] / scale);
-                xq[g * gs + lane + 32 * e] = (int8_t)(int)q;
-            }
-            if (lane == 0) xsc[g] = scale;
+        for (int it = 0; it < IT; it++) {
+            if (it >= steps) break;  // warp-uniform
+            float4 x = v[it];
+            x.x = (float)((double)w[it].x * (inv * (double)x.x));
+            x.y = (float)((double)w[it].y * (inv * (double)x.y));
+            x.z = (float)((double)w[it].z * (inv * (double)x.z));
+            x.w = (float)((double)w[it].w * (inv * (double)x.w));
+            quantize(a, x, it, xq, xsc);
         }
     }
-}
-
-struct Q8Layout {
-    int nslot;          // ring slots per warp, one unit (UNIT row records) each
-    size_t unit_bytes;  // UNIT * record bytes
 };
 
-constexpr int Q8_WARPS = 8;
+constexpr int Q8_WARPS = 8;                  // warps of a Q8_0 GEMV CTA
+constexpr int Q8_THREADS = 32 * Q8_WARPS;
 
-// Every warp streams its own units (round-robin over the CTA's contiguous
-// range) through its own ring of `nslot` shared-memory slots filled by 1-D bulk
-// copies; lane 0 issues a copy as soon as the warp has finished with a slot,
-// so nslot-1 units per warp stay in flight.  GS is the group size of the
+// The CTA's weight ring: `ns` slots of one unit (UR row records) each.
+struct Q8Ring {
+    int ns;
+    uint32_t unit_bytes;  // UR * record bytes
+};
+
+// Dynamic shared memory of a Q8_0 GEMV CTA: the ring, the input codes and
+// scales, the ring barriers, and per slot the number of units issued into it
+// and the number consumed.
+struct Q8Smem {
+    size_t xq, xsc, sxd, bars, cnt, total;
+};
+
+__host__ __device__ inline Q8Smem q8_smem(int ns, uint32_t unit_bytes, int K, int gs) {
+    Q8Smem m;
+    const size_t ng = (size_t)(K / gs);
+    m.xq = (size_t)ns * unit_bytes;
+    m.xsc = m.xq + (((size_t)K + 15) & ~size_t(15));
+    m.sxd = m.xsc + ((ng * 4 + 15) & ~size_t(15));
+    m.bars = m.sxd + ng * 8;
+    m.cnt = m.bars + 8 * (size_t)ns;
+    m.total = m.cnt + 8 * (size_t)ns;
+    return m;
+}
+
+// Q8_0 GEMV.  A unit is UR consecutive row records (for QKV and W1/W3, UR/2
+// row pairs); the CTA owns a contiguous range of units and streams them
+// through a ring of `ns` shared-memory slots with 1-D bulk copies: unit k
+// goes to slot k % ns and is consumed by warp k % Q8_WARPS, and the warp that
+// consumes a unit refills its slot at once with unit k + ns.  The first `ns`
+// copies are issued at the start, before the dependency wait (weights do not
+// depend on the previous kernel).  After the wait the warps quantize the input
+// (the listing's rule, bit-exact) into shared codes, then run their units:
+// exact int32 group dots by dp4a, (ival * sw) * sx summed per lane in double,
+// one reduce-scatter for the UR row sums, and the epilogues of the unit's rows
+// (or row pairs) on separate lanes.  GS is the group size of the
 // 64-byte-per-lane dot (32, 64 or 128, K % 64 == 0), or 0 for the generic
-// 16-byte-per-lane loop.  Dynamic shared memory:
-//   slots [Q8_WARPS][nslot][unit_bytes] | x codes [K, padded to 16] |
-//   x scales [K/gs] fp32 | x scales [K/gs] double | barriers [Q8_WARPS][nslot]
-template <int MODE, int GS>
-__global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, const Q8Layout L) {
+// 16-byte-per-lane loop.  Every wait is bounded (a.wait_ns); a CTA that gives
+// up records DERR_TIMEOUT, stops in all its warps (a shared abort flag), and
+// leaves only after every copy it issued has landed.
+template <int MODE, int GS, int UR>
+__global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, const Q8Ring R) {
     extern __shared__ __align__(128) uint8_t smem[];
-    constexpr int UNIT = (MODE == M_QKV || MODE == M_W13) ? 2 : 1;
+    constexpr bool PAIRS = MODE == M_QKV || MODE == M_W13;
+    static_assert(!PAIRS || UR % 2 == 0, "row pairs");
     __shared__ double red[Q8_WARPS];
     __shared__ unsigned long long best_s[Q8_WARPS];
     __shared__ double2 rope_cs[MODE == M_QKV ? 128 : 1];
+    __shared__ int abort_s;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int K = a.K, gs = a.gs;
+    const int K = a.K, gs = a.gs, ns = R.ns;
+    const uint32_t ub = R.unit_bytes;
     const size_t rb = a.ld;
-    const int ns = L.nslot;
-    uint8_t* slots = smem + (size_t)warp * ns * L.unit_bytes;
-    int8_t* xq = reinterpret_cast<int8_t*>(smem + (size_t)Q8_WARPS * ns * L.unit_bytes);
-    float* xsc = reinterpret_cast<float*>(xq + ((K + 15) & ~15));
-    double* sxd = reinterpret_cast<double*>((reinterpret_cast<uintptr_t>(xsc + K / gs) + 15) & ~uintptr_t(15));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sxd + ((K / gs + 1) & ~1));
-    uint64_t* full = bars + warp * ns;
-
-    const int units = a.rows / UNIT;
+    const Q8Smem lay = q8_smem(ns, ub, K, gs);
+    int8_t* xq = reinterpret_cast<int8_t*>(smem + lay.xq);
+    float* xsc = reinterpret_cast<float*>(smem + lay.xsc);
+    double* sxd = reinterpret_cast<double*>(smem + lay.sxd);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars);
+    volatile int* issued = reinterpret_cast<volatile int*>(smem + lay.cnt);  // units issued into slot s
+    int* used = const_cast<int*>(issued) + ns;                                 // units consumed from slot s
+    const int units = (a.rows + UR - 1) / UR;
     const int u0 = (int)((long long)units * blockIdx.x / gridDim.x);
     const int u1 = (int)((long long)units * (blockIdx.x + 1) / gridDim.x);
-    const int nmine = (u1 - u0 - warp + Q8_WARPS - 1) / Q8_WARPS;  // units of this warp
-    const uint8_t* Wb = static_cast<const uint8_t*>(a.W);
+    const int n = u1 - u0;
+    const uint8_t* src = static_cast<const uint8_t*>(a.W) + (size_t)u0 * ub;
     const uint64_t pol = policy_evict_first();
-    auto unit_src = [&](int k) { return Wb + (size_t)(u0 + warp + k * Q8_WARPS) * UNIT * rb; };
-
-    if (warp == 0) L2C_STAMP(0);
-    // ---- before the dependency wait: everything that earlier kernels of the
-    // step do not write.  The small loads (token/position, RMSNorm gain,
-    // embedding row, RoPE frequencies) go first, then the L2 prefetch of this
-    // CTA's weights, so that those loads do not queue behind it in HBM.
-    if (lane == 0) {
-        for (int s = 0; s < ns; s++) mbar_init(&full[s], 1);
+    // bytes of unit k of this CTA (the last unit of the matrix may be short)
+    auto unit_bytes = [&](int k) {
+        const int r0 = (u0 + k) * UR;
+        const int nr = min(UR, a.rows - r0);
+        return (uint32_t)((size_t)nr * rb);
+    };
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < ns; s++) {
+            mbar_init(&full[s], 1);
+            issued[s] = 0;
+            st_release_cta(&used[s], 0);
+        }
+        abort_s = 0;
         mbar_fence_init();
+        // test switch: withhold the first copy of CTA 0 once (a wait then runs out)
+        const bool skip0 = a.stall && blockIdx.x == 0 && n > 0 && atomicExch(a.stall, 0);
+        for (int k = 0; k < ns && k < n; k++) {
+            if (k == 0 && skip0) continue;
+            const uint32_t by = unit_bytes(k);
+            mbar_arrive_expect_tx(&full[k], by);
+            bulk_g2s(smem + (size_t)k * ub, src + (size_t)k * ub, by, &full[k], pol);
+            issued[k] = 1;
+        }
+        // and the units after the ring into L2, so that the first refills hit it
+        if (n > ns && a.prefetch_bytes) {
+            size_t by = (size_t)(n - ns) * ub;
+            if (by > a.prefetch_bytes) by = a.prefetch_bytes;
+            const size_t last = (size_t)a.rows * rb - (size_t)(u0 + ns) * ub;  // bytes left in the matrix
+            prefetch_l2_range(src + (size_t)ns * ub, (by < last ? by : last) & ~size_t(15), policy_evict_last());
+        }
     }
-    constexpr int EPL = GS > 0 ? GS / 32 : 1;
+    __syncthreads();
+    if (a.early) grid_dep_launch();
+
+    // before the dependency wait: what earlier kernels of the step do not write
     constexpr bool NORM = MODE != M_RESID;
-    constexpr int GM = Q8PreGM<EPL, NORM>::value;
-    Q8Pre<EPL, GM, NORM> pre;
-    const bool split = GS > 0 && (NORM == (a.norm_w != nullptr)) && q8_pre_fits<EPL, GM>(a, Q8_WARPS);  // CTA-uniform
+    Q8Prologue<GS == 0 ? 64 : GS, NORM, Q8_WARPS, 8> pro;
+    const bool fast = GS != 0 && (NORM == (a.norm_w != nullptr)) && pro.fits(a);  // CTA-uniform
     int token = 0, pos = 0;
     if (MODE == M_QKV) read_tp(a, token, pos);  // written before the step's first kernel
     const int8_t* eq = nullptr;
@@ -826,134 +917,132 @@ __global__ void __launch_bounds__(32 * Q8_WARPS, 1) k_gemv_q8(const GemvArgs a, 
         eq = reinterpret_cast<const int8_t*>(rec);
         es = reinterpret_cast<const float*>(rec + K);
     }
-    if (split) {
-        if (NORM) q8_pre_load<EPL, GM, NORM>(a, nullptr, nullptr, nullptr, true, pre, Q8_WARPS);
-        if (eq) q8_pre_load<EPL, GM, NORM>(a, nullptr, eq, es, false, pre, Q8_WARPS);
-    }
+    if (fast) pro.pre(a, eq, es);
     if (MODE == M_QKV) rope_table(a, pos, rope_cs);
-    if (warp == 0 && lane == 0 && a.prefetch_bytes) {
-        const size_t first = (size_t)u0 * UNIT * rb;
-        const size_t last = (size_t)u1 * UNIT * rb;
-        if (last > first) {
-            size_t bytes = last - first;
-            if (bytes > a.prefetch_bytes) bytes = a.prefetch_bytes;
-            prefetch_l2_range(Wb + first, bytes, policy_evict_last());
-        }
-    }
-    if (warp == 0) L2C_STAMP(3);
     grid_dep_wait();
-    if (!a.late_trigger) grid_dep_launch();
-    if (warp == 0) L2C_STAMP(1);
-
-    // ---- after the wait: the input written by the previous kernel, then the
-    // ring fill (its copies land while the codes are computed)
+    // after the wait: the input written by the previous kernel
     if (MODE == M_QKV && a.amax && blockIdx.x == 0 && threadIdx.x == 0) *a.amax = 0ull;
-    if (split && !eq) q8_pre_load<EPL, GM, NORM>(a, a.in, nullptr, nullptr, false, pre, Q8_WARPS);
-    // residual: lane k fetches now the x of this warp's k-th row, for the epilogue
-    float xres = 0.f;
-    if (MODE == M_RESID && lane < nmine) xres = __ldcg(a.out + u0 + warp + lane * Q8_WARPS);
-    if (warp == 0) L2C_STAMP(4);
-    auto fill_ring = [&]() {
-        if (lane == 0) {
-            for (int k = 0; k < ns && k < nmine; k++) {
-                mbar_arrive_expect_tx(&full[k], (uint32_t)L.unit_bytes);
-                bulk_g2s(slots + (size_t)k * L.unit_bytes, unit_src(k), (uint32_t)L.unit_bytes, &full[k], pol);
-            }
-        }
-    };
-    if (split) {
-        q8_pre_finish<EPL, GM, NORM>(a, pre, xq, xsc, red, fill_ring);
-    } else {
-        q8_quantize_input<NORM>(a, eq, es, xq, xsc, red);
-        fill_ring();
-    }
-    if (warp == 0) L2C_STAMP(6);
+    if (fast) pro.post(a, eq, es, xq, xsc, red);
+    else q8_quantize_input<NORM>(a, eq, es, xq, xsc, red);
     __syncthreads();
-    if (warp == 0) L2C_STAMP(7);
-    for (int g = threadIdx.x; g < K / gs; g += blockDim.x) sxd[g] = (double)xsc[g];
+    // input scales in double; for the 64-byte path times 2^896 (see q8_rows_dot64)
+    for (int g = threadIdx.x; g < K / gs; g += Q8_THREADS)
+        sxd[g] = GS != 0 ? (double)xsc[g] * 0x1p896 : (double)xsc[g];
     __syncthreads();
-    if (warp == 0) L2C_STAMP(2);
 
-    // ---- stream this warp's units
-    const int nchunk = K >> 4;   // 16-byte chunks per row
-    const int cpg = gs >> 4;     // chunks per group
+    // ---- this warp's units
+    constexpr int GRP = 32 / UR;     // lanes that hold one row's total after the reduce-scatter
+    const int my_row = lane / GRP;   // the unit row whose total this lane holds
+    const int nchunk = K >> 4;       // 16-byte chunks per row (generic loop)
+    const int cpg = gs >> 4;         // chunks per group
     const int iters = (nchunk + 31) >> 5;
     unsigned long long best = 0ull;
-    for (int k = 0; k < nmine; k++) {
-        const int s = k % ns;
-        if (!mbar_wait_bounded(&full[s], (k / ns) & 1, a.err)) {
-            // give up: let the copies already issued land before the CTA leaves
-            for (int j = k + 1; j < nmine && j < k + ns; j++) mbar_wait_bounded(&full[j % ns], (j / ns) & 1, a.err);
-            return;
+    bool gave_up = false;
+    for (int k = warp; k < n; k += Q8_WARPS) {
+        const int s = k % ns, j = k / ns;
+        // Unit k is the j-th use of slot s.  Its parity wait is only meaningful
+        // once the slot's previous unit has been consumed (then its refill, unit
+        // k, has been issued): another warp may still be on unit k - ns.
+        bool ok = true;
+        if (lane == 0 && ld_acquire_cta(&used[s]) < j) {
+            const uint64_t t0 = global_timer_ns();
+            while (ld_acquire_cta(&used[s]) < j) {
+                if (abort_s) { ok = false; break; }
+                if (global_timer_ns() - t0 > a.wait_ns) {
+                    set_error(a.err, DERR_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+            }
         }
-        const uint8_t* base = slots + (size_t)s * L.unit_bytes;
-        double acc[UNIT];
+        if (!__shfl_sync(0xffffffffu, (int)ok, 0) ||
+            !mbar_wait_bounded(&full[s], j & 1, a.err, a.wait_ns, &abort_s)) {
+            abort_s = 1;
+            gave_up = true;
+            break;
+        }
+        const int r0 = (u0 + k) * UR;              // first row of the unit
+        const int nr = min(UR, a.rows - r0);        // rows in the unit
+        // residual rows: fetched now, added in the epilogue
+        float xres = 0.f;
+        if (MODE == M_RESID && lane % GRP == 0 && my_row < nr) xres = __ldcg(a.out + r0 + my_row);
+        const uint8_t* base = smem + (size_t)s * ub;
+        double acc[UR];
         if (GS != 0) {
-            q8_rows_dot64<GS == 0 ? 64 : GS, UNIT>(base, rb, xq, sxd, K, acc);
+            q8_rows_dot64<GS == 0 ? 64 : GS, UR>(base, rb, xq, sxd, K, acc);
         } else {
 #pragma unroll
-            for (int r = 0; r < UNIT; r++) acc[r] = 0.0;
+            for (int r = 0; r < UR; r++) acc[r] = 0.0;
             for (int it = 0; it < iters; it++) {
                 const int c = lane + 32 * it;
                 const bool in = c < nchunk;
-                int dsum[UNIT];
                 int4 xv = in ? *reinterpret_cast<const int4*>(xq + 16 * c) : make_int4(0, 0, 0, 0);
 #pragma unroll
-                for (int r = 0; r < UNIT; r++) {
-                    dsum[r] = 0;
-                    if (in) {
+                for (int r = 0; r < UR; r++) {
+                    int dsum = 0;
+                    if (in && r < nr) {
                         const int4 wv = *reinterpret_cast<const int4*>(base + r * rb + 16 * c);
-                        dsum[r] = __dp4a(wv.x, xv.x, dsum[r]);
-                        dsum[r] = __dp4a(wv.y, xv.y, dsum[r]);
-                        dsum[r] = __dp4a(wv.z, xv.z, dsum[r]);
-                        dsum[r] = __dp4a(wv.w, xv.w, dsum[r]);
+                        dsum = __dp4a(wv.x, xv.x, dsum);
+                        dsum = __dp4a(wv.y, xv.y, dsum);
+                        dsum = __dp4a(wv.z, xv.z, dsum);
+                        dsum = __dp4a(wv.w, xv.w, dsum);
                     }
-                }
-                for (int o = 1; o < cpg; o <<= 1) {
-#pragma unroll
-                    for (int r = 0; r < UNIT; r++) dsum[r] += __shfl_xor_sync(0xffffffffu, dsum[r], o);
-                }
-                if (in && (c & (cpg - 1)) == 0) {
-                    const int g = c / cpg;
-#pragma unroll
-                    for (int r = 0; r < UNIT; r++) {
+                    for (int o = 1; o < cpg; o <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+                    if (in && r < nr && (c & (cpg - 1)) == 0) {
+                        const int g = c / cpg;
                         const float* sw = reinterpret_cast<const float*>(base + r * rb + K);
-                        acc[r] += (double)dsum[r] * (double)sw[g] * sxd[g];
+                        acc[r] += (double)dsum * (double)sw[g] * sxd[g];
                     }
                 }
             }
         }
-        // refill the slot with the unit ns ahead once every lane is done with it
+        // every lane is done with the slot: refill it with unit k + ns
         __syncwarp();
-        if (a.late_trigger && k + ns == nmine) grid_dep_launch();  // this warp's last copy is in
-        if (lane == 0 && k + ns < nmine) {
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive_expect_tx(&full[s], (uint32_t)L.unit_bytes);
-            bulk_g2s(slots + (size_t)s * L.unit_bytes, unit_src(k + ns), (uint32_t)L.unit_bytes, &full[s], pol);
-        }
-#pragma unroll
-        for (int r = 0; r < UNIT; r++) acc[r] = warp_sum(acc[r]);
-        const int u = u0 + warp + k * Q8_WARPS;
-        const float xo = MODE == M_RESID ? __shfl_sync(0xffffffffu, xres, k & 31) : 0.f;
         if (lane == 0) {
-            if (MODE == M_QKV) {
-                epi_qkv(a, u, (float)acc[0], (float)acc[UNIT - 1], pos, rope_cs);
-            } else if (MODE == M_W13) {
-                epi_w13(a, u, (float)acc[0], (float)acc[UNIT - 1]);
-            } else if (MODE == M_RESID) {
-                a.out[u] = (k < 32 ? xo : __ldcg(a.out + u)) + (float)acc[0];
+            if (k + ns < n) {
+                const uint32_t by = unit_bytes(k + ns);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive_expect_tx(&full[s], by);
+                bulk_g2s(smem + (size_t)s * ub, src + (size_t)(k + ns) * ub, by, &full[s], pol);
+                issued[s] = j + 2;
+            }
+            st_release_cta(&used[s], j + 1);
+        }
+        // the UR row totals: lanes [GRP*i, GRP*i + GRP) hold row i's
+        const double tot = warp_sum_scatter<UR>(acc);
+        if (PAIRS) {
+            // pair p = rows (2p, 2p+1): lane 2p*GRP takes the odd row's total from lane (2p+1)*GRP
+            const double odd = __shfl_down_sync(0xffffffffu, tot, GRP);
+            if (lane % (2 * GRP) == 0 && my_row < nr) {
+                const int pr = (r0 + my_row) / 2;
+                if (MODE == M_QKV) epi_qkv(a, pr, (float)tot, (float)odd, pos, rope_cs);
+                else epi_w13(a, pr, (float)tot, (float)odd);
+            }
+        } else if (lane % GRP == 0 && my_row < nr) {
+            const int r = r0 + my_row;
+            if (MODE == M_RESID) {
+                a.out[r] = xres + (float)tot;
             } else {
-                const float v = (float)acc[0];
-                a.out[u] = v;
+                const float v = (float)tot;
+                a.out[r] = v;
                 if (v != v) set_error(a.err, DERR_NAN);
-                const unsigned long long key = argmax_key(v, u);
+                const unsigned long long key = argmax_key(v, r);
                 best = key > best ? key : best;
             }
         }
     }
-    if (a.late_trigger) grid_dep_launch();  // (repeat triggers are harmless)
-    L2C_STAMP(8 + warp);
+    if (!a.early) grid_dep_launch();
+    // a CTA that gave up must not leave while a copy into its ring is in flight
+    if (__syncthreads_or(gave_up) && threadIdx.x == 0) {
+        for (int s = 0; s < ns; s++)
+            if (issued[s] > ld_acquire_cta(&used[s])) mbar_wait_bounded(&full[s], (issued[s] - 1) & 1, a.err, a.wait_ns);
+    }
     if (MODE == M_CLS) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+            best = other > best ? other : best;
+        }
         if (lane == 0) best_s[warp] = best;
         __syncthreads();
         if (threadIdx.x == 0) {
@@ -1029,8 +1118,43 @@ static __global__ void k_quantize_rows(const float* W, long long rows, int K, in
     }
 }
 
-// Exact int32 group dot products through the same dp4a chunk loop as the Q8_0
-// GEMV: out[r][g] = sum_k qw[r][g*gs+k] * qx[g*gs+k].  One warp per row.
+// Exact int32 group dot products, out[r][g] = sum_k qw[r][g*gs+k] *
+// qx[g*gs+k], through the Q8_0 GEMV's own chunk routine (q8_chunk_dots) for
+// GS = 32, 64, 128 with K % 64 == 0: one warp per row, the input codes staged
+// in shared memory as in the GEMV.  Dynamic shared memory: K bytes.
+template <int GS>
+__global__ void k_group_dots64(const int8_t* qw, const int8_t* qx, int rows, int K, int* out) {
+    extern __shared__ __align__(16) int8_t gx[];
+    for (int i = threadIdx.x; i < K / 16; i += blockDim.x)
+        reinterpret_cast<int4*>(gx)[i] = reinterpret_cast<const int4*>(qx)[i];
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (r >= rows) return;  // warp-uniform
+    const int n64 = K >> 6, rot = (lane >> 1) & 3;
+    const uint8_t* row = reinterpret_cast<const uint8_t*>(qw) + (size_t)r * K;
+    int* o = out + (size_t)r * (K / GS);
+    for (int t0 = 0; t0 < n64; t0 += 32) {
+        const int t = t0 + lane;
+        const bool in = t < n64;
+        int4 xv[4];
+        q8_chunk_x(gx, t, in, rot, xv);
+        int gd[GS == 32 ? 2 : 1];
+        q8_chunk_dots<GS>(row, xv, t, in, rot, gd);
+        if (!in) continue;
+        if (GS == 64) {
+            o[t] = gd[0];
+        } else if (GS == 32) {
+            o[2 * t] = gd[0];
+            o[2 * t + 1] = gd[GS == 32 ? 1 : 0];
+        } else if ((t & 1) == 0) {
+            o[t >> 1] = gd[0];
+        }
+    }
+}
+
+// Exact int32 group dot products for the other group sizes and widths, with
+// the generic GEMV's 16-byte chunk loop: one warp per row.
 static __global__ void k_group_dots(const int8_t* qw, const int8_t* qx, int rows, int K, int gs, int* out) {
     const int lane = threadIdx.x & 31;
     const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);

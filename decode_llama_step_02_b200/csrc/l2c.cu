@@ -22,7 +22,6 @@
 
 #include "../../include/l2c.h"
 #include "batched.cuh"
-#include "persistent.h"
 #include "kernels.cuh"
 
 using namespace l2c;
@@ -56,8 +55,10 @@ struct l2c_ctx {
     unsigned long long* key_scratch = nullptr;
     void* attn_part = nullptr;
     int* attn_cnt = nullptr;
-    int attn_nchunks = 16;      // CTAs per (sequence, KV head) in the fp32 attention
-    int attn_nchunks_f64 = 24;  // ... in the double attention (compute-bound: more CTAs pay)
+    int attn_ctas = 0;          // fp32 attention CTAs to aim for (0: the SM count)
+    int attn_ctas_f64 = 0;      // double attention CTAs to aim for (0: four times the SM count)
+    int attn_min_chunk = 32;    // positions per attention chunk, at least
+    int attn_nchunks_max = 1;   // chunks the partials buffer holds per (sequence, KV head)
     // graphs: [q80][gen]
     cudaGraphExec_t graph[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
     // batched Q8_0 step: quantized activations of every sequence, one graph per batch size
@@ -70,20 +71,14 @@ struct l2c_ctx {
     // tuning
     size_t pf_f32 = 32 << 10, pf_q8 = 64 << 10;  // per CTA; larger leads measured slower in the step graph
     int f32_ctas_per_sm = 1;
-    size_t q8_smem_budget = 220 << 10;  // dynamic shared memory of one Q8_0 GEMV CTA
+    size_t q8_smem_budget = 200 << 10;  // dynamic shared memory of one Q8_0 GEMV CTA (its weight ring)
+    int q8_early = 1;    // 1: Q8_0 GEMVs let the next kernel launch as soon as they start (else at their end)
+    unsigned long long wait_ns = kWaitNs;  // limit of every bounded wait in the kernels
+    int* stall = nullptr;  // test switch read by the Q8_0 q/k/v kernel of layer 0
+    long long oom_after = -1;  // test switch: device allocations after this many fail
     bool pdl = true;     // programmatic dependent launch between the step's kernels
     int late_trigger = 2;  // bit 0 fp32, bit 1 Q8_0: GEMVs let the next kernel launch only near their end
     bool graphs = true;  // replay the step as a CUDA graph (off: plain launches)
-    // persistent Q8_0 step (one launch per token), set up on first use
-    bool use_pstep = false;  // L2C_PERSISTENT=1 turns it on
-    bool pk_tried = false;
-    const void* pk = nullptr;  // nullptr: the per-layer kernels run instead
-    PLayout pl{};
-    int pk_grid = 0, pk_nchunks = 0;
-    size_t pk_pf = 0;  // L2 prefetch lead of the persistent step, bytes per CTA (0: off; measured no gain)
-    void* pk_part = nullptr;
-    unsigned* pk_sync = nullptr;  // {barrier arrivals, CTAs finished, abort flag, pad}
-    char pk_note[512] = {0};      // why the persistent step was dropped, if it was
     std::vector<void*> allocs;
     char msg[512] = {0};
     int status = L2C_OK;  // code of the last failure
@@ -111,6 +106,10 @@ static int fail(l2c_ctx* h, int code, const char* fmt, ...) {
 
 static int dalloc(l2c_ctx* h, void** p, size_t bytes) {
     if (bytes == 0) bytes = 16;
+    if (h->oom_after >= 0 && (long long)h->allocs.size() >= h->oom_after) {
+        *p = nullptr;
+        return fail(h, L2C_E_OOM, "device allocation %zu refused by L2C_TEST_OOM_AFTER", h->allocs.size());
+    }
     cudaError_t e = cudaMalloc(p, bytes);
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -167,19 +166,18 @@ struct GemvShape {
     int rows, K, unit;
 };
 
-// Ring slots per warp: as many as fit next to the input codes, 2..8.
-static Q8Layout q8_layout(const l2c_ctx* h, int K, int gs, size_t rb, int unit, size_t* smem_out) {
-    Q8Layout L = {};
-    L.unit_bytes = (size_t)unit * rb;
-    size_t fixed = (((size_t)K + 15) & ~size_t(15)) + (size_t)(K / gs) * 4 + 16 + (size_t)((K / gs + 1) & ~1) * 8;
-    size_t budget = h->q8_smem_budget;
-    int ns = (int)((budget - fixed - 16 * 8 * Q8_WARPS) / ((size_t)Q8_WARPS * L.unit_bytes));
-    L.nslot = ns < 2 ? 2 : (ns > 8 ? 8 : ns);
-    size_t b = (size_t)Q8_WARPS * L.nslot * L.unit_bytes + fixed;
-    b = (b + 15) & ~size_t(15);
-    b += 8 * (size_t)Q8_WARPS * L.nslot;
-    *smem_out = b;
-    return L;
+// The ring of a Q8_0 GEMV: as many unit slots as fit the shared-memory budget
+// next to the input codes, at least 2, at most the CTA's units.
+static Q8Ring q8_ring(const l2c_ctx* h, int K, int gs, size_t rb, int unit, int units_per_cta, size_t* smem_out) {
+    Q8Ring R = {};
+    R.unit_bytes = (uint32_t)((size_t)unit * rb);
+    const Q8Smem none = q8_smem(0, R.unit_bytes, K, gs);
+    const size_t per_slot = (size_t)R.unit_bytes + 16;  // the slot, its barrier and counters
+    int ns = h->q8_smem_budget > none.total ? (int)((h->q8_smem_budget - none.total) / per_slot) : 0;
+    if (ns > units_per_cta) ns = units_per_cta;
+    R.ns = ns < 2 ? 2 : ns;
+    *smem_out = q8_smem(R.ns, R.unit_bytes, K, gs).total;
+    return R;
 }
 
 template <int MODE>
@@ -206,16 +204,37 @@ static cudaError_t launch_gemv(l2c_ctx* h, bool q80, GemvArgs a, int unit) {
         const size_t smem = (size_t)a.K * 4 + (size_t)rows_max * ks * 4;
         return launch(h->cap, true, k_gemv_f32<MODE>, dim3(grid), dim3(F32_THREADS), smem, a, ks);
     }
-    size_t smem = 0;
-    Q8Layout L = q8_layout(h, a.K, a.gs, a.ld, unit, &smem);
+    // units of 4 rows (two row pairs for QKV and W1/W3), one row where four
+    // would leave the ring fewer than one unit per warp (the wide W2 rows)
+    const bool four = MODE != M_RESID || (size_t)4 * a.ld * Q8_WARPS <= h->q8_smem_budget;
+    const int ur = four ? 4 : 1;
+    const int q8_units = (a.rows + ur - 1) / ur;
     int grid = h->sms;
-    if (grid > units) grid = units;
+    if (grid > q8_units) grid = q8_units;
+    size_t smem = 0;
+    const Q8Ring R = q8_ring(h, a.K, a.gs, a.ld, ur, (q8_units + grid - 1) / grid, &smem);
+    a.early = h->q8_early;
     a.prefetch_bytes = h->pf_q8;
+    const dim3 g(grid), t(Q8_THREADS);
     const bool k64 = a.K % 64 == 0;
-    if (k64 && a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64>, dim3(grid), dim3(32 * Q8_WARPS), smem, a, L);
-    if (k64 && a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32>, dim3(grid), dim3(32 * Q8_WARPS), smem, a, L);
-    if (k64 && a.gs == 128) return launch(h->cap, true, k_gemv_q8<MODE, 128>, dim3(grid), dim3(32 * Q8_WARPS), smem, a, L);
-    return launch(h->cap, true, k_gemv_q8<MODE, 0>, dim3(grid), dim3(32 * Q8_WARPS), smem, a, L);
+#define L2C_Q8_LAUNCH(GS_)                                                                      \
+    return four ? launch(h->cap, true, k_gemv_q8<MODE, GS_, 4>, g, t, smem, a, R)               \
+                : launch(h->cap, true, k_gemv_q8<MODE == M_RESID ? MODE : M_RESID, GS_, 1>, g, t, smem, a, R);
+    if (k64 && a.gs == 64) L2C_Q8_LAUNCH(64)
+    if (k64 && a.gs == 32) L2C_Q8_LAUNCH(32)
+    if (k64 && a.gs == 128) L2C_Q8_LAUNCH(128)
+    L2C_Q8_LAUNCH(0)
+#undef L2C_Q8_LAUNCH
+}
+
+// Every kernel of the Q8_0 step (and of the batched step) asks for the same
+// shared-memory carveout, all of it, so that consecutive kernels never wait
+// for an SM to be reconfigured between them (that would serialize the overlap
+// of programmatic launches).  The fp32 step's kernels keep the default split:
+// their streaming loads run faster with a large L1.
+template <typename Kern>
+static cudaError_t max_carveout(Kern k) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
 }
 
 static int set_smem_limits(l2c_ctx* h) {
@@ -225,13 +244,31 @@ static int set_smem_limits(l2c_ctx* h) {
     CK(cudaFuncSetAttribute(k_gemv_f32<M_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     CK(cudaFuncSetAttribute(k_gemv_f32<M_W13>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     CK(cudaFuncSetAttribute(k_gemv_f32<M_CLS>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
-#define L2C_Q8_ATTR(GS_)                                                                                           \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_QKV, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096)); \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_W13, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+#define L2C_Q8_ATTR(GS_)                                                                                             \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_QKV, GS_, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID, GS_, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096)); \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID, GS_, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096)); \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_W13, GS_, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     L2C_Q8_ATTR(0) L2C_Q8_ATTR(32) L2C_Q8_ATTR(64) L2C_Q8_ATTR(128)
 #undef L2C_Q8_ATTR
+    {
+        cudaError_t e = attn_set_smem_limits();
+        if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "attention smem limit: %s", cudaGetErrorString(e));
+    }
+#define L2C_Q8_CARVE(GS_)                          \
+    CK(max_carveout(k_gemv_q8<M_QKV, GS_, 4>));   \
+    CK(max_carveout(k_gemv_q8<M_RESID, GS_, 4>)); \
+    CK(max_carveout(k_gemv_q8<M_RESID, GS_, 1>)); \
+    CK(max_carveout(k_gemv_q8<M_W13, GS_, 4>));   \
+    CK(max_carveout(k_gemv_q8<M_CLS, GS_, 4>));
+    L2C_Q8_CARVE(0) L2C_Q8_CARVE(32) L2C_Q8_CARVE(64) L2C_Q8_CARVE(128)
+#undef L2C_Q8_CARVE
+    CK(max_carveout(k_bgemm_q8<M_QKV>));
+    CK(max_carveout(k_bgemm_q8<M_RESID>));
+    CK(max_carveout(k_bgemm_q8<M_W13>));
+    CK(max_carveout(k_bgemm_q8<M_CLS>));
+    CK(max_carveout(k_bprep));
     h->bgemm_smem = (size_t)maxopt - 8192;
     CK(cudaFuncSetAttribute(k_bgemm_q8<M_QKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
     CK(cudaFuncSetAttribute(k_bgemm_q8<M_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
@@ -241,8 +278,36 @@ static int set_smem_limits(l2c_ctx* h) {
     return L2C_OK;
 }
 
+// Attention chunks per (sequence, KV head) for a launch over B sequences:
+// about one CTA per SM in fp32 (bandwidth-bound: long chunks, one merge) and
+// four per SM in double (more warps for its arithmetic), each chunk at least
+// attn_min_chunk positions.
+static int attn_nchunks(const l2c_ctx* h, int B, bool dbl) {
+    const int target = dbl ? (h->attn_ctas_f64 > 0 ? h->attn_ctas_f64 : 4 * h->sms)
+                           : (h->attn_ctas > 0 ? h->attn_ctas : h->sms);
+    int nc = (target + h->Hkv * B - 1) / (h->Hkv * B);
+    const int maxc = (h->S + h->attn_min_chunk - 1) / h->attn_min_chunk;
+    if (nc > maxc) nc = maxc;
+    return nc < 1 ? 1 : nc;
+}
+
+// Enqueues the attention of one layer over sequences 0..B-1 (grid z).
+static cudaError_t launch_attention(l2c_ctx* h, cudaStream_t s, bool pdl, bool dbl, const float* q, const float* kc,
+                                    const float* vc, size_t seq_stride, float* out, const int* tp, int B) {
+    AttnArgs t = {};
+    t.q = q; t.kc = kc; t.vc = vc; t.seq_stride = seq_stride;
+    t.out = out; t.tp = tp; t.tp_stride = 2;
+    t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = h->kvd; t.seq_len = h->S;
+    t.nchunks = attn_nchunks(h, B, dbl);
+    t.min_chunk = h->attn_min_chunk;
+    t.part = h->attn_part; t.count = h->attn_cnt;
+    AttnKernel ak = dbl ? attn_kernel_for<double>(h->hs, h->rep) : attn_kernel_for<float>(h->hs, h->rep);
+    const size_t smem = (size_t)(dbl ? attn_smem_for<double>(h->rep) : attn_smem_for<float>(h->rep));
+    return launch(s, pdl, ak, dim3(t.nchunks, h->Hkv, B), dim3(ATTN_THREADS), smem, t);
+}
+
 // Kernels of the step, in order within a layer.
-enum StepKernel : int { SK_QKV = 0, SK_ATTN = 1, SK_WO = 2, SK_W13 = 3, SK_W2 = 4, SK_CLS = 5, SK_STEP = 6 };
+enum StepKernel : int { SK_QKV = 0, SK_ATTN = 1, SK_WO = 2, SK_W13 = 3, SK_W2 = 4, SK_CLS = 5 };
 
 // Enqueues kernel `kind` of layer l (sequence 0) on stream s.
 static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, int l, int seq = 0) {
@@ -261,7 +326,7 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
     h->cap = s;  // launch_gemv enqueues on h->cap
     cudaError_t e = cudaSuccess;
     GemvArgs a = {};
-    a.gs = h->gs; a.tp = tp; a.err = h->err; a.vocab = h->V; a.seq_len = h->S;
+    a.gs = h->gs; a.tp = tp; a.err = h->err; a.vocab = h->V; a.seq_len = h->S; a.wait_ns = h->wait_ns;
     a.d = (int)d; a.kvd = (int)kvd; a.hs = h->hs;
     switch (kind) {
     case SK_QKV:  // RMSNorm + q/k/v + RoPE + cache write
@@ -280,19 +345,12 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
         a.kslot = kslot;
         a.vslot = vslot;
         a.freq = h->freq;
+        if (l == 0 && seq == 0) a.stall = h->stall;
         e = launch_gemv<M_QKV>(h, q80, a, 2);
         break;
-    case SK_ATTN: {
-        AttnArgs t = {};
-        t.q = q; t.kc = kslot; t.vc = vslot; t.seq_stride = (size_t)h->L * S * kvd;
-        t.out = att; t.tp = tp; t.tp_stride = 2;
-        t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = (int)kvd; t.seq_len = h->S;
-        t.nchunks = q80 ? h->attn_nchunks_f64 : h->attn_nchunks;
-        t.part = h->attn_part; t.count = h->attn_cnt; t.err = h->err;
-        AttnKernel ak = q80 ? attn_kernel_for<double>(h->hs, h->rep) : attn_kernel_for<float>(h->hs, h->rep);
-        e = launch(s, true, ak, dim3(t.nchunks, h->Hkv, 1), dim3(128), 0, t);
+    case SK_ATTN:
+        e = launch_attention(h, s, true, q80, q, kslot, vslot, (size_t)h->L * S * kvd, att, tp, 1);
         break;
-    }
     case SK_WO:  // wo + residual
         a.rows = (int)d; a.K = (int)d;
         if (q80) { a.W = h->qWo.p + (size_t)l * d * h->qWo.rb; a.ld = h->qWo.rb; }
@@ -327,77 +385,9 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
     return L2C_OK;
 }
 
-// Sets up the persistent Q8_0 step on first use; leaves h->pk null (the
-// per-layer kernels run) when the shapes or the device do not allow it: a
-// head size / GQA ratio without an instantiation, a width not a multiple of
-// 64, a group size other than 32, 64 or 128, no cooperative launch, or a ring
-// smaller than two of the largest row units.
-static int ensure_pstep(l2c_ctx* h) {
-    if (h->pk_tried) return L2C_OK;
-    h->pk_tried = true;
-    if (!h->use_pstep) return L2C_OK;
-    const void* k = pstep_kernel(h->hs, h->rep);
-    if (!k || h->d % 64 || h->h % 64 || (h->gs != 32 && h->gs != 64 && h->gs != 128)) return L2C_OK;
-    int coop = 0, maxopt = 0;
-    CK(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, h->dev));
-    CK(cudaDeviceGetAttribute(&maxopt, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->dev));
-    if (!coop) return L2C_OK;
-    size_t st = 0;
-    CK(pstep_static_smem(k, &st));
-    const int kmax = h->d > h->h ? h->d : h->h;
-    const PLayout L0 = pstep_layout(0, kmax, h->gs, h->hs, h->rep);
-    const size_t used = st + L0.total + 1024;
-    if ((size_t)maxopt <= used) return L2C_OK;
-    size_t ring = ((size_t)maxopt - used) & ~size_t(127);
-    const size_t cap = env_size("L2C_PSTEP_RING", 0);
-    if (cap && cap < ring) ring = cap & ~size_t(127);
-    const size_t umax = PS_UNIT * h->qWqkv.rb > h->qW2.rb ? PS_UNIT * h->qWqkv.rb : h->qW2.rb;
-    if (((ring / PS_PRODUCERS) & ~size_t(127)) < 2 * umax) return L2C_OK;  // two units per producer slice
-    const PLayout L = pstep_layout((uint32_t)ring, kmax, h->gs, h->hs, h->rep);
-    CK(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total));
-    int occ = 0;
-    CK(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, PS_THREADS, L.total));
-    if (occ < 1) return L2C_OK;
-    int nch = 2 * h->sms / h->Hkv;
-    nch = nch < 1 ? 1 : (nch > 64 ? 64 : nch);
-    int rc;
-    if ((rc = dalloc(h, &h->pk_part, (size_t)h->Hkv * nch * h->rep * (h->hs + 2) * sizeof(double))) ||
-        (rc = dalloc(h, (void**)&h->pk_sync, 16)))
-        return rc;
-    CK(cudaMemsetAsync(h->pk_sync, 0, 16, h->stream));
-    h->pk = k;
-    h->pl = L;
-    h->pk_grid = h->sms;
-    h->pk_nchunks = nch;
-    return L2C_OK;
-}
-
-static int launch_pstep(l2c_ctx* h) {
-    PStepArgs a = {};
-    a.Wqkv = h->qWqkv.p; a.Wo = h->qWo.p; a.W13 = h->qW13.p; a.W2 = h->qW2.p; a.Wcls = h->qWcls.p; a.E = h->qE.p;
-    a.rb_d = h->qWqkv.rb; a.rb_h = h->qW2.rb;
-    a.rms_att = h->rms_att; a.rms_ffn = h->rms_ffn; a.rms_final = h->rms_final; a.freq = h->freq;
-    a.x = h->x; a.q = h->q; a.att = h->att; a.hb = h->hb; a.logits = h->logits;
-    a.kc = h->kc; a.vc = h->vc;
-    a.d = h->d; a.hdim = h->h; a.L = h->L; a.H = h->H; a.Hkv = h->Hkv; a.hs = h->hs; a.kvd = h->kvd;
-    a.V = h->V; a.S = h->S; a.gs = h->gs;
-    a.tp = h->tp; a.amax = h->amax; a.err = h->err;
-    a.bar = h->pk_sync; a.abort_flag = reinterpret_cast<int*>(h->pk_sync + 2);
-    a.part = h->pk_part; a.count = h->attn_cnt; a.nchunks = h->pk_nchunks;
-    a.ring_bytes = h->pl.xq - h->pl.ring;  // the ring is a multiple of 128 bytes
-    a.pf_bytes = h->pk_pf;
-    cudaError_t e = pstep_launch(h->pk, h->pk_grid, a, h->pl, h->cap);
-    if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "persistent step launch: %s", cudaGetErrorString(e));
-    return L2C_OK;
-}
-
 // Enqueues one decode step of sequence 0 on h->cap (being captured).
 static int enqueue_step(l2c_ctx* h, bool q80) {
     int rc;
-    if (q80 && h->use_pstep) {
-        if ((rc = ensure_pstep(h)) != L2C_OK) return rc;
-        if (h->pk) return launch_pstep(h);
-    }
     for (int l = 0; l < h->L; l++)
         for (int k = SK_QKV; k <= SK_W2; k++)
             if ((rc = launch_step_kernel(h, h->cap, k, q80, l)) != L2C_OK) return rc;
@@ -467,20 +457,14 @@ static int bgemm(l2c_ctx* h, cudaStream_t s, int B, const Q8Mat& m, size_t row0,
 static int enqueue_batch_step(l2c_ctx* h, cudaStream_t s, int B) {
     g_pdl = h->pdl;
     const size_t d = h->d, hh = h->h, kvd = h->kvd, S = h->S;
-    AttnKernel ak = attn_kernel_for<double>(h->hs, h->rep);
     int rc;
     for (int l = 0; l < h->L; l++) {
         if ((rc = bprep(h, s, B, h->x, d, (int)d, h->rms_att + (size_t)l * d, l == 0, l == 0 ? h->amax : nullptr)))
             return rc;
         if ((rc = bgemm<M_QKV>(h, s, B, h->qWqkv, (size_t)l * (d + 2 * kvd), (int)(d + 2 * kvd), (int)d, h->q, d, l)))
             return rc;
-        AttnArgs t = {};
-        t.q = h->q; t.kc = h->kc + (size_t)l * S * kvd; t.vc = h->vc + (size_t)l * S * kvd;
-        t.seq_stride = (size_t)h->L * S * kvd; t.out = h->att; t.tp = h->tp; t.tp_stride = 2;
-        t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = (int)kvd; t.seq_len = h->S;
-        t.nchunks = h->attn_nchunks_f64;
-        t.part = h->attn_part; t.count = h->attn_cnt; t.err = h->err;
-        CK(launch(s, true, ak, dim3(t.nchunks, h->Hkv, B), dim3(128), 0, t));
+        CK(launch_attention(h, s, true, true, h->q, h->kc + (size_t)l * S * kvd, h->vc + (size_t)l * S * kvd,
+                            (size_t)h->L * S * kvd, h->att, h->tp, B));
         if ((rc = bprep(h, s, B, h->att, d, (int)d, nullptr, false, nullptr))) return rc;
         if ((rc = bgemm<M_RESID>(h, s, B, h->qWo, (size_t)l * d, (int)d, (int)d, h->x, d, l))) return rc;
         if ((rc = bprep(h, s, B, h->x, d, (int)d, h->rms_ffn + (size_t)l * d, false, nullptr))) return rc;
@@ -509,25 +493,7 @@ static int build_batch_graph(l2c_ctx* h, int B) {
     return L2C_OK;
 }
 
-static int build_graph_once(l2c_ctx* h, bool q80, bool gen);
-
-// Captures the step graph.  If the persistent Q8_0 step cannot be captured
-// (cooperative launches in graphs), the per-layer kernels take its place.
 static int build_graph(l2c_ctx* h, bool q80, bool gen) {
-    if (h->graph[q80][gen]) return L2C_OK;
-    int rc = q80 ? ensure_pstep(h) : L2C_OK;  // allocates: not while capturing
-    if (rc != L2C_OK) return rc;
-    rc = build_graph_once(h, q80, gen);
-    if (rc != L2C_OK && q80 && h->pk) {
-        snprintf(h->pk_note, sizeof(h->pk_note), "persistent step not capturable: %.400s", h->msg);
-        snprintf(h->msg, sizeof(h->msg), "%s", h->pk_note);  // readable through l2c_last_error
-        h->pk = nullptr;
-        rc = build_graph_once(h, q80, gen);
-    }
-    return rc;
-}
-
-static int build_graph_once(l2c_ctx* h, bool q80, bool gen) {
     if (h->graph[q80][gen]) return L2C_OK;
     CK(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
     int rc = enqueue_step(h, q80);
@@ -609,15 +575,13 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
     h->pdl = env_size("L2C_NO_PDL", 0) == 0;
     h->late_trigger = (int)env_size("L2C_LATE_TRIGGER", (size_t)h->late_trigger);
     h->graphs = env_size("L2C_NO_GRAPH", 0) == 0;
-    h->attn_nchunks = (int)env_size("L2C_ATTN_SPLIT", 16);
-    h->use_pstep = env_size("L2C_PERSISTENT", 0) != 0;
-    h->bgemm_stages = (int)env_size("L2C_BGEMM_STAGES", (size_t)h->bgemm_stages);
-    h->pk_pf = env_size("L2C_PSTEP_PF", h->pk_pf);
-    if (h->attn_nchunks < 1) h->attn_nchunks = 16;
-    if (h->attn_nchunks > h->S) h->attn_nchunks = h->S;
-    h->attn_nchunks_f64 = (int)env_size("L2C_ATTN_SPLIT_F64", (size_t)h->attn_nchunks_f64);
-    if (h->attn_nchunks_f64 < 1) h->attn_nchunks_f64 = 24;
-    if (h->attn_nchunks_f64 > h->S) h->attn_nchunks_f64 = h->S;
+    h->attn_ctas = (int)env_size("L2C_ATTN_CTAS", 0);
+    h->attn_ctas_f64 = (int)env_size("L2C_ATTN_CTAS_F64", 0);
+    h->attn_min_chunk = (int)env_size("L2C_ATTN_MIN_CHUNK", (size_t)h->attn_min_chunk);
+    if (h->attn_min_chunk < 1) h->attn_min_chunk = 1;
+    h->q8_early = (int)env_size("L2C_Q8_EARLY", (size_t)h->q8_early);
+    h->wait_ns = env_size("L2C_WAIT_NS", h->wait_ns);
+    if (getenv("L2C_TEST_OOM_AFTER")) h->oom_after = (long long)env_size("L2C_TEST_OOM_AFTER", 0);
     auto bail = [&](int code) { l2c_destroy(h); return code; };
     if (cudaGetDevice(&h->dev) != cudaSuccess) return bail(fail(h, L2C_E_CUDA, "no CUDA device"));
     if (cudaDeviceGetAttribute(&h->sms, cudaDevAttrMultiProcessorCount, h->dev) != cudaSuccess)
@@ -659,8 +623,10 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
     ALLOC(h->gen_count, 4);
     ALLOC(h->idx_out, 4);
     ALLOC(h->key_scratch, 8);
-    ALLOC(h->attn_part, B * (size_t)h->Hkv * (h->attn_nchunks > h->attn_nchunks_f64 ? h->attn_nchunks : h->attn_nchunks_f64) *
-                            h->rep * (h->hs + 2) * sizeof(double));
+    h->attn_nchunks_max = attn_nchunks(h, 1, true) > attn_nchunks(h, 1, false) ? attn_nchunks(h, 1, true)
+                                                                                : attn_nchunks(h, 1, false);
+    ALLOC(h->attn_part, B * (size_t)h->Hkv * h->attn_nchunks_max * h->rep * (h->hs + 2) * sizeof(double));
+    ALLOC(h->stall, 4);
     ALLOC(h->attn_cnt, B * (size_t)h->Hkv * 4);
 #undef ALLOC
     // zero state
@@ -668,6 +634,8 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
         cudaMemsetAsync(h->vc, 0, B * L * S * kvd * 4, h->stream) != cudaSuccess ||
         cudaMemsetAsync(h->attn_cnt, 0, B * (size_t)h->Hkv * 4, h->stream) != cudaSuccess ||
         cudaMemsetAsync(h->err, 0, 4, h->stream) != cudaSuccess ||
+        cudaMemsetAsync(h->stall, getenv("L2C_TEST_STALL") ? 1 : 0, 1, h->stream) != cudaSuccess ||
+        cudaMemsetAsync(reinterpret_cast<char*>(h->stall) + 1, 0, 3, h->stream) != cudaSuccess ||
         cudaMemsetAsync(h->tp, 0, B * 2 * 4, h->stream) != cudaSuccess ||
         cudaMemsetAsync(h->x, 0, B * d * 4, h->stream) != cudaSuccess)
         return bail(fail(h, L2C_E_CUDA, "memset failed"));
@@ -849,40 +817,23 @@ extern "C" int l2c_attention(l2c_ctx* h, const float* q, const float* k, const f
                              float* out) {
     if (!h || !q || !k || !v || !out || pos < 0 || pos >= h->S || (precision != 0 && precision != 1))
         return fail(h, L2C_E_ARG, "attention: need pos in [0, seq_len) and precision 0 or 1");
+    if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)out) & 15)
+        return fail(h, L2C_E_ARG, "attention: buffers must be 16-byte aligned");
     k_set_tp<<<1, 1, 0, h->stream>>>(h->tp, 0, pos);
-    AttnArgs t = {};
-    t.q = q; t.kc = k; t.vc = v; t.seq_stride = 0;
-    t.out = out; t.tp = h->tp; t.tp_stride = 2;
-    t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = h->kvd; t.seq_len = h->S;
-    t.nchunks = precision ? h->attn_nchunks_f64 : h->attn_nchunks;
-    t.part = h->attn_part; t.count = h->attn_cnt; t.err = h->err;
-    AttnKernel ak = precision ? attn_kernel_for<double>(h->hs, h->rep) : attn_kernel_for<float>(h->hs, h->rep);
-    CK(launch(h->stream, false, ak, dim3(t.nchunks, h->Hkv, 1), dim3(128), 0, t));
+    CK(launch_attention(h, h->stream, false, precision != 0, q, k, v, 0, out, h->tp, 1));
     return L2C_OK;
 }
 
 extern "C" int l2c_time_kernel(l2c_ctx* h, int kind, int q80, int iters, float* avg_ms) {
-    if (!h || kind < SK_QKV || kind > SK_STEP || iters < 1 || !avg_ms) return fail(h, L2C_E_ARG, "time_kernel: bad arguments");
+    if (!h || kind < SK_QKV || kind > SK_CLS || iters < 1 || !avg_ms) return fail(h, L2C_E_ARG, "time_kernel: bad arguments");
     if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
-    if (kind == SK_STEP) {
-        int rc = q80 ? ensure_pstep(h) : L2C_OK;
-        if (rc) return rc;
-        if (!q80 || !h->pk) return fail(h, L2C_E_STATE, "time_kernel: the step does not run as one kernel here");
-    }
     cudaEvent_t e0, e1;
     CK(cudaEventCreate(&e0));
     CK(cudaEventCreate(&e1));
     int rc = L2C_OK;
     cudaError_t er = cudaEventRecord(e0, h->stream);
     for (int i = 0; i < iters && rc == L2C_OK && er == cudaSuccess; i++) {
-        if (kind == SK_STEP) {
-            cudaStream_t saved = h->cap;
-            h->cap = h->stream;
-            rc = launch_pstep(h);
-            h->cap = saved;
-        } else {
-            rc = launch_step_kernel(h, h->stream, kind, q80 != 0, kind == SK_CLS ? 0 : i % h->L);
-        }
+        rc = launch_step_kernel(h, h->stream, kind, q80 != 0, kind == SK_CLS ? 0 : i % h->L);
     }
     if (er == cudaSuccess) er = cudaEventRecord(e1, h->stream);
     if (er == cudaSuccess) er = cudaEventSynchronize(e1);
@@ -929,7 +880,13 @@ extern "C" int l2c_q80_group_dots(l2c_ctx* h, const int8_t* qw, const int8_t* qx
     if (!h || !qw || !qx || !out || rows < 0 || K <= 0 || gs < 16 || gs > 512 || gs % 16 || K % gs)
         return fail(h, L2C_E_ARG, "group_dots: need K %% gs == 0 and gs a multiple of 16 in [16,512]");
     if (rows == 0) return L2C_OK;
-    k_group_dots<<<(rows + 7) / 8, 256, 0, h->stream>>>(qw, qx, rows, K, gs, out);
+    const bool hot = K % 64 == 0 && K <= 32768 && (gs == 32 || gs == 64 || gs == 128) &&
+                     ((uintptr_t)qw & 15) == 0 && ((uintptr_t)qx & 15) == 0;
+    const dim3 grid((rows + 7) / 8), block(256);
+    if (hot && gs == 32) k_group_dots64<32><<<grid, block, (size_t)K, h->stream>>>(qw, qx, rows, K, out);
+    else if (hot && gs == 64) k_group_dots64<64><<<grid, block, (size_t)K, h->stream>>>(qw, qx, rows, K, out);
+    else if (hot && gs == 128) k_group_dots64<128><<<grid, block, (size_t)K, h->stream>>>(qw, qx, rows, K, out);
+    else k_group_dots<<<grid, block, 0, h->stream>>>(qw, qx, rows, K, gs, out);
     CK(cudaGetLastError());
     return L2C_OK;
 }
@@ -985,7 +942,6 @@ extern "C" int l2c_sync(l2c_ctx* h) {
     if (e) {
         CK(cudaMemset(h->err, 0, 4));
         if (e & DERR_TIMEOUT) {  // an abandoned step can leave barriers and counters mid-way
-            if (h->pk_sync) CK(cudaMemset(h->pk_sync, 0, 16));
             CK(cudaMemset(h->attn_cnt, 0, (size_t)h->max_batch * h->Hkv * 4));
         }
         return fail(h, L2C_E_DEVICE, "device error word 0x%x:%s%s%s%s", e, (e & DERR_TOKEN) ? " token" : "",
@@ -993,14 +949,6 @@ extern "C" int l2c_sync(l2c_ctx* h) {
                     (e & DERR_NAN) ? " nan" : "");
     }
     return L2C_OK;
-}
-
-extern "C" int l2c_persistent(l2c_ctx* h) {
-    if (!h) return L2C_E_ARG;
-    if (!h->gs) return 0;
-    int rc = ensure_pstep(h);
-    if (rc) return rc;
-    return h->pk ? 1 : 0;
 }
 
 extern "C" void* l2c_stream(l2c_ctx* h) { return h ? (void*)h->stream : nullptr; }

@@ -159,10 +159,13 @@ L2C_API int l2c_quantize_q80(l2c_ctx* h, const float* x_dev, int64_t n, int gs, 
 
 /*
  * l2c_q80_group_dots - the exact int32 dot product of every (row, group) of
- * Q8_0 codes, computed by the same dp4a chunk loop as the Q8_0 matvec:
- * out[r][g] = sum_k qw[r][g*gs+k] * qx[g*gs+k].  qw_dev [rows][K] int8,
- * qx_dev [K] int8, out_dev [rows][K/gs] int32; K % gs == 0, gs a multiple of
- * 16 (16..512).  Asynchronous on the handle's stream.
+ * Q8_0 codes: out[r][g] = sum_k qw[r][g*gs+k] * qx[g*gs+k].  For gs = 32, 64
+ * or 128 with K % 64 == 0 (K <= 32768, 16-byte aligned qw_dev and qx_dev) it
+ * runs the Q8_0 matvec's own 64-byte chunk routine (the one every Q8_0 step
+ * uses at those group sizes); otherwise the generic matvec's 16-byte chunk
+ * loop.  qw_dev [rows][K] int8, qx_dev [K] int8, out_dev [rows][K/gs] int32;
+ * K % gs == 0, gs a multiple of 16 (16..512).  Asynchronous on the handle's
+ * stream.
  */
 L2C_API int l2c_q80_group_dots(l2c_ctx* h, const int8_t* qw_dev, const int8_t* qx_dev, int rows, int K, int gs,
                        int32_t* out_dev);
@@ -188,10 +191,11 @@ L2C_API int l2c_kv_reset(l2c_ctx* h, int seq);
  * head g = i / (n_heads / n_kv_heads), scores q_i . k_t / sqrt(head_size)
  * over t = 0..pos, softmax, and out_i = sum_t a_t v_t.  q_dev [n_heads *
  * head_size] (already rotated), k_dev and v_dev [>= pos+1][kv_dim] (one
- * layer's caches), out_dev [n_heads * head_size]; all device fp32.
- * precision: 0 accumulates in fp32 (as the fp32 step does), 1 in double (as
- * the Q8_0 step does).  pos must be in [0, seq_len).  Uses the handle's
- * scratch; asynchronous on the handle's stream.
+ * layer's caches), out_dev [n_heads * head_size]; all device fp32, 16-byte
+ * aligned (L2C_E_ARG otherwise).  precision: 0 accumulates in fp32 (as the
+ * fp32 step does), 1 in double (as the Q8_0 step does).  pos must be in
+ * [0, seq_len).  Uses the handle's scratch and position split (the same as
+ * the decode step's); asynchronous on the handle's stream.
  */
 L2C_API int l2c_attention(l2c_ctx* h, const float* q_dev, const float* k_dev, const float* v_dev, int pos,
                           int precision, float* out_dev);
@@ -209,14 +213,19 @@ L2C_API int l2c_attention(l2c_ctx* h, const float* q_dev, const float* k_dev, co
  * scratch), so this entry point takes every shape argument explicitly and
  * calls no cudaMalloc, cudaFree or allocating library routine.
  *
- * Computes exactly what l2c_attention computes, with the same kernel: for
+ * Computes what l2c_attention computes, with the same kernel but its own
+ * position split (chunks of 64 positions, where a handle picks the split from
+ * the SM count), so results agree with l2c_attention within rounding: for
  * query head i and KV head g = i / (n_heads / n_kv_heads), scores
  * q_i . k_t / sqrt(head_size) over t = 0..pos, softmax, out_i = sum a_t v_t.
  * q_dev [n_heads * head_size], k_dev and v_dev [>= pos+1][n_kv_heads *
- * head_size], out_dev [n_heads * head_size]: device fp32, owned by the
- * caller.  precision: 0 = fp32 accumulation, 1 = double.  Supported head
- * sizes and GQA ratios are those of l2c_create.  Enqueued on cuda_stream
- * (NULL = the legacy stream); returns before the kernels finish.
+ * head_size], out_dev [n_heads * head_size]: device fp32, 16-byte aligned,
+ * owned by the caller.  precision: 0 = fp32 accumulation, 1 = double.
+ * Supported head sizes and GQA ratios are those of l2c_create.  Enqueued on
+ * cuda_stream (NULL = the legacy stream); returns before the kernels finish.
+ * The kernels wait on nothing (no barrier across CTAs; the last CTA of a KV
+ * head to finish merges its chunks), so there is no device-side error to
+ * report.
  *
  * Scratch: a fixed 4 MiB device array in the library (every GPU that loads
  * the library holds it until the process exits).  A call needs
@@ -230,10 +239,14 @@ L2C_API int l2c_attention(l2c_ctx* h, const float* q_dev, const float* k_dev, co
  * clears the counters it uses before its kernel runs.
  *
  * Set-up: the first call on a device, with that device current, looks up the
- * array's device address (cudaGetSymbolAddress) and caches it; make that
- * first call before capturing work on the device's streams.
- * Errors: L2C_E_ARG (null pointer, bad shape, unsupported head size or ratio),
- * L2C_E_SCRATCH, L2C_E_CUDA.
+ * array's device address (cudaGetSymbolAddress) and sets the attention
+ * kernels' shared-memory limit (cudaFuncSetAttribute); it does so again in a
+ * new CUDA context (after a device reset, the library's module and its array
+ * are loaded anew).  Make
+ * that first call before capturing work on the device's streams.  Devices
+ * with an ordinal of 64 or more are not supported (L2C_E_CUDA).
+ * Errors: L2C_E_ARG (null or unaligned pointer, bad shape, unsupported head
+ * size or ratio), L2C_E_SCRATCH, L2C_E_CUDA.
  */
 L2C_API int l2c_attention_noalloc(const float* q_dev, const float* k_dev, const float* v_dev, int n_heads,
                                   int n_kv_heads, int head_size, int pos, int precision, float* out_dev,
@@ -245,28 +258,11 @@ L2C_API int l2c_attention_noalloc(const float* q_dev, const float* k_dev, const 
  * stores the average time per launch in ms (two CUDA events around the
  * loop).  Launch i uses layer i % n_layers, so consecutive launches stream
  * different weights.  kind: 0 = RMSNorm+QKV+RoPE, 1 = attention, 2 = wo,
- * 3 = RMSNorm+W1/W3+SwiGLU, 4 = W2, 5 = final RMSNorm+classifier,
- * 6 = the whole Q8_0 step as one persistent kernel (q80 = 1 only; L2C_E_STATE
- * where l2c_persistent() is 0).  The kernels use the handle's current
+ * 3 = RMSNorm+W1/W3+SwiGLU, 4 = W2, 5 = final RMSNorm+classifier.  The kernels use the handle's current
  * token/position and update its state (KV slot, activations) as in a step.
  * Blocks.
  */
 L2C_API int l2c_time_kernel(l2c_ctx* h, int kind, int q80, int iters, float* avg_ms);
-
-/*
- * l2c_persistent - whether the single-sequence Q8_0 step (l2c_forward_q80,
- * l2c_generate with q80) runs as ONE persistent kernel: one CTA per SM that
- * streams every weight row of the step through a shared-memory ring while
- * grid barriers order the layer phases.  The arithmetic and the results are
- * those of the per-layer kernels.  It does where the Q8_0 group size is 32, 64
- * or 128, dim and hidden_dim are multiples of 64, (head_size, n_heads /
- * n_kv_heads) has an instantiation, the device supports cooperative launches,
- * the ring fits, and the environment variable L2C_PERSISTENT=1 was set at
- * l2c_create (off by default: on the 7B shape the per-layer kernels are
- * faster).  Sets it up on first call.
- * Returns 1 or 0 (0 too before l2c_enable_q80), or a negative error code.
- */
-L2C_API int l2c_persistent(l2c_ctx* h);
 
 /* l2c_sync - waits for the handle's stream, then reads and clears the
  * device error word: L2C_E_DEVICE if a kernel recorded an error since the

@@ -58,15 +58,24 @@ def test_quantize_weight_blob_bitexact(env):
     assert np.array_equal(s.cpu().numpy(), s_ref)
 
 
-@pytest.mark.parametrize("rows,K,gs", [(7, 288, 32), (33, 4096, 64), (5, 11008, 64), (3, 768, 64), (9, 256, 128)])
+# K % 64 == 0 with gs 32 / 64 / 128 runs the Q8_0 matvec's own 64-byte chunk
+# routine (the 7B widths 4096 and 11008 among them); the others the 16-byte loop.
+@pytest.mark.parametrize("rows,K,gs", [(7, 288, 32), (33, 4096, 64), (5, 11008, 64), (3, 768, 64), (9, 256, 128),
+                                       (6, 4096, 32), (4, 11008, 32), (5, 4096, 128), (3, 11008, 128),
+                                       (4, 160, 32), (3, 96, 16)])
 def test_group_dots_bitexact(env, rows, K, gs):
     torch, l2c, dec = env
-    rng = np.random.default_rng(rows * K)
+    rng = np.random.default_rng(rows * K + gs)
     qw = rng.integers(-127, 128, (rows, K)).astype(np.int8)
     qx = rng.integers(-127, 128, K).astype(np.int8)
+    # extreme groups: +-127 everywhere gives |dot| = gs * 127^2 (both signs)
     qw[0, :] = -127
-    qx[:gs] = -127   # extreme group: 64 * 127^2
+    qx[:gs] = -127
+    qx[gs:2 * gs] = 127
+    if rows > 1:
+        qw[1, :] = 127
     ref = oracle.q80_group_dots(qw, qx, gs)
+    assert ref[0, 0] == gs * 127 * 127 and ref[0, 1] == -gs * 127 * 127
     out = torch.empty((rows, K // gs), dtype=torch.int32, device="cuda")
     dec.q80_group_dots(torch.from_numpy(qw).cuda(), torch.from_numpy(qx).cuda(), gs, out)
     dec.sync()

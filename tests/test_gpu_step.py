@@ -85,23 +85,6 @@ def test_kv_cache_slots(gpu):
         dec.close()
 
 
-@pytest.mark.parametrize("gs", [0, 32])
-def test_greedy_sequence(gpu, gs):
-    """Greedy decoding (token fed back on the device) against the oracle's greedy chain."""
-    spec = synth.TINY if not gs else synth.M15
-    steps = 256 if not gs else 128
-    tol = TOL_F32 if not gs else TOL_Q80
-    dec, orc = _pair(gpu, spec, gs)
-    toks = dec.generate(1, steps, q80=bool(gs))
-    ref_toks, ref_logits = orc.generate(1, steps, q80=bool(gs))
-    mism = np.nonzero(toks != ref_toks)[0]
-    if mism.size:
-        t = int(mism[0])
-        gap = top2_gap(ref_logits[t])
-        assert gap < tol * np.abs(ref_logits[t]).max(), (t, gap)
-    dec.close()
-
-
 def test_prefilled_cache_chunks(gpu):
     """A step at positions that span several attention chunks, on a cache prefilled with N(0,1)."""
     torch, l2c = gpu
@@ -133,87 +116,4 @@ def test_bad_arguments(gpu):
     with pytest.raises(l2c.L2CError):
         dec.generate(1, spec.seq_len + 1)
     dec.sync()
-    dec.close()
-
-
-# ---- the single-sequence Q8_0 step as one persistent kernel ------------------
-# Eligible shapes (widths multiples of 64, gs 32/64/128) run the whole step as
-# one launch; the per-layer kernels (L2C_PERSISTENT=0) must give the same
-# answers, and both must match the oracle to the Q8_0 bound above.
-Q64G = synth.ModelSpec("q64g", 256, 768, 2, 4, 1, 700, 200, 0, seed=15)
-
-
-def _dec(gpu, spec, gs, persistent, monkeypatch):
-    torch, l2c = gpu
-    monkeypatch.setenv("L2C_PERSISTENT", "1" if persistent else "0")
-    dec = l2c.Decoder(spec.cfg, torch.from_numpy(synth.blob(spec)).cuda(), spec.shared_weights)
-    dec.enable_q80(gs)
-    assert dec.persistent() == persistent
-    return dec
-
-
-@pytest.mark.parametrize("spec,gs", [(Q64, 32), (Q64, 128), (Q64G, 64)], ids=["q64-gs32", "q64-gs128", "q64g-gs64"])
-def test_q80_persistent_matches_oracle_and_layers(gpu, spec, gs, monkeypatch):
-    steps = 60
-    toks = synth.tokens(spec.seed, 22, steps, spec.vocab_size)
-    orc = oracle.Model(spec.cfg, synth.blob(spec), spec.shared_weights)
-    orc.enable_q80(gs)
-    dp = _dec(gpu, spec, gs, True, monkeypatch)
-    dl = _dec(gpu, spec, gs, False, monkeypatch)
-    for p, t in enumerate(toks):
-        got = dp.forward(int(t), p, q80=True).cpu().numpy()
-        lay = dl.forward(int(t), p, q80=True).cpu().numpy()
-        ref = orc.forward(int(t), p, q80=True)
-        assert rel_err(got, ref) <= 1e-5, p
-        assert rel_err(got, lay) <= 1e-5, p
-    k, v = dp.kv_read(steps)
-    kr, vr = orc.kv_read(steps)
-    assert rel_err(k, kr) <= 1e-6 and rel_err(v, vr) <= 1e-6
-    assert dp.persistent(), dp._msg()  # still the persistent kernel once the step graph exists
-    dp.close()
-    dl.close()
-
-
-def test_q80_persistent_prefilled_chunks(gpu, monkeypatch):
-    """Positions that split into many attention chunks, on a prefilled cache."""
-    torch, _ = gpu
-    spec = Q64G
-    dec = _dec(gpu, spec, 32, True, monkeypatch)
-    orc = oracle.Model(spec.cfg, synth.blob(spec), spec.shared_weights)
-    orc.enable_q80(32)
-    for P in (1, 63, 64, 65, 130, 199):
-        k, v = synth.kv_prefill(spec, seq=0, n_pos=P)
-        dec.kv_load(torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
-        orc.kv_load(k, v)
-        got = dec.forward(17, P, q80=True).cpu().numpy()
-        ref = orc.forward(17, P, q80=True)
-        assert rel_err(got, ref) <= 1e-5, P
-    dec.close()
-
-
-def test_q80_persistent_greedy(gpu, monkeypatch):
-    spec = Q64
-    dec = _dec(gpu, spec, 64, True, monkeypatch)
-    orc = oracle.Model(spec.cfg, synth.blob(spec), spec.shared_weights)
-    orc.enable_q80(64)
-    toks = dec.generate(3, 150, q80=True)
-    assert dec.persistent(), dec._msg()
-    ref_toks, ref_logits = orc.generate(3, 150, q80=True)
-    mism = np.nonzero(toks != ref_toks)[0]
-    if mism.size:
-        t = int(mism[0])
-        assert top2_gap(ref_logits[t]) < TOL_Q80 * np.abs(ref_logits[t]).max(), t
-    dec.close()
-
-
-def test_q80_persistent_timer(gpu, monkeypatch):
-    _, l2c = gpu
-    dec = _dec(gpu, Q64, 32, True, monkeypatch)
-    dec.forward(5, 3, q80=True)
-    assert dec.time_kernel(l2c.K_STEP, True, 3) > 0.0
-    with pytest.raises(l2c.L2CError):
-        dec.time_kernel(l2c.K_STEP, False, 1)  # the fp32 step has no single-kernel form
-    dec.close()
-    # shapes outside the persistent kernel's set keep the per-layer kernels
-    dec = _dec(gpu, synth.M15, 32, False, monkeypatch)
     dec.close()
