@@ -641,11 +641,12 @@ __device__ __forceinline__ double widen_f32_scaled(float x) {
 
 // UR rows (records at rec, stride rb) against the input codes xq: the exact
 // group dots of q8_chunk_dots, each times the row's group scale and the
-// input's group scale, summed per lane in double.  sxs holds the input scales
-// times 2^896 and the row scales are widened as sw * 2^-896, so each term is
-// the double product (ival * sw) * sx.  Requires K % 64 == 0.
+// input's group scale, summed per lane in double.  The input scales (fp32,
+// xs) are converted once per chunk and times 2^896, the row scales widened
+// as sw * 2^-896, so each term is the double product (ival * sw) * sx.
+// Requires K % 64 == 0.
 template <int GS, int UR>
-__device__ __forceinline__ void q8_rows_dot64(const uint8_t* rec, size_t rb, const int8_t* xq, const double* sxs,
+__device__ __forceinline__ void q8_rows_dot64(const uint8_t* rec, size_t rb, const int8_t* xq, const float* xs,
                                               int K, double (&acc)[UR]) {
     const int lane = threadIdx.x & 31;
     const int n64 = K >> 6;
@@ -660,9 +661,9 @@ __device__ __forceinline__ void q8_rows_dot64(const uint8_t* rec, size_t rb, con
         q8_chunk_x(xq, t, in, rot, xv);
         double sx0 = 0.0, sx1 = 0.0;
         if (in) {
-            if (GS == 64) sx0 = sxs[t];
-            else if (GS == 32) { sx0 = sxs[2 * t]; sx1 = sxs[2 * t + 1]; }
-            else sx0 = sxs[t >> 1];
+            if (GS == 64) sx0 = (double)xs[t] * 0x1p896;
+            else if (GS == 32) { sx0 = (double)xs[2 * t] * 0x1p896; sx1 = (double)xs[2 * t + 1] * 0x1p896; }
+            else sx0 = (double)xs[t >> 1] * 0x1p896;
         }
 #pragma unroll
         for (int r = 0; r < UR; r++) {
@@ -760,11 +761,21 @@ struct Q8Prologue {
         const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
         const bool resid = a.emb && blockIdx.x == 0;  // layer 0: CTA 0 stores the embedding row as x
         if (!NORM) {
-            for (int it = 0; it < steps; it++) {
-                const float4 x = load_value(a, eq, es, it);
-                if (resid && chunk(it) < a.K / 64)
-                    reinterpret_cast<float4*>(a.x_resid)[(chunk(it) * 64 + 4 * (threadIdx.x & 15)) / 4] = x;
-                quantize(a, x, it, xq, xsc);
+            // the loads of a block of steps first, all in flight, then the codes
+            constexpr int RB = 12;
+            for (int i0 = 0; i0 < steps; i0 += RB) {
+                float4 xs[RB];
+#pragma unroll
+                for (int k = 0; k < RB; k++)
+                    xs[k] = i0 + k < steps ? load_value(a, eq, es, i0 + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int k = 0; k < RB; k++) {
+                    if (i0 + k >= steps) break;  // warp-uniform
+                    const int it = i0 + k;
+                    if (resid && chunk(it) < a.K / 64)
+                        reinterpret_cast<float4*>(a.x_resid)[(chunk(it) * 64 + 4 * (threadIdx.x & 15)) / 4] = xs[k];
+                    quantize(a, xs[k], it, xq, xsc);
+                }
             }
             return;
         }
@@ -925,10 +936,10 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
     if (fast) pro.post(a, eq, es, xq, xsc, red);
     else q8_quantize_input<NORM>(a, eq, es, xq, xsc, red);
     __syncthreads();
-    // input scales in double; for the 64-byte path times 2^896 (see q8_rows_dot64)
-    for (int g = threadIdx.x; g < K / gs; g += Q8_THREADS)
-        sxd[g] = GS != 0 ? (double)xsc[g] * 0x1p896 : (double)xsc[g];
-    __syncthreads();
+    if (GS == 0) {  // the generic loop takes the input scales in double
+        for (int g = threadIdx.x; g < K / gs; g += Q8_THREADS) sxd[g] = (double)xsc[g];
+        __syncthreads();
+    }
 
     // ---- this warp's units
     constexpr int GRP = 32 / UR;     // lanes that hold one row's total after the reduce-scatter
@@ -969,7 +980,7 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
         const uint8_t* base = smem + (size_t)s * ub;
         double acc[UR];
         if (GS != 0) {
-            q8_rows_dot64<GS == 0 ? 64 : GS, UR>(base, rb, xq, sxd, K, acc);
+            q8_rows_dot64<GS == 0 ? 64 : GS, UR>(base, rb, xq, xsc, K, acc);
         } else {
 #pragma unroll
             for (int r = 0; r < UR; r++) acc[r] = 0.0;
