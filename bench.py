@@ -388,10 +388,10 @@ def run_ours(args, rank, world, local_rank):
         for kind, name in enumerate(KERNEL_NAMES):
             iters = 2 * SPEC.n_layers if kind != 5 else 8
             dec.time_kernel(kind, q80, max(4, iters // 4))  # warm
-            ms = dec.time_kernel(kind, q80, iters)
+            kms = dec.time_kernel(kind, q80, iters)
             by = kernel_bytes(kind, q80, kpos)
-            rows[name] = {"avg_launch_us": 1e3 * ms, "bytes_per_launch": by, "gbs": by / ms / 1e6,
-                          "frac_of_measured_hbm": by / ms / 1e6 / peak, "launches_timed": iters}
+            rows[name] = {"avg_launch_us": 1e3 * kms, "bytes_per_launch": by, "gbs": by / kms / 1e6,
+                          "frac_of_measured_hbm": by / kms / 1e6 / peak, "launches_timed": iters}
         kernels["q8_0" if q80 else "fp32"] = rows
     kernels["note"] = (f"each kernel alone, back to back over the layers' weights, at pos {kpos} "
                        f"(attention reads K/V of positions 0..{kpos})")

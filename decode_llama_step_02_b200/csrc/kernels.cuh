@@ -52,12 +52,13 @@ struct GemvArgs {
     const int* tp;           // {token, pos}
     unsigned long long* amax;  // argmax key (classifier); reset by layer 0
     int* err;
-    size_t prefetch_bytes;   // fp32: L2 prefetch issued before the dependency wait
+    size_t prefetch_bytes;   // L2 prefetch of the CTA's first weights, issued before the dependency wait
     int late_trigger;        // fp32: 1 = let the next kernel launch only after this CTA's last weight loads
-    int early;               // Q8_0: 1 = let the next kernel launch as soon as this one starts
+    int early;               // Q8_0: 1 = let the next kernel launch as soon as this one starts (else at its end)
     unsigned long long wait_ns;  // limit of every barrier wait
     int* stall;              // test switch (Q8_0): CTA 0 withholds one ring copy once if *stall != 0
 };
+
 
 // ----------------------------------------------------------------- epilogues --
 
@@ -815,112 +816,83 @@ struct Q8Prologue {
 constexpr int Q8_WARPS = 8;                  // warps of a Q8_0 GEMV CTA
 constexpr int Q8_THREADS = 32 * Q8_WARPS;
 
-// The CTA's weight ring: `ns` slots of one unit (UR row records) each.
+// A Q8_0 GEMV CTA's rings: `ns` slots per warp of one unit (UNIT row
+// records) each.
 struct Q8Ring {
     int ns;
-    uint32_t unit_bytes;  // UR * record bytes
+    uint32_t unit_bytes;  // UNIT * record bytes
 };
 
-// Dynamic shared memory of a Q8_0 GEMV CTA: the ring, the input codes and
-// scales, the ring barriers, and per slot the number of units issued into it
-// and the number consumed.
+// Q8_0 GEMV.  A unit is one row record, or a row pair for QKV and W1/W3
+// (UNIT rows); the CTA owns a contiguous range of units and warp w takes its
+// units w, w + 8, ..., streaming them with 1-D bulk copies through its own
+// ring of `ns` shared-memory slots: its parity waits follow its own copies in
+// order, and it refills a slot as soon as it has read it.  Before the
+// dependency wait the kernel loads what no earlier kernel of the step writes
+// (the RMSNorm gain, the embedding row on layer 0, the RoPE table) and
+// prefetches the first a.prefetch_bytes of the CTA's weights into L2; right
+// after it, the rings are filled and the input is quantized (the listing's
+// rule, bit-exact) into shared codes.  Then per unit: exact int32 group dots
+// by dp4a, (ival * sw) * sx summed per lane in double, one reduce-scatter for
+// the unit's row sums, the epilogue.  GS is the group size of the
+// 64-byte-per-lane dot (32, 64 or 128, K % 64 == 0), or 0 for the generic
+// 16-byte-per-lane loop.  Every wait is bounded (a.wait_ns); a warp that gives
+// up records DERR_TIMEOUT, makes the others stop (a shared abort flag) and
+// lets its copies in flight land before the CTA leaves.  Dynamic shared
+// memory: the rings [Q8_WARPS][ns][unit], the input codes and scales, the
+// barriers.
 struct Q8Smem {
-    size_t xq, xsc, sxd, bars, cnt, total;
+    size_t xq, xsc, sxd, bars, total;
 };
 
 __host__ __device__ inline Q8Smem q8_smem(int ns, uint32_t unit_bytes, int K, int gs) {
     Q8Smem m;
     const size_t ng = (size_t)(K / gs);
-    m.xq = (size_t)ns * unit_bytes;
+    m.xq = (size_t)Q8_WARPS * ns * unit_bytes;
     m.xsc = m.xq + (((size_t)K + 15) & ~size_t(15));
     m.sxd = m.xsc + ((ng * 4 + 15) & ~size_t(15));
-    m.bars = m.sxd + ng * 8;
-    m.cnt = m.bars + 8 * (size_t)ns;
-    m.total = m.cnt + 8 * (size_t)ns;
+    m.bars = m.sxd + ng * 8;  // the double scales: generic path only
+    m.total = m.bars + 8 * (size_t)Q8_WARPS * ns;
     return m;
 }
 
-// Q8_0 GEMV.  A unit is UR consecutive row records (for QKV and W1/W3, UR/2
-// row pairs); the CTA owns a contiguous range of units and streams them
-// through a ring of `ns` shared-memory slots with 1-D bulk copies: unit k
-// goes to slot k % ns and is consumed by warp k % Q8_WARPS, and the warp that
-// consumes a unit refills its slot at once with unit k + ns.  The first `ns`
-// copies are issued at the start, before the dependency wait (weights do not
-// depend on the previous kernel).  After the wait the warps quantize the input
-// (the listing's rule, bit-exact) into shared codes, then run their units:
-// exact int32 group dots by dp4a, (ival * sw) * sx summed per lane in double,
-// one reduce-scatter for the UR row sums, and the epilogues of the unit's rows
-// (or row pairs) on separate lanes.  GS is the group size of the
-// 64-byte-per-lane dot (32, 64 or 128, K % 64 == 0), or 0 for the generic
-// 16-byte-per-lane loop.  Every wait is bounded (a.wait_ns); a CTA that gives
-// up records DERR_TIMEOUT, stops in all its warps (a shared abort flag), and
-// leaves only after every copy it issued has landed.
-template <int MODE, int GS, int UR>
+template <int MODE, int GS>
 __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, const Q8Ring R) {
     extern __shared__ __align__(128) uint8_t smem[];
-    constexpr bool PAIRS = MODE == M_QKV || MODE == M_W13;
-    static_assert(!PAIRS || UR % 2 == 0, "row pairs");
+    constexpr int UNIT = (MODE == M_QKV || MODE == M_W13) ? 2 : 1;
     __shared__ double red[Q8_WARPS];
     __shared__ unsigned long long best_s[Q8_WARPS];
     __shared__ double2 rope_cs[MODE == M_QKV ? 128 : 1];
     __shared__ int abort_s;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int K = a.K, gs = a.gs, ns = R.ns;
-    const uint32_t ub = R.unit_bytes;
+    const uint32_t ub = R.unit_bytes;  // UNIT * record bytes
     const size_t rb = a.ld;
     const Q8Smem lay = q8_smem(ns, ub, K, gs);
+    uint8_t* slots = smem + (size_t)warp * ns * ub;
     int8_t* xq = reinterpret_cast<int8_t*>(smem + lay.xq);
     float* xsc = reinterpret_cast<float*>(smem + lay.xsc);
-    double* sxd = reinterpret_cast<double*>(smem + lay.sxd);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars);
-    volatile int* issued = reinterpret_cast<volatile int*>(smem + lay.cnt);  // units issued into slot s
-    int* used = const_cast<int*>(issued) + ns;                                 // units consumed from slot s
-    const int units = (a.rows + UR - 1) / UR;
+    double* sxd = reinterpret_cast<double*>(smem + lay.sxd);  // generic path only
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars) + warp * ns;
+    const int units = a.rows / UNIT;
     const int u0 = (int)((long long)units * blockIdx.x / gridDim.x);
     const int u1 = (int)((long long)units * (blockIdx.x + 1) / gridDim.x);
-    const int n = u1 - u0;
-    const uint8_t* src = static_cast<const uint8_t*>(a.W) + (size_t)u0 * ub;
+    const int nmine = (u1 - u0 - warp + Q8_WARPS - 1) / Q8_WARPS;  // units of this warp
+    const uint8_t* Wb = static_cast<const uint8_t*>(a.W);
     const uint64_t pol = policy_evict_first();
-    // bytes of unit k of this CTA (the last unit of the matrix may be short)
-    auto unit_bytes = [&](int k) {
-        const int r0 = (u0 + k) * UR;
-        const int nr = min(UR, a.rows - r0);
-        return (uint32_t)((size_t)nr * rb);
-    };
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < ns; s++) {
-            mbar_init(&full[s], 1);
-            issued[s] = 0;
-            st_release_cta(&used[s], 0);
-        }
-        abort_s = 0;
+    auto unit_src = [&](int k) { return Wb + (size_t)(u0 + warp + k * Q8_WARPS) * ub; };
+    if (lane == 0) {
+        for (int s = 0; s < ns; s++) mbar_init(&full[s], 1);
         mbar_fence_init();
-        // test switch: withhold the first copy of CTA 0 once (a wait then runs out)
-        const bool skip0 = a.stall && blockIdx.x == 0 && n > 0 && atomicExch(a.stall, 0);
-        for (int k = 0; k < ns && k < n; k++) {
-            if (k == 0 && skip0) continue;
-            const uint32_t by = unit_bytes(k);
-            mbar_arrive_expect_tx(&full[k], by);
-            bulk_g2s(smem + (size_t)k * ub, src + (size_t)k * ub, by, &full[k], pol);
-            issued[k] = 1;
-        }
-        // and the units after the ring into L2, so that the first refills hit it
-        if (n > ns && a.prefetch_bytes) {
-            size_t by = (size_t)(n - ns) * ub;
-            if (by > a.prefetch_bytes) by = a.prefetch_bytes;
-            const size_t last = (size_t)a.rows * rb - (size_t)(u0 + ns) * ub;  // bytes left in the matrix
-            prefetch_l2_range(src + (size_t)ns * ub, (by < last ? by : last) & ~size_t(15), policy_evict_last());
-        }
     }
-    __syncthreads();
+    if (threadIdx.x == 0) abort_s = 0;
     if (a.early) grid_dep_launch();
-
     // before the dependency wait: what earlier kernels of the step do not write
     constexpr bool NORM = MODE != M_RESID;
     Q8Prologue<GS == 0 ? 64 : GS, NORM, Q8_WARPS, 8> pro;
-    const bool fast = GS != 0 && (NORM == (a.norm_w != nullptr)) && pro.fits(a);  // CTA-uniform
+    const bool fast = GS != 0 && (NORM == (a.norm_w != nullptr)) && pro.fits(a);
     int token = 0, pos = 0;
-    if (MODE == M_QKV) read_tp(a, token, pos);  // written before the step's first kernel
+    if (MODE == M_QKV) read_tp(a, token, pos);
     const int8_t* eq = nullptr;
     const float* es = nullptr;
     if (a.emb) {
@@ -930,68 +902,59 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
     }
     if (fast) pro.pre(a, eq, es);
     if (MODE == M_QKV) rope_table(a, pos, rope_cs);
+    if (threadIdx.x == 0 && a.prefetch_bytes && u1 > u0) {
+        size_t bytes = (size_t)(u1 - u0) * ub;
+        if (bytes > a.prefetch_bytes) bytes = a.prefetch_bytes;
+        prefetch_l2_range(Wb + (size_t)u0 * ub, bytes, policy_evict_last());
+    }
+    __syncthreads();  // barrier inits visible
     grid_dep_wait();
-    // after the wait: the input written by the previous kernel
+    // test switch: CTA 0's warp 0 withholds its first copy once (a wait then runs out)
+    bool skip0 = false;
+    if (threadIdx.x == 0) skip0 = a.stall && blockIdx.x == 0 && nmine > 0 && atomicExch(a.stall, 0);
+    if (lane == 0) {
+        for (int k = 0; k < ns && k < nmine; k++) {
+            if (k == 0 && skip0) continue;
+            mbar_arrive_expect_tx(&full[k], ub);
+            bulk_g2s(slots + (size_t)k * ub, unit_src(k), ub, &full[k], pol);
+        }
+    }
     if (MODE == M_QKV && a.amax && blockIdx.x == 0 && threadIdx.x == 0) *a.amax = 0ull;
+    // residual: lane j fetches the x of this warp's j-th unit, for the epilogue
+    float xres = 0.f;
+    if (MODE == M_RESID && lane < nmine) xres = __ldcg(a.out + u0 + warp + lane * Q8_WARPS);
     if (fast) pro.post(a, eq, es, xq, xsc, red);
     else q8_quantize_input<NORM>(a, eq, es, xq, xsc, red);
     __syncthreads();
-    if (GS == 0) {  // the generic loop takes the input scales in double
+    if (GS == 0) {
         for (int g = threadIdx.x; g < K / gs; g += Q8_THREADS) sxd[g] = (double)xsc[g];
         __syncthreads();
     }
 
-    // ---- this warp's units
-    constexpr int GRP = 32 / UR;     // lanes that hold one row's total after the reduce-scatter
-    const int my_row = lane / GRP;   // the unit row whose total this lane holds
-    const int nchunk = K >> 4;       // 16-byte chunks per row (generic loop)
-    const int cpg = gs >> 4;         // chunks per group
-    const int iters = (nchunk + 31) >> 5;
+    const int nchunk = K >> 4, cpg = gs >> 4, iters = (nchunk + 31) >> 5;
     unsigned long long best = 0ull;
-    bool gave_up = false;
-    for (int k = warp; k < n; k += Q8_WARPS) {
-        const int s = k % ns, j = k / ns;
-        // Unit k is the j-th use of slot s.  Its parity wait is only meaningful
-        // once the slot's previous unit has been consumed (then its refill, unit
-        // k, has been issued): another warp may still be on unit k - ns.
-        bool ok = true;
-        if (lane == 0 && ld_acquire_cta(&used[s]) < j) {
-            const uint64_t t0 = global_timer_ns();
-            while (ld_acquire_cta(&used[s]) < j) {
-                if (abort_s) { ok = false; break; }
-                if (global_timer_ns() - t0 > a.wait_ns) {
-                    set_error(a.err, DERR_TIMEOUT);
-                    ok = false;
-                    break;
-                }
-            }
-        }
-        if (!__shfl_sync(0xffffffffu, (int)ok, 0) ||
-            !mbar_wait_bounded(&full[s], j & 1, a.err, a.wait_ns, &abort_s)) {
+    int k = 0;
+    for (; k < nmine; k++) {
+        const int s = k % ns;
+        if (!mbar_wait_bounded(&full[s], (k / ns) & 1, a.err, a.wait_ns, &abort_s)) {
             abort_s = 1;
-            gave_up = true;
             break;
         }
-        const int r0 = (u0 + k) * UR;              // first row of the unit
-        const int nr = min(UR, a.rows - r0);        // rows in the unit
-        // residual rows: fetched now, added in the epilogue
-        float xres = 0.f;
-        if (MODE == M_RESID && lane % GRP == 0 && my_row < nr) xres = __ldcg(a.out + r0 + my_row);
-        const uint8_t* base = smem + (size_t)s * ub;
-        double acc[UR];
+        const uint8_t* base = slots + (size_t)s * ub;
+        double acc[UNIT];
         if (GS != 0) {
-            q8_rows_dot64<GS == 0 ? 64 : GS, UR>(base, rb, xq, xsc, K, acc);
+            q8_rows_dot64<GS == 0 ? 64 : GS, UNIT>(base, rb, xq, xsc, K, acc);
         } else {
 #pragma unroll
-            for (int r = 0; r < UR; r++) acc[r] = 0.0;
+            for (int r = 0; r < UNIT; r++) acc[r] = 0.0;
             for (int it = 0; it < iters; it++) {
                 const int c = lane + 32 * it;
                 const bool in = c < nchunk;
                 int4 xv = in ? *reinterpret_cast<const int4*>(xq + 16 * c) : make_int4(0, 0, 0, 0);
 #pragma unroll
-                for (int r = 0; r < UR; r++) {
+                for (int r = 0; r < UNIT; r++) {
                     int dsum = 0;
-                    if (in && r < nr) {
+                    if (in) {
                         const int4 wv = *reinterpret_cast<const int4*>(base + r * rb + 16 * c);
                         dsum = __dp4a(wv.x, xv.x, dsum);
                         dsum = __dp4a(wv.y, xv.y, dsum);
@@ -999,7 +962,7 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
                         dsum = __dp4a(wv.w, xv.w, dsum);
                     }
                     for (int o = 1; o < cpg; o <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
-                    if (in && r < nr && (c & (cpg - 1)) == 0) {
+                    if (in && (c & (cpg - 1)) == 0) {
                         const int g = c / cpg;
                         const float* sw = reinterpret_cast<const float*>(base + r * rb + K);
                         acc[r] += (double)dsum * (double)sw[g] * sxd[g];
@@ -1007,53 +970,40 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
                 }
             }
         }
-        // every lane is done with the slot: refill it with unit k + ns
+        // refill the slot with the unit ns ahead once every lane is done with it
         __syncwarp();
-        if (lane == 0) {
-            if (k + ns < n) {
-                const uint32_t by = unit_bytes(k + ns);
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                mbar_arrive_expect_tx(&full[s], by);
-                bulk_g2s(smem + (size_t)s * ub, src + (size_t)(k + ns) * ub, by, &full[s], pol);
-                issued[s] = j + 2;
-            }
-            st_release_cta(&used[s], j + 1);
+        if (lane == 0 && k + ns < nmine) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive_expect_tx(&full[s], ub);
+            bulk_g2s(slots + (size_t)s * ub, unit_src(k + ns), ub, &full[s], pol);
         }
-        // the UR row totals: lanes [GRP*i, GRP*i + GRP) hold row i's
-        const double tot = warp_sum_scatter<UR>(acc);
-        if (PAIRS) {
-            // pair p = rows (2p, 2p+1): lane 2p*GRP takes the odd row's total from lane (2p+1)*GRP
-            const double odd = __shfl_down_sync(0xffffffffu, tot, GRP);
-            if (lane % (2 * GRP) == 0 && my_row < nr) {
-                const int pr = (r0 + my_row) / 2;
-                if (MODE == M_QKV) epi_qkv(a, pr, (float)tot, (float)odd, pos, rope_cs);
-                else epi_w13(a, pr, (float)tot, (float)odd);
+        const double tot = warp_sum_scatter<UNIT>(acc);  // UNIT = 2: lanes 16..31 hold row 1
+        const int u = u0 + warp + k * Q8_WARPS;
+        const float xo = MODE == M_RESID ? __shfl_sync(0xffffffffu, xres, k & 31) : 0.f;
+        if (UNIT == 2) {
+            const double odd = __shfl_down_sync(0xffffffffu, tot, 16);
+            if (lane == 0) {
+                if (MODE == M_QKV) epi_qkv(a, u, (float)tot, (float)odd, pos, rope_cs);
+                else epi_w13(a, u, (float)tot, (float)odd);
             }
-        } else if (lane % GRP == 0 && my_row < nr) {
-            const int r = r0 + my_row;
+        } else if (lane == 0) {
             if (MODE == M_RESID) {
-                a.out[r] = xres + (float)tot;
+                a.out[u] = (k < 32 ? xo : __ldcg(a.out + u)) + (float)tot;
             } else {
                 const float v = (float)tot;
-                a.out[r] = v;
+                a.out[u] = v;
                 if (v != v) set_error(a.err, DERR_NAN);
-                const unsigned long long key = argmax_key(v, r);
+                const unsigned long long key = argmax_key(v, u);
                 best = key > best ? key : best;
             }
         }
     }
     if (!a.early) grid_dep_launch();
-    // a CTA that gave up must not leave while a copy into its ring is in flight
-    if (__syncthreads_or(gave_up) && threadIdx.x == 0) {
-        for (int s = 0; s < ns; s++)
-            if (issued[s] > ld_acquire_cta(&used[s])) mbar_wait_bounded(&full[s], (issued[s] - 1) & 1, a.err, a.wait_ns);
-    }
+    // a warp that gave up lets its copies in flight land before the CTA leaves
+    if (k < nmine && lane == 0)
+        for (int j = k; j < nmine && j < k + ns; j++)
+            if (!(j == 0 && skip0)) mbar_wait_bounded(&full[j % ns], (j / ns) & 1, a.err, a.wait_ns);
     if (MODE == M_CLS) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-            best = other > best ? other : best;
-        }
         if (lane == 0) best_s[warp] = best;
         __syncthreads();
         if (threadIdx.x == 0) {

@@ -71,8 +71,8 @@ struct l2c_ctx {
     // tuning
     size_t pf_f32 = 32 << 10, pf_q8 = 64 << 10;  // per CTA; larger leads measured slower in the step graph
     int f32_ctas_per_sm = 1;
-    size_t q8_smem_budget = 200 << 10;  // dynamic shared memory of one Q8_0 GEMV CTA (its weight ring)
-    int q8_early = 1;    // 1: Q8_0 GEMVs let the next kernel launch as soon as they start (else at their end)
+    size_t q8_smem_budget = 220 << 10;  // dynamic shared memory of one Q8_0 GEMV CTA (its rings)
+    int q8_early = 0;    // 1: Q8_0 GEMVs let the next kernel launch as soon as they start (else at their end)
     unsigned long long wait_ns = kWaitNs;  // limit of every bounded wait in the kernels
     int* stall = nullptr;  // test switch read by the Q8_0 q/k/v kernel of layer 0
     long long oom_after = -1;  // test switch: device allocations after this many fail
@@ -166,19 +166,8 @@ struct GemvShape {
     int rows, K, unit;
 };
 
-// The ring of a Q8_0 GEMV: as many unit slots as fit the shared-memory budget
-// next to the input codes, at least 2, at most the CTA's units.
-static Q8Ring q8_ring(const l2c_ctx* h, int K, int gs, size_t rb, int unit, int units_per_cta, size_t* smem_out) {
-    Q8Ring R = {};
-    R.unit_bytes = (uint32_t)((size_t)unit * rb);
-    const Q8Smem none = q8_smem(0, R.unit_bytes, K, gs);
-    const size_t per_slot = (size_t)R.unit_bytes + 16;  // the slot, its barrier and counters
-    int ns = h->q8_smem_budget > none.total ? (int)((h->q8_smem_budget - none.total) / per_slot) : 0;
-    if (ns > units_per_cta) ns = units_per_cta;
-    R.ns = ns < 2 ? 2 : ns;
-    *smem_out = q8_smem(R.ns, R.unit_bytes, K, gs).total;
-    return R;
-}
+// Kernels of the step, in order within a layer.
+enum StepKernel : int { SK_QKV = 0, SK_ATTN = 1, SK_WO = 2, SK_W13 = 3, SK_W2 = 4, SK_CLS = 5 };
 
 template <int MODE>
 static cudaError_t launch_gemv(l2c_ctx* h, bool q80, GemvArgs a, int unit) {
@@ -204,27 +193,23 @@ static cudaError_t launch_gemv(l2c_ctx* h, bool q80, GemvArgs a, int unit) {
         const size_t smem = (size_t)a.K * 4 + (size_t)rows_max * ks * 4;
         return launch(h->cap, true, k_gemv_f32<MODE>, dim3(grid), dim3(F32_THREADS), smem, a, ks);
     }
-    // units of 4 rows (two row pairs for QKV and W1/W3), one row where four
-    // would leave the ring fewer than one unit per warp (the wide W2 rows)
-    const bool four = MODE != M_RESID || (size_t)4 * a.ld * Q8_WARPS <= h->q8_smem_budget;
-    const int ur = four ? 4 : 1;
-    const int q8_units = (a.rows + ur - 1) / ur;
-    int grid = h->sms;
-    if (grid > q8_units) grid = q8_units;
-    size_t smem = 0;
-    const Q8Ring R = q8_ring(h, a.K, a.gs, a.ld, ur, (q8_units + grid - 1) / grid, &smem);
+    // units of UNIT rows, as many ring slots per warp as fit (2..8)
+    const int grid = h->sms < units ? h->sms : units;
+    Q8Ring R = {};
+    R.unit_bytes = (uint32_t)((size_t)unit * a.ld);
+    const size_t fixed = q8_smem(0, R.unit_bytes, a.K, a.gs).total;
+    const size_t per = (size_t)Q8_WARPS * (R.unit_bytes + 8);
+    const int ns = h->q8_smem_budget > fixed ? (int)((h->q8_smem_budget - fixed) / per) : 0;
+    R.ns = ns < 2 ? 2 : (ns > 8 ? 8 : ns);
+    const size_t smem = q8_smem(R.ns, R.unit_bytes, a.K, a.gs).total;
     a.early = h->q8_early;
     a.prefetch_bytes = h->pf_q8;
     const dim3 g(grid), t(Q8_THREADS);
     const bool k64 = a.K % 64 == 0;
-#define L2C_Q8_LAUNCH(GS_)                                                                      \
-    return four ? launch(h->cap, true, k_gemv_q8<MODE, GS_, 4>, g, t, smem, a, R)               \
-                : launch(h->cap, true, k_gemv_q8<MODE == M_RESID ? MODE : M_RESID, GS_, 1>, g, t, smem, a, R);
-    if (k64 && a.gs == 64) L2C_Q8_LAUNCH(64)
-    if (k64 && a.gs == 32) L2C_Q8_LAUNCH(32)
-    if (k64 && a.gs == 128) L2C_Q8_LAUNCH(128)
-    L2C_Q8_LAUNCH(0)
-#undef L2C_Q8_LAUNCH
+    if (k64 && a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64>, g, t, smem, a, R);
+    if (k64 && a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32>, g, t, smem, a, R);
+    if (k64 && a.gs == 128) return launch(h->cap, true, k_gemv_q8<MODE, 128>, g, t, smem, a, R);
+    return launch(h->cap, true, k_gemv_q8<MODE, 0>, g, t, smem, a, R);
 }
 
 // Every kernel of the Q8_0 step (and of the batched step) asks for the same
@@ -244,24 +229,22 @@ static int set_smem_limits(l2c_ctx* h) {
     CK(cudaFuncSetAttribute(k_gemv_f32<M_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     CK(cudaFuncSetAttribute(k_gemv_f32<M_W13>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     CK(cudaFuncSetAttribute(k_gemv_f32<M_CLS>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
-#define L2C_Q8_ATTR(GS_)                                                                                             \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_QKV, GS_, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID, GS_, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096)); \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID, GS_, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096)); \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_W13, GS_, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+#define L2C_Q8_ATTR(GS_)                                                                                          \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_QKV, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096)); \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_W13, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     L2C_Q8_ATTR(0) L2C_Q8_ATTR(32) L2C_Q8_ATTR(64) L2C_Q8_ATTR(128)
 #undef L2C_Q8_ATTR
     {
         cudaError_t e = attn_set_smem_limits();
         if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "attention smem limit: %s", cudaGetErrorString(e));
     }
-#define L2C_Q8_CARVE(GS_)                          \
-    CK(max_carveout(k_gemv_q8<M_QKV, GS_, 4>));   \
-    CK(max_carveout(k_gemv_q8<M_RESID, GS_, 4>)); \
-    CK(max_carveout(k_gemv_q8<M_RESID, GS_, 1>)); \
-    CK(max_carveout(k_gemv_q8<M_W13, GS_, 4>));   \
-    CK(max_carveout(k_gemv_q8<M_CLS, GS_, 4>));
+#define L2C_Q8_CARVE(GS_)                      \
+    CK(max_carveout(k_gemv_q8<M_QKV, GS_>));   \
+    CK(max_carveout(k_gemv_q8<M_RESID, GS_>)); \
+    CK(max_carveout(k_gemv_q8<M_W13, GS_>));   \
+    CK(max_carveout(k_gemv_q8<M_CLS, GS_>));
     L2C_Q8_CARVE(0) L2C_Q8_CARVE(32) L2C_Q8_CARVE(64) L2C_Q8_CARVE(128)
 #undef L2C_Q8_CARVE
     CK(max_carveout(k_bgemm_q8<M_QKV>));
@@ -306,10 +289,7 @@ static cudaError_t launch_attention(l2c_ctx* h, cudaStream_t s, bool pdl, bool d
     return launch(s, pdl, ak, dim3(t.nchunks, h->Hkv, B), dim3(ATTN_THREADS), smem, t);
 }
 
-// Kernels of the step, in order within a layer.
-enum StepKernel : int { SK_QKV = 0, SK_ATTN = 1, SK_WO = 2, SK_W13 = 3, SK_W2 = 4, SK_CLS = 5 };
-
-// Enqueues kernel `kind` of layer l (sequence 0) on stream s.
+// Enqueues kernel `kind` of layer l (sequence seq) on stream s.
 static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, int l, int seq = 0) {
     g_pdl = h->pdl;
     const size_t d = h->d, kvd = h->kvd, hh = h->h, S = h->S;
