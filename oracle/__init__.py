@@ -61,6 +61,7 @@ def lib():
             "orc_q80_group_dots": (None, [vp, vp, vp, i32, i32, i32]),
             "orc_matvec_q80": (None, [vp, vp, vp, vp, vp, i32, i32, i32]),
             "orc_argmax": (i32, [vp, i32]),
+            "orc_sample": (i32, [vp, i32, ctypes.c_float, ctypes.c_float, ctypes.c_double]),
             "orc_blob_floats": (sz, [vp, i32]),
             "orc_create": (vp, [vp, vp, sz, i32, i32]),
             "orc_enable_q80": (i32, [vp, i32]),
@@ -191,6 +192,12 @@ def matvec_q80(qw, sw, qx, sx, gs: int):
 def argmax(x) -> int:
     x = _f32(x)
     return lib().orc_argmax(_p(x), x.size)
+
+
+def sample(z, temperature: float, topp: float, coin: float) -> int:
+    """Temperature / top-p / multinomial draw with the given coin (orc_sample)."""
+    z = _f32(z)
+    return lib().orc_sample(_p(z), z.size, float(temperature), float(topp), float(coin))
 
 
 def blob_floats(cfg, shared_weights: int) -> int:

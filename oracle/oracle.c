@@ -17,6 +17,8 @@
  *   [qa]    "Karpathy 技術學習庫 - Q&A 問答集", 技術細節: KV Cache 在 C 中如何
  *           管理, 為什麼 QKV 的維度不同 (GQA), RoPE 在 C 中的實作, 跳過
  *           freq_cis, shared_weights 參數的作用; 效能相關: 13B+ overflow.
+ *   [essay] "LLM底层原理与工程实践：从参数文件到C语言推理" (m.mht18.com),
+ *           §3.2 (sampling with a temperature after the logits).
  *
  * Readings where the pages are silent (each repeated where it is used):
  *   RMSNorm eps = 1e-5 inside the square root; RoPE base 10000 on adjacent
@@ -260,6 +262,68 @@ int orc_argmax(const float* x, int n) {
     int best = 0;
     for (int i = 1; i < n; i++) if (x[i] > x[best]) best = i;
     return best;
+}
+
+static int cmp_desc(const void* a, const void* b) {
+    const double x = *(const double*)a, y = *(const double*)b;
+    return x < y ? 1 : (x > y ? -1 : 0);
+}
+
+/* Sampling after the logits [essay §3.2: a temperature divides the logits
+ * before the softmax; port 智能家居控制案例: the greedy sample_argmax].  The
+ * pages give no more, so the reading taken is:
+ *   temperature == 0: the greedy argmax.
+ *   otherwise weights q_i = exp((z_i - max z) / T) in double (the softmax
+ *   up to its normalisation Z = sum q_i);
+ *   topp < 1 restricts the draw to the smallest set of most probable tokens
+ *   whose weight reaches topp * Z (every token tied with the last one taken
+ *   is in the set): tau = the weight at which the running sum, over the
+ *   weights sorted in decreasing order, first reaches topp * Z, and the set
+ *   is {i : q_i >= tau};
+ *   the draw uses the caller's coin u in [0, 1): the first index i, in index
+ *   order, of the set at which the running sum of the set's weights exceeds
+ *   u * Z_set (the last index of the set if rounding leaves none). */
+int orc_sample(const float* z, int n, float temperature, float topp, double coin) {
+    if (n <= 0) return -1;
+    if (temperature == 0.0f) return orc_argmax(z, n);
+    float mx = z[0];
+    for (int i = 1; i < n; i++) if (z[i] > mx) mx = z[i];
+    double* q = (double*)malloc(sizeof(double) * (size_t)n);
+    double Z = 0.0;
+    for (int i = 0; i < n; i++) {
+        q[i] = exp(((double)z[i] - (double)mx) / (double)temperature);
+        Z += q[i];
+    }
+    double tau = 0.0;
+    if (topp < 1.0f) {
+        double* sorted = (double*)malloc(sizeof(double) * (size_t)n);
+        memcpy(sorted, q, sizeof(double) * (size_t)n);
+        qsort(sorted, (size_t)n, sizeof(double), cmp_desc);
+        const double target = (double)topp * Z;
+        double cum = 0.0;
+        tau = sorted[n - 1];
+        for (int k = 0; k < n; k++) {
+            cum += sorted[k];
+            if (cum >= target) {
+                tau = sorted[k];
+                break;
+            }
+        }
+        free(sorted);
+    }
+    double zset = 0.0;
+    for (int i = 0; i < n; i++) if (q[i] >= tau) zset += q[i];
+    const double target = coin * zset;
+    double cum = 0.0;
+    int last = -1, pick = -1;
+    for (int i = 0; i < n && pick < 0; i++) {
+        if (q[i] < tau) continue;
+        cum += q[i];
+        last = i;
+        if (cum > target) pick = i;
+    }
+    free(q);
+    return pick >= 0 ? pick : last;
 }
 
 /* ---------------------------------------------------------------- model -- */

@@ -47,6 +47,7 @@ void orc_q80_group_dots(int32_t* out, const int8_t* qx, const int8_t* qw, int n,
 void orc_matvec_q80(float* o, const int8_t* qx, const float* sx, const int8_t* qw, const float* sw,
                     int n, int d, int gs);
 int orc_argmax(const float* x, int n);
+int orc_sample(const float* z, int n, float temperature, float topp, double coin);
 
 /* ---- whole model ---- */
 size_t orc_blob_floats(const orc_config* c, int shared_weights);

@@ -34,6 +34,9 @@ MUTANTS = {
     "argmax_last_tie": ("if (x[i] > x[best]) best = i;", "if (x[i] >= x[best]) best = i;"),
     "wrong_norm_weight": ("orc_rmsnorm(m->xb, x, m->w_att + l * d, d);", "orc_rmsnorm(m->xb, x, m->w_ffn + l * d, d);"),
     "swiglu_operands_swapped": ("orc_swiglu(m->hb, m->hb2, h);", "orc_swiglu(m->hb2, m->hb, h); memcpy(m->hb, m->hb2, sizeof(float) * (size_t)h);"),
+    "sample_temperature_multiplies": ("((double)z[i] - (double)mx) / (double)temperature", "((double)z[i] - (double)mx) * (double)temperature"),
+    "sample_topp_excludes_ties": ("for (int i = 0; i < n; i++) if (q[i] >= tau) zset += q[i];", "for (int i = 0; i < n; i++) if (q[i] > tau || (q[i] == tau && i == 0)) zset += q[i];"),
+    "sample_coin_not_scaled": ("const double target = coin * zset;", "const double target = coin;"),
 }
 
 
@@ -52,6 +55,7 @@ def test_pins_catch_planted_mistake(name):
         subprocess.check_call(["gcc", *oracle.CFLAGS, "-o", so, msrc, "-lm"])
         env = dict(os.environ, ORACLE_LIB_PATH=so, OMP_NUM_THREADS="2")
         r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                            "tests/test_oracle_pins.py", "tests/test_oracle_forward.py"],
+                            "tests/test_oracle_pins.py", "tests/test_oracle_forward.py",
+                            "tests/test_oracle_sampling.py"],
                            cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
         assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
