@@ -20,7 +20,7 @@ L2C_OK, L2C_E_ARG, L2C_E_OOM, L2C_E_CUDA, L2C_E_DEVICE, L2C_E_STATE, L2C_E_SCRAT
 # every symbol declared in include/l2c.h
 EXPORTS = (
     "l2c_blob_floats", "l2c_create", "l2c_enable_q80", "l2c_forward", "l2c_forward_q80", "l2c_argmax",
-    "l2c_generate", "l2c_forward_batch", "l2c_quantize_q80", "l2c_q80_group_dots", "l2c_kv_load",
+    "l2c_generate", "l2c_sample", "l2c_forward_batch", "l2c_quantize_q80", "l2c_q80_group_dots", "l2c_kv_load",
     "l2c_kv_read", "l2c_kv_reset", "l2c_attention", "l2c_attention_noalloc", "l2c_time_kernel", "l2c_sync", "l2c_stream", "l2c_last_status", "l2c_last_error",
     "l2c_destroy",
 )
@@ -59,6 +59,8 @@ def lib():
             "l2c_forward_q80": (vp, [vp, i32, i32]),
             "l2c_argmax": (i32, [vp, vp, i32, ctypes.POINTER(ctypes.c_int)]),
             "l2c_generate": (i32, [vp, i32, i32, i32, i32, vp]),
+            "l2c_sample": (i32, [vp, vp, i32, ctypes.c_float, ctypes.c_float, ctypes.c_double,
+                                 ctypes.POINTER(ctypes.c_int)]),
             "l2c_forward_batch": (i32, [vp, i32, vp, vp, i32, vp]),
             "l2c_quantize_q80": (i32, [vp, vp, i64, i32, vp, vp]),
             "l2c_q80_group_dots": (i32, [vp, vp, vp, i32, i32, i32, vp]),
@@ -157,6 +159,13 @@ class Decoder:
     def argmax(self, logits) -> int:
         out = ctypes.c_int()
         self._check(lib().l2c_argmax(self._h, _ptr(logits), logits.numel(), ctypes.byref(out)))
+        return out.value
+
+    def sample(self, logits, temperature: float, topp: float, coin: float) -> int:
+        """The token drawn from device logits with temperature / top-p and the given coin (l2c_sample)."""
+        out = ctypes.c_int()
+        self._check(lib().l2c_sample(self._h, _ptr(logits), int(logits.numel()), float(temperature), float(topp),
+                                     float(coin), ctypes.byref(out)))
         return out.value
 
     def generate(self, token0: int, steps: int, q80: bool = False, pos0: int = 0) -> np.ndarray:

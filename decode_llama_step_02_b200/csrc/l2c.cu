@@ -22,6 +22,7 @@
 
 #include "../../include/l2c.h"
 #include "batched.cuh"
+#include "sampling.cuh"
 #include "kernels.cuh"
 
 using namespace l2c;
@@ -53,6 +54,8 @@ struct l2c_ctx {
     int* gen_count = nullptr;
     int* idx_out = nullptr;
     unsigned long long* key_scratch = nullptr;
+    double* sample_q = nullptr;  // weights of l2c_sample, sample_n doubles (allocated on first use)
+    size_t sample_n = 0;
     void* attn_part = nullptr;
     int* attn_cnt = nullptr;
     int attn_ctas = 0;          // fp32 attention CTAs to aim for (0: the SM count)
@@ -836,6 +839,26 @@ extern "C" int l2c_argmax(l2c_ctx* h, const float* logits, int n, int* out_idx) 
     if (grid > h->sms) grid = h->sms;
     k_argmax<<<grid, 256, 0, h->stream>>>(logits, n, h->key_scratch, h->err);
     k_argmax_index<<<1, 1, 0, h->stream>>>(h->key_scratch, h->idx_out);
+    CK(cudaGetLastError());
+    int rc = l2c_sync(h);
+    if (rc) return rc;
+    CK(cudaMemcpy(out_idx, h->idx_out, 4, cudaMemcpyDeviceToHost));
+    return L2C_OK;
+}
+
+extern "C" int l2c_sample(l2c_ctx* h, const float* logits, int n, float temperature, float topp, double coin,
+                          int* out_idx) {
+    if (!h || !logits || n <= 0 || !out_idx || !(temperature >= 0.0f) || !(topp > 0.0f) ||
+        !(coin >= 0.0 && coin < 1.0))
+        return fail(h, L2C_E_ARG, "sample: need n > 0, temperature >= 0, topp > 0 and a coin in [0, 1)");
+    if (temperature == 0.0f) return l2c_argmax(h, logits, n, out_idx);
+    if (h->sample_n < (size_t)n) {
+        int rc;
+        if ((rc = dalloc(h, (void**)&h->sample_q, (size_t)n * sizeof(double))) != L2C_OK) return rc;
+        h->sample_n = (size_t)n;
+    }
+    k_sample<<<1, SAMPLE_THREADS, 0, h->stream>>>(logits, n, temperature, topp, coin, nullptr, h->sample_q, h->idx_out,
+                                                  h->err);
     CK(cudaGetLastError());
     int rc = l2c_sync(h);
     if (rc) return rc;

@@ -131,6 +131,24 @@ L2C_API const float* l2c_forward_q80(l2c_ctx* h, int token, int pos);
 L2C_API int l2c_argmax(l2c_ctx* h, const float* logits_dev, int n, int* out_idx_host);
 
 /*
+ * l2c_sample - the token draw after the logits: a temperature divides the
+ * logits before the softmax ("LLM底层原理与工程实践" §3.2), temperature 0 is the
+ * greedy sample_argmax of [port] 智能家居控制案例 (l2c_argmax).  Otherwise
+ * (reading taken where the pages stop): weights q_i = exp((z_i - max z) / T)
+ * in double; top-p keeps the smallest set of most probable tokens whose
+ * weight reaches topp * sum q, every token tied with the last one included
+ * (topp >= 1: all tokens); the coin u picks the first index, in index order,
+ * of the set at which the running weight exceeds u * the set's weight.
+ * logits_dev [n] device fp32 (e.g. the logits of l2c_forward, on the same
+ * stream); temperature >= 0, topp > 0, coin in [0, 1) (the caller draws it:
+ * the library keeps no random state).  Blocks until the index is on the host.
+ * A NaN logit gives L2C_E_DEVICE.  The first call with a larger n allocates
+ * a scratch row of n doubles in the handle.
+ */
+L2C_API int l2c_sample(l2c_ctx* h, const float* logits_dev, int n, float temperature, float topp, double coin,
+                       int* out_idx_host);
+
+/*
  * l2c_generate - greedy decoding with the token fed back on the device:
  * tok_0 = token0; for t = 0..steps-1: logits = forward(tok_t, pos0 + t),
  * tok_{t+1} = argmax(logits).  tokens_out_host[t] = tok_{t+1}.
