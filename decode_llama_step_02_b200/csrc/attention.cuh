@@ -196,21 +196,24 @@ __device__ __forceinline__ void attn_batch(int n, KV kv, const Acc (&qr)[REP][4]
             widen4<Acc>(kr[i], kw);
             sp[i] = kw[0] * qr[h][0] + kw[1] * qr[h][1] + kw[2] * qr[h][2] + kw[3] * qr[h][3];
         }
-        const Acc tot = warp_sum_scatter<PB>(sp);  // lane l: position (l / (32/PB)) % PB
-        Acc sc[PB];
-        Acc mx = -INFINITY;
+        // lane l holds the score of position (l / (32/PB)) % PB of the batch:
+        // the batch max comes from the lanes of the other positions, and each
+        // lane takes the exponential of its own position only (one exp per
+        // lane instead of PB), then the weights are broadcast
+        const Acc tot = warp_sum_scatter<PB>(sp);
+        const int mine = ((threadIdx.x & 31) / (32 / PB)) % PB;
+        const Acc sc = mine < n ? tot * scale : (Acc)-INFINITY;
+        Acc mx = sc;
 #pragma unroll
-        for (int i = 0; i < PB; i++) {
-            const Acc si = __shfl_sync(0xffffffffu, tot, i * (32 / PB));
-            sc[i] = i < n ? si * scale : (Acc)-INFINITY;
-            mx = max(mx, sc[i]);
-        }
+        for (int sh = 32 / PB; sh < 32; sh <<= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, sh));
         const Acc mnew = max(m[h], mx);
-        const Acc alpha = exp(m[h] - mnew);  // exp(-inf) = 0 on the warp's first batch
+        // exp(-inf) = 0 on the warp's first batch; an unchanged max scales by 1
+        const Acc alpha = mnew == m[h] ? (Acc)1 : exp(m[h] - mnew);
+        const Acc pm = exp(sc - mnew);  // masked positions: exp(-inf) = 0
         Acc ps = 0, w4[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int i = 0; i < PB; i++) {
-            const Acc p = exp(sc[i] - mnew);  // masked positions: exp(-inf) = 0
+            const Acc p = __shfl_sync(0xffffffffu, pm, i * (32 / PB));
             Acc vw[4];
             widen4<Acc>(kv(i, 1), vw);
             ps += p;

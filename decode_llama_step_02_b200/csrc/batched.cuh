@@ -151,6 +151,65 @@ __host__ __device__ inline BLayout make_blayout(int kc, int gs, int ns) {
     return L;
 }
 
+// The epilogue of a batched GEMM CTA: its rows r0 .. r0+nrows-1 of every
+// live sequence sit in `so` (fp32, rounded once).  Threads tid of nt (named
+// barrier `bar`, nt threads) take (row unit, sequence) pairs:
+//   QKV: RoPE of q and k, K/V cache write at each sequence's own position
+//   W13: hb = silu(W1 x) * (W3 x) (interleaved rows)
+//   RESID: out += v;  CLS: logits and a per-sequence argmax key.
+template <int MODE>
+__device__ __forceinline__ void bgemm_epilogue(const BGemmArgs& a, int r0, int nrows, const float (*so)[BMAX + 1],
+                                               unsigned long long* best_s, int tid, int nt, int bar) {
+    if (MODE == M_QKV || MODE == M_W13) {
+        for (int i = tid; i < (nrows / 2) * a.B; i += nt) {
+            const int up = i / a.B, b = i % a.B;
+            const int r = r0 + 2 * up;
+            const float v0 = so[2 * up][b], v1 = so[2 * up + 1][b];
+            if (MODE == M_W13) {
+                a.out[(size_t)b * a.out_stride + r / 2] = (float)(silu_d((double)v0) * (double)v1);
+            } else {
+                int pos = a.tp[2 * b + 1];
+                if (pos < 0 || pos >= a.seq_len) pos = 0;  // flagged by the prep kernel
+                if (r < a.d) {
+                    float o0, o1;
+                    rope_pair(v0, v1, r % a.hs, pos, a.freq, o0, o1);
+                    a.out[(size_t)b * a.out_stride + r] = o0;
+                    a.out[(size_t)b * a.out_stride + r + 1] = o1;
+                } else if (r < a.d + a.kvd) {
+                    const int j = r - a.d;
+                    float o0, o1;
+                    rope_pair(v0, v1, j % a.hs, pos, a.freq, o0, o1);
+                    float* k = a.kc_base + (size_t)b * a.seq_stride + (size_t)pos * a.kvd;
+                    k[j] = o0;
+                    k[j + 1] = o1;
+                } else {
+                    const int j = r - a.d - a.kvd;
+                    float* v = a.vc_base + (size_t)b * a.seq_stride + (size_t)pos * a.kvd;
+                    v[j] = v0;
+                    v[j + 1] = v1;
+                }
+            }
+        }
+    } else {
+        for (int i = tid; i < nrows * a.B; i += nt) {
+            const int rr = i / a.B, b = i % a.B;
+            const float v = so[rr][b];
+            float* o = a.out + (size_t)b * a.out_stride + r0 + rr;
+            if (MODE == M_RESID) {
+                *o = *o + v;
+            } else {
+                *o = v;
+                if (v != v) set_error(a.err, DERR_NAN);
+                atomicMax(&best_s[b], argmax_key(v, r0 + rr));
+            }
+        }
+        if (MODE == M_CLS) {
+            asm volatile("bar.sync %0, %1;" :: "r"(bar), "r"(nt) : "memory");
+            if (tid < a.B && best_s[tid]) atomicMax(&a.amax[tid], best_s[tid]);
+        }
+    }
+}
+
 // grid = ceil(rows / BG_ROWS) CTAs of (BG_WARPS + 1) warps; the last warp is
 // the producer (its 32 lanes issue the stage's bulk copies).
 template <int MODE>
@@ -293,56 +352,7 @@ __global__ void __launch_bounds__(32 * (BG_WARPS + 1)) k_bgemm_q8(const BGemmArg
         stage_out[wr0 + gid + 8][8 * n + 2 * tig + 1] = (float)acc[n][3];
     }
     asm volatile("bar.sync 1, %0;" :: "r"(32 * BG_WARPS) : "memory");
-    // epilogue: thread t takes (row unit, sequence) pairs
-    const int nt = 32 * BG_WARPS;
-    if (MODE == M_QKV || MODE == M_W13) {
-        for (int i = threadIdx.x; i < (nrows / 2) * a.B; i += nt) {
-            const int up = i / a.B, b = i % a.B;
-            const int r = r0 + 2 * up;
-            const float v0 = stage_out[2 * up][b], v1 = stage_out[2 * up + 1][b];
-            if (MODE == M_W13) {
-                a.out[(size_t)b * a.out_stride + r / 2] = (float)(silu_d((double)v0) * (double)v1);
-            } else {
-                int pos = a.tp[2 * b + 1];
-                if (pos < 0 || pos >= a.seq_len) pos = 0;  // flagged by the prep kernel
-                if (r < a.d) {
-                    float o0, o1;
-                    rope_pair(v0, v1, r % a.hs, pos, a.freq, o0, o1);
-                    a.out[(size_t)b * a.out_stride + r] = o0;
-                    a.out[(size_t)b * a.out_stride + r + 1] = o1;
-                } else if (r < a.d + a.kvd) {
-                    const int j = r - a.d;
-                    float o0, o1;
-                    rope_pair(v0, v1, j % a.hs, pos, a.freq, o0, o1);
-                    float* k = a.kc_base + (size_t)b * a.seq_stride + (size_t)pos * a.kvd;
-                    k[j] = o0;
-                    k[j + 1] = o1;
-                } else {
-                    const int j = r - a.d - a.kvd;
-                    float* v = a.vc_base + (size_t)b * a.seq_stride + (size_t)pos * a.kvd;
-                    v[j] = v0;
-                    v[j + 1] = v1;
-                }
-            }
-        }
-    } else {
-        for (int i = threadIdx.x; i < nrows * a.B; i += nt) {
-            const int rr = i / a.B, b = i % a.B;
-            const float v = stage_out[rr][b];
-            float* o = a.out + (size_t)b * a.out_stride + r0 + rr;
-            if (MODE == M_RESID) {
-                *o = *o + v;
-            } else {
-                *o = v;
-                if (v != v) set_error(a.err, DERR_NAN);
-                atomicMax(&best_s[b], argmax_key(v, r0 + rr));
-            }
-        }
-        if (MODE == M_CLS) {
-            asm volatile("bar.sync 1, %0;" :: "r"(32 * BG_WARPS) : "memory");
-            if (threadIdx.x < a.B && best_s[threadIdx.x]) atomicMax(&a.amax[threadIdx.x], best_s[threadIdx.x]);
-        }
-    }
+    bgemm_epilogue<MODE>(a, r0, nrows, stage_out, best_s, threadIdx.x, 32 * BG_WARPS, 1);
 }
 
 }  // namespace l2c
