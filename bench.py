@@ -15,6 +15,7 @@ rank (one per GPU) runs an independent replica: batch-1 decode does not shard.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -39,6 +40,8 @@ METRIC = "decode tokens/s at batch 1 (fp32 & Q8_0) on 1 B200; achieved HBM GB/s 
 UNIT = "tokens/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+# fp32 FMA peak from unit counts and clock: 148 SMs x 128 FP32 lanes x 2 flop x 1.965 GHz
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 # ------------------------------------------------------------ byte accounting --
@@ -530,10 +533,14 @@ def run_extra(args):
                                "buckets": flushed}}), flush=True)
         dec.close()
 
+    if args.extra in ("all", "prefill"):
+        run_prefill(torch, l2c, ev, stream)
     if args.extra not in ("all", "batch"):
         return 0
-    # GQA-7B, 32 sequences, one batched Q8_0 step
+    # GQA-7B, 32 sequences, one batched step (Q8_0 and fp32)
     spec, B = synth.GQA7B, 32
+    if args.layers:
+        spec = dataclasses.replace(spec, name=f"GQA-7B-width-{args.layers}L", n_layers=args.layers)
     blob = device_blob(torch, spec)
     dec = l2c.Decoder(spec.cfg, blob, spec.shared_weights, max_batch=B)
     del blob
@@ -549,31 +556,80 @@ def run_extra(args):
     tk = torch.from_numpy(toks.astype(np.int32)).cuda()
     ps = torch.from_numpy(pos.astype(np.int32)).cuda()
     out = torch.empty((B, spec.vocab_size), dtype=torch.float32, device="cuda")
-    for _ in range(3):
-        dec.forward_batch(tk, ps, out, q80=True)
-    dec.sync()
-    reps = 10
-    a, b = ev(), ev()
-    a.record(stream)
-    for _ in range(reps):
-        dec.forward_batch(tk, ps, out, q80=True)
-    b.record(stream)
-    torch.cuda.synchronize()
-    dec.sync()
-    ms = a.elapsed_time(b) / reps
     d, h, L, H, Hkv, V, S = spec.cfg
     kvd = Hkv * (d // H)
-    wbytes = bytes_per_token(True, -1, spec, GS)  # weights only (pos -1: no KV)
     kvbytes = float(sum(8.0 * L * (int(p) + 1) * kvd for p in pos))
-    by = wbytes + kvbytes
-    print(json.dumps({
-        "extra": True, "config": spec.name + " batch 32", "variant": f"q8_0 gs={GS}", "ms_per_step": ms,
-        "tokens_per_s": B / ms * 1e3, "bytes_per_step": by, "weight_bytes": wbytes, "kv_bytes": kvbytes,
-        "gbs": by / ms / 1e6, "frac_of_measured_hbm": by / ms / 1e6 / peak, "frac_of_8tbs": by / ms / 1e6 / NOMINAL_HBM_GBS,
-        "inputs": "tokens uniform (stream 2), positions uniform in [0, 2047] (stream 3), caches prefilled N(0,1)",
-        "timing": f"CUDA events around {reps} batched steps (l2c_forward_batch), device-resident inputs"}), flush=True)
+    for q80 in (True, False):
+        for _ in range(3):
+            dec.forward_batch(tk, ps, out, q80=q80)
+        dec.sync()
+        reps = 10
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(reps):
+            dec.forward_batch(tk, ps, out, q80=q80)
+        b.record(stream)
+        torch.cuda.synchronize()
+        dec.sync()
+        ms = a.elapsed_time(b) / reps
+        wbytes = bytes_per_token(q80, -1, spec, GS)  # weights only (pos -1: no KV)
+        by = wbytes + kvbytes
+        line = {
+            "extra": True, "config": spec.name + " batch 32", "variant": f"q8_0 gs={GS}" if q80 else "fp32",
+            "ms_per_step": ms, "tokens_per_s": B / ms * 1e3, "bytes_per_step": by, "weight_bytes": wbytes,
+            "kv_bytes": kvbytes, "gbs": by / ms / 1e6, "frac_of_measured_hbm": by / ms / 1e6 / peak,
+            "frac_of_8tbs": by / ms / 1e6 / NOMINAL_HBM_GBS,
+            "inputs": "tokens uniform (stream 2), positions uniform in [0, 2047] (stream 3), caches prefilled N(0,1)",
+            "timing": f"CUDA events around {reps} batched steps (l2c_forward_batch), device-resident inputs"}
+        if not q80:
+            fl = 2.0 * B * matvec_params(spec)
+            line["gemm_flops_per_step"] = fl
+            line["gemm_tflops"] = fl / ms / 1e9
+            line["frac_of_fp32_fma_peak"] = fl / ms / 1e9 / FP32_FMA_TFLOPS
+        print(json.dumps(line), flush=True)
     dec.close()
     return 0
+
+
+def matvec_params(spec) -> float:
+    """Weights one token multiplies: every matvec of the step (classifier included)."""
+    d, h, L, H, Hkv, V, S = spec.cfg
+    kvd = Hkv * (d // H)
+    return float(L * (2 * d * d + 2 * d * kvd + 3 * d * h) + V * d)
+
+
+def run_prefill(torch, l2c, ev, stream):
+    """A 128-token prompt on the 7B shape (l2c_prefill: 4 GEMM chunks of 32
+    tokens), fp32 and Q8_0 GS=64, timed with CUDA events around whole calls."""
+    n = 128
+    blob = device_blob(torch)
+    dec = l2c.Decoder(SPEC.cfg, blob, SPEC.shared_weights)
+    del blob
+    torch.cuda.empty_cache()
+    dec.enable_q80(GS)
+    toks = synth.tokens(SPEC.seed, 4, n, SPEC.vocab_size)
+    last = torch.empty(SPEC.vocab_size, dtype=torch.float32, device="cuda")
+    for q80 in (False, True):
+        dec.prefill(toks, 0, q80=q80, logits_last=last)  # warm-up: buffers, module loading
+        reps, ts = 3, []
+        for _ in range(reps):
+            a, b = ev(), ev()
+            a.record(stream)
+            dec.prefill(toks, 0, q80=q80, logits_last=last)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ms = statistics.median(ts)
+        fl = 2.0 * n * matvec_params(SPEC)
+        line = {"extra": True, "config": SPEC.name + " prefill", "variant": f"q8_0 gs={GS}" if q80 else "fp32",
+                "prompt_tokens": n, "chunks": (n + 31) // 32, "ms_per_prompt": ms, "tokens_per_s": n / ms * 1e3,
+                "matvec_flops": fl, "tflops": fl / ms / 1e9,
+                "decode_equivalent": "the same prompt fed token by token costs n decode steps (see the bench line)",
+                "timing": f"CUDA events around l2c_prefill, median of {reps}; weights larger than L2"}
+        if not q80:
+            line["frac_of_fp32_fma_peak"] = fl / ms / 1e9 / FP32_FMA_TFLOPS
+        print(json.dumps(line), flush=True)
+    dec.close()
 
 
 def main():
@@ -583,15 +639,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--extra", nargs="?", const="all", choices=("all", "small", "batch"),
-                    help="the other workloads (small: tiny, 15M, 110M position curves; batch: GQA-7B batch 32), "
-                         "not bench lines")
+    ap.add_argument("--extra", nargs="?", const="all", choices=("all", "small", "batch", "prefill"),
+                    help="the other workloads (small: tiny, 15M, 110M position curves; batch: GQA-7B batch 32; "
+                         "prefill: a 128-token 7B prompt), not bench lines")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling case: the 7B widths with this many layers (not a bench line)")
     args = ap.parse_args()
     if args.layers:
         global SPEC
-        import dataclasses
         SPEC = dataclasses.replace(synth.L7B, name=f"7B-width-{args.layers}L", n_layers=args.layers)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -20,7 +20,7 @@ L2C_OK, L2C_E_ARG, L2C_E_OOM, L2C_E_CUDA, L2C_E_DEVICE, L2C_E_STATE, L2C_E_SCRAT
 # every symbol declared in include/l2c.h
 EXPORTS = (
     "l2c_blob_floats", "l2c_create", "l2c_enable_q80", "l2c_forward", "l2c_forward_q80", "l2c_argmax",
-    "l2c_generate", "l2c_sample", "l2c_forward_batch", "l2c_quantize_q80", "l2c_q80_group_dots", "l2c_kv_load",
+    "l2c_generate", "l2c_sample", "l2c_forward_batch", "l2c_prefill", "l2c_quantize_q80", "l2c_q80_group_dots", "l2c_kv_load",
     "l2c_kv_read", "l2c_kv_reset", "l2c_attention", "l2c_attention_noalloc", "l2c_time_kernel", "l2c_sync", "l2c_stream", "l2c_last_status", "l2c_last_error",
     "l2c_destroy",
 )
@@ -62,6 +62,7 @@ def lib():
             "l2c_sample": (i32, [vp, vp, i32, ctypes.c_float, ctypes.c_float, ctypes.c_double,
                                  ctypes.POINTER(ctypes.c_int)]),
             "l2c_forward_batch": (i32, [vp, i32, vp, vp, i32, vp]),
+            "l2c_prefill": (i32, [vp, i32, i32, vp, i32, i32, vp]),
             "l2c_quantize_q80": (i32, [vp, vp, i64, i32, vp, vp]),
             "l2c_q80_group_dots": (i32, [vp, vp, vp, i32, i32, i32, vp]),
             "l2c_kv_load": (i32, [vp, i32, i32, vp, vp]),
@@ -177,6 +178,13 @@ class Decoder:
     def forward_batch(self, tokens, pos, logits_out, q80: bool = True):
         self._check(lib().l2c_forward_batch(self._h, int(tokens.numel() if hasattr(tokens, "numel") else tokens.size),
                                             _ptr(tokens), _ptr(pos), int(q80), _ptr(logits_out)))
+
+    def prefill(self, tokens, pos0: int = 0, q80: bool = False, logits_last=None, seq: int = 0):
+        """Prompt tokens (host int32) at positions pos0.. of sequence seq, as GEMMs
+        (l2c_prefill); the last token's logits go to logits_last (device, optional)."""
+        toks = np.ascontiguousarray(tokens, dtype=np.int32)
+        self._check(lib().l2c_prefill(self._h, int(seq), int(toks.size), toks.ctypes.data, int(pos0), int(q80),
+                                      _ptr(logits_last) if logits_last is not None else None))
 
     # -- KV cache
     def kv_load(self, k, v, seq: int = 0):

@@ -50,6 +50,8 @@ struct AttnArgs {
     int H, Hkv, hs, kvd, seq_len;
     int nchunks;         // gridDim.x: the positions 0..pos are split into at most this many chunks
     int min_chunk;       // ... of at least this many positions each
+    int shared_kv;       // 1: every entry reads one cache (the tokens of a prompt chunk, positions rising from
+                         // entry 0's): rows from entry 0's position on come from the kernel before
     void* part;          // partials [B][Hkv][nchunks][rep][hs+2] (Acc)
     int* count;          // [B][Hkv] arrival counters (zero between launches)
 };
@@ -79,8 +81,15 @@ __device__ __forceinline__ void widen4(const float4 v, Acc (&w)[4]) {
     }
 }
 
-constexpr int ATTN_WARPS = 4;
+constexpr int ATTN_WARPS = 4;       // warps of a double-precision attention CTA
 constexpr int ATTN_THREADS = 32 * ATTN_WARPS;
+constexpr int ATTN_WARPS_F32 = 8;   // warps of an fp32 attention CTA (one CTA per SM: more loads in flight)
+
+// Threads of an attention CTA of accumulator type Acc.
+template <typename Acc>
+constexpr int attn_threads() {
+    return sizeof(Acc) == 8 ? ATTN_THREADS : 32 * ATTN_WARPS_F32;
+}
 constexpr int ATTN_NB = 3;  // batches in each lane's shared-memory ring
 
 // Positions a warp loads at once (one batch): fewer in double or when the
@@ -109,7 +118,7 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 // The merge of a work item's four warps and of the chunks of (b, g); every
 // thread of the CTA calls it after its warp's online softmax is done.
-template <typename Acc, int HS, int REP>
+template <typename Acc, int HS, int REP, int NW>
 __device__ __forceinline__ void attn_finish(const AttnArgs& a, int c, int g, int b, int nact, const Acc (&m)[REP],
                                             const Acc (&l)[REP], const Acc (&o)[REP][4], Acc (*sm_m)[REP],
                                             Acc (*sm_l)[REP], Acc (*sm_o)[REP][HS], int* last_s) {
@@ -131,14 +140,14 @@ __device__ __forceinline__ void attn_finish(const AttnArgs& a, int c, int g, int
     }
     __syncthreads();
     Acc* part = static_cast<Acc*>(a.part) + ((((size_t)b * a.Hkv + g) * a.nchunks + c) * REP) * (HS + 2);
-    for (int i = tid; i < REP * HS; i += ATTN_THREADS) {
+    for (int i = tid; i < REP * HS; i += (32 * NW)) {
         const int h = i / HS, e = i % HS;
         Acc M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < ATTN_WARPS; w++) M = max(M, sm_m[w][h]);
+        for (int w = 0; w < NW; w++) M = max(M, sm_m[w][h]);
         Acc L = 0, O = 0;
 #pragma unroll
-        for (int w = 0; w < ATTN_WARPS; w++) {
+        for (int w = 0; w < NW; w++) {
             const Acc f = sm_m[w][h] == -INFINITY ? (Acc)0 : exp(sm_m[w][h] - M);
             L += sm_l[w][h] * f;
             O += sm_o[w][h][e] * f;
@@ -163,7 +172,7 @@ __device__ __forceinline__ void attn_finish(const AttnArgs& a, int c, int g, int
     if (!*last_s) return;
     __threadfence();
     const Acc* p0 = static_cast<const Acc*>(a.part) + (((size_t)b * a.Hkv + g) * a.nchunks * REP) * (HS + 2);
-    for (int i = tid; i < REP * HS; i += ATTN_THREADS) {
+    for (int i = tid; i < REP * HS; i += (32 * NW)) {
         const int h = i / HS, e = i % HS;
         Acc M = -INFINITY;
         for (int k = 0; k < nact; k++) M = max(M, __ldcg(p0 + ((size_t)k * REP + h) * (HS + 2) + HS));
@@ -227,10 +236,19 @@ __device__ __forceinline__ void attn_batch(int n, KV kv, const Acc (&qr)[REP][4]
 }
 
 // The work item of CTA (c, g, b): its chunk [t0, t1) and the number of
-// active chunks of sequence b; false when this CTA has no positions.
-__device__ __forceinline__ bool attn_item(const AttnArgs& a, int c, int b, int& t0, int& t1, int& nact, int& pos) {
+// active chunks of sequence b; false when this CTA has no positions.  Rows
+// before `fresh` were written before the step (readable before the
+// dependency wait): all rows before the entry's own position, or with a
+// shared cache those before entry 0's position.
+__device__ __forceinline__ bool attn_item(const AttnArgs& a, int c, int b, int& t0, int& t1, int& nact, int& pos,
+                                          int& fresh) {
     pos = a.tp[b * a.tp_stride + 1];  // written before the step: readable before the wait
     if (pos < 0 || pos >= a.seq_len) pos = 0;  // the q/k/v kernel has flagged it
+    fresh = pos;
+    if (a.shared_kv) {
+        const int p0 = a.tp[1];
+        fresh = p0 < 0 ? 0 : (p0 < pos ? p0 : pos);
+    }
     const int T = pos + 1;
     nact = (T + a.min_chunk - 1) / a.min_chunk;
     if (nact > a.nchunks) nact = a.nchunks;
@@ -247,25 +265,26 @@ struct AttnPBF {  // fp32 kernel: positions per batch
     static constexpr int value = REP >= 3 ? 4 : 8;
 };
 
-// fp32 attention, grid (nchunks, Hkv, B), ATTN_THREADS threads, no dynamic
-// shared memory (the fp32 step's kernels keep the default L1 / shared split).
-// The chunk's positions go in batches of PB to the four warps in turn; a lane
+// fp32 attention, grid (nchunks, Hkv, B), 32 * ATTN_WARPS_F32 threads, no
+// dynamic shared memory (the fp32 step's kernels keep the default L1 / shared
+// split).  The chunk's positions go in batches of PB to the warps in turn; a lane
 // holds one float4 of each K and V row slice (hs <= 128) in registers, and
 // every warp keeps the next batch's 128-bit loads in flight while it computes
 // the current one.
 template <int HS, int REP>
-__global__ void __launch_bounds__(ATTN_THREADS) k_attention_f32(const AttnArgs a) {
+__global__ void __launch_bounds__(32 * ATTN_WARPS_F32) k_attention_f32(const AttnArgs a) {
     constexpr int V4 = HS / 4;
     constexpr int PB = AttnPBF<REP>::value;
     static_assert(HS % 4 == 0 && HS <= 128, "head size");
-    __shared__ float sm_m[ATTN_WARPS][REP], sm_l[ATTN_WARPS][REP];
-    __shared__ float sm_o[ATTN_WARPS][REP][HS];
+    __shared__ float sm_m[ATTN_WARPS_F32][REP], sm_l[ATTN_WARPS_F32][REP];
+    __shared__ float sm_o[ATTN_WARPS_F32][REP][HS];
     __shared__ int last_s;
     const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool lane_on = lane < V4;
     int t0, t1, nact, pos;
-    if (!attn_item(a, c, b, t0, t1, nact, pos)) return;
+    int fresh;
+    if (!attn_item(a, c, b, t0, t1, nact, pos, fresh)) return;
     const int nb = (t1 - t0 + PB - 1) / PB;
     const float* kc = a.kc + (size_t)b * a.seq_stride + (size_t)g * HS + 4 * lane;
     const float* vc = a.vc + (size_t)b * a.seq_stride + (size_t)g * HS + 4 * lane;
@@ -283,9 +302,9 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention_f32(const AttnArgs a
     };
     float4 ka[PB], va[PB], kb[PB], vb[PB];
     int bi = warp;
-    // the warp's first batch, if all its rows precede the current position,
-    // is read before the wait (only row pos comes from the kernel before)
-    const bool early = bi < nb && t0 + (bi + 1) * PB <= pos;
+    // the warp's first batch, if all its rows precede `fresh` (rows from
+    // there on come from the kernel before), is read before the wait
+    const bool early = bi < nb && t0 + (bi + 1) * PB <= fresh;
     if (early) load(bi, ka, va);
     grid_dep_wait();
     grid_dep_launch();
@@ -308,17 +327,17 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention_f32(const AttnArgs a
     }
     // two register buffers: batch bi in (ka, va), the next one loading into (kb, vb)
     while (bi < nb) {
-        if (bi + ATTN_WARPS < nb) load(bi + ATTN_WARPS, kb, vb);
+        if (bi + ATTN_WARPS_F32 < nb) load(bi + ATTN_WARPS_F32, kb, vb);
         attn_batch<float, REP, PB>(min(PB, t1 - (t0 + bi * PB)),
                                    [&](int i, int kv) { return kv ? va[i] : ka[i]; }, qr, scale, m, l, o);
-        bi += ATTN_WARPS;
+        bi += ATTN_WARPS_F32;
         if (bi >= nb) break;
-        if (bi + ATTN_WARPS < nb) load(bi + ATTN_WARPS, ka, va);
+        if (bi + ATTN_WARPS_F32 < nb) load(bi + ATTN_WARPS_F32, ka, va);
         attn_batch<float, REP, PB>(min(PB, t1 - (t0 + bi * PB)),
                                    [&](int i, int kv) { return kv ? vb[i] : kb[i]; }, qr, scale, m, l, o);
-        bi += ATTN_WARPS;
+        bi += ATTN_WARPS_F32;
     }
-    attn_finish<float, HS, REP>(a, c, g, b, nact, m, l, o, sm_m, sm_l, sm_o, &last_s);
+    attn_finish<float, HS, REP, ATTN_WARPS_F32>(a, c, g, b, nact, m, l, o, sm_m, sm_l, sm_o, &last_s);
 }
 
 // grid (nchunks, Hkv, B), ATTN_THREADS threads, attn_ring_bytes<Acc, REP>()
@@ -342,7 +361,8 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool lane_on = lane < V4;
     int t0, t1, nact, pos;
-    if (!attn_item(a, c, b, t0, t1, nact, pos)) return;
+    int fresh;
+    if (!attn_item(a, c, b, t0, t1, nact, pos, fresh)) return;
     const int nb = (t1 - t0 + PB - 1) / PB;   // batches of the chunk; warp w takes w, w+4, ...
     const float* kc = a.kc + (size_t)b * a.seq_stride + (size_t)g * HS + 4 * (lane_on ? lane : 0);
     const float* vc = a.vc + (size_t)b * a.seq_stride + (size_t)g * HS + 4 * (lane_on ? lane : 0);
@@ -364,9 +384,9 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
         }
         cp_async_commit();
     };
-    // a batch whose rows all precede the current position (only row pos comes
-    // from the kernel before) may be copied before the dependency wait
-    auto before_wait_ok = [&](int jj) { return t0 + (warp + ATTN_WARPS * jj + 1) * PB <= pos; };
+    // a batch whose rows all precede `fresh` (rows from there on come from
+    // the kernel before) may be copied before the dependency wait
+    auto before_wait_ok = [&](int jj) { return t0 + (warp + ATTN_WARPS * jj + 1) * PB <= fresh; };
     int nissued = 0;
     while (nissued < ATTN_NB - 1 && before_wait_ok(nissued)) issue(nissued++);
     grid_dep_wait();
@@ -414,7 +434,7 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
 #pragma unroll
             for (int h = 0; h < REP; h++) o[h][0] = o[h][1] = o[h][2] = o[h][3] = (Acc)NAN;
     }
-    attn_finish<Acc, HS, REP>(a, c, g, b, nact, m, l, o, sm_m, sm_l, sm_o, &last_s);
+    attn_finish<Acc, HS, REP, ATTN_WARPS>(a, c, g, b, nact, m, l, o, sm_m, sm_l, sm_o, &last_s);
 }
 
 typedef void (*AttnKernel)(const AttnArgs);

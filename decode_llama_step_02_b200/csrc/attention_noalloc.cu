@@ -132,7 +132,8 @@ extern "C" int l2c_attention_noalloc(const float* q_dev, const float* k_dev, con
     t.min_chunk = kChunk;
     t.part = scratch + 256 + cnt_bytes; t.count = counters;
     const int smem = precision ? attn_smem_for<double>(rep) : attn_smem_for<float>(rep);
-    ak<<<dim3(nchunks, n_kv_heads, 1), ATTN_THREADS, smem, s>>>(t);
+    const int threads = precision ? attn_threads<double>() : attn_threads<float>();
+    ak<<<dim3(nchunks, n_kv_heads, 1), threads, smem, s>>>(t);
     if (cudaGetLastError() != cudaSuccess) return L2C_E_CUDA;
     return L2C_OK;
 }

@@ -101,7 +101,8 @@ __global__ void __launch_bounds__(256) k_bprep(const BPrepArgs a) {
 struct BGemmArgs {
     const uint8_t* W;       // Q8_0 row records [rows][rb]
     size_t rb;
-    int rows, K, gs, kc;    // kc: K bytes per stage (a multiple of 32 and of gs, dividing K)
+    int rows, K, gs, kc;    // kc: K bytes per stage (a multiple of 32 and of gs, dividing K; 4 groups'
+                            // multiple unless kc == K)
     int B;                  // live sequences (<= BMAX); codes of the others are zero
     const int8_t* xq;       // [BMAX][kq_stride]
     const double* xs;       // [BMAX][ks_stride] activation scales in double
@@ -222,7 +223,11 @@ __global__ void __launch_bounds__(32 * (BG_WARPS + 1)) k_bgemm_q8(const BGemmArg
     const int nrows = min(BG_ROWS, a.rows - r0);
     const int nchunks = a.K / a.kc;
     const int gpc = a.kc / a.gs;                 // groups per chunk
-    const size_t sc_bytes = (size_t)gpc * 4;     // scale bytes per row per chunk (multiple of 16 by construction)
+    const size_t sc_bytes = (size_t)gpc * 4;     // scale bytes per row per chunk
+    // copy sizes: multiples of 16 bytes (with one chunk, kc == K, the copy runs
+    // into the padding of the weight record / of the activation scale row)
+    const uint32_t wsc_copy = (uint32_t)((sc_bytes + 15) & ~size_t(15));
+    const uint32_t xsc_copy = (uint32_t)((2 * sc_bytes + 15) & ~size_t(15));
     uint64_t* full = reinterpret_cast<uint64_t*>(bsm + (size_t)L.ns * L.stage_bytes);
     uint64_t* empty = full + L.ns;
 
@@ -249,8 +254,7 @@ __global__ void __launch_bounds__(32 * (BG_WARPS + 1)) k_bgemm_q8(const BGemmArg
         }
         // activations come from the prep kernel: wait for it before copying them
         grid_dep_wait();
-        const uint32_t bytes_stage =
-            (uint32_t)((size_t)nrows * (a.kc + sc_bytes) + (size_t)BMAX * (a.kc + 2 * sc_bytes));
+        const uint32_t bytes_stage = (uint32_t)((size_t)nrows * (a.kc + wsc_copy) + (size_t)BMAX * (a.kc + xsc_copy));
         bool ok = true;
         int issued = 0;
         for (int c = 0; c < nchunks && ok; c++) {
@@ -267,15 +271,15 @@ __global__ void __launch_bounds__(32 * (BG_WARPS + 1)) k_bgemm_q8(const BGemmArg
             for (int r = lane; r < nrows; r += 32) {
                 const uint8_t* rec = Wb + (size_t)r * a.rb;
                 bulk_g2s(st + L.w_off + (size_t)r * L.kcp, rec + (size_t)c * a.kc, a.kc, &full[s], pol_w);
-                bulk_g2s(st + L.ws_off + (size_t)r * ((sc_bytes + 15) & ~size_t(15)),
-                         rec + a.K + (size_t)c * sc_bytes, (uint32_t)sc_bytes, &full[s], pol_w);
+                bulk_g2s(st + L.ws_off + (size_t)r * wsc_copy, rec + a.K + (size_t)c * sc_bytes, wsc_copy, &full[s],
+                         pol_w);
             }
             for (int b = lane; b < BMAX; b += 32) {
                 bulk_g2s(st + L.x_off + (size_t)b * L.kcp, a.xq + (size_t)b * a.kq_stride + (size_t)c * a.kc, a.kc,
                          &full[s], pol_x);
-                bulk_g2s(st + L.xs_off + (size_t)b * ((2 * sc_bytes + 15) & ~size_t(15)),
+                bulk_g2s(st + L.xs_off + (size_t)b * xsc_copy,
                          reinterpret_cast<const uint8_t*>(a.xs + (size_t)b * a.ks_stride) + (size_t)c * 2 * sc_bytes,
-                         (uint32_t)(2 * sc_bytes), &full[s], pol_x);
+                         xsc_copy, &full[s], pol_x);
             }
             issued = c + 1;
         }
@@ -342,7 +346,10 @@ __global__ void __launch_bounds__(32 * (BG_WARPS + 1)) k_bgemm_q8(const BGemmArg
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
     }
-    if (!ok) return;
+    // every consumer warp meets the others here, including one that gave up
+    // on a wait (the error word is set): then all of them leave together
+    const SyncNamed cons{1, 32 * BG_WARPS};
+    if (cons.sync_or(!ok)) return;
     // results of this warp's rows -> shared staging (fp32, rounded once)
 #pragma unroll
     for (int n = 0; n < 4; n++) {
@@ -351,8 +358,182 @@ __global__ void __launch_bounds__(32 * (BG_WARPS + 1)) k_bgemm_q8(const BGemmArg
         stage_out[wr0 + gid + 8][8 * n + 2 * tig] = (float)acc[n][2];
         stage_out[wr0 + gid + 8][8 * n + 2 * tig + 1] = (float)acc[n][3];
     }
-    asm volatile("bar.sync 1, %0;" :: "r"(32 * BG_WARPS) : "memory");
+    cons.sync();
     bgemm_epilogue<MODE>(a, r0, nrows, stage_out, best_s, threadIdx.x, 32 * BG_WARPS, 1);
+}
+
+
+// ---------------------------------------------------------------- fp32 path --
+//
+// The fp32 batched step (B <= BMAX sequences, or the tokens of a prompt chunk)
+// has the same shape with fp32 operands: prep_f32 writes each row's RMSNorm
+// (or the embedding row) in fp32, and gemm_f32 multiplies in fp32 on the CUDA
+// cores (FFMA: each weight element feeds B multiply-adds, so at B = 32 the
+// GEMM is bound by the FMA pipes rather than by HBM), with the epilogues above.
+// The attention output and hb feed their GEMMs directly (no norm).
+
+constexpr int BF_ROWS = 32;               // weight rows per CTA
+constexpr int BF_KT = 64;                 // K per stage
+constexpr int BF_PITCH = BF_KT + 4;       // floats per shared row: conflict-free 16-byte reads
+constexpr int BF_STAGES = 3;
+constexpr int BF_THREADS = 128;
+constexpr int BF_STAGE_FLOATS = (BF_ROWS + BMAX) * BF_PITCH;
+constexpr int BF_SMEM = BF_STAGES * BF_STAGE_FLOATS * 4;
+
+struct BPrepF32Args {
+    const float* in;        // [B][in_stride] (x)
+    size_t in_stride;
+    const float* norm_w;    // RMSNorm gain
+    const float* emb;       // layer 0: fp32 embedding table [vocab][K], else nullptr
+    float* x_resid;         // layer 0: receives the embedding rows [B][K]
+    float* out;             // [B][out_stride] normalized rows
+    size_t out_stride;
+    int K;
+    const int* tp;
+    int vocab;
+    unsigned long long* amax;  // reset per sequence on layer 0
+    int* err;
+};
+
+// CTA (b, y) of a (B, Y) grid: sequence b's row (the embedding row on layer
+// 0), its RMSNorm sum over the whole row in every CTA of the sequence, then
+// w * (inv * x) in double, rounded once, for the y-th of Y equal ranges.
+__global__ void __launch_bounds__(256) k_bprep_f32(const BPrepF32Args a) {
+    extern __shared__ float bpf_x[];
+    __shared__ double red[32];
+    const int b = blockIdx.x;
+    const int K = a.K;
+    const int i0 = (int)((long long)K * blockIdx.y / gridDim.y);
+    const int i1 = (int)((long long)K * (blockIdx.y + 1) / gridDim.y);
+    grid_dep_wait();
+    grid_dep_launch();
+    const float* in = a.in + (size_t)b * a.in_stride;
+    if (a.emb) {
+        int token = a.tp[2 * b];
+        if (token < 0 || token >= a.vocab) {
+            if (threadIdx.x == 0) set_error(a.err, DERR_TOKEN);
+            token = 0;
+        }
+        in = a.emb + (size_t)token * K;
+        if (a.amax && threadIdx.x == 0 && blockIdx.y == 0) a.amax[b] = 0ull;
+    }
+    for (int i = threadIdx.x; i < K; i += blockDim.x) {
+        const float v = in[i];
+        bpf_x[i] = v;
+        if (a.emb && i >= i0 && i < i1) a.x_resid[(size_t)b * K + i] = v;
+    }
+    __syncthreads();
+    double ss = 0.0;
+    for (int i = threadIdx.x; i < K; i += blockDim.x) ss += (double)bpf_x[i] * (double)bpf_x[i];
+    ss = block_sum(ss, red);
+    const double inv = 1.0 / sqrt(ss / (double)K + 1e-5);
+    float* out = a.out + (size_t)b * a.out_stride;
+    for (int i = i0 + (int)threadIdx.x; i < i1; i += blockDim.x)
+        out[i] = (float)((double)a.norm_w[i] * (inv * (double)bpf_x[i]));
+}
+
+// 16-byte global -> shared asynchronous copy; with on == false nothing is
+// read and the destination is zero-filled.
+__device__ __forceinline__ void bf_cp16(float* dst, const float* src, bool on, uint64_t pol) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;"
+                 :: "r"(smem_u32(dst)), "l"(src), "r"(on ? 16 : 0), "l"(pol) : "memory");
+}
+
+// grid = ceil(rows / BF_ROWS) CTAs of BF_THREADS threads, BF_SMEM bytes of
+// dynamic shared memory.  CTA i computes rows i*BF_ROWS .. +BF_ROWS-1 for
+// every sequence: Y[b][r] = sum_k W[r][k] X[b][k] in fp32 FMAs.  Stages of
+// BF_KT columns of W (this CTA's rows) and of X (all BMAX rows; rows >= B and
+// columns >= K are zero-filled) stream through a BF_STAGES-deep cp.async
+// ring.  Thread t computes rows 2*(t/8) + {0, 1} for sequences
+// t%8 + {0, 8, 16, 24} in k order, reading 4 consecutive k of each at once.
+// a.W holds the fp32 rows (a.rb bytes apart); X is [B][x_stride].
+template <int MODE>
+__global__ void __launch_bounds__(BF_THREADS) k_bgemm_f32(const BGemmArgs a, const float* X, size_t x_stride) {
+    extern __shared__ __align__(16) float fsm[];
+    __shared__ float stage_out[BF_ROWS][BMAX + 1];
+    __shared__ unsigned long long best_s[BMAX];
+    const int tid = threadIdx.x;
+    const int r0 = blockIdx.x * BF_ROWS;
+    const int nrows = min(BF_ROWS, a.rows - r0);
+    const int K = a.K;
+    const int nkt = (K + BF_KT - 1) / BF_KT;
+    const float* W = reinterpret_cast<const float*>(a.W) + (size_t)r0 * (a.rb / 4);
+    const size_t ldw = a.rb / 4;
+    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_x = policy_evict_last();
+    if (tid < BMAX) best_s[tid] = 0ull;
+    if (tid == 0 && a.prefetch_bytes) {  // weights do not depend on earlier kernels
+        size_t bytes = (size_t)nrows * a.rb;
+        if (bytes > a.prefetch_bytes) bytes = a.prefetch_bytes;
+        prefetch_l2_range(W, bytes & ~size_t(15), policy_evict_last());
+    }
+    grid_dep_wait();
+    grid_dep_launch();
+    auto load = [&](int t) {
+        float* st = fsm + (size_t)(t % BF_STAGES) * BF_STAGE_FLOATS;
+        const int k0 = t * BF_KT;
+#pragma unroll
+        for (int j = 0; j < (BF_ROWS * BF_KT / 4) / BF_THREADS; j++) {
+            const int idx = tid + j * BF_THREADS;
+            const int r = idx / (BF_KT / 4), c4 = idx % (BF_KT / 4);
+            const int k = k0 + 4 * c4;
+            const bool on = r < nrows && k < K;
+            bf_cp16(st + r * BF_PITCH + 4 * c4, on ? W + (size_t)r * ldw + k : W, on, pol_w);
+        }
+#pragma unroll
+        for (int j = 0; j < (BMAX * BF_KT / 4) / BF_THREADS; j++) {
+            const int idx = tid + j * BF_THREADS;
+            const int b = idx / (BF_KT / 4), c4 = idx % (BF_KT / 4);
+            const int k = k0 + 4 * c4;
+            const bool on = b < a.B && k < K;
+            bf_cp16(st + (BF_ROWS + b) * BF_PITCH + 4 * c4, on ? X + (size_t)b * x_stride + k : X, on, pol_x);
+        }
+    };
+#pragma unroll
+    for (int t = 0; t < BF_STAGES - 1; t++) {
+        if (t < nkt) load(t);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    const int sg = tid & 7, rp = tid >> 3;
+    float acc[2][4];
+#pragma unroll
+    for (int i = 0; i < 2; i++) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    for (int t = 0; t < nkt; t++) {
+        asm volatile("cp.async.wait_group %0;" :: "n"(BF_STAGES - 2) : "memory");
+        __syncthreads();  // stage t landed for every thread; stage t-1 is free
+        if (t + BF_STAGES - 1 < nkt) load(t + BF_STAGES - 1);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        const float* wt = fsm + (size_t)(t % BF_STAGES) * BF_STAGE_FLOATS;
+        const float* xt = wt + BF_ROWS * BF_PITCH;
+        // the stage's 16 steps of 4 columns, fully unrolled so that the shared
+        // loads of later steps issue ahead of the FMAs of earlier ones
+        const float* wr = wt + (2 * rp) * BF_PITCH;
+        const float* xr = xt + sg * BF_PITCH;
+#pragma unroll
+        for (int kk = 0; kk < BF_KT; kk += 4) {
+            const float4 w0 = *reinterpret_cast<const float4*>(wr + kk);
+            const float4 w1 = *reinterpret_cast<const float4*>(wr + BF_PITCH + kk);
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const float4 xv = *reinterpret_cast<const float4*>(xr + 8 * j * BF_PITCH + kk);
+                acc[0][j] = fmaf(w0.x, xv.x, acc[0][j]);
+                acc[0][j] = fmaf(w0.y, xv.y, acc[0][j]);
+                acc[0][j] = fmaf(w0.z, xv.z, acc[0][j]);
+                acc[0][j] = fmaf(w0.w, xv.w, acc[0][j]);
+                acc[1][j] = fmaf(w1.x, xv.x, acc[1][j]);
+                acc[1][j] = fmaf(w1.y, xv.y, acc[1][j]);
+                acc[1][j] = fmaf(w1.z, xv.z, acc[1][j]);
+                acc[1][j] = fmaf(w1.w, xv.w, acc[1][j]);
+            }
+        }
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 2; i++)
+#pragma unroll
+        for (int j = 0; j < 4; j++) stage_out[2 * rp + i][sg + 8 * j] = acc[i][j];
+    __syncthreads();
+    bgemm_epilogue<MODE>(a, r0, nrows, stage_out, best_s, tid, BF_THREADS, 1);
 }
 
 }  // namespace l2c

@@ -32,6 +32,18 @@ struct Q8Mat {
     size_t rb = 0;  // record bytes per row
 };
 
+// Activations of a batched step over entries 0..B-1 (sequences of the
+// handle, or the tokens of a prompt chunk) and where their KV caches are.
+struct BatchBufs {
+    float *x = nullptr, *q = nullptr, *att = nullptr, *hb = nullptr, *logits = nullptr;
+    int* tp = nullptr;                   // [cap][2] token, pos
+    unsigned long long* amax = nullptr;  // [cap] argmax keys
+    void* part = nullptr;                // attention partials
+    int* cnt = nullptr;                  // attention arrival counters [cap][Hkv] (zero between launches)
+    size_t cache_off = 0;                // floats from sequence 0's cache to entry 0's
+    size_t seq_stride = 0;               // floats between entries' caches (0: one cache shared by all)
+};
+
 struct l2c_ctx {
     l2c_config c{};
     int shared = 1, max_batch = 1;
@@ -68,7 +80,12 @@ struct l2c_ctx {
     int8_t* bxq = nullptr;
     double* bxs = nullptr;
     size_t bkq = 0, bks = 0;  // strides (bytes of codes, floats of scales) per sequence
-    std::vector<cudaGraphExec_t> bgraph;  // index B (1..max_batch)
+    std::vector<cudaGraphExec_t> bgraph;  // Q8_0, index B (1..max_batch)
+    std::vector<cudaGraphExec_t> bgraph_f32;  // fp32, index B
+    BatchBufs bb;            // the handle's sequences (x, q, ... above)
+    BatchBufs pb;            // prompt chunks of l2c_prefill (allocated on first use, BMAX entries)
+    float* xb = nullptr;     // fp32 batched step: normalized input rows [BMAX][xbs]
+    size_t xbs = 0;
     size_t bgemm_smem = 64 << 10;         // dynamic shared memory a batched GEMM CTA may take
     int bgemm_stages = 3;                 // ring stages (deeper rings cost the second CTA per SM)
     // tuning
@@ -261,6 +278,16 @@ static int set_smem_limits(l2c_ctx* h) {
     CK(cudaFuncSetAttribute(k_bgemm_q8<M_W13>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
     CK(cudaFuncSetAttribute(k_bgemm_q8<M_CLS>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 8192));
     CK(cudaFuncSetAttribute(k_bprep, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+    CK(cudaFuncSetAttribute(k_bprep_f32, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
+    CK(max_carveout(k_bprep_f32));
+    CK(cudaFuncSetAttribute(k_bgemm_f32<M_QKV>, cudaFuncAttributeMaxDynamicSharedMemorySize, BF_SMEM));
+    CK(cudaFuncSetAttribute(k_bgemm_f32<M_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, BF_SMEM));
+    CK(cudaFuncSetAttribute(k_bgemm_f32<M_W13>, cudaFuncAttributeMaxDynamicSharedMemorySize, BF_SMEM));
+    CK(cudaFuncSetAttribute(k_bgemm_f32<M_CLS>, cudaFuncAttributeMaxDynamicSharedMemorySize, BF_SMEM));
+    CK(max_carveout(k_bgemm_f32<M_QKV>));
+    CK(max_carveout(k_bgemm_f32<M_RESID>));
+    CK(max_carveout(k_bgemm_f32<M_W13>));
+    CK(max_carveout(k_bgemm_f32<M_CLS>));
     return L2C_OK;
 }
 
@@ -271,7 +298,9 @@ static int set_smem_limits(l2c_ctx* h) {
 static int attn_nchunks(const l2c_ctx* h, int B, bool dbl) {
     const int target = dbl ? (h->attn_ctas_f64 > 0 ? h->attn_ctas_f64 : 4 * h->sms)
                            : (h->attn_ctas > 0 ? h->attn_ctas : h->sms);
-    int nc = (target + h->Hkv * B - 1) / (h->Hkv * B);
+    // double: enough CTAs to fill the SMs several times (arithmetic-bound);
+    // fp32: at most `target` CTAs of 8 warps (one per SM: no SM gets two)
+    int nc = dbl ? (target + h->Hkv * B - 1) / (h->Hkv * B) : target / (h->Hkv * B);
     const int maxc = (h->S + h->attn_min_chunk - 1) / h->attn_min_chunk;
     if (nc > maxc) nc = maxc;
     return nc < 1 ? 1 : nc;
@@ -279,17 +308,19 @@ static int attn_nchunks(const l2c_ctx* h, int B, bool dbl) {
 
 // Enqueues the attention of one layer over sequences 0..B-1 (grid z).
 static cudaError_t launch_attention(l2c_ctx* h, cudaStream_t s, bool pdl, bool dbl, const float* q, const float* kc,
-                                    const float* vc, size_t seq_stride, float* out, const int* tp, int B) {
+                                    const float* vc, size_t seq_stride, float* out, const int* tp, int B,
+                                    void* part, int* cnt, bool shared_kv = false) {
     AttnArgs t = {};
     t.q = q; t.kc = kc; t.vc = vc; t.seq_stride = seq_stride;
     t.out = out; t.tp = tp; t.tp_stride = 2;
     t.H = h->H; t.Hkv = h->Hkv; t.hs = h->hs; t.kvd = h->kvd; t.seq_len = h->S;
     t.nchunks = attn_nchunks(h, B, dbl);
     t.min_chunk = h->attn_min_chunk;
-    t.part = h->attn_part; t.count = h->attn_cnt;
+    t.part = part; t.count = cnt; t.shared_kv = shared_kv ? 1 : 0;
     AttnKernel ak = dbl ? attn_kernel_for<double>(h->hs, h->rep) : attn_kernel_for<float>(h->hs, h->rep);
     const size_t smem = (size_t)(dbl ? attn_smem_for<double>(h->rep) : attn_smem_for<float>(h->rep));
-    return launch(s, pdl, ak, dim3(t.nchunks, h->Hkv, B), dim3(ATTN_THREADS), smem, t);
+    const int threads = dbl ? attn_threads<double>() : attn_threads<float>();
+    return launch(s, pdl, ak, dim3(t.nchunks, h->Hkv, B), dim3(threads), smem, t);
 }
 
 // Enqueues kernel `kind` of layer l (sequence seq) on stream s.
@@ -332,7 +363,8 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
         e = launch_gemv<M_QKV>(h, q80, a, 2);
         break;
     case SK_ATTN:
-        e = launch_attention(h, s, true, q80, q, kslot, vslot, (size_t)h->L * S * kvd, att, tp, 1);
+        e = launch_attention(h, s, true, q80, q, kslot, vslot, (size_t)h->L * S * kvd, att, tp, 1, h->attn_part,
+                             h->attn_cnt + (size_t)seq * h->Hkv);
         break;
     case SK_WO:  // wo + residual
         a.rows = (int)d; a.K = (int)d;
@@ -380,11 +412,14 @@ static int enqueue_step(l2c_ctx* h, bool q80) {
 // ------------------------------------------------------------- batched step --
 
 // K bytes per GEMM stage: a multiple of 32 (the MMA k) and of 4*gs (16-byte
-// scale copies) that divides K, at most 512.
+// scale copies) that divides K, at most 512; else the whole row in one stage
+// (K a multiple of 32 up to 2048: its scale copies run into the records'
+// padding).
 static int batched_kc(int K, int gs) {
     int unit = 4 * gs > 32 ? 4 * gs : 32;
     for (int kc = 512 - 512 % unit; kc >= unit; kc -= unit)
         if (K % kc == 0) return kc;
+    if (K % 32 == 0 && K % gs == 0 && K <= 2048) return K;
     return 0;
 }
 
@@ -398,32 +433,72 @@ static int ensure_batched(l2c_ctx* h) {
     if ((rc = dalloc(h, (void**)&h->bxs, (size_t)BMAX * h->bks * 8)) != L2C_OK) return rc;
     CK(cudaMemsetAsync(h->bxq, 0, (size_t)BMAX * h->bkq, h->stream));
     CK(cudaMemsetAsync(h->bxs, 0, (size_t)BMAX * h->bks * 8, h->stream));
-    h->bgraph.assign((size_t)h->max_batch + 1, nullptr);
     return L2C_OK;
 }
 
-static int bprep(l2c_ctx* h, cudaStream_t s, int B, const float* in, size_t in_stride, int K, const float* norm,
-                 bool emb, unsigned long long* amax) {
+static int ensure_batched_f32(l2c_ctx* h) {
+    if (h->xb) return L2C_OK;
+    h->xbs = ((size_t)h->d + 3) & ~size_t(3);
+    int rc;
+    if ((rc = dalloc(h, (void**)&h->xb, (size_t)BMAX * h->xbs * 4)) != L2C_OK) return rc;
+    CK(cudaMemsetAsync(h->xb, 0, (size_t)BMAX * h->xbs * 4, h->stream));
+    return L2C_OK;
+}
+
+// The activations of l2c_prefill's prompt chunks (BMAX tokens each).
+static int ensure_prefill(l2c_ctx* h) {
+    if (h->pb.x) return L2C_OK;
+    BatchBufs& p = h->pb;
+    const size_t d = h->d, hh = h->h, V = h->V;
+    const size_t part = (size_t)BMAX * h->Hkv * h->attn_nchunks_max * h->rep * (h->hs + 2) * sizeof(double);
+    int rc;
+    if ((rc = dalloc(h, (void**)&p.x, BMAX * d * 4)) != L2C_OK) return rc;
+    if ((rc = dalloc(h, (void**)&p.q, BMAX * d * 4)) != L2C_OK) return rc;
+    if ((rc = dalloc(h, (void**)&p.att, BMAX * d * 4)) != L2C_OK) return rc;
+    if ((rc = dalloc(h, (void**)&p.hb, BMAX * hh * 4)) != L2C_OK) return rc;
+    if ((rc = dalloc(h, (void**)&p.logits, BMAX * V * 4)) != L2C_OK) return rc;
+    if ((rc = dalloc(h, (void**)&p.tp, BMAX * 2 * 4)) != L2C_OK) return rc;
+    if ((rc = dalloc(h, (void**)&p.amax, BMAX * 8)) != L2C_OK) return rc;
+    if ((rc = dalloc(h, &p.part, part)) != L2C_OK) return rc;
+    if ((rc = dalloc(h, (void**)&p.cnt, (size_t)BMAX * h->Hkv * 4)) != L2C_OK) return rc;
+    CK(cudaMemsetAsync(p.cnt, 0, (size_t)BMAX * h->Hkv * 4, h->stream));
+    CK(cudaMemsetAsync(p.tp, 0, BMAX * 2 * 4, h->stream));
+    return L2C_OK;
+}
+
+static int bprep(l2c_ctx* h, cudaStream_t s, int B, const BatchBufs& bb, const float* in, size_t in_stride, int K,
+                 const float* norm, bool emb, unsigned long long* amax) {
     BPrepArgs p = {};
     p.in = in; p.in_stride = in_stride; p.norm_w = norm;
-    p.emb = emb ? h->qE.p : nullptr; p.emb_rb = h->qE.rb; p.x_resid = h->x;
+    p.emb = emb ? h->qE.p : nullptr; p.emb_rb = h->qE.rb; p.x_resid = bb.x;
     p.K = K; p.gs = h->gs; p.xq = h->bxq; p.xs = h->bxs; p.kq_stride = h->bkq; p.ks_stride = h->bks;
-    p.tp = h->tp; p.vocab = h->V; p.seq_len = h->S; p.amax = amax; p.err = h->err;
+    p.tp = bb.tp; p.vocab = h->V; p.seq_len = h->S; p.amax = amax; p.err = h->err;
     CK(launch(s, true, k_bprep, dim3(B, BPREP_SPLIT), dim3(256), (size_t)K * 4, p));
     return L2C_OK;
 }
 
-template <int MODE>
-static int bgemm(l2c_ctx* h, cudaStream_t s, int B, const Q8Mat& m, size_t row0, int rows, int K, float* out,
-                 size_t out_stride, int l) {
+// The epilogue fields of a batched GEMM over rows [row0, row0 + rows) of a
+// layer-l matrix.
+static BGemmArgs bgemm_args(l2c_ctx* h, int B, const BatchBufs& bb, int rows, int K, float* out, size_t out_stride,
+                            int l) {
     BGemmArgs g = {};
-    g.W = m.p + row0 * m.rb; g.rb = m.rb; g.rows = rows; g.K = K; g.gs = h->gs; g.kc = batched_kc(K, h->gs);
-    g.B = B; g.xq = h->bxq; g.xs = h->bxs; g.kq_stride = h->bkq; g.ks_stride = h->bks;
+    g.rows = rows; g.K = K; g.gs = h->gs; g.B = B;
     g.out = out; g.out_stride = out_stride;
-    g.kc_base = h->kc + (size_t)l * h->S * h->kvd; g.vc_base = h->vc + (size_t)l * h->S * h->kvd;
-    g.seq_stride = (size_t)h->L * h->S * h->kvd;
+    g.kc_base = h->kc + bb.cache_off + (size_t)l * h->S * h->kvd;
+    g.vc_base = h->vc + bb.cache_off + (size_t)l * h->S * h->kvd;
+    g.seq_stride = bb.seq_stride;
     g.freq = h->freq; g.d = h->d; g.kvd = h->kvd; g.hs = h->hs; g.seq_len = h->S;
-    g.tp = h->tp; g.amax = h->amax; g.err = h->err; g.prefetch_bytes = h->pf_q8;
+    g.tp = bb.tp; g.amax = bb.amax; g.err = h->err;
+    return g;
+}
+
+template <int MODE>
+static int bgemm(l2c_ctx* h, cudaStream_t s, int B, const BatchBufs& bb, const Q8Mat& m, size_t row0, int rows,
+                 int K, float* out, size_t out_stride, int l) {
+    BGemmArgs g = bgemm_args(h, B, bb, rows, K, out, out_stride, l);
+    g.W = m.p + row0 * m.rb; g.rb = m.rb; g.kc = batched_kc(K, h->gs);
+    g.xq = h->bxq; g.xs = h->bxs; g.kq_stride = h->bkq; g.ks_stride = h->bks;
+    g.prefetch_bytes = h->pf_q8;
     // as many ring stages as the shared memory holds (2..16): the weight slices
     // of one stage are small, so the depth sets the bytes in flight
     BLayout L = make_blayout(g.kc, h->gs, 1);
@@ -436,33 +511,90 @@ static int bgemm(l2c_ctx* h, cudaStream_t s, int B, const Q8Mat& m, size_t row0,
     return L2C_OK;
 }
 
-// One batched Q8_0 step of sequences 0..B-1 on stream s.
-static int enqueue_batch_step(l2c_ctx* h, cudaStream_t s, int B) {
+// fp32: RMSNorm (or the layer-0 embedding row and its norm) of entries 0..B-1 -> h->xb.
+static int bprep_f32(l2c_ctx* h, cudaStream_t s, int B, const BatchBufs& bb, const float* norm, bool emb,
+                     unsigned long long* amax) {
+    BPrepF32Args p = {};
+    p.in = bb.x; p.in_stride = h->d; p.norm_w = norm;
+    p.emb = emb ? h->E : nullptr; p.x_resid = bb.x;
+    p.out = h->xb; p.out_stride = h->xbs; p.K = h->d;
+    p.tp = bb.tp; p.vocab = h->V; p.amax = amax; p.err = h->err;
+    CK(launch(s, true, k_bprep_f32, dim3(B, BPREP_SPLIT), dim3(256), (size_t)h->d * 4, p));
+    return L2C_OK;
+}
+
+template <int MODE>
+static int bgemm_f32(l2c_ctx* h, cudaStream_t s, int B, const BatchBufs& bb, const float* W, int rows, int K,
+                     const float* X, size_t x_stride, float* out, size_t out_stride, int l) {
+    BGemmArgs g = bgemm_args(h, B, bb, rows, K, out, out_stride, l);
+    g.W = reinterpret_cast<const uint8_t*>(W); g.rb = (size_t)K * 4;
+    g.prefetch_bytes = h->pf_f32;
+    const int grid = (rows + BF_ROWS - 1) / BF_ROWS;
+    CK(launch(s, true, k_bgemm_f32<MODE>, dim3(grid), dim3(BF_THREADS), (size_t)BF_SMEM, g, X, x_stride));
+    return L2C_OK;
+}
+
+// One batched step of entries 0..B-1 of `bb` on stream s: Q8_0 (int8 tensor
+// cores, double group sums) or fp32 (FFMA).  With shared_kv every entry
+// reads and writes one cache (a prompt chunk).
+static int enqueue_batch_step(l2c_ctx* h, cudaStream_t s, int B, const BatchBufs& bb, bool q80, bool shared_kv) {
     g_pdl = h->pdl;
     const size_t d = h->d, hh = h->h, kvd = h->kvd, S = h->S;
     int rc;
     for (int l = 0; l < h->L; l++) {
-        if ((rc = bprep(h, s, B, h->x, d, (int)d, h->rms_att + (size_t)l * d, l == 0, l == 0 ? h->amax : nullptr)))
-            return rc;
-        if ((rc = bgemm<M_QKV>(h, s, B, h->qWqkv, (size_t)l * (d + 2 * kvd), (int)(d + 2 * kvd), (int)d, h->q, d, l)))
-            return rc;
-        CK(launch_attention(h, s, true, true, h->q, h->kc + (size_t)l * S * kvd, h->vc + (size_t)l * S * kvd,
-                            (size_t)h->L * S * kvd, h->att, h->tp, B));
-        if ((rc = bprep(h, s, B, h->att, d, (int)d, nullptr, false, nullptr))) return rc;
-        if ((rc = bgemm<M_RESID>(h, s, B, h->qWo, (size_t)l * d, (int)d, (int)d, h->x, d, l))) return rc;
-        if ((rc = bprep(h, s, B, h->x, d, (int)d, h->rms_ffn + (size_t)l * d, false, nullptr))) return rc;
-        if ((rc = bgemm<M_W13>(h, s, B, h->qW13, (size_t)l * 2 * hh, (int)(2 * hh), (int)d, h->hb, hh, l))) return rc;
-        if ((rc = bprep(h, s, B, h->hb, hh, (int)hh, nullptr, false, nullptr))) return rc;
-        if ((rc = bgemm<M_RESID>(h, s, B, h->qW2, (size_t)l * d, (int)d, (int)hh, h->x, d, l))) return rc;
+        const float* kl = h->kc + bb.cache_off + (size_t)l * S * kvd;
+        const float* vl = h->vc + bb.cache_off + (size_t)l * S * kvd;
+        if (q80) {
+            if ((rc = bprep(h, s, B, bb, bb.x, d, (int)d, h->rms_att + (size_t)l * d, l == 0,
+                            l == 0 ? bb.amax : nullptr)))
+                return rc;
+            if ((rc = bgemm<M_QKV>(h, s, B, bb, h->qWqkv, (size_t)l * (d + 2 * kvd), (int)(d + 2 * kvd), (int)d,
+                                   bb.q, d, l)))
+                return rc;
+        } else {
+            if ((rc = bprep_f32(h, s, B, bb, h->rms_att + (size_t)l * d, l == 0, l == 0 ? bb.amax : nullptr)))
+                return rc;
+            if ((rc = bgemm_f32<M_QKV>(h, s, B, bb, h->Wqkv + (size_t)l * (d + 2 * kvd) * d, (int)(d + 2 * kvd),
+                                       (int)d, h->xb, h->xbs, bb.q, d, l)))
+                return rc;
+        }
+        CK(launch_attention(h, s, true, q80, bb.q, kl, vl, bb.seq_stride, bb.att, bb.tp, B, bb.part, bb.cnt,
+                            shared_kv));
+        if (q80) {
+            if ((rc = bprep(h, s, B, bb, bb.att, d, (int)d, nullptr, false, nullptr))) return rc;
+            if ((rc = bgemm<M_RESID>(h, s, B, bb, h->qWo, (size_t)l * d, (int)d, (int)d, bb.x, d, l))) return rc;
+            if ((rc = bprep(h, s, B, bb, bb.x, d, (int)d, h->rms_ffn + (size_t)l * d, false, nullptr))) return rc;
+            if ((rc = bgemm<M_W13>(h, s, B, bb, h->qW13, (size_t)l * 2 * hh, (int)(2 * hh), (int)d, bb.hb, hh, l)))
+                return rc;
+            if ((rc = bprep(h, s, B, bb, bb.hb, hh, (int)hh, nullptr, false, nullptr))) return rc;
+            if ((rc = bgemm<M_RESID>(h, s, B, bb, h->qW2, (size_t)l * d, (int)d, (int)hh, bb.x, d, l))) return rc;
+        } else {
+            if ((rc = bgemm_f32<M_RESID>(h, s, B, bb, h->Wo + (size_t)l * d * d, (int)d, (int)d, bb.att, d, bb.x, d,
+                                         l)))
+                return rc;
+            if ((rc = bprep_f32(h, s, B, bb, h->rms_ffn + (size_t)l * d, false, nullptr))) return rc;
+            if ((rc = bgemm_f32<M_W13>(h, s, B, bb, h->W13 + (size_t)l * 2 * hh * d, (int)(2 * hh), (int)d, h->xb,
+                                       h->xbs, bb.hb, hh, l)))
+                return rc;
+            if ((rc = bgemm_f32<M_RESID>(h, s, B, bb, h->W2 + (size_t)l * d * hh, (int)d, (int)hh, bb.hb, hh, bb.x,
+                                         d, l)))
+                return rc;
+        }
     }
-    if ((rc = bprep(h, s, B, h->x, d, (int)d, h->rms_final, false, nullptr))) return rc;
-    return bgemm<M_CLS>(h, s, B, h->qWcls, 0, h->V, (int)d, h->logits, (size_t)h->V, 0);
+    if (q80) {
+        if ((rc = bprep(h, s, B, bb, bb.x, d, (int)d, h->rms_final, false, nullptr))) return rc;
+        return bgemm<M_CLS>(h, s, B, bb, h->qWcls, 0, h->V, (int)d, bb.logits, (size_t)h->V, 0);
+    }
+    if ((rc = bprep_f32(h, s, B, bb, h->rms_final, false, nullptr))) return rc;
+    return bgemm_f32<M_CLS>(h, s, B, bb, h->Wcls, h->V, (int)d, h->xb, h->xbs, bb.logits, (size_t)h->V, 0);
 }
 
-static int build_batch_graph(l2c_ctx* h, int B) {
-    if (h->bgraph[B]) return L2C_OK;
+static int build_batch_graph(l2c_ctx* h, int B, bool q80) {
+    std::vector<cudaGraphExec_t>& gv = q80 ? h->bgraph : h->bgraph_f32;
+    if (gv.size() < (size_t)h->max_batch + 1) gv.assign((size_t)h->max_batch + 1, nullptr);
+    if (gv[B]) return L2C_OK;
     CK(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
-    int rc = enqueue_batch_step(h, h->cap, B);
+    int rc = enqueue_batch_step(h, h->cap, B, h->bb, q80, false);
     cudaGraph_t g = nullptr;
     cudaError_t e = cudaStreamEndCapture(h->cap, &g);
     if (rc != L2C_OK) {
@@ -470,7 +602,7 @@ static int build_batch_graph(l2c_ctx* h, int B) {
         return rc;
     }
     if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "batched capture failed: %s", cudaGetErrorString(e));
-    e = cudaGraphInstantiate(&h->bgraph[B], g, 0);
+    e = cudaGraphInstantiate(&gv[B], g, 0);
     cudaGraphDestroy(g);
     if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "batched graph instantiate: %s", cudaGetErrorString(e));
     return L2C_OK;
@@ -612,6 +744,10 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
     ALLOC(h->stall, 4);
     ALLOC(h->attn_cnt, B * (size_t)h->Hkv * 4);
 #undef ALLOC
+    h->bb.x = h->x; h->bb.q = h->q; h->bb.att = h->att; h->bb.hb = h->hb; h->bb.logits = h->logits;
+    h->bb.tp = h->tp; h->bb.amax = h->amax; h->bb.part = h->attn_part; h->bb.cnt = h->attn_cnt;
+    h->bb.cache_off = 0;
+    h->bb.seq_stride = L * S * kvd;
     // zero state
     if (cudaMemsetAsync(h->kc, 0, B * L * S * kvd * 4, h->stream) != cudaSuccess ||
         cudaMemsetAsync(h->vc, 0, B * L * S * kvd * 4, h->stream) != cudaSuccess ||
@@ -758,7 +894,7 @@ extern "C" int l2c_forward_batch(l2c_ctx* h, int B, const int32_t* tokens, const
     if (!h || !tokens || !pos || !logits_out || B < 1 || B > h->max_batch)
         return fail(h, L2C_E_ARG, "forward_batch: need 1 <= B <= max_batch and non-null arrays");
     if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
-    if (q80 && B > BMAX) return fail(h, L2C_E_ARG, "forward_batch: the Q8_0 batched step takes at most %d sequences", BMAX);
+    if (B > BMAX) return fail(h, L2C_E_ARG, "forward_batch: the batched step takes at most %d sequences", BMAX);
     const bool tok_dev = is_device_ptr(tokens), pos_dev = is_device_ptr(pos);
     if (!tok_dev && !pos_dev) {
         for (int b = 0; b < B; b++) {
@@ -777,23 +913,57 @@ extern "C" int l2c_forward_batch(l2c_ctx* h, int B, const int32_t* tokens, const
         if (batched_kc(h->d, h->gs) == 0 || batched_kc(h->h, h->gs) == 0 || h->gs % 32)
             return fail(h, L2C_E_ARG, "batched Q8_0 step needs gs a multiple of 32 and widths it tiles");
         if ((rc = ensure_batched(h))) return rc;
-        if (h->graphs) {
-            if ((rc = build_batch_graph(h, B))) return rc;
-            CK(cudaGraphLaunch(h->bgraph[B], h->stream));
-        } else if ((rc = enqueue_batch_step(h, h->stream, B))) {
-            return rc;
-        }
-    } else {
-        // fp32: the single-sequence kernels, one sequence after another
-        for (int b = 0; b < B; b++) {
-            for (int l = 0; l < h->L; l++)
-                for (int k = SK_QKV; k <= SK_W2; k++)
-                    if ((rc = launch_step_kernel(h, h->stream, k, false, l, b))) return rc;
-            if ((rc = launch_step_kernel(h, h->stream, SK_CLS, false, 0, b))) return rc;
-        }
+    } else if ((rc = ensure_batched_f32(h))) {
+        return rc;
+    }
+    if (h->graphs) {
+        if ((rc = build_batch_graph(h, B, q80 != 0))) return rc;
+        CK(cudaGraphLaunch((q80 ? h->bgraph : h->bgraph_f32)[B], h->stream));
+    } else if ((rc = enqueue_batch_step(h, h->stream, B, h->bb, q80 != 0, false))) {
+        return rc;
     }
     CK(cudaMemcpyAsync(logits_out, h->logits, (size_t)B * h->V * 4, cudaMemcpyDeviceToDevice, h->stream));
     return L2C_OK;
+}
+
+extern "C" int l2c_prefill(l2c_ctx* h, int seq, int n, const int32_t* tokens, int pos0, int q80,
+                           float* logits_last) {
+    if (!h || !tokens || n < 1 || seq < 0 || seq >= h->max_batch || pos0 < 0 || (long long)pos0 + n > h->S)
+        return fail(h, L2C_E_ARG, "prefill: need n >= 1, a sequence of the handle and pos0 + n <= seq_len");
+    if (is_device_ptr(tokens)) return fail(h, L2C_E_ARG, "prefill: tokens must be host memory");
+    for (int i = 0; i < n; i++)
+        if (tokens[i] < 0 || tokens[i] >= h->V) return fail(h, L2C_E_ARG, "token[%d]=%d out of range", i, tokens[i]);
+    if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
+    int rc;
+    if (q80) {
+        if (batched_kc(h->d, h->gs) == 0 || batched_kc(h->h, h->gs) == 0 || h->gs % 32)
+            return fail(h, L2C_E_ARG, "Q8_0 prefill needs gs a multiple of 32 and widths the batched GEMM tiles");
+        if ((rc = ensure_batched(h))) return rc;
+    } else if ((rc = ensure_batched_f32(h))) {
+        return rc;
+    }
+    if ((rc = ensure_prefill(h))) return rc;
+    BatchBufs bb = h->pb;
+    bb.cache_off = (size_t)seq * h->L * h->S * h->kvd;
+    bb.seq_stride = 0;  // one cache: every token of a chunk reads and writes sequence seq's
+    int tp[2 * BMAX];
+    int last = 0;
+    for (int c0 = 0; c0 < n; c0 += BMAX) {
+        const int B = n - c0 < BMAX ? n - c0 : BMAX;
+        for (int i = 0; i < B; i++) {
+            tp[2 * i] = tokens[c0 + i];
+            tp[2 * i + 1] = pos0 + c0 + i;
+        }
+        // a copy, not a kernel: the chunk's kernels start after every earlier
+        // kernel has finished, so rows of earlier chunks are complete
+        CK(cudaMemcpyAsync(bb.tp, tp, (size_t)B * 8, cudaMemcpyHostToDevice, h->stream));
+        if ((rc = enqueue_batch_step(h, h->stream, B, bb, q80 != 0, true))) return rc;
+        last = B - 1;
+    }
+    if (logits_last)
+        CK(cudaMemcpyAsync(logits_last, bb.logits + (size_t)last * h->V, (size_t)h->V * 4, cudaMemcpyDeviceToDevice,
+                           h->stream));
+    return l2c_sync(h);
 }
 
 extern "C" int l2c_attention(l2c_ctx* h, const float* q, const float* k, const float* v, int pos, int precision,
@@ -803,7 +973,7 @@ extern "C" int l2c_attention(l2c_ctx* h, const float* q, const float* k, const f
     if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)out) & 15)
         return fail(h, L2C_E_ARG, "attention: buffers must be 16-byte aligned");
     k_set_tp<<<1, 1, 0, h->stream>>>(h->tp, 0, pos);
-    CK(launch_attention(h, h->stream, false, precision != 0, q, k, v, 0, out, h->tp, 1));
+    CK(launch_attention(h, h->stream, false, precision != 0, q, k, v, 0, out, h->tp, 1, h->attn_part, h->attn_cnt));
     return L2C_OK;
 }
 
@@ -974,6 +1144,8 @@ extern "C" void l2c_destroy(l2c_ctx* h) {
     for (int a = 0; a < 2; a++)
         for (int b = 0; b < 2; b++)
             if (h->graph[a][b]) cudaGraphExecDestroy(h->graph[a][b]);
+    for (cudaGraphExec_t g : h->bgraph_f32)
+        if (g) cudaGraphExecDestroy(g);
     for (cudaGraphExec_t g : h->bgraph)
         if (g) cudaGraphExecDestroy(g);
     for (void* p : h->allocs) cudaFree(p);

@@ -160,11 +160,31 @@ L2C_API int l2c_generate(l2c_ctx* h, int token0, int pos0, int steps, int q80, i
 /*
  * l2c_forward_batch - B independent sequences, one token each: sequence b
  * runs the step with tokens[b] at position pos[b] against its own KV cache.
- * tokens, pos: host or device int32 [B]; B <= max_batch.  logits_out_dev:
- * device [B][vocab_size].  q80 selects the Q8_0 path.
+ * Each matvec of the step runs as one GEMM over the B sequences (Q8_0: int8
+ * tensor cores, exact int32 group dots, double group sums; fp32: fp32 FMAs).
+ * tokens, pos: host or device int32 [B]; B <= max_batch and B <= 32.
+ * logits_out_dev: device [B][vocab_size].  q80 selects the Q8_0 path.
  */
 L2C_API int l2c_forward_batch(l2c_ctx* h, int B, const int32_t* tokens, const int32_t* pos, int q80,
                       float* logits_out_dev);
+
+/*
+ * l2c_prefill - a prompt at once: tokens[0..n-1] at positions pos0..pos0+n-1
+ * of sequence seq.  The pages feed a prompt through forward one token at a
+ * time ([port] 智能家居控制案例: encode, then forward(tokens[0], 0), ...);
+ * this computes the same K/V cache rows and logits as those n steps, in
+ * chunks of up to 32 tokens that run as GEMMs (each weight row read once per
+ * chunk), with causal attention: token i of a chunk attends to positions
+ * 0..pos0+i of the sequence's cache, which holds the rows of earlier chunks
+ * and calls.  Same arithmetic per element as the batched step: Q8_0 on the
+ * int8 tensor cores with double group sums; fp32 with fp32 FMAs.
+ * tokens: host int32 [n]; 0 <= seq < max_batch; n >= 1; pos0 + n <= seq_len.
+ * logits_last_dev: device [vocab_size] receives the logits of the last token
+ * (NULL: not written).  q80 = 1 needs l2c_enable_q80 with gs a multiple of 32
+ * that the batched GEMM tiles (else L2C_E_ARG).  The first call allocates the
+ * chunk activations in the handle.  Blocks until the cache is written.
+ */
+L2C_API int l2c_prefill(l2c_ctx* h, int seq, int n, const int32_t* tokens, int pos0, int q80, float* logits_last_dev);
 
 /*
  * l2c_quantize_q80 - quantize() of [port] §1 INT8量化压缩 on n device
