@@ -64,11 +64,13 @@ __device__ __forceinline__ double widen_scaled(float x) {
 }
 constexpr double kTwo896 = 0x1p896;
 
-__device__ __forceinline__ bool nonfinite4(const float4 v) {
-    return ((__float_as_uint(v.x) & 0x7f800000u) == 0x7f800000u) |
-           ((__float_as_uint(v.y) & 0x7f800000u) == 0x7f800000u) |
-           ((__float_as_uint(v.z) & 0x7f800000u) == 0x7f800000u) |
-           ((__float_as_uint(v.w) & 0x7f800000u) == 0x7f800000u);
+// chk + v * 0 over the four elements: NaN once any element is infinite or
+// NaN (the widening above would turn those into finite doubles), else chk.
+__device__ __forceinline__ float nonfinite_fold(const float4 v, float chk) {
+    chk = __fmaf_rn(v.x, 0.f, chk);
+    chk = __fmaf_rn(v.y, 0.f, chk);
+    chk = __fmaf_rn(v.z, 0.f, chk);
+    return __fmaf_rn(v.w, 0.f, chk);
 }
 
 template <typename Acc>
@@ -174,14 +176,23 @@ __device__ __forceinline__ void attn_finish(const AttnArgs& a, int c, int g, int
     const Acc* p0 = static_cast<const Acc*>(a.part) + (((size_t)b * a.Hkv + g) * a.nchunks * REP) * (HS + 2);
     for (int i = tid; i < REP * HS; i += (32 * NW)) {
         const int h = i / HS, e = i % HS;
-        Acc M = -INFINITY;
-        for (int k = 0; k < nact; k++) M = max(M, __ldcg(p0 + ((size_t)k * REP + h) * (HS + 2) + HS));
-        Acc Ls = 0, Os = 0;
-        for (int k = 0; k < nact; k++) {
+        Acc M = -INFINITY, Ls = 0, Os = 0;
+        auto term = [&](int k) {
             const Acc* pk = p0 + ((size_t)k * REP + h) * (HS + 2);
             const Acc f = exp(__ldcg(pk + HS) - M);
             Ls += __ldcg(pk + HS + 1) * f;
             Os += __ldcg(pk + e) * f;
+        };
+        if (sizeof(Acc) == 8) {
+            // double: up to 4 CTAs per SM, so many chunks; unrolled, the chunks'
+            // loads (independent of one another) are in flight together
+#pragma unroll 8
+            for (int k = 0; k < nact; k++) M = max(M, __ldcg(p0 + ((size_t)k * REP + h) * (HS + 2) + HS));
+#pragma unroll 8
+            for (int k = 0; k < nact; k++) term(k);
+        } else {
+            for (int k = 0; k < nact; k++) M = max(M, __ldcg(p0 + ((size_t)k * REP + h) * (HS + 2) + HS));
+            for (int k = 0; k < nact; k++) term(k);
         }
         a.out[(size_t)b * a.H * HS + ((size_t)g * REP + h) * HS + e] = (float)(Os / Ls);
     }
@@ -410,7 +421,10 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
         l[h] = 0;
         o[h][0] = o[h][1] = o[h][2] = o[h][3] = 0;
     }
-    bool bad = false;  // a non-finite K/V element (double path)
+    // non-finite K/V elements (double path): x * 0 is NaN exactly for an
+    // infinite or NaN x, so one FMA per element (on the FMA pipe, which this
+    // kernel leaves idle) folds every element into chk
+    float chk = 0.f;
     for (int jj = 0;; jj++) {
         const int bi = warp + ATTN_WARPS * jj;
         if (bi >= nb) break;
@@ -419,7 +433,7 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
         const int slot = jj % ATTN_NB;
         if (DBL) {
 #pragma unroll
-            for (int i = 0; i < PB; i++) bad |= nonfinite4(*ent(slot, i, 0)) | nonfinite4(*ent(slot, i, 1));
+            for (int i = 0; i < PB; i++) chk = nonfinite_fold(*ent(slot, i, 1), nonfinite_fold(*ent(slot, i, 0), chk));
         }
         attn_batch<Acc, REP, PB>(min(PB, t1 - (t0 + bi * PB)), [&](int i, int kv) { return *ent(slot, i, kv); }, qr,
                                  scale, m, l, o);
@@ -430,7 +444,7 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
         for (int h = 0; h < REP; h++) {
             o[h][0] *= (Acc)kTwo896; o[h][1] *= (Acc)kTwo896; o[h][2] *= (Acc)kTwo896; o[h][3] *= (Acc)kTwo896;
         }
-        if (__any_sync(0xffffffffu, bad))
+        if (__any_sync(0xffffffffu, chk != chk))
 #pragma unroll
             for (int h = 0; h < REP; h++) o[h][0] = o[h][1] = o[h][2] = o[h][3] = (Acc)NAN;
     }

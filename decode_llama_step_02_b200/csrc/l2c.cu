@@ -70,8 +70,9 @@ struct l2c_ctx {
     size_t sample_n = 0;
     void* attn_part = nullptr;
     int* attn_cnt = nullptr;
-    int attn_ctas = 0;          // fp32 attention CTAs to aim for (0: the SM count)
-    int attn_ctas_f64 = 0;      // double attention CTAs to aim for (0: four times the SM count)
+    int attn_ctas = 0;          // fp32 attention CTAs to aim for (0: all that are resident at once)
+    int attn_ctas_f64 = 0;      // double attention CTAs to aim for (0: all that are resident at once)
+    int attn_occ_f32 = 1, attn_occ_f64 = 4;  // resident CTAs per SM of this shape's attention kernels
     int attn_min_chunk = 32;    // positions per attention chunk, at least
     int attn_nchunks_max = 1;   // chunks the partials buffer holds per (sequence, KV head)
     // graphs: [q80][gen]
@@ -291,16 +292,20 @@ static int set_smem_limits(l2c_ctx* h) {
     return L2C_OK;
 }
 
-// Attention chunks per (sequence, KV head) for a launch over B sequences:
-// about one CTA per SM in fp32 (bandwidth-bound: long chunks, one merge) and
-// four per SM in double (more warps for its arithmetic), each chunk at least
+// Attention chunks per (sequence, KV head) for a launch over B sequences: at
+// most as many CTAs as are resident at once (the 7B shape: one 8-warp CTA per
+// SM in fp32, four 4-warp CTAs per SM in double), each chunk at least
 // attn_min_chunk positions.
 static int attn_nchunks(const l2c_ctx* h, int B, bool dbl) {
-    const int target = dbl ? (h->attn_ctas_f64 > 0 ? h->attn_ctas_f64 : 4 * h->sms)
-                           : (h->attn_ctas > 0 ? h->attn_ctas : h->sms);
-    // double: enough CTAs to fill the SMs several times (arithmetic-bound);
-    // fp32: at most `target` CTAs of 8 warps (one per SM: no SM gets two)
-    int nc = dbl ? (target + h->Hkv * B - 1) / (h->Hkv * B) : target / (h->Hkv * B);
+    const int target = dbl ? (h->attn_ctas_f64 > 0 ? h->attn_ctas_f64 : h->attn_occ_f64 * h->sms)
+                           : (h->attn_ctas > 0 ? h->attn_ctas : h->attn_occ_f32 * h->sms);
+    // at most `target` CTAs, so that all of them are resident at once (a
+    // second wave of a few CTAs would double the kernel's tail); but when that
+    // leaves a single chunk per (sequence, KV head) (many sequences), the next
+    // count up: one chunk serialises a whole sequence in one CTA
+    const int per = h->Hkv * B;
+    int nc = target / per;
+    if (nc < 2) nc = (target + per - 1) / per;
     const int maxc = (h->S + h->attn_min_chunk - 1) / h->attn_min_chunk;
     if (nc > maxc) nc = maxc;
     return nc < 1 ? 1 : nc;
@@ -499,14 +504,16 @@ static int bgemm(l2c_ctx* h, cudaStream_t s, int B, const BatchBufs& bb, const Q
     g.W = m.p + row0 * m.rb; g.rb = m.rb; g.kc = batched_kc(K, h->gs);
     g.xq = h->bxq; g.xs = h->bxs; g.kq_stride = h->bkq; g.ks_stride = h->bks;
     g.prefetch_bytes = h->pf_q8;
-    // as many ring stages as the shared memory holds (2..16): the weight slices
-    // of one stage are small, so the depth sets the bytes in flight
+    // ring stages: the depth sets the bytes in flight.  A grid of more CTAs
+    // than SMs keeps bgemm_stages (two CTAs per SM then share the shared
+    // memory); a grid of at most one CTA per SM takes as many as fit (up to 8)
+    const int grid = (rows + BG_ROWS - 1) / BG_ROWS;
     BLayout L = make_blayout(g.kc, h->gs, 1);
+    const int cap = grid <= h->sms ? 8 : h->bgemm_stages;
     int ns = (int)(h->bgemm_smem / (L.stage_bytes + 16));
-    ns = ns < 2 ? 2 : (ns > h->bgemm_stages ? h->bgemm_stages : ns);
+    ns = ns < 2 ? 2 : (ns > cap ? cap : ns);
     L = make_blayout(g.kc, h->gs, ns);
     size_t smem = (size_t)L.ns * L.stage_bytes + 16 * (size_t)L.ns;
-    int grid = (rows + BG_ROWS - 1) / BG_ROWS;
     CK(launch(s, true, k_bgemm_q8<MODE>, dim3(grid), dim3(32 * (BG_WARPS + 1)), smem, g, L));
     return L2C_OK;
 }
@@ -703,6 +710,18 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
         return bail(L2C_E_CUDA);
     if (cudaStreamCreateWithFlags(&h->cap, cudaStreamNonBlocking) != cudaSuccess) return bail(L2C_E_CUDA);
     if ((rc = set_smem_limits(h)) != L2C_OK) return bail(rc);
+    {  // resident attention CTAs per SM (the default chunk counts keep every CTA resident)
+        int occ = 0;
+        AttnKernel kf = attn_kernel_for<float>(h->hs, h->rep), kd = attn_kernel_for<double>(h->hs, h->rep);
+        if (kf && cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kf, attn_threads<float>(), 0) == cudaSuccess &&
+            occ > 0)
+            h->attn_occ_f32 = occ;
+        if (kd && cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kd, attn_threads<double>(),
+                                                                attn_smem_for<double>(h->rep)) == cudaSuccess &&
+            occ > 0)
+            h->attn_occ_f64 = occ;
+        cudaGetLastError();
+    }
 
     const size_t d = h->d, hh = h->h, L = h->L, kvd = h->kvd, V = h->V, S = h->S, B = max_batch;
     const size_t rq = d + 2 * kvd;

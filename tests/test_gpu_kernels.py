@@ -132,3 +132,35 @@ def test_attention_matches_oracle(H, Hkv, hs, S, positions):
             got = out.cpu().numpy()
             assert np.abs(got - ref).max() <= tol * np.abs(ref).max(), (pos, precision)
     dec.close()
+
+
+@pytest.mark.parametrize("precision", [0, 1], ids=["fp32", "double"])
+@pytest.mark.parametrize("where,value", [("k", np.inf), ("k", np.nan), ("v", np.nan), ("v", np.inf)])
+def test_attention_nonfinite_kv_is_not_finite(precision, where, value):
+    """A non-finite K or V element at a position the query reaches leaves the heads of
+    its KV head non-finite (the double path detects it: its integer widening alone
+    would turn it into a large finite value) and every other head finite."""
+    torch, l2c = need_gpu()
+    H, Hkv, hs, S, pos = 8, 4, 16, 300, 250
+    d = H * hs
+    spec = synth.ModelSpec("attn-nf", d, 4 * d, 1, H, Hkv, 64, S, 1, seed=9)
+    dec = l2c.Decoder(spec.cfg, synth.blob(spec), 1)
+    kc, vc = synth.kv_prefill(spec, seq=0, n_pos=S)
+    kc, vc = kc[0].copy(), vc[0].copy()
+    g = 2  # KV head hit: query heads 4 and 5
+    (kc if where == "k" else vc)[137, g * hs + 5] = value
+    q = np.random.default_rng(1).standard_normal(d).astype(np.float32)
+    rep = H // Hkv
+    for h in range(g * rep, (g + 1) * rep):
+        q[h * hs + 5] = 1.0  # an infinite key then scores +inf in both heads
+    out = torch.empty(d, dtype=torch.float32, device="cuda")
+    dec.attention(torch.from_numpy(q).cuda(), torch.from_numpy(kc).cuda(), torch.from_numpy(vc).cuda(), pos, out,
+                  precision)
+    dec.sync()
+    got = out.cpu().numpy().reshape(H, hs)
+    for h in range(H):
+        if h // rep == g:
+            assert not np.isfinite(got[h]).all(), h
+        else:
+            assert np.isfinite(got[h]).all(), h
+    dec.close()
