@@ -6,14 +6,15 @@
 // Work item (chunk c, KV head g, sequence b): the positions [t0, t1) of the
 // chunk, for the rep = H/Hkv query heads that share KV head g (heads
 // g*rep .. g*rep+rep-1: contiguous groups), so every K/V row is read once per
-// group.  One CTA of four warps per item.  Each warp takes batches of
-// positions in turn and runs an online softmax over them (scores from one
-// reduce-scatter per head, running max, rescaled weighted V sum) while the
-// next two batches stream into shared memory (cp.async, per lane); then the
-// warps merge their states.  Rows before the current position do not depend
-// on the kernel that precedes attention in the step, so a warp's first
-// batches are copied before the dependency wait when they do not contain the
-// current position's row.
+// group.  One CTA per item: 8 warps in fp32 (K/V batches in registers), 4
+// in double (K/V batches streamed into per-lane shared-memory rings with
+// cp.async).  Each warp takes batches of positions in turn and runs an online
+// softmax over them (scores from one reduce-scatter per head, running max,
+// rescaled weighted V sum) while its next batches load; then the warps merge
+// their states.  Rows before the current position do not depend on the
+// kernel that precedes attention in the step, so a warp's first batches are
+// read before the dependency wait when they do not contain a row the kernel
+// before writes.
 //
 // Each active chunk writes its (o, m, l) per head; the last CTA to arrive for
 // (b, g) (an atomic counter, no spin-wait) merges them:
@@ -120,7 +121,7 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
 
-// The merge of a work item's four warps and of the chunks of (b, g); every
+// The merge of a work item's NW warps and of the chunks of (b, g); every
 // thread of the CTA calls it after its warp's online softmax is done.
 template <typename Acc, int HS, int REP, int NW>
 __device__ __forceinline__ void attn_finish(const AttnArgs& a, int c, int g, int b, int nact, const Acc (&m)[REP],
@@ -128,7 +129,7 @@ __device__ __forceinline__ void attn_finish(const AttnArgs& a, int c, int g, int
                                             Acc (*sm_l)[REP], Acc (*sm_o)[REP][HS], int* last_s) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const bool lane_on = lane < HS / 4;
-    // merge the four warps' states (a warp without positions has m = -inf, l = 0)
+    // merge the warps' states (a warp without positions has m = -inf, l = 0)
     if (lane == 0) {
 #pragma unroll
         for (int h = 0; h < REP; h++) {
@@ -355,7 +356,7 @@ __global__ void __launch_bounds__(32 * ATTN_WARPS_F32) k_attention_f32(const Att
 
 // grid (nchunks, Hkv, B), ATTN_THREADS threads, attn_ring_bytes<Acc, REP>()
 // bytes of dynamic shared memory: CTA (c, g, b) runs work item (c, g, b).
-// The chunk's positions go in batches of PB to the four warps in turn; a lane
+// The chunk's positions go in batches of PB to the ATTN_WARPS warps in turn; a lane
 // owns one float4 of each K and V row slice (hs <= 128) and streams it into
 // its own ring of ATTN_NB batches in shared memory with cp.async, so two
 // batches are in flight while it computes a third, without holding them in
