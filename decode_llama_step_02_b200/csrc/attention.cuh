@@ -98,10 +98,11 @@ constexpr int ATTN_NB = 3;  // batches in each lane's shared-memory ring
 // Positions a warp loads at once (one batch): fewer when the query group is
 // large, to bound the registers of the batch being computed.  In double,
 // batches of 8 (two CTAs per SM with their 96 KB rings) measured faster than
-// batches of 4 (four CTAs per SM) or 2.
+// batches of 4 (four CTAs per SM) or 2 for MHA, and 4 faster than 2 or 1 at a
+// GQA ratio of 4.
 template <typename Acc, int REP>
 struct AttnPB {
-    static constexpr int value = sizeof(Acc) == 8 ? (REP >= 4 ? 2 : 8) : (REP >= 3 ? 4 : 8);
+    static constexpr int value = sizeof(Acc) == 8 ? (REP >= 8 ? 2 : (REP >= 4 ? 4 : 8)) : (REP >= 3 ? 4 : 8);
 };
 
 // Dynamic shared memory of an attention CTA: per warp ATTN_NB batches of PB
