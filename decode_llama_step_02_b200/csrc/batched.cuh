@@ -375,8 +375,8 @@ __global__ void __launch_bounds__(32 * (BG_WARPS + 1)) k_bgemm_q8(const BGemmArg
 constexpr int BF_ROWS = 32;               // weight rows per CTA
 constexpr int BF_KT = 64;                 // K per stage
 constexpr int BF_PITCH = BF_KT + 4;       // floats per shared row: conflict-free 16-byte reads
-constexpr int BF_STAGES = 3;
-constexpr int BF_THREADS = 128;
+constexpr int BF_STAGES = 4;               // 70 KB: three CTAs per SM (measured best of 2..8)
+constexpr int BF_THREADS = 64;
 constexpr int BF_STAGE_FLOATS = (BF_ROWS + BMAX) * BF_PITCH;
 constexpr int BF_SMEM = BF_STAGES * BF_STAGE_FLOATS * 4;
 
@@ -444,9 +444,12 @@ __device__ __forceinline__ void bf_cp16(float* dst, const float* src, bool on, u
 // every sequence: Y[b][r] = sum_k W[r][k] X[b][k] in fp32 FMAs.  Stages of
 // BF_KT columns of W (this CTA's rows) and of X (all BMAX rows; rows >= B and
 // columns >= K are zero-filled) stream through a BF_STAGES-deep cp.async
-// ring.  Thread t computes rows 2*(t/8) + {0, 1} for sequences
-// t%8 + {0, 8, 16, 24} in k order, reading 4 consecutive k of each at once.
-// a.W holds the fp32 rows (a.rb bytes apart); X is [B][x_stride].
+// ring.  Thread t computes rows t/8 + {0, 8, 16, 24} for sequences
+// t%8 + {0, 8, 16, 24} in k order, reading 4 consecutive k of each at once
+// (16-byte shared loads: a 4 x 4 tile does 64 FMAs per 8 loads, against 32
+// per 6 for 2 x 4; the shared-memory pipe, four wavefronts per 16-byte warp
+// load, is the limit).  a.W holds the fp32 rows (a.rb bytes apart); X is
+// [B][x_stride].
 template <int MODE>
 __global__ void __launch_bounds__(BF_THREADS) k_bgemm_f32(const BGemmArgs a, const float* X, size_t x_stride) {
     extern __shared__ __align__(16) float fsm[];
@@ -494,10 +497,10 @@ __global__ void __launch_bounds__(BF_THREADS) k_bgemm_f32(const BGemmArgs a, con
         if (t < nkt) load(t);
         asm volatile("cp.async.commit_group;" ::: "memory");
     }
-    const int sg = tid & 7, rp = tid >> 3;
-    float acc[2][4];
+    const int sg = tid & 7, rp = tid >> 3;  // rows rp + 8i, sequences sg + 8j
+    float acc[4][4];
 #pragma unroll
-    for (int i = 0; i < 2; i++) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    for (int i = 0; i < 4; i++) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
     for (int t = 0; t < nkt; t++) {
         asm volatile("cp.async.wait_group %0;" :: "n"(BF_STAGES - 2) : "memory");
         __syncthreads();  // stage t landed for every thread; stage t-1 is free
@@ -507,31 +510,31 @@ __global__ void __launch_bounds__(BF_THREADS) k_bgemm_f32(const BGemmArgs a, con
         const float* xt = wt + BF_ROWS * BF_PITCH;
         // the stage's 16 steps of 4 columns, fully unrolled so that the shared
         // loads of later steps issue ahead of the FMAs of earlier ones
-        const float* wr = wt + (2 * rp) * BF_PITCH;
+        const float* wr = wt + rp * BF_PITCH;
         const float* xr = xt + sg * BF_PITCH;
 #pragma unroll
         for (int kk = 0; kk < BF_KT; kk += 4) {
-            const float4 w0 = *reinterpret_cast<const float4*>(wr + kk);
-            const float4 w1 = *reinterpret_cast<const float4*>(wr + BF_PITCH + kk);
+            float4 wv[4], xv[4];
 #pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const float4 xv = *reinterpret_cast<const float4*>(xr + 8 * j * BF_PITCH + kk);
-                acc[0][j] = fmaf(w0.x, xv.x, acc[0][j]);
-                acc[0][j] = fmaf(w0.y, xv.y, acc[0][j]);
-                acc[0][j] = fmaf(w0.z, xv.z, acc[0][j]);
-                acc[0][j] = fmaf(w0.w, xv.w, acc[0][j]);
-                acc[1][j] = fmaf(w1.x, xv.x, acc[1][j]);
-                acc[1][j] = fmaf(w1.y, xv.y, acc[1][j]);
-                acc[1][j] = fmaf(w1.z, xv.z, acc[1][j]);
-                acc[1][j] = fmaf(w1.w, xv.w, acc[1][j]);
-            }
+            for (int i = 0; i < 4; i++) wv[i] = *reinterpret_cast<const float4*>(wr + 8 * i * BF_PITCH + kk);
+#pragma unroll
+            for (int j = 0; j < 4; j++) xv[j] = *reinterpret_cast<const float4*>(xr + 8 * j * BF_PITCH + kk);
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    acc[i][j] = fmaf(wv[i].x, xv[j].x, acc[i][j]);
+                    acc[i][j] = fmaf(wv[i].y, xv[j].y, acc[i][j]);
+                    acc[i][j] = fmaf(wv[i].z, xv[j].z, acc[i][j]);
+                    acc[i][j] = fmaf(wv[i].w, xv[j].w, acc[i][j]);
+                }
         }
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 #pragma unroll
-    for (int i = 0; i < 2; i++)
+    for (int i = 0; i < 4; i++)
 #pragma unroll
-        for (int j = 0; j < 4; j++) stage_out[2 * rp + i][sg + 8 * j] = acc[i][j];
+        for (int j = 0; j < 4; j++) stage_out[rp + 8 * i][sg + 8 * j] = acc[i][j];
     __syncthreads();
     bgemm_epilogue<MODE>(a, r0, nrows, stage_out, best_s, tid, BF_THREADS, 1);
 }
