@@ -429,6 +429,21 @@ def run_ours(args, rank, world, local_rank):
            "h2d_bytes_per_step": 2 * len(POSITIONS) * 8,          # token + position per decode step
            "d2h_bytes_per_step": 2 * len(POSITIONS) * SPEC.vocab_size * 4}
 
+    # ---- the hot path's other rows on this GPU, device-timed, not part of `value`:
+    # a 128-token prompt on this decoder (l2c_prefill), then the GQA-7B batch of
+    # 32 sequences (l2c_forward_batch) on a second model once this one is freed
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    rows = {}
+    if not args.no_rows:
+        rows["prefill_7b_128_tokens"] = measure_prefill(torch, dec, ev, stream)
+    dec.close()
+    dec = None
+    torch.cuda.empty_cache()
+    if not args.no_rows:
+        rows["batch_gqa7b_32_sequences"] = measure_batch(torch, l2c, ev, stream, peak, args.layers, reps=5)
+
     # ---- CPU oracle beside it (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -445,13 +460,12 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": "f32 | i8*i8->i32 with f64 group sums", "data": "synthetic",
         "config": workload_config(), "roofline": roof, "roofline_q8_0": roof_q8,
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_token * 2 * len(POSITIONS) * args.steps,
-        "clocks": clk.summary(), "variants": variants, "kernels": kernels,
+        "clocks": clk.summary(), "variants": variants, "kernels": kernels, "rows": rows,
         "context": "pages' CPU figures: ~110 tok/s 15M int8 on an M1 MacBook Air; ~0.8 tok/s 7B fp32 on a "
                    "16-core Ryzen 9 7950X; ~4 tok/s 7B on a 96-thread server",
     }
     if rank == 0:
         print(json.dumps(out), flush=True)
-    dec.close()
     return 0
 
 
@@ -537,10 +551,18 @@ def run_extra(args):
         run_prefill(torch, l2c, ev, stream)
     if args.extra not in ("all", "batch"):
         return 0
-    # GQA-7B, 32 sequences, one batched step (Q8_0 and fp32)
+    for line in measure_batch(torch, l2c, ev, stream, peak, args.layers, reps=10):
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def measure_batch(torch, l2c, ev, stream, peak, layers=0, reps=10):
+    """GQA-7B, 32 sequences at positions U[0, 2047] on caches prefilled N(0,1):
+    one batched step (l2c_forward_batch), Q8_0 and fp32, timed with CUDA events
+    around `reps` steps.  Returns one record per variant."""
     spec, B = synth.GQA7B, 32
-    if args.layers:
-        spec = dataclasses.replace(spec, name=f"GQA-7B-width-{args.layers}L", n_layers=args.layers)
+    if layers:
+        spec = dataclasses.replace(spec, name=f"GQA-7B-width-{layers}L", n_layers=layers)
     blob = device_blob(torch, spec)
     dec = l2c.Decoder(spec.cfg, blob, spec.shared_weights, max_batch=B)
     del blob
@@ -559,11 +581,11 @@ def run_extra(args):
     d, h, L, H, Hkv, V, S = spec.cfg
     kvd = Hkv * (d // H)
     kvbytes = float(sum(8.0 * L * (int(p) + 1) * kvd for p in pos))
+    lines = []
     for q80 in (True, False):
         for _ in range(3):
             dec.forward_batch(tk, ps, out, q80=q80)
         dec.sync()
-        reps = 10
         a, b = ev(), ev()
         a.record(stream)
         for _ in range(reps):
@@ -586,9 +608,9 @@ def run_extra(args):
             line["gemm_flops_per_step"] = fl
             line["gemm_tflops"] = fl / ms / 1e9
             line["frac_of_fp32_fma_peak"] = fl / ms / 1e9 / FP32_FMA_TFLOPS
-        print(json.dumps(line), flush=True)
+        lines.append(line)
     dec.close()
-    return 0
+    return lines
 
 
 def matvec_params(spec) -> float:
@@ -599,19 +621,28 @@ def matvec_params(spec) -> float:
 
 
 def run_prefill(torch, l2c, ev, stream):
-    """A 128-token prompt on the 7B shape (l2c_prefill: 4 GEMM chunks of 32
-    tokens), fp32 and Q8_0 GS=64, timed with CUDA events around whole calls."""
-    n = 128
+    """A 128-token prompt on the 7B shape, fp32 and Q8_0 GS=64 (one JSON line each)."""
     blob = device_blob(torch)
     dec = l2c.Decoder(SPEC.cfg, blob, SPEC.shared_weights)
     del blob
     torch.cuda.empty_cache()
     dec.enable_q80(GS)
+    for line in measure_prefill(torch, dec, ev, stream):
+        print(json.dumps(line), flush=True)
+    dec.close()
+
+
+def measure_prefill(torch, dec, ev, stream, n=128, reps=3):
+    """A prompt of n tokens at positions 0..n-1 of sequence 0 (l2c_prefill: GEMM
+    chunks of 32 tokens), fp32 and Q8_0, timed with CUDA events around whole calls
+    (median of reps).  Overwrites the cache rows 0..n-1.  Returns one record per
+    variant."""
     toks = synth.tokens(SPEC.seed, 4, n, SPEC.vocab_size)
     last = torch.empty(SPEC.vocab_size, dtype=torch.float32, device="cuda")
+    lines = []
     for q80 in (False, True):
         dec.prefill(toks, 0, q80=q80, logits_last=last)  # warm-up: buffers, module loading
-        reps, ts = 3, []
+        ts = []
         for _ in range(reps):
             a, b = ev(), ev()
             a.record(stream)
@@ -628,8 +659,8 @@ def run_prefill(torch, l2c, ev, stream):
                 "timing": f"CUDA events around l2c_prefill, median of {reps}; weights larger than L2"}
         if not q80:
             line["frac_of_fp32_fma_peak"] = fl / ms / 1e9 / FP32_FMA_TFLOPS
-        print(json.dumps(line), flush=True)
-    dec.close()
+        lines.append(line)
+    return lines
 
 
 def main():
@@ -639,6 +670,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true",
+                    help="skip the prefill and batched-step records of the bench line")
     ap.add_argument("--extra", nargs="?", const="all", choices=("all", "small", "batch", "prefill"),
                     help="the other workloads (small: tiny, 15M, 110M position curves; batch: GQA-7B batch 32; "
                          "prefill: a 128-token 7B prompt), not bench lines")
