@@ -65,6 +65,8 @@ def lib():
             "orc_blob_floats": (sz, [vp, i32]),
             "orc_create": (vp, [vp, vp, sz, i32, i32]),
             "orc_enable_q80": (i32, [vp, i32]),
+            "orc_enable_kv8": (i32, [vp]),
+            "orc_kv8_row": (None, [vp, i32, i32]),
             "orc_forward": (i32, [vp, i32, i32, i32, i32, vp]),
             "orc_kv_load": (i32, [vp, i32, i32, vp, vp]),
             "orc_kv_read": (i32, [vp, i32, i32, vp, vp]),
@@ -189,6 +191,13 @@ def matvec_q80(qw, sw, qx, sx, gs: int):
     return o
 
 
+def kv8_row(row, gs: int) -> np.ndarray:
+    """A K/V row as the int8 KV cache keeps it: quantize() per gs group, then code * scale."""
+    r = _f32(row).copy()
+    lib().orc_kv8_row(_p(r), r.size, int(gs))
+    return r
+
+
 def argmax(x) -> int:
     x = _f32(x)
     return lib().orc_argmax(_p(x), x.size)
@@ -223,6 +232,11 @@ class Model:
         if lib().orc_enable_q80(self._h, gs) != 0:
             raise ValueError("orc_enable_q80 failed")
         self.gs = gs
+
+    def enable_kv8(self):
+        """int8 KV cache: K/V rows kept as Q8_0 groups of head_size (orc_enable_kv8)."""
+        if lib().orc_enable_kv8(self._h) != 0:
+            raise ValueError("orc_enable_kv8 failed")
 
     def forward(self, token: int, pos: int, q80: bool = False, seq: int = 0) -> np.ndarray:
         out = np.empty(self.vocab, dtype=np.float32)

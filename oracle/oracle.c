@@ -220,6 +220,15 @@ void orc_dequantize(const int8_t* q, const float* s, int64_t n, int gs, float* o
     for (int64_t i = 0; i < n; i++) out[i] = (float)q[i] * s[i / gs];
 }
 
+/* A KV row of n values in place: quantize() in groups of gs, then code * scale. */
+void orc_kv8_row(float* row, int n, int gs) {
+    int8_t* q = (int8_t*)malloc((size_t)n);
+    float* sc = (float*)malloc(sizeof(float) * (size_t)(n / gs + 1));
+    if (q && sc && orc_quantize(row, n, gs, q, sc) == 0) orc_dequantize(q, sc, n, gs, row);
+    free(q);
+    free(sc);
+}
+
 /* Exact int32 dot products of every (row, group):
  * out[i][g] = sum_{k<gs} qw[i][g*gs+k] * qx[g*gs+k].  qw is [d][n]. */
 void orc_q80_group_dots(int32_t* out, const int8_t* qx, const int8_t* qw, int n, int d, int gs) {
@@ -333,6 +342,7 @@ typedef struct { int8_t* q; float* s; } orc_qt;
 struct orc_model {
     orc_config c;
     int shared, n_seq, gs;
+    int kv8; /* 1: the KV cache holds Q8_0 rows (see orc_enable_kv8) */
     const float *E, *w_att, *wq, *wk, *wv, *wo, *w_ffn, *w1, *w2, *w3, *w_final, *wcls;
     orc_qt qE, qwq, qwk, qwv, qwo, qw1, qw2, qw3, qwcls;
     float *kcache, *vcache; /* [n_seq][L][S][kv_dim] */
@@ -486,6 +496,10 @@ int orc_forward(orc_model* m, int seq, int token, int pos, int q80, float* logit
         }
         orc_rope(m->q, d, hs, pos);
         orc_rope(k, kvd, hs, pos);
+        if (m->kv8) {
+            orc_kv8_row(k, kvd, hs);
+            orc_kv8_row(v, kvd, hs);
+        }
         orc_attention(m->xb, m->q, kc, vc, pos, H, Hkv, hs);
         if (q80) orc_qmatvec(m, m->xb2, m->xb, &m->qwo, l, d, d);
         else orc_matvec(m->xb2, m->xb, m->wo + l * (size_t)d * d, d, d);
@@ -512,14 +526,41 @@ int orc_forward(orc_model* m, int seq, int token, int pos, int q80, float* logit
 int orc_kv_load(orc_model* m, int seq, int n_pos, const float* k, const float* v) {
     const orc_config* c = &m->c;
     if (seq < 0 || seq >= m->n_seq || n_pos < 0 || n_pos > c->seq_len) return -1;
-    size_t kvd = (size_t)c->n_kv_heads * (size_t)(c->dim / c->n_heads);
+    int hs = c->dim / c->n_heads;
+    size_t kvd = (size_t)c->n_kv_heads * (size_t)hs;
     size_t L = (size_t)c->n_layers, S = (size_t)c->seq_len;
     for (size_t l = 0; l < L; l++) {
         size_t dst = (((size_t)seq * L + l) * S) * kvd;
         size_t src = l * (size_t)n_pos * kvd;
         if (k) memcpy(m->kcache + dst, k + src, sizeof(float) * (size_t)n_pos * kvd);
         if (v) memcpy(m->vcache + dst, v + src, sizeof(float) * (size_t)n_pos * kvd);
+        if (m->kv8)
+            for (int t = 0; t < n_pos; t++) {
+                if (k) orc_kv8_row(m->kcache + dst + (size_t)t * kvd, (int)kvd, hs);
+                if (v) orc_kv8_row(m->vcache + dst + (size_t)t * kvd, (int)kvd, hs);
+            }
     }
+    return 0;
+}
+
+/* int8 KV cache (reading of the int8 KV cache variant; the pages give none):
+ * every K and V row, when it is stored, becomes Q8_0 groups of head_size
+ * values (one group per KV head), quantized with the quantize() rule of
+ * [port §1], and attention reads code * scale (one fp32 multiply).  The
+ * cache keeps those dequantized values in fp32, which is the same arithmetic
+ * as keeping the codes and scales.  Enabling it quantizes the rows already in
+ * the cache. */
+int orc_enable_kv8(orc_model* m) {
+    const orc_config* c = &m->c;
+    int hs = c->dim / c->n_heads;
+    size_t kvd = (size_t)c->n_kv_heads * (size_t)hs;
+    size_t rows = (size_t)m->n_seq * (size_t)c->n_layers * (size_t)c->seq_len;
+    if (!m->kv8)
+        for (size_t r = 0; r < rows; r++) {
+            orc_kv8_row(m->kcache + r * kvd, (int)kvd, hs);
+            orc_kv8_row(m->vcache + r * kvd, (int)kvd, hs);
+        }
+    m->kv8 = 1;
     return 0;
 }
 

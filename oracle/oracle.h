@@ -55,6 +55,9 @@ size_t orc_blob_floats(const orc_config* c, int shared_weights);
 orc_model* orc_create(const orc_config* c, const float* blob, size_t blob_floats, int shared_weights,
                       int n_seq);
 int orc_enable_q80(orc_model* m, int gs);
+/* int8 KV cache: K and V rows stored as Q8_0 groups of head_size values. */
+int orc_enable_kv8(orc_model* m);
+void orc_kv8_row(float* row, int n, int gs);
 int orc_forward(orc_model* m, int seq, int token, int pos, int q80, float* logits);
 int orc_kv_load(orc_model* m, int seq, int n_pos, const float* k, const float* v);
 int orc_kv_reset(orc_model* m, int seq);

@@ -50,7 +50,14 @@ def _q8_fake(M, gs, quantize):
     return (q.astype(np.float64) * np.repeat(s.astype(np.float64), gs)).reshape(M.shape)
 
 
-def prefill_logits(cfg, blob, shared, tokens, q80_gs=0, quantize=None):
+def _kv8(M, hs, quantize):
+    """K or V rows [T][kvd] as an int8 KV cache keeps them: Q8_0 groups of one head
+    (hs values), code * scale rounded to fp32."""
+    q, s = quantize(M.astype(np.float32).ravel(), hs)
+    return f32(q.astype(np.float64) * np.repeat(s.astype(np.float64), hs)).reshape(M.shape)
+
+
+def prefill_logits(cfg, blob, shared, tokens, q80_gs=0, quantize=None, kv8=False):
     d, h, L, H, Hkv, V, S = cfg
     hs = d // H
     rep = H // Hkv
@@ -85,6 +92,8 @@ def prefill_logits(cfg, blob, shared, tokens, q80_gs=0, quantize=None):
         Q = rope(mm(Xn, W["wq"][l]), H)
         K = rope(mm(Xn, W["wk"][l]), Hkv)
         Vv = mm(Xn, W["wv"][l])
+        if kv8:
+            K, Vv = _kv8(K, hs, quantize), _kv8(Vv, hs, quantize)
         Kr = np.repeat(K.reshape(T, Hkv, hs), rep, axis=1)
         Vr = np.repeat(Vv.reshape(T, Hkv, hs), rep, axis=1)
         Qh = Q.reshape(T, H, hs)

@@ -33,6 +33,10 @@ MUTANTS = {
     "no_rope_on_k": ("orc_rope(k, kvd, hs, pos);", ""),
     "argmax_last_tie": ("if (x[i] > x[best]) best = i;", "if (x[i] >= x[best]) best = i;"),
     "wrong_norm_weight": ("orc_rmsnorm(m->xb, x, m->w_att + l * d, d);", "orc_rmsnorm(m->xb, x, m->w_ffn + l * d, d);"),
+    "kv8_before_rope": ("        orc_rope(k, kvd, hs, pos);\n        if (m->kv8) {\n            orc_kv8_row(k, kvd, hs);",
+                        "        if (m->kv8) orc_kv8_row(k, kvd, hs);\n        orc_rope(k, kvd, hs, pos);\n        if (m->kv8) {"),
+    "kv8_v_not_quantized": ("            orc_kv8_row(v, kvd, hs);\n        }", "        }"),
+    "kv8_one_group_per_row": ("            orc_kv8_row(k, kvd, hs);\n", "            orc_kv8_row(k, kvd, kvd);\n"),
     "swiglu_operands_swapped": ("orc_swiglu(m->hb, m->hb2, h);", "orc_swiglu(m->hb2, m->hb, h); memcpy(m->hb, m->hb2, sizeof(float) * (size_t)h);"),
     "sample_temperature_multiplies": ("((double)z[i] - (double)mx) / (double)temperature", "((double)z[i] - (double)mx) * (double)temperature"),
     "sample_topp_excludes_ties": ("for (int i = 0; i < n; i++) if (q[i] >= tau) zset += q[i];", "for (int i = 0; i < n; i++) if (q[i] > tau || (q[i] == tau && i == 0)) zset += q[i];"),
@@ -56,6 +60,6 @@ def test_pins_catch_planted_mistake(name):
         env = dict(os.environ, ORACLE_LIB_PATH=so, OMP_NUM_THREADS="2")
         r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                             "tests/test_oracle_pins.py", "tests/test_oracle_forward.py",
-                            "tests/test_oracle_sampling.py"],
+                            "tests/test_oracle_sampling.py", "tests/test_oracle_kv8.py"],
                            cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
         assert r.returncode != 0, f"mutant {name} survived the pins:\n{r.stdout[-2000:]}"
