@@ -438,6 +438,7 @@ def run_ours(args, rank, world, local_rank):
     rows = {}
     if not args.no_rows:
         rows["prefill_7b_128_tokens"] = measure_prefill(torch, dec, ev, stream)
+        rows["q8_0_int8_kv_cache"] = measure_kv8(torch, dec, stream, peak)
     dec.close()
     dec = None
     torch.cuda.empty_cache()
@@ -630,6 +631,40 @@ def run_prefill(torch, l2c, ev, stream):
     for line in measure_prefill(torch, dec, ev, stream):
         print(json.dumps(line), flush=True)
     dec.close()
+
+
+def kv8_bytes_per_token(pos: int, spec=None, gs=GS) -> float:
+    """Algorithmic bytes of one Q8_0 step reading the int8 KV cache: the Q8_0
+    weights and vectors, plus codes (1 byte) and one fp32 scale per head row
+    for K and V of positions 0..pos."""
+    d, h, L, H, Hkv, V, S = (spec or SPEC).cfg
+    kvd = Hkv * (d // H)
+    return bytes_per_token(True, -1, spec, gs) + 2.0 * L * (pos + 1) * (kvd + 4 * Hkv)
+
+
+def measure_kv8(torch, dec, stream, peak, reps=20):
+    """The Q8_0 step with the int8 KV cache (l2c_enable_kv8: every row already in
+    the cache is quantized) at the bench positions: the median of `reps`
+    individually timed graph replays per position.  Leaves the cache on."""
+    dec.enable_kv8()
+    out = {}
+    for p in POSITIONS:
+        for _ in range(3):
+            dec.forward_ptr(TOKEN, p, True)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        torch.cuda.synchronize()
+        for a, b in evs:
+            a.record(stream)
+            dec.forward_ptr(TOKEN, p, True)
+            b.record(stream)
+        torch.cuda.synchronize()
+        t = statistics.median([a.elapsed_time(b) for a, b in evs])
+        by = kv8_bytes_per_token(p)
+        out[f"pos{p}"] = {"ms_per_token_median": t, "tokens_per_s": 1e3 / t, "bytes_per_token": by,
+                          "gbs": by / t / 1e6, "frac_of_measured_hbm": by / t / 1e6 / peak,
+                          "frac_of_8tbs_roofline": by / t / 1e6 / NOMINAL_HBM_GBS, "replays": reps}
+    dec.sync()
+    return out
 
 
 def measure_prefill(torch, dec, ev, stream, n=128, reps=3):

@@ -20,7 +20,7 @@ L2C_OK, L2C_E_ARG, L2C_E_OOM, L2C_E_CUDA, L2C_E_DEVICE, L2C_E_STATE, L2C_E_SCRAT
 # every symbol declared in include/l2c.h
 EXPORTS = (
     "l2c_blob_floats", "l2c_create", "l2c_enable_q80", "l2c_forward", "l2c_forward_q80", "l2c_argmax",
-    "l2c_generate", "l2c_sample", "l2c_forward_batch", "l2c_prefill", "l2c_quantize_q80", "l2c_q80_group_dots", "l2c_kv_load",
+    "l2c_generate", "l2c_sample", "l2c_forward_batch", "l2c_prefill", "l2c_enable_kv8", "l2c_quantize_q80", "l2c_q80_group_dots", "l2c_kv_load",
     "l2c_kv_read", "l2c_kv_reset", "l2c_attention", "l2c_attention_noalloc", "l2c_time_kernel", "l2c_sync", "l2c_stream", "l2c_last_status", "l2c_last_error",
     "l2c_destroy",
 )
@@ -63,6 +63,7 @@ def lib():
                                  ctypes.POINTER(ctypes.c_int)]),
             "l2c_forward_batch": (i32, [vp, i32, vp, vp, i32, vp]),
             "l2c_prefill": (i32, [vp, i32, i32, vp, i32, i32, vp]),
+            "l2c_enable_kv8": (i32, [vp, i32]),
             "l2c_quantize_q80": (i32, [vp, vp, i64, i32, vp, vp]),
             "l2c_q80_group_dots": (i32, [vp, vp, vp, i32, i32, i32, vp]),
             "l2c_kv_load": (i32, [vp, i32, i32, vp, vp]),
@@ -187,6 +188,10 @@ class Decoder:
                                       _ptr(logits_last) if logits_last is not None else None))
 
     # -- KV cache
+    def enable_kv8(self, on: bool = True):
+        """The int8 KV cache (K/V rows as Q8_0 groups of one head) on or off (l2c_enable_kv8)."""
+        self._check(lib().l2c_enable_kv8(self._h, int(on)))
+
     def kv_load(self, k, v, seq: int = 0):
         n_pos = k.shape[1]
         self._check(lib().l2c_kv_load(self._h, int(seq), int(n_pos), _ptr(k), _ptr(v)))

@@ -55,6 +55,14 @@ struct AttnArgs {
                          // entry 0's): rows from entry 0's position on come from the kernel before
     void* part;          // partials [B][Hkv][nchunks][rep][hs+2] (Acc)
     int* count;          // [B][Hkv] arrival counters (zero between launches)
+    // int8 KV cache (the double kernel's KV8 form): this layer's codes of
+    // sequence 0 ([S][kvd], sequence b at + b*seq_stride) and scales
+    // ([S][Hkv], sequence b at + b*sc_seq_stride)
+    const int8_t* kq;
+    const int8_t* vq;
+    const float* ks;
+    const float* vs;
+    size_t sc_seq_stride;
 };
 
 // x * 2^-896 as a double, exactly, for every finite float x (see above).
@@ -118,7 +126,21 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool on, 
     asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;"
                  :: "r"(smem_u32(dst)), "l"(src), "r"(on ? 16 : 0), "l"(pol) : "memory");
 }
+// 4-byte form (int8 KV cache codes and scales)
+__device__ __forceinline__ void cp_async4(void* dst, const void* src, bool on) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" :: "r"(smem_u32(dst)), "l"(src), "r"(on ? 4 : 0)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+// A ring entry of the int8 KV cache: .x holds four codes (little-endian), .y
+// their head's scale; the values are code * scale (fp32 multiplies).
+__device__ __forceinline__ float4 kv8_decode(const float4 e) {
+    const uint32_t c = __float_as_uint(e.x);
+    const float s = e.y;
+    return make_float4(__fmul_rn((float)(int8_t)(c & 0xffu), s), __fmul_rn((float)(int8_t)((c >> 8) & 0xffu), s),
+                       __fmul_rn((float)(int8_t)((c >> 16) & 0xffu), s), __fmul_rn((float)(int8_t)(c >> 24), s));
+}
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
 
@@ -362,7 +384,7 @@ __global__ void __launch_bounds__(32 * ATTN_WARPS_F32) k_attention_f32(const Att
 // its own ring of ATTN_NB batches in shared memory with cp.async, so two
 // batches are in flight while it computes a third, without holding them in
 // registers (each lane reads back only what it copied: no synchronisation).
-template <typename Acc, int HS, int REP>
+template <typename Acc, int HS, int REP, bool KV8 = false>
 __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
     constexpr bool DBL = sizeof(Acc) == 8;
     constexpr int V4 = HS / 4;  // float4 per row slice (<= 32: one per lane)
@@ -382,9 +404,18 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
     const float* kc = a.kc + (size_t)b * a.seq_stride + (size_t)g * HS + 4 * (lane_on ? lane : 0);
     const float* vc = a.vc + (size_t)b * a.seq_stride + (size_t)g * HS + 4 * (lane_on ? lane : 0);
     const uint64_t pol = policy_evict_first();
+    // KV8: this lane's four codes and its head's scale of each K / V row
+    const int8_t* kq = KV8 ? a.kq + (size_t)b * a.seq_stride + (size_t)g * HS + 4 * (lane_on ? lane : 0) : nullptr;
+    const int8_t* vq = KV8 ? a.vq + (size_t)b * a.seq_stride + (size_t)g * HS + 4 * (lane_on ? lane : 0) : nullptr;
+    const float* ksc = KV8 ? a.ks + (size_t)b * a.sc_seq_stride + g : nullptr;
+    const float* vsc = KV8 ? a.vs + (size_t)b * a.sc_seq_stride + g : nullptr;
     float4* ring = aring + (size_t)warp * ATTN_NB * PB * 2 * 32;
     // ring entry of (slot, position i, K or V) for this lane
     auto ent = [&](int slot, int i, int kv) -> float4* { return ring + ((slot * PB + i) * 2 + kv) * 32 + lane; };
+    // its values (KV8: decoded from the codes and the scale)
+    auto val = [&](int slot, int i, int kv) -> float4 {
+        return KV8 ? kv8_decode(*ent(slot, i, kv)) : *ent(slot, i, kv);
+    };
     // copies of the warp's jj-th batch into slot jj % ATTN_NB; always one commit group
     auto issue = [&](int jj) {
         const int bi = warp + ATTN_WARPS * jj;
@@ -394,8 +425,16 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
             const int t = t0 + bi * PB + i;
             const bool on = lane_on && bi < nb && t < t1;
             const size_t off = on ? (size_t)t * a.kvd : 0;
-            cp_async16(ent(slot, i, 0), kc + off, on, pol);
-            cp_async16(ent(slot, i, 1), vc + off, on, pol);
+            if (KV8) {
+                const size_t so = on ? (size_t)t * a.Hkv : 0;
+                cp_async4(&ent(slot, i, 0)->x, kq + off, on);
+                cp_async4(&ent(slot, i, 0)->y, ksc + so, on);
+                cp_async4(&ent(slot, i, 1)->x, vq + off, on);
+                cp_async4(&ent(slot, i, 1)->y, vsc + so, on);
+            } else {
+                cp_async16(ent(slot, i, 0), kc + off, on, pol);
+                cp_async16(ent(slot, i, 1), vc + off, on, pol);
+            }
         }
         cp_async_commit();
     };
@@ -437,9 +476,9 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
         const int slot = jj % ATTN_NB;
         if (DBL) {
 #pragma unroll
-            for (int i = 0; i < PB; i++) chk = nonfinite_fold(*ent(slot, i, 1), nonfinite_fold(*ent(slot, i, 0), chk));
+            for (int i = 0; i < PB; i++) chk = nonfinite_fold(val(slot, i, 1), nonfinite_fold(val(slot, i, 0), chk));
         }
-        attn_batch<Acc, REP, PB>(min(PB, t1 - (t0 + bi * PB)), [&](int i, int kv) { return *ent(slot, i, kv); }, qr,
+        attn_batch<Acc, REP, PB>(min(PB, t1 - (t0 + bi * PB)), [&](int i, int kv) { return val(slot, i, kv); }, qr,
                                  scale, m, l, o);
     }
     cp_async_wait<0>();  // no copy of this lane may land after the CTA leaves
@@ -480,6 +519,15 @@ inline AttnKernel attn_kernel_for(int hs, int rep) {
     return nullptr;
 }
 
+// The double kernel reading the int8 KV cache, for (hs, rep).
+inline AttnKernel attn_kernel_kv8(int hs, int rep) {
+#define L2C_ATTN_Q(HS_, REP_) \
+    if (hs == HS_ && rep == REP_) return k_attention<double, HS_, REP_, true>;
+    L2C_ATTN_SHAPES(L2C_ATTN_Q)
+#undef L2C_ATTN_Q
+    return nullptr;
+}
+
 // Dynamic shared memory of the attention instantiation for a GQA ratio (the
 // fp32 kernel has none).
 template <typename Acc>
@@ -508,6 +556,17 @@ inline cudaError_t attn_set_smem_limits() {
         return e;
     L2C_ATTN_SHAPES(L2C_ATTN_ATTR)
 #undef L2C_ATTN_ATTR
+#define L2C_ATTN_ATTR_Q(HS_, REP_)                                                                                \
+    if ((e = cudaFuncSetAttribute(k_attention<double, HS_, REP_, true>,                                           \
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, attn_ring_bytes<double, REP_>())) != \
+        cudaSuccess)                                                                                              \
+        return e;                                                                                                 \
+    if ((e = cudaFuncSetAttribute(k_attention<double, HS_, REP_, true>,                                           \
+                                  cudaFuncAttributePreferredSharedMemoryCarveout,                                 \
+                                  (int)cudaSharedmemCarveoutMaxShared)) != cudaSuccess)                           \
+        return e;
+    L2C_ATTN_SHAPES(L2C_ATTN_ATTR_Q)
+#undef L2C_ATTN_ATTR_Q
     return e;
 }
 

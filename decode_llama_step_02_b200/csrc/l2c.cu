@@ -22,6 +22,7 @@
 
 #include "../../include/l2c.h"
 #include "batched.cuh"
+#include "kvcache.cuh"
 #include "sampling.cuh"
 #include "kernels.cuh"
 
@@ -83,6 +84,10 @@ struct l2c_ctx {
     size_t bkq = 0, bks = 0;  // strides (bytes of codes, floats of scales) per sequence
     std::vector<cudaGraphExec_t> bgraph;  // Q8_0, index B (1..max_batch)
     std::vector<cudaGraphExec_t> bgraph_f32;  // fp32, index B
+    // int8 KV cache (l2c_enable_kv8): codes [max_batch][L][S][kvd], scales [max_batch][L][S][Hkv]
+    bool kv8 = false;
+    int8_t *kq8 = nullptr, *vq8 = nullptr;
+    float *ks8 = nullptr, *vs8 = nullptr;
     BatchBufs bb;            // the handle's sequences (x, q, ... above)
     BatchBufs pb;            // prompt chunks of l2c_prefill (allocated on first use, BMAX entries)
     float* xb = nullptr;     // fp32 batched step: normalized input rows [BMAX][xbs]
@@ -314,7 +319,7 @@ static int attn_nchunks(const l2c_ctx* h, int B, bool dbl) {
 // Enqueues the attention of one layer over sequences 0..B-1 (grid z).
 static cudaError_t launch_attention(l2c_ctx* h, cudaStream_t s, bool pdl, bool dbl, const float* q, const float* kc,
                                     const float* vc, size_t seq_stride, float* out, const int* tp, int B,
-                                    void* part, int* cnt, bool shared_kv = false) {
+                                    void* part, int* cnt, bool shared_kv = false, bool kv8 = false) {
     AttnArgs t = {};
     t.q = q; t.kc = kc; t.vc = vc; t.seq_stride = seq_stride;
     t.out = out; t.tp = tp; t.tp_stride = 2;
@@ -323,9 +328,30 @@ static cudaError_t launch_attention(l2c_ctx* h, cudaStream_t s, bool pdl, bool d
     t.min_chunk = h->attn_min_chunk;
     t.part = part; t.count = cnt; t.shared_kv = shared_kv ? 1 : 0;
     AttnKernel ak = dbl ? attn_kernel_for<double>(h->hs, h->rep) : attn_kernel_for<float>(h->hs, h->rep);
+    if (kv8 && dbl) {
+        // the int8 cache of the same rows: codes at the same element offset,
+        // scales at one per (row, KV head)
+        const size_t eo = (size_t)(kc - h->kc);
+        t.kq = h->kq8 + eo; t.vq = h->vq8 + eo;
+        t.ks = h->ks8 + eo / h->hs; t.vs = h->vs8 + eo / h->hs;
+        t.sc_seq_stride = seq_stride / h->hs;
+        ak = attn_kernel_kv8(h->hs, h->rep);
+    }
     const size_t smem = (size_t)(dbl ? attn_smem_for<double>(h->rep) : attn_smem_for<float>(h->rep));
     const int threads = dbl ? attn_threads<double>() : attn_threads<float>();
     return launch(s, pdl, ak, dim3(t.nchunks, h->Hkv, B), dim3(threads), smem, t);
+}
+
+// The int8 cache arguments for fp32 rows starting at kc / vc (rows of the
+// handle's cache; the int8 rows sit at the same row index).
+static Kv8Args kv8_args(l2c_ctx* h, float* kc, float* vc) {
+    Kv8Args k8 = {};
+    const size_t eo = (size_t)(kc - h->kc);
+    k8.kc = kc; k8.vc = vc;
+    k8.kq = h->kq8 + eo; k8.vq = h->vq8 + eo;
+    k8.ks = h->ks8 + eo / h->hs; k8.vs = h->vs8 + eo / h->hs;
+    k8.kvd = h->kvd; k8.hs = h->hs; k8.n_kv_heads = h->Hkv; k8.seq_len = h->S;
+    return k8;
 }
 
 // Enqueues kernel `kind` of layer l (sequence seq) on stream s.
@@ -368,8 +394,16 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
         e = launch_gemv<M_QKV>(h, q80, a, 2);
         break;
     case SK_ATTN:
+        if (h->kv8) {
+            // the row just written at pos into the int8 cache (and its fp32 row
+            // to code * scale, as kv_read returns it)
+            Kv8Args k8 = kv8_args(h, kslot, vslot);
+            k8.pos = tp + 1;
+            e = launch(s, true, k_kv8_rows, dim3(1, 2 * h->Hkv), dim3(32), 0, k8);
+            if (e != cudaSuccess) break;
+        }
         e = launch_attention(h, s, true, q80, q, kslot, vslot, (size_t)h->L * S * kvd, att, tp, 1, h->attn_part,
-                             h->attn_cnt + (size_t)seq * h->Hkv);
+                             h->attn_cnt + (size_t)seq * h->Hkv, false, h->kv8);
         break;
     case SK_WO:  // wo + residual
         a.rows = (int)d; a.K = (int)d;
@@ -874,6 +908,7 @@ static const float* forward_impl(l2c_ctx* h, int token, int pos, bool q80) {
     if (token < 0 || token >= h->V) { fail(h, L2C_E_ARG, "token %d not in [0,%d)", token, h->V); return nullptr; }
     if (pos < 0 || pos >= h->S) { fail(h, L2C_E_ARG, "pos %d not in [0,%d)", pos, h->S); return nullptr; }
     if (q80 && !h->gs) { fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)"); return nullptr; }
+    if (!q80 && h->kv8) { fail(h, L2C_E_STATE, "the int8 KV cache serves the Q8_0 step"); return nullptr; }
     if (h->graphs && build_graph(h, q80, false) != L2C_OK) return nullptr;
     k_set_tp<<<1, 1, 0, h->stream>>>(h->tp, token, pos);
     cudaError_t e = cudaSuccess;
@@ -898,6 +933,7 @@ extern "C" int l2c_generate(l2c_ctx* h, int token0, int pos0, int steps, int q80
     if (token0 < 0 || token0 >= h->V) return fail(h, L2C_E_ARG, "token %d not in [0,%d)", token0, h->V);
     if (pos0 < 0 || pos0 + steps > h->S) return fail(h, L2C_E_ARG, "pos0 + steps exceeds seq_len");
     if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
+    if (!q80 && h->kv8) return fail(h, L2C_E_STATE, "the int8 KV cache serves the Q8_0 step");
     if (steps == 0) return L2C_OK;
     int rc = build_graph(h, q80 != 0, true);
     if (rc) return rc;
@@ -914,6 +950,7 @@ extern "C" int l2c_forward_batch(l2c_ctx* h, int B, const int32_t* tokens, const
         return fail(h, L2C_E_ARG, "forward_batch: need 1 <= B <= max_batch and non-null arrays");
     if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
     if (B > BMAX) return fail(h, L2C_E_ARG, "forward_batch: the batched step takes at most %d sequences", BMAX);
+    if (h->kv8) return fail(h, L2C_E_STATE, "forward_batch: not with the int8 KV cache (l2c_enable_kv8)");
     const bool tok_dev = is_device_ptr(tokens), pos_dev = is_device_ptr(pos);
     if (!tok_dev && !pos_dev) {
         for (int b = 0; b < B; b++) {
@@ -953,6 +990,7 @@ extern "C" int l2c_prefill(l2c_ctx* h, int seq, int n, const int32_t* tokens, in
     for (int i = 0; i < n; i++)
         if (tokens[i] < 0 || tokens[i] >= h->V) return fail(h, L2C_E_ARG, "token[%d]=%d out of range", i, tokens[i]);
     if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
+    if (h->kv8) return fail(h, L2C_E_STATE, "prefill: not with the int8 KV cache (l2c_enable_kv8)");
     int rc;
     if (q80) {
         if (batched_kc(h->d, h->gs) == 0 || batched_kc(h->h, h->gs) == 0 || h->gs % 32)
@@ -1094,9 +1132,47 @@ extern "C" int l2c_kv_load(l2c_ctx* h, int seq, int n_pos, const float* k, const
     for (size_t l = 0; l < L; l++) {
         if (k) CK(cudaMemcpyAsync(h->kc + base + l * S * kvd, k + l * n_pos * kvd, n_pos * kvd * 4, kk, h->stream));
         if (v) CK(cudaMemcpyAsync(h->vc + base + l * S * kvd, v + l * n_pos * kvd, n_pos * kvd * 4, kv, h->stream));
+        if (h->kv8) {  // the loaded rows into the int8 cache (both K and V, as a step stores them)
+            Kv8Args k8 = kv8_args(h, h->kc + base + l * S * kvd, h->vc + base + l * S * kvd);
+            k_kv8_rows<<<dim3((unsigned)n_pos, 2 * h->Hkv), 32, 0, h->stream>>>(k8);
+            CK(cudaGetLastError());
+        }
     }
     CK(cudaStreamSynchronize(h->stream));
     return L2C_OK;
+}
+
+extern "C" int l2c_enable_kv8(l2c_ctx* h, int on) {
+    if (!h) return L2C_E_ARG;
+    if (on && (h->hs % 4 || h->hs > 128 || !attn_kernel_kv8(h->hs, h->rep)))
+        return fail(h, L2C_E_ARG, "int8 KV cache: head size %d / GQA ratio %d not built", h->hs, h->rep);
+    if ((bool)on == h->kv8) return L2C_OK;
+    int rc;
+    if (on && !h->kq8) {
+        const size_t rows = (size_t)h->max_batch * h->L * h->S;
+        if ((rc = dalloc(h, (void**)&h->kq8, rows * h->kvd)) != L2C_OK) return rc;
+        if ((rc = dalloc(h, (void**)&h->vq8, rows * h->kvd)) != L2C_OK) return rc;
+        if ((rc = dalloc(h, (void**)&h->ks8, rows * h->Hkv * 4)) != L2C_OK) return rc;
+        if ((rc = dalloc(h, (void**)&h->vs8, rows * h->Hkv * 4)) != L2C_OK) return rc;
+    }
+    if (on) {  // every row already in the cache into the int8 cache
+        const size_t rows = (size_t)h->max_batch * h->L * h->S;
+        for (size_t r0 = 0; r0 < rows; r0 += 65535) {
+            const size_t n = rows - r0 < 65535 ? rows - r0 : 65535;
+            Kv8Args k8 = kv8_args(h, h->kc + r0 * h->kvd, h->vc + r0 * h->kvd);
+            k_kv8_rows<<<dim3((unsigned)n, 2 * h->Hkv), 32, 0, h->stream>>>(k8);
+            CK(cudaGetLastError());
+        }
+    }
+    // the step graphs were captured for the other cache
+    for (int a = 0; a < 2; a++)
+        for (int b = 0; b < 2; b++)
+            if (h->graph[a][b]) {
+                cudaGraphExecDestroy(h->graph[a][b]);
+                h->graph[a][b] = nullptr;
+            }
+    h->kv8 = on != 0;
+    return l2c_sync(h);
 }
 
 extern "C" int l2c_kv_read(l2c_ctx* h, int seq, int n_pos, float* k, float* v) {
@@ -1116,12 +1192,15 @@ extern "C" int l2c_kv_read(l2c_ctx* h, int seq, int n_pos, float* k, float* v) {
 extern "C" int l2c_kv_reset(l2c_ctx* h, int seq) {
     if (!h || seq < -1 || seq >= h->max_batch) return fail(h, L2C_E_ARG, "kv_reset: bad sequence");
     const size_t n = (size_t)h->L * h->S * h->kvd;
-    if (seq < 0) {
-        CK(cudaMemsetAsync(h->kc, 0, n * h->max_batch * 4, h->stream));
-        CK(cudaMemsetAsync(h->vc, 0, n * h->max_batch * 4, h->stream));
-    } else {
-        CK(cudaMemsetAsync(h->kc + (size_t)seq * n, 0, n * 4, h->stream));
-        CK(cudaMemsetAsync(h->vc + (size_t)seq * n, 0, n * 4, h->stream));
+    const size_t s0 = seq < 0 ? 0 : (size_t)seq, ns = seq < 0 ? (size_t)h->max_batch : 1;
+    CK(cudaMemsetAsync(h->kc + s0 * n, 0, n * ns * 4, h->stream));
+    CK(cudaMemsetAsync(h->vc + s0 * n, 0, n * ns * 4, h->stream));
+    if (h->kq8) {  // codes 0, scales 0: the int8 cache reads 0 as well
+        const size_t nsc = n / h->hs;
+        CK(cudaMemsetAsync(h->kq8 + s0 * n, 0, n * ns, h->stream));
+        CK(cudaMemsetAsync(h->vq8 + s0 * n, 0, n * ns, h->stream));
+        CK(cudaMemsetAsync(h->ks8 + s0 * nsc, 0, nsc * ns * 4, h->stream));
+        CK(cudaMemsetAsync(h->vs8 + s0 * nsc, 0, nsc * ns * 4, h->stream));
     }
     return L2C_OK;
 }

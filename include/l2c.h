@@ -187,6 +187,25 @@ L2C_API int l2c_forward_batch(l2c_ctx* h, int B, const int32_t* tokens, const in
 L2C_API int l2c_prefill(l2c_ctx* h, int seq, int n, const int32_t* tokens, int pos0, int q80, float* logits_last_dev);
 
 /*
+ * l2c_enable_kv8 - the int8 KV cache (on = 1) or the fp32 one (on = 0).  The
+ * pages give no int8 KV cache; the reading: every K and V row, when it is
+ * stored, becomes Q8_0 groups of head_size values (one per KV head) with the
+ * quantize() rule of [port] §1, and attention reads code * scale (one fp32
+ * multiply).  It serves the Q8_0 step (l2c_forward_q80, l2c_generate with
+ * q80 = 1), whose attention then streams the codes and scales (a quarter of
+ * the bytes); the fp32 cache rows are overwritten with the same code * scale
+ * values (l2c_kv_read returns those).  Enabling it quantizes every row
+ * already in the cache (all sequences); l2c_kv_load quantizes the rows it
+ * loads.  The first call allocates the codes (2 * max_batch * n_layers *
+ * seq_len * kv_dim bytes) and scales.  While it is on, the fp32 step
+ * (l2c_forward, l2c_generate with q80 = 0), l2c_forward_batch and
+ * l2c_prefill return L2C_E_STATE.
+ * Errors: L2C_E_ARG for a head size / GQA ratio without an attention kernel
+ * (head_size a multiple of 4, at most 128); L2C_E_OOM.  Blocks.
+ */
+L2C_API int l2c_enable_kv8(l2c_ctx* h, int on);
+
+/*
  * l2c_quantize_q80 - quantize() of [port] §1 INT8量化压缩 on n device
  * floats: for each group of gs values, s[g] = max|x| / 127 (fp32) and
  * q[i] = round(x[i] / s[g]) (fp32 quotient, half away from zero); a group of

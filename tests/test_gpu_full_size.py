@@ -48,6 +48,16 @@ def test_7b_step_matches_oracle():
             assert err <= (TOL_Q80 if q80 else TOL_F32), (q80, P, err)
             if q80:
                 assert err <= 1e-5, (P, err)
+    # the int8 KV cache on both sides: every row in the cache is quantized, then the
+    # Q8_0 steps (each writes its slot through the int8 store) keep reproducing the
+    # oracle's codes (1e-5)
+    dec.enable_kv8()
+    orc.enable_kv8()
+    for P in (0, 512, P_MAX):
+        got = dec.forward(1, P, q80=True).cpu().numpy()
+        ref = orc.forward(1, P, q80=True)
+        err = rel_err(got, ref)
+        assert err <= 1e-5, ("kv8", P, err)
     dec.close()
     orc.close()
 
