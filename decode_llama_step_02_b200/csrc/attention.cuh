@@ -412,9 +412,13 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
     float4* ring = aring + (size_t)warp * ATTN_NB * PB * 2 * 32;
     // ring entry of (slot, position i, K or V) for this lane
     auto ent = [&](int slot, int i, int kv) -> float4* { return ring + ((slot * PB + i) * 2 + kv) * 32 + lane; };
-    // its values (KV8: decoded from the codes and the scale)
+    // its values (KV8: this lane's codes, decoded with the head's scale, which
+    // lane 0 alone copies into its own entry)
     auto val = [&](int slot, int i, int kv) -> float4 {
-        return KV8 ? kv8_decode(*ent(slot, i, kv)) : *ent(slot, i, kv);
+        if (!KV8) return *ent(slot, i, kv);
+        float4 e = *ent(slot, i, kv);
+        e.y = (ring + ((slot * PB + i) * 2 + kv) * 32)->y;
+        return kv8_decode(e);
     };
     // copies of the warp's jj-th batch into slot jj % ATTN_NB; always one commit group
     auto issue = [&](int jj) {
@@ -426,11 +430,14 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
             const bool on = lane_on && bi < nb && t < t1;
             const size_t off = on ? (size_t)t * a.kvd : 0;
             if (KV8) {
-                const size_t so = on ? (size_t)t * a.Hkv : 0;
+                const bool pos_on = bi < nb && t < t1;
+                const size_t so = pos_on ? (size_t)t * a.Hkv : 0;
                 cp_async4(&ent(slot, i, 0)->x, kq + off, on);
-                cp_async4(&ent(slot, i, 0)->y, ksc + so, on);
                 cp_async4(&ent(slot, i, 1)->x, vq + off, on);
-                cp_async4(&ent(slot, i, 1)->y, vsc + so, on);
+                if (lane == 0) {
+                    cp_async4(&ent(slot, i, 0)->y, ksc + so, pos_on);
+                    cp_async4(&ent(slot, i, 1)->y, vsc + so, pos_on);
+                }
             } else {
                 cp_async16(ent(slot, i, 0), kc + off, on, pol);
                 cp_async16(ent(slot, i, 1), vc + off, on, pol);
@@ -472,6 +479,7 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
         const int bi = warp + ATTN_WARPS * jj;
         if (bi >= nb) break;
         cp_async_wait<ATTN_NB - 2>();  // batch jj has landed (this lane's copies)
+        if (KV8) __syncwarp();         // ... and lane 0's scales, for every lane
         issue(jj + ATTN_NB - 1);       // into the slot read in the previous round
         const int slot = jj % ATTN_NB;
         if (DBL) {
