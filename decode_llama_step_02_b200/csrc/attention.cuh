@@ -133,6 +133,36 @@ __device__ __forceinline__ void cp_async4(void* dst, const void* src, bool on) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
+// One head's K or V row (hs <= 128 values at x) into the int8 KV cache with
+// one warp: quantize() of "超精简LLM部署" §1 over the whole row (the group is the
+// head), codes to q, the scale to *sc, and code * scale back over x.  A
+// non-finite element makes the scale NaN (every read of the group is NaN).
+__device__ __forceinline__ void kv8_store_head(float* x, int8_t* q, float* sc, int hs) {
+    const int lane = threadIdx.x & 31;
+    float v[4];
+    float m = 0.f;
+    bool bad = false;
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+        const int i = lane + 32 * e;
+        v[e] = i < hs ? x[i] : 0.f;
+        m = fmaxf(m, fabsf(v[e]));
+        bad |= !isfinite(v[e]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float scale = __any_sync(0xffffffffu, bad) ? __int_as_float(0x7fc00000) : m / 127.0f;
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+        const int i = lane + 32 * e;
+        if (i >= hs) break;
+        const int code = scale != 0.f && scale == scale ? (int)roundf(v[e] / scale) : 0;
+        q[i] = (int8_t)code;
+        x[i] = __fmul_rn((float)code, scale);
+    }
+    if (lane == 0) *sc = scale;
+}
+
 // A ring entry of the int8 KV cache: .x holds four codes (little-endian), .y
 // their head's scale; the values are code * scale (fp32 multiplies).
 __device__ __forceinline__ float4 kv8_decode(const float4 e) {
@@ -452,6 +482,22 @@ __global__ void __launch_bounds__(ATTN_THREADS) k_attention(const AttnArgs a) {
     while (nissued < ATTN_NB - 1 && before_wait_ok(nissued)) issue(nissued++);
     grid_dep_wait();
     grid_dep_launch();
+    if (KV8 && t1 == pos + 1) {
+        // this CTA's chunk holds the current position: its warp 0 stores the
+        // K and V rows at pos of head g (written by the q/k/v kernel, fp32)
+        // into the int8 cache, and the fp32 rows as code * scale, before any
+        // warp copies that row (the copies of earlier rows are unaffected)
+        if (warp == 0) {
+            kv8_store_head(const_cast<float*>(a.kc) + (size_t)b * a.seq_stride + (size_t)pos * a.kvd + (size_t)g * HS,
+                           const_cast<int8_t*>(a.kq) + (size_t)b * a.seq_stride + (size_t)pos * a.kvd + (size_t)g * HS,
+                           const_cast<float*>(a.ks) + (size_t)b * a.sc_seq_stride + (size_t)pos * a.Hkv + g, HS);
+            kv8_store_head(const_cast<float*>(a.vc) + (size_t)b * a.seq_stride + (size_t)pos * a.kvd + (size_t)g * HS,
+                           const_cast<int8_t*>(a.vq) + (size_t)b * a.seq_stride + (size_t)pos * a.kvd + (size_t)g * HS,
+                           const_cast<float*>(a.vs) + (size_t)b * a.sc_seq_stride + (size_t)pos * a.Hkv + g, HS);
+            __threadfence();
+        }
+        __syncthreads();
+    }
     while (nissued < ATTN_NB - 1) issue(nissued++);
 
     const float* q = a.q + (size_t)b * a.H * HS + (size_t)g * REP * HS;

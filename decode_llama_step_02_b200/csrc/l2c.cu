@@ -350,7 +350,7 @@ static Kv8Args kv8_args(l2c_ctx* h, float* kc, float* vc) {
     k8.kc = kc; k8.vc = vc;
     k8.kq = h->kq8 + eo; k8.vq = h->vq8 + eo;
     k8.ks = h->ks8 + eo / h->hs; k8.vs = h->vs8 + eo / h->hs;
-    k8.kvd = h->kvd; k8.hs = h->hs; k8.n_kv_heads = h->Hkv; k8.seq_len = h->S;
+    k8.kvd = h->kvd; k8.hs = h->hs; k8.n_kv_heads = h->Hkv;
     return k8;
 }
 
@@ -393,15 +393,7 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
         if (l == 0 && seq == 0) a.stall = h->stall;
         e = launch_gemv<M_QKV>(h, q80, a, 2);
         break;
-    case SK_ATTN:
-        if (h->kv8) {
-            // the row just written at pos into the int8 cache (and its fp32 row
-            // to code * scale, as kv_read returns it)
-            Kv8Args k8 = kv8_args(h, kslot, vslot);
-            k8.pos = tp + 1;
-            e = launch(s, true, k_kv8_rows, dim3(1, 2 * h->Hkv), dim3(32), 0, k8);
-            if (e != cudaSuccess) break;
-        }
+    case SK_ATTN:  // with the int8 KV cache the attention also stores the row at pos
         e = launch_attention(h, s, true, q80, q, kslot, vslot, (size_t)h->L * S * kvd, att, tp, 1, h->attn_part,
                              h->attn_cnt + (size_t)seq * h->Hkv, false, h->kv8);
         break;
