@@ -728,6 +728,8 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
     h->attn_min_chunk = (int)env_size("L2C_ATTN_MIN_CHUNK", (size_t)h->attn_min_chunk);
     if (h->attn_min_chunk < 1) h->attn_min_chunk = 1;
     h->q8_early = (int)env_size("L2C_Q8_EARLY", (size_t)h->q8_early);
+    h->bgemm_stages = (int)env_size("L2C_BGEMM_STAGES", (size_t)h->bgemm_stages);
+    if (h->bgemm_stages < 2) h->bgemm_stages = 2;
     h->wait_ns = env_size("L2C_WAIT_NS", h->wait_ns);
     if (getenv("L2C_TEST_OOM_AFTER")) h->oom_after = (long long)env_size("L2C_TEST_OOM_AFTER", 0);
     auto bail = [&](int code) { l2c_destroy(h); return code; };
