@@ -116,3 +116,27 @@ def test_prefill_rejects_bad_arguments():
     assert e.value.code == l2c.L2C_E_STATE
     dec.close()
     orc.close()
+
+
+def test_prefill_second_sequence_of_a_batch_handle():
+    """A prompt into sequence 1 of a two-sequence handle: its cache rows and last
+    logits match the oracle's sequence 1; sequence 0's cache stays untouched."""
+    torch, l2c = need_gpu()
+    spec = synth.M15
+    b = synth.blob(spec)
+    dec = l2c.Decoder(spec.cfg, torch.from_numpy(b).cuda(), spec.shared_weights, max_batch=2)
+    orc = oracle.Model(spec.cfg, b, spec.shared_weights, n_seq=2)
+    toks = synth.tokens(spec.seed, 54, 37, spec.vocab_size)
+    last = torch.empty(spec.vocab_size, dtype=torch.float32, device="cuda")
+    dec.prefill(toks, 0, logits_last=last, seq=1)
+    ref = None
+    for i, t in enumerate(toks):
+        ref = orc.forward(int(t), i, seq=1)
+    assert rel_err(last.cpu().numpy(), ref) <= TOL_F32
+    k, v = dec.kv_read(37, seq=1)
+    kr, vr = orc.kv_read(37, seq=1)
+    assert rel_err(k, kr) <= 1e-5 and rel_err(v, vr) <= 1e-5
+    k0, v0 = dec.kv_read(37, seq=0)
+    assert not np.any(k0) and not np.any(v0)
+    dec.close()
+    orc.close()
