@@ -57,6 +57,7 @@ def lib():
             "orc_silu": (ctypes.c_double, [ctypes.c_double]),
             "orc_swiglu": (None, [vp, vp, i32]),
             "orc_quantize": (i32, [vp, i64, i32, vp, vp]),
+            "orc_quantize4": (i32, [vp, i64, i32, vp, vp]),
             "orc_dequantize": (None, [vp, vp, i64, i32, vp]),
             "orc_q80_group_dots": (None, [vp, vp, vp, i32, i32, i32]),
             "orc_matvec_q80": (None, [vp, vp, vp, vp, vp, i32, i32, i32]),
@@ -65,6 +66,7 @@ def lib():
             "orc_blob_floats": (sz, [vp, i32]),
             "orc_create": (vp, [vp, vp, sz, i32, i32]),
             "orc_enable_q80": (i32, [vp, i32]),
+            "orc_enable_q40": (i32, [vp, i32]),
             "orc_enable_kv8": (i32, [vp]),
             "orc_kv8_row": (None, [vp, i32, i32]),
             "orc_forward": (i32, [vp, i32, i32, i32, i32, vp]),
@@ -163,6 +165,16 @@ def quantize(x, gs: int):
     return q, s
 
 
+def quantize4(x, gs: int):
+    """Q4_0: (codes int8 [n] in [-7, 7], scales fp32 [n/gs])."""
+    x = _f32(x).ravel()
+    q = np.empty(x.size, dtype=np.int8)
+    s = np.empty(x.size // gs, dtype=np.float32)
+    if lib().orc_quantize4(_p(x), x.size, gs, _p(q), _p(s)) != 0:
+        raise ValueError("n must be a multiple of gs")
+    return q, s
+
+
 def dequantize(q, s, gs: int):
     q = np.ascontiguousarray(q, dtype=np.int8)
     s = _f32(s)
@@ -227,20 +239,31 @@ class Model:
         if not self._h:
             raise ValueError("orc_create rejected the config or blob size")
         self.gs = 0
+        self.gs4 = 0
 
     def enable_q80(self, gs: int):
         if lib().orc_enable_q80(self._h, gs) != 0:
             raise ValueError("orc_enable_q80 failed")
         self.gs = gs
 
+    def enable_q40(self, gs: int):
+        """Q4_0 weights (orc_enable_q40); their matvec inputs stay Q8_0."""
+        if lib().orc_enable_q40(self._h, gs) != 0:
+            raise ValueError("orc_enable_q40 failed")
+        self.gs4 = gs
+
     def enable_kv8(self):
         """int8 KV cache: K/V rows kept as Q8_0 groups of head_size (orc_enable_kv8)."""
         if lib().orc_enable_kv8(self._h) != 0:
             raise ValueError("orc_enable_kv8 failed")
 
-    def forward(self, token: int, pos: int, q80: bool = False, seq: int = 0) -> np.ndarray:
+    @staticmethod
+    def _wf(q80, q40):
+        return 2 if q40 else int(bool(q80))
+
+    def forward(self, token: int, pos: int, q80: bool = False, seq: int = 0, q40: bool = False) -> np.ndarray:
         out = np.empty(self.vocab, dtype=np.float32)
-        if lib().orc_forward(self._h, seq, token, pos, int(q80), _p(out)) != 0:
+        if lib().orc_forward(self._h, seq, token, pos, self._wf(q80, q40), _p(out)) != 0:
             raise ValueError("orc_forward rejected its arguments")
         return out
 
@@ -261,10 +284,10 @@ class Model:
         lib().orc_kv_reset(self._h, seq)
 
     def generate(self, token0: int, steps: int, q80: bool = False, pos0: int = 0, seq: int = 0,
-                 keep_logits: bool = True):
+                 keep_logits: bool = True, q40: bool = False):
         toks = np.empty(steps, dtype=np.int32)
         lg = np.empty((steps, self.vocab), dtype=np.float32) if keep_logits else None
-        rc = lib().orc_generate(self._h, seq, token0, pos0, steps, int(q80), _p(toks),
+        rc = lib().orc_generate(self._h, seq, token0, pos0, steps, self._wf(q80, q40), _p(toks),
                                 _p(lg) if lg is not None else None)
         if rc != 0:
             raise ValueError("orc_generate failed")

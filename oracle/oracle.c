@@ -26,7 +26,9 @@
  *   1/sqrt(hs) over positions 0..pos inclusive; query head i uses KV head
  *   i / (n_heads/n_kv_heads); SwiGLU = silu(W1 x) * (W3 x); Q8_0 covers every
  *   matvec weight and the embedding table, and every matvec input is
- *   quantized at the same group size; an all-zero group has scale 0, codes 0.
+ *   quantized at the same group size; an all-zero group has scale 0, codes 0;
+ *   Q4_0 is the same rule with codes in [-7, 7] (scale = max|x| / 7) on the
+ *   same tensors, its matvec inputs still Q8_0.
  *
  * Arithmetic: fp32 storage; sums in double, rounded to fp32 once per step
  * (orc_set_fp32_accum(1) gives the pages' fp32 loops instead).  Every offset
@@ -188,12 +190,13 @@ void orc_swiglu(float* hb, const float* hb2, int n) {
     }
 }
 
-/* Q8_0 quantize [port §1 INT8量化压缩, the quantize() listing]: for each
- * group of gs consecutive values, wmax = max|x|, scale = wmax / 127 (fp32),
- * q = (int8) round(x / scale) with the quotient in fp32 and C round() (half
- * away from zero).  Reading where the listing divides 0 by 0: a group whose
- * wmax is 0 gets scale 0 and all codes 0.  Returns -1 if n % gs != 0. */
-int orc_quantize(const float* x, int64_t n, int gs, int8_t* q, float* s) {
+/* Quantize [port §1 INT8量化压缩, the quantize() listing] with the largest
+ * code qmax as a parameter: for each group of gs consecutive values,
+ * wmax = max|x|, scale = wmax / qmax (fp32), q = (int8) round(x / scale) with
+ * the quotient in fp32 and C round() (half away from zero).  Reading where
+ * the listing divides 0 by 0: a group whose wmax is 0 gets scale 0 and all
+ * codes 0.  Returns -1 if n % gs != 0. */
+static int orc_quantize_qmax(const float* x, int64_t n, int gs, float qmax, int8_t* q, float* s) {
     if (gs <= 0 || n % gs != 0) return -1;
     int64_t ng = n / gs;
     #pragma omp parallel for schedule(static)
@@ -204,7 +207,7 @@ int orc_quantize(const float* x, int64_t n, int gs, int8_t* q, float* s) {
             float val = fabsf(xg[i]);
             if (val > wmax) wmax = val;
         }
-        float scale = wmax / 127.0f;
+        float scale = wmax / qmax;
         s[g] = scale;
         for (int i = 0; i < gs; i++) {
             if (scale == 0.0f) { q[g * gs + i] = 0; continue; }
@@ -213,6 +216,19 @@ int orc_quantize(const float* x, int64_t n, int gs, int8_t* q, float* s) {
         }
     }
     return 0;
+}
+
+/* Q8_0 [port §1, the quantize() listing]: qmax = 127. */
+int orc_quantize(const float* x, int64_t n, int gs, int8_t* q, float* s) {
+    return orc_quantize_qmax(x, n, gs, 127.0f, q, s);
+}
+
+/* Q4_0 [news 技术深度解析, the 整数量化路径 item: runq.c with 4-bit integer
+ * groups, "like llama.cpp's"; the page gives no rule].  Reading: the Q8_0
+ * rule above with 4-bit codes, qmax = 7: scale = wmax / 7 in fp32, codes
+ * round(x / scale) in [-7, 7], one fp32 scale per group of gs. */
+int orc_quantize4(const float* x, int64_t n, int gs, int8_t* q, float* s) {
+    return orc_quantize_qmax(x, n, gs, 7.0f, q, s);
 }
 
 /* x ~= q * scale of its group, one fp32 multiply per element. */
@@ -339,12 +355,19 @@ int orc_sample(const float* z, int n, float temperature, float topp, double coin
 
 typedef struct { int8_t* q; float* s; } orc_qt;
 
+/* One quantized copy of the weights: every matvec weight and the embedding
+ * table in groups of gs (gs = 0: not made). */
+typedef struct {
+    int gs;
+    orc_qt E, wq, wk, wv, wo, w1, w2, w3, wcls;
+} orc_qset;
+
 struct orc_model {
     orc_config c;
-    int shared, n_seq, gs;
+    int shared, n_seq;
     int kv8; /* 1: the KV cache holds Q8_0 rows (see orc_enable_kv8) */
     const float *E, *w_att, *wq, *wk, *wv, *wo, *w_ffn, *w1, *w2, *w3, *w_final, *wcls;
-    orc_qt qE, qwq, qwk, qwv, qwo, qw1, qw2, qw3, qwcls;
+    orc_qset q8, q4; /* Q8_0 (orc_enable_q80) and Q4_0 (orc_enable_q40) */
     float *kcache, *vcache; /* [n_seq][L][S][kv_dim] */
     float *x, *xb, *xb2, *hb, *hb2, *q;
     int8_t* aq; /* activation codes, max(dim, hidden) */
@@ -418,44 +441,67 @@ orc_model* orc_create(const orc_config* c, const float* blob, size_t blob_floats
     return m;
 }
 
-static int orc_qt_make(orc_qt* t, const float* w, size_t n, int gs) {
+static int orc_qt_make(orc_qt* t, const float* w, size_t n, int gs, int four) {
     t->q = (int8_t*)malloc(n);
     t->s = (float*)malloc(sizeof(float) * (n / (size_t)gs));
     if (!t->q || !t->s) return -1;
-    return orc_quantize(w, (int64_t)n, gs, t->q, t->s);
+    return four ? orc_quantize4(w, (int64_t)n, gs, t->q, t->s) : orc_quantize(w, (int64_t)n, gs, t->q, t->s);
 }
 
 static void orc_qt_free(orc_qt* t) { free(t->q); free(t->s); t->q = NULL; t->s = NULL; }
 
-/* Quantizes every matvec weight and the embedding table to Q8_0 with group
- * size gs (groups run along the flattened tensor, which is along rows since
- * every input width is a multiple of gs).  A tied classifier shares E's codes. */
-int orc_enable_q80(orc_model* m, int gs) {
+static void orc_qset_free(orc_qset* z, int shared) {
+    orc_qt_free(&z->E);
+    orc_qt_free(&z->wq); orc_qt_free(&z->wk); orc_qt_free(&z->wv); orc_qt_free(&z->wo);
+    orc_qt_free(&z->w1); orc_qt_free(&z->w2); orc_qt_free(&z->w3);
+    if (!shared) orc_qt_free(&z->wcls);
+    z->gs = 0;
+}
+
+/* Quantizes every matvec weight and the embedding table with group size gs
+ * (groups run along the flattened tensor, which is along rows since every
+ * input width is a multiple of gs), Q8_0 codes or (four = 1) Q4_0 codes.  A
+ * tied classifier shares E's codes. */
+static int orc_qset_make(orc_model* m, orc_qset* z, int gs, int four) {
     const orc_config* c = &m->c;
     size_t d = (size_t)c->dim, h = (size_t)c->hidden_dim, L = (size_t)c->n_layers;
     size_t hs = d / (size_t)c->n_heads, kvd = (size_t)c->n_kv_heads * hs, V = (size_t)c->vocab_size;
     if (gs <= 0 || d % (size_t)gs || h % (size_t)gs) return -1;
-    if (m->gs) return m->gs == gs ? 0 : -1;
+    if (z->gs) return z->gs == gs ? 0 : -1;
     int rc = 0;
-    rc |= orc_qt_make(&m->qE, m->E, V * d, gs);
-    rc |= orc_qt_make(&m->qwq, m->wq, L * d * d, gs);
-    rc |= orc_qt_make(&m->qwk, m->wk, L * kvd * d, gs);
-    rc |= orc_qt_make(&m->qwv, m->wv, L * kvd * d, gs);
-    rc |= orc_qt_make(&m->qwo, m->wo, L * d * d, gs);
-    rc |= orc_qt_make(&m->qw1, m->w1, L * h * d, gs);
-    rc |= orc_qt_make(&m->qw2, m->w2, L * d * h, gs);
-    rc |= orc_qt_make(&m->qw3, m->w3, L * h * d, gs);
-    if (m->shared) m->qwcls = m->qE;
-    else rc |= orc_qt_make(&m->qwcls, m->wcls, V * d, gs);
-    if (rc) return -1;
-    m->gs = gs;
+    rc |= orc_qt_make(&z->E, m->E, V * d, gs, four);
+    rc |= orc_qt_make(&z->wq, m->wq, L * d * d, gs, four);
+    rc |= orc_qt_make(&z->wk, m->wk, L * kvd * d, gs, four);
+    rc |= orc_qt_make(&z->wv, m->wv, L * kvd * d, gs, four);
+    rc |= orc_qt_make(&z->wo, m->wo, L * d * d, gs, four);
+    rc |= orc_qt_make(&z->w1, m->w1, L * h * d, gs, four);
+    rc |= orc_qt_make(&z->w2, m->w2, L * d * h, gs, four);
+    rc |= orc_qt_make(&z->w3, m->w3, L * h * d, gs, four);
+    if (m->shared) z->wcls = z->E;
+    else rc |= orc_qt_make(&z->wcls, m->wcls, V * d, gs, four);
+    if (rc) {
+        z->gs = 1; /* any nonzero: free what was made */
+        orc_qset_free(z, m->shared);
+        return -1;
+    }
+    z->gs = gs;
     return 0;
 }
 
-/* matvec through Q8_0: quantize the input at the model's group size, then
- * the exact-int32 group matvec on layer l of a stacked [L][d][n] tensor. */
-static void orc_qmatvec(orc_model* m, float* o, const float* x, const orc_qt* t, size_t l, int n, int d) {
-    int gs = m->gs;
+/* Q8_0 weights [port §1; hub §量化支持]. */
+int orc_enable_q80(orc_model* m, int gs) { return orc_qset_make(m, &m->q8, gs, 0); }
+
+/* Q4_0 weights [news 技术深度解析, 整数量化路径] (the reading of orc_quantize4);
+ * the inputs of their matvecs are Q8_0 at the same group size, as in the
+ * Q8_0 step. */
+int orc_enable_q40(orc_model* m, int gs) { return orc_qset_make(m, &m->q4, gs, 1); }
+
+/* matvec through a quantized set: quantize the input to Q8_0 at the set's
+ * group size, then the exact-int32 group matvec on layer l of a stacked
+ * [L][d][n] tensor. */
+static void orc_qmatvec(orc_model* m, const orc_qset* z, float* o, const float* x, const orc_qt* t, size_t l, int n,
+                        int d) {
+    int gs = z->gs;
     orc_quantize(x, n, gs, m->aq, m->as);
     size_t off = l * (size_t)d * (size_t)n;
     orc_matvec_q80(o, m->aq, m->as, t->q + off, t->s + off / (size_t)gs, n, d, gs);
@@ -466,17 +512,20 @@ static void orc_qmatvec(orc_model* m, float* o, const float* x, const orc_qt* t,
  * per layer RMSNorm, q/k/v matvecs with k and v written straight into the
  * cache slot [layer][pos], RoPE on q and k, attention over 0..pos, wo matvec
  * plus residual, RMSNorm, SwiGLU FFN plus residual; final RMSNorm and the
- * classifier matvec (the embedding table when tied, qa §shared_weights). */
+ * classifier matvec (the embedding table when tied, qa §shared_weights).
+ * q80 picks the weights: 0 fp32, 1 the Q8_0 set, 2 the Q4_0 set. */
 int orc_forward(orc_model* m, int seq, int token, int pos, int q80, float* logits) {
     const orc_config* c = &m->c;
     if (seq < 0 || seq >= m->n_seq || token < 0 || token >= c->vocab_size || pos < 0 ||
         pos >= c->seq_len || !logits) return -1;
-    if (q80 && !m->gs) return -1;
+    if (q80 < 0 || q80 > 2) return -1;
+    const orc_qset* z = q80 == 2 ? &m->q4 : (q80 ? &m->q8 : NULL);
+    if (z && !z->gs) return -1;
     int d = c->dim, h = c->hidden_dim, H = c->n_heads, Hkv = c->n_kv_heads;
     int hs = d / H, kvd = Hkv * hs;
     size_t L = (size_t)c->n_layers, S = (size_t)c->seq_len;
     float* x = m->x;
-    if (q80) orc_dequantize(m->qE.q + (size_t)token * d, m->qE.s + (size_t)token * d / m->gs, d, m->gs, x);
+    if (z) orc_dequantize(z->E.q + (size_t)token * d, z->E.s + (size_t)token * d / z->gs, d, z->gs, x);
     else memcpy(x, m->E + (size_t)token * d, sizeof(float) * (size_t)d);
     for (size_t l = 0; l < L; l++) {
         size_t loff = ((size_t)seq * L + l) * S * (size_t)kvd;
@@ -485,10 +534,10 @@ int orc_forward(orc_model* m, int seq, int token, int pos, int q80, float* logit
         float* k = kc + (size_t)pos * kvd;
         float* v = vc + (size_t)pos * kvd;
         orc_rmsnorm(m->xb, x, m->w_att + l * d, d);
-        if (q80) {
-            orc_qmatvec(m, m->q, m->xb, &m->qwq, l, d, d);
-            orc_qmatvec(m, k, m->xb, &m->qwk, l, d, kvd);
-            orc_qmatvec(m, v, m->xb, &m->qwv, l, d, kvd);
+        if (z) {
+            orc_qmatvec(m, z, m->q, m->xb, &z->wq, l, d, d);
+            orc_qmatvec(m, z, k, m->xb, &z->wk, l, d, kvd);
+            orc_qmatvec(m, z, v, m->xb, &z->wv, l, d, kvd);
         } else {
             orc_matvec(m->q, m->xb, m->wq + l * (size_t)d * d, d, d);
             orc_matvec(k, m->xb, m->wk + l * (size_t)kvd * d, d, kvd);
@@ -501,24 +550,24 @@ int orc_forward(orc_model* m, int seq, int token, int pos, int q80, float* logit
             orc_kv8_row(v, kvd, hs);
         }
         orc_attention(m->xb, m->q, kc, vc, pos, H, Hkv, hs);
-        if (q80) orc_qmatvec(m, m->xb2, m->xb, &m->qwo, l, d, d);
+        if (z) orc_qmatvec(m, z, m->xb2, m->xb, &z->wo, l, d, d);
         else orc_matvec(m->xb2, m->xb, m->wo + l * (size_t)d * d, d, d);
         for (int i = 0; i < d; i++) x[i] += m->xb2[i];
         orc_rmsnorm(m->xb, x, m->w_ffn + l * d, d);
-        if (q80) {
-            orc_qmatvec(m, m->hb, m->xb, &m->qw1, l, d, h);
-            orc_qmatvec(m, m->hb2, m->xb, &m->qw3, l, d, h);
+        if (z) {
+            orc_qmatvec(m, z, m->hb, m->xb, &z->w1, l, d, h);
+            orc_qmatvec(m, z, m->hb2, m->xb, &z->w3, l, d, h);
         } else {
             orc_matvec(m->hb, m->xb, m->w1 + l * (size_t)h * d, d, h);
             orc_matvec(m->hb2, m->xb, m->w3 + l * (size_t)h * d, d, h);
         }
         orc_swiglu(m->hb, m->hb2, h);
-        if (q80) orc_qmatvec(m, m->xb, m->hb, &m->qw2, l, h, d);
+        if (z) orc_qmatvec(m, z, m->xb, m->hb, &z->w2, l, h, d);
         else orc_matvec(m->xb, m->hb, m->w2 + l * (size_t)d * h, h, d);
         for (int i = 0; i < d; i++) x[i] += m->xb[i];
     }
     orc_rmsnorm(x, x, m->w_final, d);
-    if (q80) orc_qmatvec(m, logits, x, &m->qwcls, 0, d, c->vocab_size);
+    if (z) orc_qmatvec(m, z, logits, x, &z->wcls, 0, d, c->vocab_size);
     else orc_matvec(logits, x, m->wcls, d, c->vocab_size);
     return 0;
 }
@@ -606,12 +655,8 @@ int orc_generate(orc_model* m, int seq, int token0, int pos0, int steps, int q80
 
 void orc_destroy(orc_model* m) {
     if (!m) return;
-    if (m->gs) {
-        orc_qt_free(&m->qE);
-        orc_qt_free(&m->qwq); orc_qt_free(&m->qwk); orc_qt_free(&m->qwv); orc_qt_free(&m->qwo);
-        orc_qt_free(&m->qw1); orc_qt_free(&m->qw2); orc_qt_free(&m->qw3);
-        if (!m->shared) orc_qt_free(&m->qwcls);
-    }
+    if (m->q8.gs) orc_qset_free(&m->q8, m->shared);
+    if (m->q4.gs) orc_qset_free(&m->q4, m->shared);
     free(m->kcache); free(m->vcache);
     free(m->x); free(m->xb); free(m->xb2); free(m->hb); free(m->hb2); free(m->q);
     free(m->aq); free(m->as);

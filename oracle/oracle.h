@@ -11,7 +11,7 @@
  * accumulated in double and rounded to fp32 once at the end of its step.
  * orc_set_fp32_accum(1) switches these sums to the pages' plain fp32
  * left-to-right loops, to show how far the pages' own rounding sits from the
- * double result.  Q8_0 codes and int32 group dot products are exact.
+ * double result.  Q8_0 / Q4_0 codes and int32 group dot products are exact.
  */
 #ifndef L2C_ORACLE_H
 #define L2C_ORACLE_H
@@ -42,6 +42,8 @@ void orc_attention(float* out, const float* q, const float* kc, const float* vc,
 double orc_silu(double z);
 void orc_swiglu(float* hb, const float* hb2, int n);
 int orc_quantize(const float* x, int64_t n, int gs, int8_t* q, float* s);
+/* Q4_0: the same rule with scale = max|x| / 7, codes in [-7, 7] (one int8 each). */
+int orc_quantize4(const float* x, int64_t n, int gs, int8_t* q, float* s);
 void orc_dequantize(const int8_t* q, const float* s, int64_t n, int gs, float* out);
 void orc_q80_group_dots(int32_t* out, const int8_t* qx, const int8_t* qw, int n, int d, int gs);
 void orc_matvec_q80(float* o, const int8_t* qx, const float* sx, const int8_t* qw, const float* sw,
@@ -55,9 +57,12 @@ size_t orc_blob_floats(const orc_config* c, int shared_weights);
 orc_model* orc_create(const orc_config* c, const float* blob, size_t blob_floats, int shared_weights,
                       int n_seq);
 int orc_enable_q80(orc_model* m, int gs);
+/* Q4_0 weights (matvec inputs stay Q8_0 at the same group size). */
+int orc_enable_q40(orc_model* m, int gs);
 /* int8 KV cache: K and V rows stored as Q8_0 groups of head_size values. */
 int orc_enable_kv8(orc_model* m);
 void orc_kv8_row(float* row, int n, int gs);
+/* q80: 0 fp32 weights, 1 the Q8_0 set, 2 the Q4_0 set. */
 int orc_forward(orc_model* m, int seq, int token, int pos, int q80, float* logits);
 int orc_kv_load(orc_model* m, int seq, int n_pos, const float* k, const float* v);
 int orc_kv_reset(orc_model* m, int seq);

@@ -5,7 +5,8 @@ The whole sequence at once, in float64 NumPy: causal-masked attention over a
 e^{i pos freq} (the PyTorch "freqs_cis" form the karpathy-notes Q&A page
 contrasts with llama2.c's on-the-fly cosf/sinf), grouped-query attention as
 multi-head attention over K/V repeated per query head, and Q8_0 matvecs as
-matrix products of dequantized operands.  Row t of its logits must equal the
+matrix products of dequantized operands (Q4_0 weights the same way, their inputs
+Q8_0).  Row t of its logits must equal the
 decode step at position t fed the same tokens.
 
 Values are float64 between the points where the decode step stores fp32
@@ -57,7 +58,11 @@ def _kv8(M, hs, quantize):
     return f32(q.astype(np.float64) * np.repeat(s.astype(np.float64), hs)).reshape(M.shape)
 
 
-def prefill_logits(cfg, blob, shared, tokens, q80_gs=0, quantize=None, kv8=False):
+def prefill_logits(cfg, blob, shared, tokens, q80_gs=0, quantize=None, kv8=False, wquantize=None):
+    """Logits [T][V].  q80_gs: quantized weights and matvec inputs at that group size,
+    the inputs (and the int8 KV rows) through `quantize`, the weights and the embedding
+    table through `wquantize` (default: `quantize`; the Q4_0 weights pass their own)."""
+    wquantize = wquantize or quantize
     d, h, L, H, Hkv, V, S = cfg
     hs = d // H
     rep = H // Hkv
@@ -80,10 +85,10 @@ def prefill_logits(cfg, blob, shared, tokens, q80_gs=0, quantize=None, kv8=False
         if not q80_gs:
             return f32(Xin @ M.T)
         Xq = np.stack([_q8_fake(r, q80_gs, quantize) for r in Xin.astype(np.float32)])
-        return f32(Xq @ _q8_fake(M, q80_gs, quantize).T)
+        return f32(Xq @ _q8_fake(M, q80_gs, wquantize).T)
 
     if q80_gs:
-        X = _q8_fake(W["E"], q80_gs, quantize)[tokens]
+        X = _q8_fake(W["E"], q80_gs, wquantize)[tokens]
     else:
         X = W["E"][tokens].copy()
     mask = np.triu(np.full((T, T), -np.inf), 1)

@@ -14,12 +14,14 @@ ODD = synth.ModelSpec("odd", 48, 100, 2, 6, 2, 50, 24, 0, seed=10, wsigma=0.2, n
 ODDQ = synth.ModelSpec("oddq", 48, 112, 2, 6, 2, 50, 24, 0, seed=10, wsigma=0.2, nsigma=0.1)
 
 
-def _decode_all(spec, toks, q80=False, gs=0):
+def _decode_all(spec, toks, q80=False, gs=0, q40=False):
     b = synth.blob(spec)
     m = oracle.Model(spec.cfg, b, spec.shared_weights)
     if q80:
         m.enable_q80(gs)
-    return np.stack([m.forward(int(t), p, q80=q80) for p, t in enumerate(toks)]), b
+    if q40:
+        m.enable_q40(gs)
+    return np.stack([m.forward(int(t), p, q80=q80, q40=q40) for p, t in enumerate(toks)]), b
 
 
 @pytest.mark.parametrize("spec,T", [(BRUTE, 8), (ODD, 24), (synth.TINY, 40), (synth.M15, 24)],
@@ -41,6 +43,34 @@ def test_decode_equals_prefill_q80(spec, gs, T):
     # both formulations round to fp32 at the same points, so every Q8_0 code is decided
     # on the same fp32 value: the codes agree and only double rounding noise remains
     assert np.abs(got - ref).max() <= 2e-6 * scale
+
+
+@pytest.mark.parametrize("spec,gs,T", [(ODDQ, 16, 12), (synth.M15, 32, 12)], ids=["oddq", "15M"])
+def test_decode_equals_prefill_q40(spec, gs, T):
+    toks = synth.tokens(spec.seed, 8, T, spec.vocab_size)
+    got, b = _decode_all(spec, toks, q40=True, gs=gs)
+    ref = prefill_logits(spec.cfg, b, spec.shared_weights, toks, q80_gs=gs, quantize=oracle.quantize,
+                         wquantize=oracle.quantize4)
+    assert np.abs(got - ref).max() <= 2e-6 * np.abs(ref).max()
+
+
+def test_q40_coarser_than_q80_and_q80_set_untouched():
+    """Q4_0 moves the logits further from fp32 than Q8_0 does; enabling it beside the
+    Q8_0 set (another group size) leaves the Q8_0 step as it was."""
+    spec = synth.M15
+    toks = synth.tokens(spec.seed, 9, 8, spec.vocab_size)
+    f, b = _decode_all(spec, toks)
+    q8, _ = _decode_all(spec, toks, q80=True, gs=32)
+    q4, _ = _decode_all(spec, toks, q40=True, gs=32)
+    e8, e4 = np.abs(f - q8).max(), np.abs(f - q4).max()
+    assert e8 < e4 <= 0.5 * np.abs(f).max()
+    m = oracle.Model(spec.cfg, b, spec.shared_weights)
+    m.enable_q80(32)
+    m.enable_q40(96)
+    both = np.stack([m.forward(int(t), p, q80=True) for p, t in enumerate(toks)])
+    assert np.array_equal(both, q8)
+    with pytest.raises(ValueError):
+        m.enable_q40(32)  # already made with another group size
 
 
 def test_q80_close_to_fp32():

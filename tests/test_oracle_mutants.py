@@ -27,7 +27,11 @@ MUTANTS = {
     "gqa_mapping": ("int g = h / rep;", "int g = h % n_kv_heads;"),
     "silu_sign": ("return z / (1.0 + exp(-z));", "return z / (1.0 + exp(z));"),
     "quant_round_half_even": ("q[g * gs + i] = (int8_t)round((double)quot);", "q[g * gs + i] = (int8_t)rint((double)quot);"),
-    "quant_scale_128": ("float scale = wmax / 127.0f;", "float scale = wmax / 128.0f;"),
+    "quant_scale_128": ("return orc_quantize_qmax(x, n, gs, 127.0f, q, s);", "return orc_quantize_qmax(x, n, gs, 128.0f, q, s);"),
+    "q4_scale_8": ("return orc_quantize_qmax(x, n, gs, 7.0f, q, s);", "return orc_quantize_qmax(x, n, gs, 8.0f, q, s);"),
+    "q4_set_holds_q8_codes": ("return four ? orc_quantize4(", "return 0 ? orc_quantize4("),
+    "q4_embedding_row_from_fp32": ("    if (z) orc_dequantize(z->E.q + (size_t)token * d, z->E.s + (size_t)token * d / z->gs, d, z->gs, x);\n    else memcpy(",
+                                   "    if (z && z == &m->q8) orc_dequantize(m->q8.E.q + (size_t)token * d, m->q8.E.s + (size_t)token * d / m->q8.gs, d, m->q8.gs, x);\n    else memcpy("),
     "q80_drop_sx": ("vd += (double)ival * (double)srow[g] * (double)sx[g];", "vd += (double)ival * (double)srow[g];"),
     "no_attn_residual": ("for (int i = 0; i < d; i++) x[i] += m->xb2[i];", "for (int i = 0; i < d; i++) x[i] = m->xb2[i];"),
     "no_rope_on_k": ("orc_rope(k, kvd, hs, pos);", ""),

@@ -215,6 +215,53 @@ def test_quantize_bounds_and_error():
         oracle.quantize(np.zeros(33, np.float32), 32)
 
 
+def _golden_q4_cases():
+    cases, cur = [], None
+    for ln in open(os.path.join(GOLDEN, "q40_quantize_cases.txt")):
+        ln = ln.strip()
+        if not ln or ln.startswith("#"):
+            continue
+        key, *vals = ln.split()
+        if key == "case":
+            cur = {"name": vals[0]}
+            cases.append(cur)
+        else:
+            cur[key] = vals
+    return cases
+
+
+@pytest.mark.parametrize("case", _golden_q4_cases(), ids=lambda c: c["name"])
+def test_quantize4_cases(case):
+    gs = int(case["gs"][0])
+    x = np.array([float(v) for v in case["x"]], np.float32)
+    q, s = oracle.quantize4(x, gs)
+    assert q.tolist() == [int(v) for v in case["q"]]
+    np.testing.assert_allclose(s, [float(v) for v in case["scale"]], rtol=1e-7, atol=0)
+
+
+def test_quantize4_is_the_nearest_code():
+    """Every Q4_0 code is the integer in [-7, 7] nearest to x / scale (brute force over
+    the 15 codes; ties, which random inputs do not hit, aside), the group's largest
+    magnitude maps to +-7, and the scale is max|x| / 7 in fp32."""
+    for gs in (32, 64, 128):
+        x = (rng.standard_normal(128 * 20) * rng.uniform(0.01, 10, 128 * 20)).astype(np.float32)
+        q, s = oracle.quantize4(x, gs)
+        g = x.reshape(-1, gs)
+        np.testing.assert_array_equal(s, (np.abs(g).max(1) / np.float32(7)).astype(np.float32))
+        quot = (g / s[:, None]).astype(np.float32).astype(np.float64)
+        codes = np.arange(-7, 8, dtype=np.float64)
+        best = codes[np.argmin(np.abs(quot[..., None] - codes), axis=-1)]
+        np.testing.assert_array_equal(q.reshape(-1, gs), best)
+        imax = np.argmax(np.abs(g), axis=1)
+        assert np.all(np.abs(q.reshape(-1, gs)[np.arange(len(g)), imax]) == 7)
+        deq = oracle.dequantize(q, s, gs).reshape(-1, gs).astype(np.float64)
+        assert np.all(np.abs(deq - g) <= s[:, None].astype(np.float64) * (0.5 + 1e-5))
+    q, s = oracle.quantize4(np.zeros(64, np.float32), 32)
+    assert not q.any() and not s.any()
+    with pytest.raises(ValueError):
+        oracle.quantize4(np.zeros(33, np.float32), 32)
+
+
 def test_group_dots_brute_force():
     gs, n, d = 32, 96, 5
     qw = rng.integers(-127, 128, (d, n)).astype(np.int8)
