@@ -58,16 +58,27 @@ def bytes_per_token(q80: bool, pos: int, spec=None, gs=GS) -> float:
     return (1 + 4.0 / gs) * (mats + d) + 4.0 * (2 * L * d + d) + kv
 
 
-def kernel_bytes(kind: int, q80: bool, pos: int, spec=None, gs=GS) -> float:
+def q40_bytes_per_token(pos: int, spec=None, gs=GS) -> float:
+    """Algorithmic bytes of one Q4_0 decode step: every weight once as 4-bit codes
+    plus one fp32 scale per group, the embedding row (int8-wide codes and scales),
+    the norm gains, the fp32 KV cache for positions 0..pos."""
+    d, h, L, H, Hkv, V, S = (spec or SPEC).cfg
+    kvd = Hkv * (d // H)
+    mats = L * (2 * d * d + 2 * d * kvd + 3 * d * h) + V * d
+    return (0.5 + 4.0 / gs) * mats + (1 + 4.0 / gs) * d + 4.0 * (2 * L * d + d) + 8.0 * L * (pos + 1) * kvd
+
+
+def kernel_bytes(kind: int, q80, pos: int, spec=None, gs=GS) -> float:
     """Algorithmic bytes of one launch of step kernel `kind` (the numbering of
     l2c_time_kernel: 0 RMSNorm+QKV+RoPE, 1 attention, 2 wo, 3 RMSNorm+W1/W3+SwiGLU,
     4 W2, 5 final RMSNorm+classifier): its weights once (Q8_0: codes plus fp32
     group scales), plus the vectors it reads and writes; attention: K and V of
-    positions 0..pos, q and the output."""
+    positions 0..pos, q and the output.  q80: 0 fp32, 1 Q8_0, 2 Q4_0 (half a
+    byte per weight plus the scales)."""
     spec = spec or SPEC
     d, h, L, H, Hkv, V, S = spec.cfg
     kvd = Hkv * (d // H)
-    bpw = (1 + 4.0 / gs) if q80 else 4.0
+    bpw = ((0.5 if int(q80) == 2 else 1.0) + 4.0 / gs) if q80 else 4.0
     if kind == 0:
         return (d + 2 * kvd) * d * bpw + 4.0 * (2 * d + d + 2 * kvd)
     if kind == 1:
@@ -438,6 +449,7 @@ def run_ours(args, rank, world, local_rank):
     rows = {}
     if not args.no_rows:
         rows["prefill_7b_128_tokens"] = measure_prefill(torch, dec, ev, stream)
+        rows["q4_0_weights"] = measure_q40(torch, dec, stream, peak)
         rows["q8_0_int8_kv_cache"] = measure_kv8(torch, dec, stream, peak)
     dec.close()
     dec = None
@@ -663,6 +675,45 @@ def measure_kv8(torch, dec, stream, peak, reps=20):
         out[f"pos{p}"] = {"ms_per_token_median": t, "tokens_per_s": 1e3 / t, "bytes_per_token": by,
                           "gbs": by / t / 1e6, "frac_of_measured_hbm": by / t / 1e6 / peak,
                           "frac_of_8tbs_roofline": by / t / 1e6 / NOMINAL_HBM_GBS, "replays": reps}
+    dec.sync()
+    return out
+
+
+def measure_q40(torch, dec, stream, peak, reps=20):
+    """The Q4_0 step (l2c_enable_q40, GS as the Q8_0 step) at the bench positions:
+    the median of `reps` individually timed graph replays per position, and each
+    kernel alone at the last position (l2c_time_kernel), as for the main variants."""
+    dec.enable_q40(GS)
+    out = {}
+    for p in POSITIONS:
+        for _ in range(3):
+            dec.forward_ptr(TOKEN, p, q40=True)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        torch.cuda.synchronize()
+        for a, b in evs:
+            a.record(stream)
+            dec.forward_ptr(TOKEN, p, q40=True)
+            b.record(stream)
+        torch.cuda.synchronize()
+        ts = [a.elapsed_time(b) for a, b in evs]
+        t = statistics.median(ts)
+        by = q40_bytes_per_token(p)
+        out[f"pos{p}"] = {"ms_per_token_median": t, "ms_p10": pct(ts, 0.1), "ms_p90": pct(ts, 0.9),
+                          "tokens_per_s": 1e3 / t, "bytes_per_token": by,
+                          "gbs": by / t / 1e6, "frac_of_measured_hbm": by / t / 1e6 / peak,
+                          "frac_of_8tbs_roofline": by / t / 1e6 / NOMINAL_HBM_GBS, "replays": reps}
+    kpos = POSITIONS[-1]
+    dec.forward_ptr(TOKEN, kpos, q40=True)
+    kern = {}
+    for kind, name in enumerate(KERNEL_NAMES):
+        iters = 2 * SPEC.n_layers if kind != 5 else 8
+        dec.time_kernel(kind, 2, max(4, iters // 4))  # warm
+        kms = dec.time_kernel(kind, 2, iters)
+        by = kernel_bytes(kind, 2, kpos)
+        kern[name] = {"avg_launch_us": 1e3 * kms, "bytes_per_launch": by, "gbs": by / kms / 1e6,
+                      "frac_of_measured_hbm": by / kms / 1e6 / peak, "launches_timed": iters}
+    out["kernels_pos%d" % kpos] = kern
+    out["gs"] = GS
     dec.sync()
     return out
 

@@ -19,7 +19,8 @@ L2C_OK, L2C_E_ARG, L2C_E_OOM, L2C_E_CUDA, L2C_E_DEVICE, L2C_E_STATE, L2C_E_SCRAT
 
 # every symbol declared in include/l2c.h
 EXPORTS = (
-    "l2c_blob_floats", "l2c_create", "l2c_enable_q80", "l2c_forward", "l2c_forward_q80", "l2c_argmax",
+    "l2c_blob_floats", "l2c_create", "l2c_enable_q80", "l2c_enable_q40", "l2c_forward", "l2c_forward_q80",
+    "l2c_forward_q40", "l2c_argmax",
     "l2c_generate", "l2c_sample", "l2c_forward_batch", "l2c_prefill", "l2c_enable_kv8", "l2c_quantize_q80", "l2c_q80_group_dots", "l2c_kv_load",
     "l2c_kv_read", "l2c_kv_reset", "l2c_attention", "l2c_attention_noalloc", "l2c_time_kernel", "l2c_sync", "l2c_stream", "l2c_last_status", "l2c_last_error",
     "l2c_destroy",
@@ -55,8 +56,10 @@ def lib():
             "l2c_blob_floats": (sz, [vp, i32]),
             "l2c_create": (i32, [vp, vp, sz, i32, i32, vp, ctypes.POINTER(vp)]),
             "l2c_enable_q80": (i32, [vp, i32]),
+            "l2c_enable_q40": (i32, [vp, i32]),
             "l2c_forward": (vp, [vp, i32, i32]),
             "l2c_forward_q80": (vp, [vp, i32, i32]),
+            "l2c_forward_q40": (vp, [vp, i32, i32]),
             "l2c_argmax": (i32, [vp, vp, i32, ctypes.POINTER(ctypes.c_int)]),
             "l2c_generate": (i32, [vp, i32, i32, i32, i32, vp]),
             "l2c_sample": (i32, [vp, vp, i32, ctypes.c_float, ctypes.c_float, ctypes.c_double,
@@ -144,18 +147,27 @@ class Decoder:
     def enable_q80(self, gs: int):
         self._check(lib().l2c_enable_q80(self._h, int(gs)))
 
+    def enable_q40(self, gs: int):
+        """Q4_0 weights (l2c_enable_q40): 4-bit codes, scale = max|x| / 7 per group of gs."""
+        self._check(lib().l2c_enable_q40(self._h, int(gs)))
+
+    @staticmethod
+    def _wf(q80, q40):
+        """Weight format of the C ABI: 0 fp32, 1 Q8_0, 2 Q4_0."""
+        return 2 if q40 else int(q80)
+
     # -- steps
-    def forward_ptr(self, token: int, pos: int, q80: bool = False) -> int:
-        f = lib().l2c_forward_q80 if q80 else lib().l2c_forward
+    def forward_ptr(self, token: int, pos: int, q80: bool = False, q40: bool = False) -> int:
+        f = (lib().l2c_forward, lib().l2c_forward_q80, lib().l2c_forward_q40)[self._wf(q80, q40)]
         p = f(self._h, int(token), int(pos))
         if not p:
             raise L2CError(lib().l2c_last_status(self._h), self._msg())
         return p
 
-    def forward(self, token: int, pos: int, q80: bool = False):
+    def forward(self, token: int, pos: int, q80: bool = False, q40: bool = False):
         """Enqueues one step; returns a zero-copy torch view of the device logits."""
         import torch
-        p = self.forward_ptr(token, pos, q80)
+        p = self.forward_ptr(token, pos, q80, q40)
         return torch.as_tensor(_DevArray(p, (self.vocab,), "<f4", 0), device="cuda")
 
     def argmax(self, logits) -> int:
@@ -170,9 +182,9 @@ class Decoder:
                                      float(coin), ctypes.byref(out)))
         return out.value
 
-    def generate(self, token0: int, steps: int, q80: bool = False, pos0: int = 0) -> np.ndarray:
+    def generate(self, token0: int, steps: int, q80: bool = False, pos0: int = 0, q40: bool = False) -> np.ndarray:
         toks = np.empty(steps, dtype=np.int32)
-        self._check(lib().l2c_generate(self._h, int(token0), int(pos0), int(steps), int(q80),
+        self._check(lib().l2c_generate(self._h, int(token0), int(pos0), int(steps), self._wf(q80, q40),
                                        toks.ctypes.data))
         return toks
 
@@ -219,15 +231,16 @@ class Decoder:
         rows, K = qw.shape
         self._check(lib().l2c_q80_group_dots(self._h, _ptr(qw), _ptr(qx), int(rows), int(K), int(gs), _ptr(out)))
 
-    def time_kernel(self, kind: int, q80: bool, iters: int) -> float:
-        """Average ms per launch of one kernel of the step run alone (l2c_time_kernel)."""
+    def time_kernel(self, kind: int, q80, iters: int) -> float:
+        """Average ms per launch of one kernel of the step run alone (l2c_time_kernel);
+        q80: 0 / False fp32, 1 / True Q8_0, 2 Q4_0."""
         ms = ctypes.c_float()
         self._check(lib().l2c_time_kernel(self._h, int(kind), int(q80), int(iters), ctypes.byref(ms)))
         return ms.value
 
-    def set_position(self, token: int, pos: int, q80: bool = False):
+    def set_position(self, token: int, pos: int, q80: bool = False, q40: bool = False):
         """Runs one step at (token, pos) so that the handle's state holds them."""
-        self.forward_ptr(token, pos, q80)
+        self.forward_ptr(token, pos, q80, q40)
 
     def close(self):
         if getattr(self, "_h", None):

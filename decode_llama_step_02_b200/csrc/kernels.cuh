@@ -685,6 +685,67 @@ __device__ __forceinline__ void q8_rows_dot64(const uint8_t* rec, size_t rb, con
     }
 }
 
+// Q4_0 row records: [K/2 bytes of 4-bit codes | K/GS fp32 scales | pad to
+// 16 B].  The values 32t..32t+31 (chunk t) sit in the 16 bytes at 16t: byte
+// b holds value 32t+b in its low nibble and 32t+16+b in its high nibble, each
+// as code + 8 (1..15 for codes in [-7, 7]).
+__host__ __device__ inline size_t q4_record_bytes(int K, int gs) {
+    return (size_t)K / 2 + (((size_t)(K / gs) * 4 + 15) & ~size_t(15));
+}
+
+// UR Q4_0 rows (records at rec, stride rb) against the Q8_0 input codes xq:
+// per lane chunk t one 16-byte load of a row and two of the input (its
+// halves read in the order h = j ^ r, r = bit 2 of the lane, so that the
+// eight lanes of a quarter-warp touch distinct 16-byte bank groups).  The
+// low nibbles of a row chunk pair with input half 0, the high ones with half
+// 1; the chunk's exact dot is sum((code + 8) * x) - corr[t], corr[t] = 8 *
+// (sum of the chunk's input codes), and the CPG = GS/32 chunks of a group
+// (consecutive lanes) add up with shuffles.  Each group's exact int32 dot
+// times the row's group scale and the input's, summed per lane in double as
+// in q8_rows_dot64.  Requires K % 32 == 0, GS in {32, 64, 128}, K % GS == 0.
+template <int GS, int UR>
+__device__ __forceinline__ void q4_rows_dot32(const uint8_t* rec, size_t rb, const int8_t* xq, const float* xs,
+                                              const int* corr, int K, double (&acc)[UR]) {
+    constexpr int CPG = GS / 32;
+    const int lane = threadIdx.x & 31;
+    const int n32 = K >> 5;
+    const int r = (lane >> 2) & 1;
+#pragma unroll
+    for (int u = 0; u < UR; u++) acc[u] = 0.0;
+#pragma unroll 2
+    for (int t0 = 0; t0 < n32; t0 += 32) {
+        const int t = t0 + lane;
+        const bool in = t < n32;
+        int4 xv[2];
+#pragma unroll
+        for (int j = 0; j < 2; j++)
+            xv[j] = in ? *reinterpret_cast<const int4*>(xq + 32 * t + 16 * (j ^ r)) : make_int4(0, 0, 0, 0);
+        const int cr = in ? corr[t] : 0;
+        const bool head = in && (t & (CPG - 1)) == 0;  // the lane that holds its group's dot
+        const double sx = head ? (double)xs[t / CPG] * 0x1p896 : 0.0;
+#pragma unroll
+        for (int u = 0; u < UR; u++) {
+            const uint8_t* row = rec + u * rb;
+            const int4 wv = in ? *reinterpret_cast<const int4*>(row + 16 * t) : make_int4(0, 0, 0, 0);
+            int dd = -cr;
+#pragma unroll
+            for (int j = 0; j < 2; j++) {
+                const int sh = 4 * (j ^ r);
+                dd = __dp4a((int)(((uint32_t)wv.x >> sh) & 0x0f0f0f0fu), xv[j].x, dd);
+                dd = __dp4a((int)(((uint32_t)wv.y >> sh) & 0x0f0f0f0fu), xv[j].y, dd);
+                dd = __dp4a((int)(((uint32_t)wv.z >> sh) & 0x0f0f0f0fu), xv[j].z, dd);
+                dd = __dp4a((int)(((uint32_t)wv.w >> sh) & 0x0f0f0f0fu), xv[j].w, dd);
+            }
+#pragma unroll
+            for (int o = 1; o < CPG; o <<= 1) dd += __shfl_xor_sync(0xffffffffu, dd, o);
+            if (head) {
+                const float* sw = reinterpret_cast<const float*>(row + K / 2);
+                acc[u] = fma(i2d_exact(dd) * widen_f32_scaled(sw[t / CPG]), sx, acc[u]);
+            }
+        }
+    }
+}
+
 // Input quantization of the 64-byte-per-lane Q8_0 path (K % 64 == 0, GS 32,
 // 64 or 128), split around the dependency wait.  The input is taken in chunks
 // of 64 values, two per warp step: half-warp h of warp w takes chunk
@@ -845,18 +906,21 @@ struct Q8Smem {
     size_t xq, xsc, sxd, bars, total;
 };
 
+// sxd holds the input's double scales (generic Q8_0 path) or the Q4_0
+// chunk corrections (K/32 ints).
 __host__ __device__ inline Q8Smem q8_smem(int ns, uint32_t unit_bytes, int K, int gs) {
     Q8Smem m;
     const size_t ng = (size_t)(K / gs);
+    const size_t aux = ng * 8 > (size_t)(K / 32) * 4 ? ng * 8 : (size_t)(K / 32) * 4;
     m.xq = (size_t)Q8_WARPS * ns * unit_bytes;
     m.xsc = m.xq + (((size_t)K + 15) & ~size_t(15));
     m.sxd = m.xsc + ((ng * 4 + 15) & ~size_t(15));
-    m.bars = m.sxd + ng * 8;  // the double scales: generic path only
+    m.bars = m.sxd + ((aux + 7) & ~size_t(7));
     m.total = m.bars + 8 * (size_t)Q8_WARPS * ns;
     return m;
 }
 
-template <int MODE, int GS>
+template <int MODE, int GS, bool W4 = false>
 __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, const Q8Ring R) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int UNIT = (MODE == M_QKV || MODE == M_W13) ? 2 : 1;
@@ -896,7 +960,9 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
     const int8_t* eq = nullptr;
     const float* es = nullptr;
     if (a.emb) {
-        const uint8_t* rec = static_cast<const uint8_t*>(a.emb) + (size_t)token * a.ld;
+        // the embedding rows are Q8_0-layout records (holding 4-bit codes beside Q4_0 weights)
+        const size_t erb = W4 ? (size_t)K + (((size_t)(K / gs) * 4 + 15) & ~size_t(15)) : rb;
+        const uint8_t* rec = static_cast<const uint8_t*>(a.emb) + (size_t)token * erb;
         eq = reinterpret_cast<const int8_t*>(rec);
         es = reinterpret_cast<const float*>(rec + K);
     }
@@ -930,6 +996,23 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
         for (int g = threadIdx.x; g < K / gs; g += Q8_THREADS) sxd[g] = (double)xsc[g];
         __syncthreads();
     }
+    int* corr = reinterpret_cast<int*>(smem + lay.sxd);  // Q4_0: 8 * (sum of the input codes) per 32-chunk
+    if (W4) {
+        for (int t = threadIdx.x; t < K / 32; t += Q8_THREADS) {
+            const int4 c0 = *reinterpret_cast<const int4*>(xq + 32 * t);
+            const int4 c1 = *reinterpret_cast<const int4*>(xq + 32 * t + 16);
+            int sum = __dp4a(c0.x, 0x01010101, 0);
+            sum = __dp4a(c0.y, 0x01010101, sum);
+            sum = __dp4a(c0.z, 0x01010101, sum);
+            sum = __dp4a(c0.w, 0x01010101, sum);
+            sum = __dp4a(c1.x, 0x01010101, sum);
+            sum = __dp4a(c1.y, 0x01010101, sum);
+            sum = __dp4a(c1.z, 0x01010101, sum);
+            sum = __dp4a(c1.w, 0x01010101, sum);
+            corr[t] = 8 * sum;
+        }
+        __syncthreads();
+    }
 
     const int nchunk = K >> 4, cpg = gs >> 4, iters = (nchunk + 31) >> 5;
     unsigned long long best = 0ull;
@@ -942,7 +1025,9 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
         }
         const uint8_t* base = slots + (size_t)s * ub;
         double acc[UNIT];
-        if (GS != 0) {
+        if (W4) {
+            q4_rows_dot32<GS == 0 ? 32 : GS, UNIT>(base, rb, xq, xsc, corr, K, acc);
+        } else if (GS != 0) {
             q8_rows_dot64<GS == 0 ? 64 : GS, UNIT>(base, rb, xq, xsc, K, acc);
         } else {
 #pragma unroll
@@ -1076,6 +1161,41 @@ static __global__ void k_quantize_rows(const float* W, long long rows, int K, in
         uint8_t* rec = out + (size_t)r * rb;
         quantize_group_warp(W + (size_t)r * K + (size_t)g * gs, gs, reinterpret_cast<int8_t*>(rec) + g * gs,
                             reinterpret_cast<float*>(rec + K) + g);
+    }
+}
+
+// Re-lays an fp32 matrix [rows][K] as Q4_0: one warp per (row, group) with
+// the 4-bit rule (scale = max|x| / 7 in fp32, code = round(x / scale), half
+// away from zero, in [-7, 7]; a zero group gets scale 0, codes 0).  wide = 0:
+// packed records (q4_record_bytes: code + 8 in nibbles, chunk layout of
+// q4_rows_dot32); wide = 1: the Q8_0 record layout [K int8 codes | scales |
+// pad] holding the 4-bit codes (the embedding table, read one row at a time
+// by the Q8_0 input path).  gs is a multiple of 32.
+static __global__ void k_quantize_rows_q4(const float* W, long long rows, int K, int gs, uint8_t* out, size_t rb,
+                                          int wide) {
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    const int ng = K / gs, lane = threadIdx.x & 31;
+    const long long total = rows * ng;
+    for (long long t = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < total; t += warps) {
+        const long long r = t / ng;
+        const int g = (int)(t % ng);
+        const float* x = W + (size_t)r * K + (size_t)g * gs;
+        uint8_t* rec = out + (size_t)r * rb;
+        float m = 0.f;
+        for (int i = lane; i < gs; i += 32) m = fmaxf(m, fabsf(x[i]));
+        m = warp_max(m);
+        const float scale = m / 7.0f;
+        for (int i0 = 0; i0 < gs; i0 += 32) {
+            const int code = scale == 0.f ? 0 : (int)roundf(x[i0 + lane] / scale);
+            if (wide) {
+                reinterpret_cast<int8_t*>(rec)[g * gs + i0 + lane] = (int8_t)code;
+            } else {
+                const int hi = __shfl_down_sync(0xffffffffu, code, 16);
+                if (lane < 16)
+                    rec[(size_t)(g * gs + i0) / 2 + lane] = (uint8_t)((code + 8) | ((hi + 8) << 4));
+            }
+        }
+        if (lane == 0) reinterpret_cast<float*>(rec + (wide ? (size_t)K : (size_t)K / 2))[g] = scale;
     }
 }
 

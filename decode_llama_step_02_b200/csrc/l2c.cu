@@ -57,6 +57,9 @@ struct l2c_ctx {
     // Q8_0 weights
     int gs = 0;
     Q8Mat qE, qWqkv, qWo, qW13, qW2, qWcls;
+    // Q4_0 weights (packed records; the embedding as Q8_0-layout records of 4-bit codes)
+    int gs4 = 0;
+    Q8Mat q4E, q4Wqkv, q4Wo, q4W13, q4W2, q4Wcls;
     // state
     float *kc = nullptr, *vc = nullptr;
     float *x = nullptr, *q = nullptr, *att = nullptr, *hb = nullptr, *logits = nullptr;
@@ -76,8 +79,8 @@ struct l2c_ctx {
     int attn_occ_f32 = 1, attn_occ_f64 = 4;  // resident CTAs per SM of this shape's attention kernels
     int attn_min_chunk = 32;    // positions per attention chunk, at least
     int attn_nchunks_max = 1;   // chunks the partials buffer holds per (sequence, KV head)
-    // graphs: [q80][gen]
-    cudaGraphExec_t graph[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+    // graphs: [weight format: fp32, Q8_0, Q4_0][gen]
+    cudaGraphExec_t graph[3][2] = {{nullptr, nullptr}, {nullptr, nullptr}, {nullptr, nullptr}};
     // batched Q8_0 step: quantized activations of every sequence, one graph per batch size
     int8_t* bxq = nullptr;
     double* bxs = nullptr;
@@ -195,11 +198,14 @@ struct GemvShape {
 // Kernels of the step, in order within a layer.
 enum StepKernel : int { SK_QKV = 0, SK_ATTN = 1, SK_WO = 2, SK_W13 = 3, SK_W2 = 4, SK_CLS = 5 };
 
+// Weight formats of the single-sequence step.
+enum WeightFormat : int { WF_F32 = 0, WF_Q80 = 1, WF_Q40 = 2 };
+
 template <int MODE>
-static cudaError_t launch_gemv(l2c_ctx* h, bool q80, GemvArgs a, int unit) {
+static cudaError_t launch_gemv(l2c_ctx* h, int wf, GemvArgs a, int unit) {
     const int units = a.rows / unit;
-    a.late_trigger = (h->late_trigger >> (q80 ? 1 : 0)) & 1;
-    if (!q80) {
+    a.late_trigger = (h->late_trigger >> (wf != WF_F32 ? 1 : 0)) & 1;
+    if (wf == WF_F32) {
         int grid = h->sms * h->f32_ctas_per_sm;
         if (grid > units) grid = units;
         a.prefetch_bytes = h->pf_f32;
@@ -231,6 +237,11 @@ static cudaError_t launch_gemv(l2c_ctx* h, bool q80, GemvArgs a, int unit) {
     a.early = h->q8_early;
     a.prefetch_bytes = h->pf_q8;
     const dim3 g(grid), t(Q8_THREADS);
+    if (wf == WF_Q40) {  // gs 32, 64 or 128 (l2c_enable_q40)
+        if (a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64, true>, g, t, smem, a, R);
+        if (a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32, true>, g, t, smem, a, R);
+        return launch(h->cap, true, k_gemv_q8<MODE, 128, true>, g, t, smem, a, R);
+    }
     const bool k64 = a.K % 64 == 0;
     if (k64 && a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64>, g, t, smem, a, R);
     if (k64 && a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32>, g, t, smem, a, R);
@@ -262,6 +273,17 @@ static int set_smem_limits(l2c_ctx* h) {
     CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     L2C_Q8_ATTR(0) L2C_Q8_ATTR(32) L2C_Q8_ATTR(64) L2C_Q8_ATTR(128)
 #undef L2C_Q8_ATTR
+#define L2C_Q4_ATTR(GS_)                                                                                                \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_QKV, GS_, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID, GS_, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096)); \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_W13, GS_, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(max_carveout(k_gemv_q8<M_QKV, GS_, true>));                                                                      \
+    CK(max_carveout(k_gemv_q8<M_RESID, GS_, true>));                                                                    \
+    CK(max_carveout(k_gemv_q8<M_W13, GS_, true>));                                                                      \
+    CK(max_carveout(k_gemv_q8<M_CLS, GS_, true>));
+    L2C_Q4_ATTR(32) L2C_Q4_ATTR(64) L2C_Q4_ATTR(128)
+#undef L2C_Q4_ATTR
     {
         cudaError_t e = attn_set_smem_limits();
         if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "attention smem limit: %s", cudaGetErrorString(e));
@@ -355,7 +377,15 @@ static Kv8Args kv8_args(l2c_ctx* h, float* kc, float* vc) {
 }
 
 // Enqueues kernel `kind` of layer l (sequence seq) on stream s.
-static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, int l, int seq = 0) {
+static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, int wf, int l, int seq = 0) {
+    const bool q80 = wf != WF_F32;  // quantized weights (Q8_0 or Q4_0)
+    const bool w4 = wf == WF_Q40;
+    const Q8Mat& mE = w4 ? h->q4E : h->qE;
+    const Q8Mat& mQKV = w4 ? h->q4Wqkv : h->qWqkv;
+    const Q8Mat& mO = w4 ? h->q4Wo : h->qWo;
+    const Q8Mat& m13 = w4 ? h->q4W13 : h->qW13;
+    const Q8Mat& m2 = w4 ? h->q4W2 : h->qW2;
+    const Q8Mat& mCls = w4 ? h->q4Wcls : h->qWcls;
     g_pdl = h->pdl;
     const size_t d = h->d, kvd = h->kvd, hh = h->h, S = h->S;
     const size_t cache_off = (size_t)seq * h->L * S * kvd;
@@ -371,18 +401,18 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
     h->cap = s;  // launch_gemv enqueues on h->cap
     cudaError_t e = cudaSuccess;
     GemvArgs a = {};
-    a.gs = h->gs; a.tp = tp; a.err = h->err; a.vocab = h->V; a.seq_len = h->S; a.wait_ns = h->wait_ns;
+    a.gs = w4 ? h->gs4 : h->gs; a.tp = tp; a.err = h->err; a.vocab = h->V; a.seq_len = h->S; a.wait_ns = h->wait_ns;
     a.d = (int)d; a.kvd = (int)kvd; a.hs = h->hs;
     switch (kind) {
     case SK_QKV:  // RMSNorm + q/k/v + RoPE + cache write
         a.rows = (int)(d + 2 * kvd);
         a.K = (int)d;
-        if (q80) { a.W = h->qWqkv.p + (size_t)l * a.rows * h->qWqkv.rb; a.ld = h->qWqkv.rb; }
+        if (q80) { a.W = mQKV.p + (size_t)l * a.rows * mQKV.rb; a.ld = mQKV.rb; }
         else { a.W = h->Wqkv + (size_t)l * a.rows * d; a.ld = d; }
         a.in = x;
         a.norm_w = h->rms_att + (size_t)l * d;
         if (l == 0) {
-            a.emb = q80 ? (const void*)h->qE.p : (const void*)h->E;
+            a.emb = q80 ? (const void*)mE.p : (const void*)h->E;
             a.x_resid = x;
             a.amax = amax;
         }
@@ -391,7 +421,7 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
         a.vslot = vslot;
         a.freq = h->freq;
         if (l == 0 && seq == 0) a.stall = h->stall;
-        e = launch_gemv<M_QKV>(h, q80, a, 2);
+        e = launch_gemv<M_QKV>(h, wf, a, 2);
         break;
     case SK_ATTN:  // with the int8 KV cache the attention also stores the row at pos
         e = launch_attention(h, s, true, q80, q, kslot, vslot, (size_t)h->L * S * kvd, att, tp, 1, h->attn_part,
@@ -399,31 +429,31 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
         break;
     case SK_WO:  // wo + residual
         a.rows = (int)d; a.K = (int)d;
-        if (q80) { a.W = h->qWo.p + (size_t)l * d * h->qWo.rb; a.ld = h->qWo.rb; }
+        if (q80) { a.W = mO.p + (size_t)l * d * mO.rb; a.ld = mO.rb; }
         else { a.W = h->Wo + (size_t)l * d * d; a.ld = d; }
         a.in = att; a.out = x;
-        e = launch_gemv<M_RESID>(h, q80, a, 1);
+        e = launch_gemv<M_RESID>(h, wf, a, 1);
         break;
     case SK_W13:  // RMSNorm + W1/W3 + SwiGLU
         a.rows = (int)(2 * hh); a.K = (int)d;
-        if (q80) { a.W = h->qW13.p + (size_t)l * 2 * hh * h->qW13.rb; a.ld = h->qW13.rb; }
+        if (q80) { a.W = m13.p + (size_t)l * 2 * hh * m13.rb; a.ld = m13.rb; }
         else { a.W = h->W13 + (size_t)l * 2 * hh * d; a.ld = d; }
         a.in = x; a.norm_w = h->rms_ffn + (size_t)l * d; a.out = hb;
-        e = launch_gemv<M_W13>(h, q80, a, 2);
+        e = launch_gemv<M_W13>(h, wf, a, 2);
         break;
     case SK_W2:  // W2 + residual
         a.rows = (int)d; a.K = (int)hh;
-        if (q80) { a.W = h->qW2.p + (size_t)l * d * h->qW2.rb; a.ld = h->qW2.rb; }
+        if (q80) { a.W = m2.p + (size_t)l * d * m2.rb; a.ld = m2.rb; }
         else { a.W = h->W2 + (size_t)l * d * hh; a.ld = hh; }
         a.in = hb; a.out = x;
-        e = launch_gemv<M_RESID>(h, q80, a, 1);
+        e = launch_gemv<M_RESID>(h, wf, a, 1);
         break;
     default:  // final RMSNorm + classifier + argmax
         a.rows = h->V; a.K = (int)d;
-        if (q80) { a.W = h->qWcls.p; a.ld = h->qWcls.rb; }
+        if (q80) { a.W = mCls.p; a.ld = mCls.rb; }
         else { a.W = h->Wcls; a.ld = d; }
         a.in = x; a.norm_w = h->rms_final; a.out = h->logits + (size_t)seq * h->V; a.amax = amax;
-        e = launch_gemv<M_CLS>(h, q80, a, 1);
+        e = launch_gemv<M_CLS>(h, wf, a, 1);
         break;
     }
     h->cap = saved;
@@ -432,12 +462,12 @@ static int launch_step_kernel(l2c_ctx* h, cudaStream_t s, int kind, bool q80, in
 }
 
 // Enqueues one decode step of sequence 0 on h->cap (being captured).
-static int enqueue_step(l2c_ctx* h, bool q80) {
+static int enqueue_step(l2c_ctx* h, int wf) {
     int rc;
     for (int l = 0; l < h->L; l++)
         for (int k = SK_QKV; k <= SK_W2; k++)
-            if ((rc = launch_step_kernel(h, h->cap, k, q80, l)) != L2C_OK) return rc;
-    return launch_step_kernel(h, h->cap, SK_CLS, q80, 0);
+            if ((rc = launch_step_kernel(h, h->cap, k, wf, l)) != L2C_OK) return rc;
+    return launch_step_kernel(h, h->cap, SK_CLS, wf, 0);
 }
 
 // ------------------------------------------------------------- batched step --
@@ -641,10 +671,10 @@ static int build_batch_graph(l2c_ctx* h, int B, bool q80) {
     return L2C_OK;
 }
 
-static int build_graph(l2c_ctx* h, bool q80, bool gen) {
-    if (h->graph[q80][gen]) return L2C_OK;
+static int build_graph(l2c_ctx* h, int wf, bool gen) {
+    if (h->graph[wf][gen]) return L2C_OK;
     CK(cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal));
-    int rc = enqueue_step(h, q80);
+    int rc = enqueue_step(h, wf);
     if (rc == L2C_OK && gen) {
         cudaError_t e = launch(h->cap, false, k_advance, dim3(1), dim3(1), 0, h->tp,
                                (const unsigned long long*)h->amax, h->gen_tokens, h->gen_count);
@@ -657,7 +687,7 @@ static int build_graph(l2c_ctx* h, bool q80, bool gen) {
         return rc;
     }
     if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "capture failed: %s", cudaGetErrorString(e));
-    e = cudaGraphInstantiate(&h->graph[q80][gen], g, 0);
+    e = cudaGraphInstantiate(&h->graph[wf][gen], g, 0);
     cudaGraphDestroy(g);
     if (e != cudaSuccess) return fail(h, L2C_E_CUDA, "graph instantiate: %s", cudaGetErrorString(e));
     return L2C_OK;
@@ -895,23 +925,69 @@ extern "C" int l2c_enable_q80(l2c_ctx* h, int gs) {
     return L2C_OK;
 }
 
+// ---------------------------------------------------------------- Q4_0 set --
+
+// Q4_0 records of an fp32 matrix [rows][K]: packed (the GEMV weights) or, for
+// the embedding table, the Q8_0 record layout holding the 4-bit codes.
+static int make_q4(l2c_ctx* h, Q8Mat& m, const float* W, size_t rows, int K, bool wide) {
+    m.rb = wide ? record_bytes(K, h->gs4) : q4_record_bytes(K, h->gs4);
+    int rc = dalloc(h, (void**)&m.p, rows * m.rb);
+    if (rc) return rc;
+    CK(cudaMemsetAsync(m.p, 0, rows * m.rb, h->stream));
+    long long groups = (long long)rows * (K / h->gs4);
+    long long blocks = (groups + 7) / 8;
+    int grid = (int)(blocks < 65535LL * 16 ? blocks : 65535LL * 16);
+    k_quantize_rows_q4<<<grid, 256, 0, h->stream>>>(W, (long long)rows, K, h->gs4, m.p, m.rb, wide ? 1 : 0);
+    CK(cudaGetLastError());
+    return L2C_OK;
+}
+
+extern "C" int l2c_enable_q40(l2c_ctx* h, int gs) {
+    if (!h) return L2C_E_ARG;
+    if (h->gs4) return h->gs4 == gs ? L2C_OK : fail(h, L2C_E_STATE, "Q4_0 already enabled with gs=%d", h->gs4);
+    if ((gs != 32 && gs != 64 && gs != 128) || h->d % gs || h->h % gs)
+        return fail(h, L2C_E_ARG, "Q4_0: gs=%d must be 32, 64 or 128 and divide dim and hidden_dim", gs);
+    h->gs4 = gs;
+    const size_t d = h->d, hh = h->h, L = h->L, kvd = h->kvd, V = h->V;
+    int rc;
+    if ((rc = make_q4(h, h->q4E, h->E, V, (int)d, true)) ||
+        (rc = make_q4(h, h->q4Wqkv, h->Wqkv, L * (d + 2 * kvd), (int)d, false)) ||
+        (rc = make_q4(h, h->q4Wo, h->Wo, L * d, (int)d, false)) ||
+        (rc = make_q4(h, h->q4W13, h->W13, L * 2 * hh, (int)d, false)) ||
+        (rc = make_q4(h, h->q4W2, h->W2, L * d, (int)hh, false)) ||
+        (rc = make_q4(h, h->q4Wcls, h->Wcls, V, (int)d, false))) {
+        h->gs4 = 0;
+        return rc;
+    }
+    CK(cudaStreamSynchronize(h->stream));
+    return L2C_OK;
+}
+
 // ------------------------------------------------------------------ forward --
 
-static const float* forward_impl(l2c_ctx* h, int token, int pos, bool q80) {
+// Whether the weights of format wf are made, and the int8 KV cache (which
+// serves the quantized steps) allows the step; 0 if so, else the failure code.
+static int step_ready(l2c_ctx* h, int wf) {
+    if (wf == WF_Q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
+    if (wf == WF_Q40 && !h->gs4) return fail(h, L2C_E_STATE, "Q4_0 weights not made (l2c_enable_q40)");
+    if (wf == WF_F32 && h->kv8) return fail(h, L2C_E_STATE, "the int8 KV cache serves the quantized steps");
+    return L2C_OK;
+}
+
+static const float* forward_impl(l2c_ctx* h, int token, int pos, int wf) {
     if (!h) return nullptr;
     if (token < 0 || token >= h->V) { fail(h, L2C_E_ARG, "token %d not in [0,%d)", token, h->V); return nullptr; }
     if (pos < 0 || pos >= h->S) { fail(h, L2C_E_ARG, "pos %d not in [0,%d)", pos, h->S); return nullptr; }
-    if (q80 && !h->gs) { fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)"); return nullptr; }
-    if (!q80 && h->kv8) { fail(h, L2C_E_STATE, "the int8 KV cache serves the Q8_0 step"); return nullptr; }
-    if (h->graphs && build_graph(h, q80, false) != L2C_OK) return nullptr;
+    if (step_ready(h, wf) != L2C_OK) return nullptr;
+    if (h->graphs && build_graph(h, wf, false) != L2C_OK) return nullptr;
     k_set_tp<<<1, 1, 0, h->stream>>>(h->tp, token, pos);
     cudaError_t e = cudaSuccess;
     if (h->graphs) {
-        e = cudaGraphLaunch(h->graph[q80][0], h->stream);
+        e = cudaGraphLaunch(h->graph[wf][0], h->stream);
     } else {
         cudaStream_t saved = h->cap;
         h->cap = h->stream;
-        int rc = enqueue_step(h, q80);
+        int rc = enqueue_step(h, wf);
         h->cap = saved;
         if (rc != L2C_OK) return nullptr;
     }
@@ -919,21 +995,23 @@ static const float* forward_impl(l2c_ctx* h, int token, int pos, bool q80) {
     return h->logits;
 }
 
-extern "C" const float* l2c_forward(l2c_ctx* h, int token, int pos) { return forward_impl(h, token, pos, false); }
-extern "C" const float* l2c_forward_q80(l2c_ctx* h, int token, int pos) { return forward_impl(h, token, pos, true); }
+extern "C" const float* l2c_forward(l2c_ctx* h, int token, int pos) { return forward_impl(h, token, pos, WF_F32); }
+extern "C" const float* l2c_forward_q80(l2c_ctx* h, int token, int pos) { return forward_impl(h, token, pos, WF_Q80); }
+extern "C" const float* l2c_forward_q40(l2c_ctx* h, int token, int pos) { return forward_impl(h, token, pos, WF_Q40); }
 
 extern "C" int l2c_generate(l2c_ctx* h, int token0, int pos0, int steps, int q80, int32_t* tokens_out) {
     if (!h || !tokens_out || steps < 0) return L2C_E_ARG;
+    if (q80 < WF_F32 || q80 > WF_Q40) return fail(h, L2C_E_ARG, "generate: weight format %d not in {0,1,2}", q80);
     if (token0 < 0 || token0 >= h->V) return fail(h, L2C_E_ARG, "token %d not in [0,%d)", token0, h->V);
     if (pos0 < 0 || pos0 + steps > h->S) return fail(h, L2C_E_ARG, "pos0 + steps exceeds seq_len");
-    if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
-    if (!q80 && h->kv8) return fail(h, L2C_E_STATE, "the int8 KV cache serves the Q8_0 step");
+    int rc = step_ready(h, q80);
+    if (rc) return rc;
     if (steps == 0) return L2C_OK;
-    int rc = build_graph(h, q80 != 0, true);
+    rc = build_graph(h, q80, true);
     if (rc) return rc;
     k_set_tp<<<1, 1, 0, h->stream>>>(h->tp, token0, pos0);
     CK(cudaMemsetAsync(h->gen_count, 0, 4, h->stream));
-    for (int t = 0; t < steps; t++) CK(cudaGraphLaunch(h->graph[q80 != 0][1], h->stream));
+    for (int t = 0; t < steps; t++) CK(cudaGraphLaunch(h->graph[q80][1], h->stream));
     CK(cudaMemcpyAsync(tokens_out, h->gen_tokens, (size_t)steps * 4, cudaMemcpyDeviceToHost, h->stream));
     return l2c_sync(h);
 }
@@ -942,6 +1020,7 @@ extern "C" int l2c_forward_batch(l2c_ctx* h, int B, const int32_t* tokens, const
                                  float* logits_out) {
     if (!h || !tokens || !pos || !logits_out || B < 1 || B > h->max_batch)
         return fail(h, L2C_E_ARG, "forward_batch: need 1 <= B <= max_batch and non-null arrays");
+    if (q80 < 0 || q80 > 1) return fail(h, L2C_E_ARG, "forward_batch: q80 must be 0 or 1 (Q4_0 serves the single-sequence step)");
     if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
     if (B > BMAX) return fail(h, L2C_E_ARG, "forward_batch: the batched step takes at most %d sequences", BMAX);
     if (h->kv8) return fail(h, L2C_E_STATE, "forward_batch: not with the int8 KV cache (l2c_enable_kv8)");
@@ -983,6 +1062,7 @@ extern "C" int l2c_prefill(l2c_ctx* h, int seq, int n, const int32_t* tokens, in
     if (is_device_ptr(tokens)) return fail(h, L2C_E_ARG, "prefill: tokens must be host memory");
     for (int i = 0; i < n; i++)
         if (tokens[i] < 0 || tokens[i] >= h->V) return fail(h, L2C_E_ARG, "token[%d]=%d out of range", i, tokens[i]);
+    if (q80 < 0 || q80 > 1) return fail(h, L2C_E_ARG, "prefill: q80 must be 0 or 1 (Q4_0 serves the single-sequence step)");
     if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
     if (h->kv8) return fail(h, L2C_E_STATE, "prefill: not with the int8 KV cache (l2c_enable_kv8)");
     int rc;
@@ -1029,15 +1109,17 @@ extern "C" int l2c_attention(l2c_ctx* h, const float* q, const float* k, const f
 }
 
 extern "C" int l2c_time_kernel(l2c_ctx* h, int kind, int q80, int iters, float* avg_ms) {
-    if (!h || kind < SK_QKV || kind > SK_CLS || iters < 1 || !avg_ms) return fail(h, L2C_E_ARG, "time_kernel: bad arguments");
-    if (q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
+    if (!h || kind < SK_QKV || kind > SK_CLS || iters < 1 || !avg_ms || q80 < WF_F32 || q80 > WF_Q40)
+        return fail(h, L2C_E_ARG, "time_kernel: bad arguments");
+    if (q80 == WF_Q80 && !h->gs) return fail(h, L2C_E_STATE, "Q8_0 weights not made (l2c_enable_q80)");
+    if (q80 == WF_Q40 && !h->gs4) return fail(h, L2C_E_STATE, "Q4_0 weights not made (l2c_enable_q40)");
     cudaEvent_t e0, e1;
     CK(cudaEventCreate(&e0));
     CK(cudaEventCreate(&e1));
     int rc = L2C_OK;
     cudaError_t er = cudaEventRecord(e0, h->stream);
     for (int i = 0; i < iters && rc == L2C_OK && er == cudaSuccess; i++) {
-        rc = launch_step_kernel(h, h->stream, kind, q80 != 0, kind == SK_CLS ? 0 : i % h->L);
+        rc = launch_step_kernel(h, h->stream, kind, q80, kind == SK_CLS ? 0 : i % h->L);
     }
     if (er == cudaSuccess) er = cudaEventRecord(e1, h->stream);
     if (er == cudaSuccess) er = cudaEventSynchronize(e1);
@@ -1159,7 +1241,7 @@ extern "C" int l2c_enable_kv8(l2c_ctx* h, int on) {
         }
     }
     // the step graphs were captured for the other cache
-    for (int a = 0; a < 2; a++)
+    for (int a = 0; a < 3; a++)
         for (int b = 0; b < 2; b++)
             if (h->graph[a][b]) {
                 cudaGraphExecDestroy(h->graph[a][b]);

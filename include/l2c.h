@@ -104,6 +104,20 @@ L2C_API int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_flo
 L2C_API int l2c_enable_q80(l2c_ctx* h, int gs);
 
 /*
+ * l2c_enable_q40 - makes a Q4_0 weight set, beside the fp32 and Q8_0 ones.
+ * "技术深度解析" (ainews.cool llama2.c article), 整数量化路径: runq.c with 4-bit
+ * integer groups; the page gives no rule, so the reading is quantize() of
+ * [port] §1 with 4-bit codes: per group of gs values along a row, scale =
+ * max|x| / 7 (fp32) and code = round(x / scale), in [-7, 7].  The same
+ * tensors as l2c_enable_q80 (every matvec weight and the embedding table);
+ * the GEMVs stream two codes per byte plus one fp32 scale per group.  gs must
+ * be 32, 64 or 128 and divide dim and hidden_dim (else L2C_E_ARG).  Calling
+ * it again with the same gs is a no-op; another gs gives L2C_E_STATE.
+ * L2C_E_OOM if the device memory runs out.  Blocks.
+ */
+L2C_API int l2c_enable_q40(l2c_ctx* h, int gs);
+
+/*
  * l2c_forward - forward(transformer, token, pos) of run.c ([port]
  * 智能家居控制案例): one decode step of sequence 0 in fp32.  Embedding row,
  * then per layer RMSNorm, q/k/v matvecs, RoPE as cos/sin(pos*freq) computed
@@ -122,6 +136,12 @@ L2C_API const float* l2c_forward(l2c_ctx* h, int token, int pos);
  * sum over groups of the exact int32 group dot times both scales.  NULL also
  * when l2c_enable_q80 has not been called. */
 L2C_API const float* l2c_forward_q80(l2c_ctx* h, int token, int pos);
+
+/* l2c_forward_q40 - the same step through the Q4_0 weights: every matvec input
+ * is quantized to Q8_0 at the Q4_0 group size, and each output is the sum
+ * over groups of the exact int32 dot of the 4-bit and 8-bit codes times both
+ * scales.  NULL also when l2c_enable_q40 has not been called. */
+L2C_API const float* l2c_forward_q40(l2c_ctx* h, int token, int pos);
 
 /*
  * l2c_argmax - sample_argmax() of [port] 智能家居控制案例: the index of the
@@ -152,7 +172,8 @@ L2C_API int l2c_sample(l2c_ctx* h, const float* logits_dev, int n, float tempera
  * l2c_generate - greedy decoding with the token fed back on the device:
  * tok_0 = token0; for t = 0..steps-1: logits = forward(tok_t, pos0 + t),
  * tok_{t+1} = argmax(logits).  tokens_out_host[t] = tok_{t+1}.
- * q80 selects the Q8_0 path.  pos0 + steps must not exceed seq_len.
+ * q80 picks the weights: 0 fp32, 1 Q8_0, 2 Q4_0 (other values: L2C_E_ARG;
+ * weights not made: L2C_E_STATE).  pos0 + steps must not exceed seq_len.
  * Blocks until the tokens are on the host.
  */
 L2C_API int l2c_generate(l2c_ctx* h, int token0, int pos0, int steps, int q80, int32_t* tokens_out_host);
@@ -163,7 +184,8 @@ L2C_API int l2c_generate(l2c_ctx* h, int token0, int pos0, int steps, int q80, i
  * Each matvec of the step runs as one GEMM over the B sequences (Q8_0: int8
  * tensor cores, exact int32 group dots, double group sums; fp32: fp32 FMAs).
  * tokens, pos: host or device int32 [B]; B <= max_batch and B <= 32.
- * logits_out_dev: device [B][vocab_size].  q80 selects the Q8_0 path.
+ * logits_out_dev: device [B][vocab_size].  q80 = 1 selects the Q8_0 path
+ * (0 fp32; other values, Q4_0 included, give L2C_E_ARG).
  */
 L2C_API int l2c_forward_batch(l2c_ctx* h, int B, const int32_t* tokens, const int32_t* pos, int q80,
                       float* logits_out_dev);
@@ -181,7 +203,8 @@ L2C_API int l2c_forward_batch(l2c_ctx* h, int B, const int32_t* tokens, const in
  * tokens: host int32 [n]; 0 <= seq < max_batch; n >= 1; pos0 + n <= seq_len.
  * logits_last_dev: device [vocab_size] receives the logits of the last token
  * (NULL: not written).  q80 = 1 needs l2c_enable_q80 with gs a multiple of 32
- * that the batched GEMM tiles (else L2C_E_ARG).  The first call allocates the
+ * that the batched GEMM tiles (else L2C_E_ARG); q80 is 0 or 1 (Q4_0 serves
+ * the single-sequence step only: L2C_E_ARG).  The first call allocates the
  * chunk activations in the handle.  Blocks until the cache is written.
  */
 L2C_API int l2c_prefill(l2c_ctx* h, int seq, int n, const int32_t* tokens, int pos0, int q80, float* logits_last_dev);
@@ -191,8 +214,8 @@ L2C_API int l2c_prefill(l2c_ctx* h, int seq, int n, const int32_t* tokens, int p
  * pages give no int8 KV cache; the reading: every K and V row, when it is
  * stored, becomes Q8_0 groups of head_size values (one per KV head) with the
  * quantize() rule of [port] §1, and attention reads code * scale (one fp32
- * multiply).  It serves the Q8_0 step (l2c_forward_q80, l2c_generate with
- * q80 = 1), whose attention then streams the codes and scales (a quarter of
+ * multiply).  It serves the quantized steps (l2c_forward_q80, l2c_forward_q40,
+ * l2c_generate with q80 = 1 or 2), whose attention then streams the codes and scales (a quarter of
  * the bytes); the fp32 cache rows are overwritten with the same code * scale
  * values (l2c_kv_read returns those).  Enabling it quantizes every row
  * already in the cache (all sequences); l2c_kv_load quantizes the rows it
@@ -310,8 +333,8 @@ L2C_API int l2c_attention_noalloc(const float* q_dev, const float* k_dev, const 
                                   void* cuda_stream);
 
 /*
- * l2c_time_kernel - measurement hook: runs kernel `kind` of the fp32 (q80 = 0)
- * or Q8_0 step alone, iters times back to back on the handle's stream, and
+ * l2c_time_kernel - measurement hook: runs kernel `kind` of the fp32 (q80 = 0),
+ * Q8_0 (1) or Q4_0 (2) step alone, iters times back to back on the handle's stream, and
  * stores the average time per launch in ms (two CUDA events around the
  * loop).  Launch i uses layer i % n_layers, so consecutive launches stream
  * different weights.  kind: 0 = RMSNorm+QKV+RoPE, 1 = attention, 2 = wo,

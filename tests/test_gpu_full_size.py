@@ -1,6 +1,6 @@
 """Full-size workloads in the launch configuration bench.py times, on outputs the
-oracle computes one step at a time: the 7B shape (fp32 and Q8_0 GS=64, a cache
-prefilled to 512 positions) and the GQA 7B-width batch of 32 sequences (Q8_0
+oracle computes one step at a time: the 7B shape (fp32, Q8_0 GS=64 and Q4_0
+GS=64, a cache prefilled to 2048 positions) and the GQA 7B-width batch of 32 sequences (Q8_0
 GS=64, ragged positions, 4 sequences sampled for the oracle)."""
 import numpy as np
 import pytest
@@ -48,6 +48,14 @@ def test_7b_step_matches_oracle():
             assert err <= (TOL_Q80 if q80 else TOL_F32), (q80, P, err)
             if q80:
                 assert err <= 1e-5, (P, err)
+    # the Q4_0 weights (GS=64) on the same cache
+    dec.enable_q40(64)
+    orc.enable_q40(64)
+    for P in (0, 512, P_MAX):
+        got = dec.forward(1, P, q40=True).cpu().numpy()
+        ref = orc.forward(1, P, q40=True)
+        err = rel_err(got, ref)
+        assert err <= 1e-5, ("q40", P, err)
     # the int8 KV cache on both sides: every row in the cache is quantized, then the
     # Q8_0 steps (each writes its slot through the int8 store) keep reproducing the
     # oracle's codes (1e-5)
