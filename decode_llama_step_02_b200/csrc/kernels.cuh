@@ -686,9 +686,12 @@ __device__ __forceinline__ void q8_rows_dot64(const uint8_t* rec, size_t rb, con
 }
 
 // Q4_0 row records: [K/2 bytes of 4-bit codes | K/GS fp32 scales | pad to
-// 16 B].  The values 32t..32t+31 (chunk t) sit in the 16 bytes at 16t: byte
-// b holds value 32t+b in its low nibble and 32t+16+b in its high nibble, each
-// as code + 8 (1..15 for codes in [-7, 7]).
+// 16 B], each code stored as code + 8 (1..15 for codes in [-7, 7]).  Two
+// layouts of the code bytes: with K % 64 == 0 the values 64t..64t+63 (chunk
+// t) sit in the 32 bytes at 32t, byte b holding value 64t+b in its low
+// nibble and 64t+32+b in its high one (q4_rows_dot64); otherwise (K an odd
+// multiple of 32, GS = 32) the values 32t..32t+31 sit in the 16 bytes at 16t,
+// byte b holding 32t+b low and 32t+16+b high (q4_rows_dot32).
 __host__ __device__ inline size_t q4_record_bytes(int K, int gs) {
     return (size_t)K / 2 + (((size_t)(K / gs) * 4 + 15) & ~size_t(15));
 }
@@ -741,6 +744,89 @@ __device__ __forceinline__ void q4_rows_dot32(const uint8_t* rec, size_t rb, con
             if (head) {
                 const float* sw = reinterpret_cast<const float*>(row + K / 2);
                 acc[u] = fma(i2d_exact(dd) * widen_f32_scaled(sw[t / CPG]), sx, acc[u]);
+            }
+        }
+    }
+}
+
+// d + sum of the four byte products of a (unsigned bytes) and b (signed bytes).
+__device__ __forceinline__ int dp4a_us(uint32_t a, int b, int d) {
+    int r;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(d));
+    return r;
+}
+
+// UR Q4_0 rows in the 64-value chunk layout against the Q8_0 input codes xq.
+// Lane chunk t: two 16-byte loads of a row (halves h) and four of the input
+// (quarters f).  Quarter f pairs with the low (f < 2) or high nibbles of half
+// f & 1.  The loads are rotated so that the eight lanes of a quarter-warp
+// touch distinct 16-byte bank groups: with rot = bit 2 of the lane | (bit 1 of
+// the lane) << 1, input slot j holds quarter j ^ rot and row register jj half
+// jj ^ (rot & 1), so slot j pairs with register j & 1 and a nibble picked by
+// a per-lane mask.  The high nibbles are taken in place (byte = 16 * code),
+// so one AND per word: sum over slots 0-1 and 2-3 with unsigned-by-signed
+// dp4a, then lo + (hi >> 4) - corr per group (corr = 8 * the input codes'
+// sum over 32 values).  Group scaling as in q8_rows_dot64.  Requires K % 64
+// == 0, GS in {32, 64, 128}.
+template <int GS, int UR>
+__device__ __forceinline__ void q4_rows_dot64(const uint8_t* rec, size_t rb, const int8_t* xq, const float* xs,
+                                              const int* corr, int K, double (&acc)[UR]) {
+    const int lane = threadIdx.x & 31;
+    const int n64 = K >> 6;
+    const int rot = ((lane >> 2) & 1) | (lane & 2);
+    const uint32_t mA = (rot >> 1) ? 0xf0f0f0f0u : 0x0f0f0f0fu;  // nibble of slots 0, 1
+    const uint32_t mB = ~mA;                                      // nibble of slots 2, 3
+#pragma unroll
+    for (int u = 0; u < UR; u++) acc[u] = 0.0;
+#pragma unroll 2
+    for (int t0 = 0; t0 < n64; t0 += 32) {
+        const int t = t0 + lane;
+        const bool in = t < n64;
+        int4 xv[4];
+#pragma unroll
+        for (int j = 0; j < 4; j++)
+            xv[j] = in ? *reinterpret_cast<const int4*>(xq + 64 * t + 16 * (j ^ rot)) : make_int4(0, 0, 0, 0);
+        const int2 cr = in ? *reinterpret_cast<const int2*>(corr + 2 * t) : make_int2(0, 0);
+        double sx0 = 0.0, sx1 = 0.0;
+        if (in) {
+            if (GS == 64) sx0 = (double)xs[t] * 0x1p896;
+            else if (GS == 32) { sx0 = (double)xs[2 * t] * 0x1p896; sx1 = (double)xs[2 * t + 1] * 0x1p896; }
+            else sx0 = (double)xs[t >> 1] * 0x1p896;
+        }
+#pragma unroll
+        for (int u = 0; u < UR; u++) {
+            const uint8_t* row = rec + u * rb;
+            int4 wv[2];
+#pragma unroll
+            for (int jj = 0; jj < 2; jj++)
+                wv[jj] = in ? *reinterpret_cast<const int4*>(row + 32 * t + 16 * (jj ^ (rot & 1)))
+                            : make_int4(0, 0, 0, 0);
+            int sA = 0, sB = 0;
+#pragma unroll
+            for (int j = 0; j < 2; j++) {
+                const int4 w = wv[j];
+                sA = dp4a_us((uint32_t)w.x & mA, xv[j].x, sA);
+                sA = dp4a_us((uint32_t)w.y & mA, xv[j].y, sA);
+                sA = dp4a_us((uint32_t)w.z & mA, xv[j].z, sA);
+                sA = dp4a_us((uint32_t)w.w & mA, xv[j].w, sA);
+                sB = dp4a_us((uint32_t)w.x & mB, xv[j + 2].x, sB);
+                sB = dp4a_us((uint32_t)w.y & mB, xv[j + 2].y, sB);
+                sB = dp4a_us((uint32_t)w.z & mB, xv[j + 2].z, sB);
+                sB = dp4a_us((uint32_t)w.w & mB, xv[j + 2].w, sB);
+            }
+            const int lo = (rot >> 1) ? sB : sA;         // quarters 0, 1: values 64t..64t+31
+            const int hi = ((rot >> 1) ? sA : sB) >> 4;  // quarters 2, 3 (16 * code, exact shift)
+            const float* sw = reinterpret_cast<const float*>(row + K / 2);
+            if (GS == 32) {
+                if (in) {
+                    acc[u] = fma(i2d_exact(lo - cr.x) * widen_f32_scaled(sw[2 * t]), sx0, acc[u]);
+                    acc[u] = fma(i2d_exact(hi - cr.y) * widen_f32_scaled(sw[2 * t + 1]), sx1, acc[u]);
+                }
+            } else {
+                int dd = lo + hi - (cr.x + cr.y);
+                if (GS == 128) dd += __shfl_xor_sync(0xffffffffu, dd, 1);
+                if (in && (GS == 64 || (t & 1) == 0))
+                    acc[u] = fma(i2d_exact(dd) * widen_f32_scaled(sw[GS == 64 ? t : (t >> 1)]), sx0, acc[u]);
             }
         }
     }
@@ -920,7 +1006,7 @@ __host__ __device__ inline Q8Smem q8_smem(int ns, uint32_t unit_bytes, int K, in
     return m;
 }
 
-template <int MODE, int GS, bool W4 = false>
+template <int MODE, int GS, int W4 = 0>
 __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, const Q8Ring R) {
     extern __shared__ __align__(128) uint8_t smem[];
     constexpr int UNIT = (MODE == M_QKV || MODE == M_W13) ? 2 : 1;
@@ -1025,7 +1111,9 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
         }
         const uint8_t* base = slots + (size_t)s * ub;
         double acc[UNIT];
-        if (W4) {
+        if (W4 == 2) {
+            q4_rows_dot64<GS == 0 ? 64 : GS, UNIT>(base, rb, xq, xsc, corr, K, acc);
+        } else if (W4 == 1) {
             q4_rows_dot32<GS == 0 ? 32 : GS, UNIT>(base, rb, xq, xsc, corr, K, acc);
         } else if (GS != 0) {
             q8_rows_dot64<GS == 0 ? 64 : GS, UNIT>(base, rb, xq, xsc, K, acc);
@@ -1164,38 +1252,57 @@ static __global__ void k_quantize_rows(const float* W, long long rows, int K, in
     }
 }
 
-// Re-lays an fp32 matrix [rows][K] as Q4_0: one warp per (row, group) with
-// the 4-bit rule (scale = max|x| / 7 in fp32, code = round(x / scale), half
-// away from zero, in [-7, 7]; a zero group gets scale 0, codes 0).  wide = 0:
-// packed records (q4_record_bytes: code + 8 in nibbles, chunk layout of
-// q4_rows_dot32); wide = 1: the Q8_0 record layout [K int8 codes | scales |
-// pad] holding the 4-bit codes (the embedding table, read one row at a time
-// by the Q8_0 input path).  gs is a multiple of 32.
+// Re-lays an fp32 matrix [rows][K] as Q4_0 with the 4-bit rule (scale =
+// max|x| / 7 in fp32, code = round(x / scale), half away from zero, in
+// [-7, 7]; a zero group gets scale 0, codes 0).  mode 0: packed records in the
+// 32-value chunk layout (gs a multiple of 32); mode 2: packed records in the
+// 64-value chunk layout (K % 64 == 0); mode 1: the Q8_0 record layout [K int8
+// codes | scales | pad] holding the 4-bit codes (the embedding table, read one
+// row at a time by the Q8_0 input path).  One warp per task of `span` values
+// of a row (whole groups and whole chunks): lane l takes the values
+// i0 + l and i0 + half + l of each step i0 (half = 16 or 32 for the chunk
+// layouts), which share one byte of a packed record.
 static __global__ void k_quantize_rows_q4(const float* W, long long rows, int K, int gs, uint8_t* out, size_t rb,
-                                          int wide) {
+                                          int mode) {
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
-    const int ng = K / gs, lane = threadIdx.x & 31;
-    const long long total = rows * ng;
+    const int lane = threadIdx.x & 31;
+    const int span = mode == 2 && gs < 64 ? 64 : gs;  // 64: two groups of 32 share each byte
+    const int tasks = K / span;
+    const long long total = rows * tasks;
     for (long long t = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < total; t += warps) {
-        const long long r = t / ng;
-        const int g = (int)(t % ng);
-        const float* x = W + (size_t)r * K + (size_t)g * gs;
+        const long long r = t / tasks;
+        const int base = (int)(t % tasks) * span;
+        const float* x = W + (size_t)r * K + base;
         uint8_t* rec = out + (size_t)r * rb;
-        float m = 0.f;
-        for (int i = lane; i < gs; i += 32) m = fmaxf(m, fabsf(x[i]));
-        m = warp_max(m);
-        const float scale = m / 7.0f;
-        for (int i0 = 0; i0 < gs; i0 += 32) {
-            const int code = scale == 0.f ? 0 : (int)roundf(x[i0 + lane] / scale);
-            if (wide) {
-                reinterpret_cast<int8_t*>(rec)[g * gs + i0 + lane] = (int8_t)code;
-            } else {
-                const int hi = __shfl_down_sync(0xffffffffu, code, 16);
-                if (lane < 16)
-                    rec[(size_t)(g * gs + i0) / 2 + lane] = (uint8_t)((code + 8) | ((hi + 8) << 4));
+        float* sc = reinterpret_cast<float*>(rec + (mode == 1 ? (size_t)K : (size_t)K / 2));
+        // the scales of the task's groups (one, or two of 32 values)
+        float m0 = 0.f, m1 = 0.f;
+        for (int i = lane; i < span; i += 32) {
+            if (span > gs && i >= gs) m1 = fmaxf(m1, fabsf(x[i]));
+            else m0 = fmaxf(m0, fabsf(x[i]));
+        }
+        m0 = warp_max(m0);
+        m1 = warp_max(m1);
+        const float s0 = m0 / 7.0f, s1 = m1 / 7.0f;
+        auto code = [&](int i) {
+            const float sc_i = (span > gs && i >= gs) ? s1 : s0;
+            return sc_i == 0.f ? 0 : (int)roundf(x[i] / sc_i);
+        };
+        if (mode == 1) {
+            for (int i = lane; i < span; i += 32) reinterpret_cast<int8_t*>(rec)[base + i] = (int8_t)code(i);
+        } else {
+            const int half = mode == 2 ? 32 : 16;
+            for (int i0 = 0; i0 < span; i0 += 2 * half) {
+                // lane l < half writes byte (base + i0) / 2 + l: value i0 + l low, i0 + half + l high
+                const int lo = code(i0 + lane);
+                const int hi = mode == 2 ? code(i0 + 32 + lane) : __shfl_down_sync(0xffffffffu, lo, 16);
+                if (lane < half) rec[(size_t)(base + i0) / 2 + lane] = (uint8_t)((lo + 8) | ((hi + 8) << 4));
             }
         }
-        if (lane == 0) reinterpret_cast<float*>(rec + (wide ? (size_t)K : (size_t)K / 2))[g] = scale;
+        if (lane == 0) {
+            sc[base / gs] = s0;
+            if (span > gs) sc[base / gs + 1] = s1;
+        }
     }
 }
 

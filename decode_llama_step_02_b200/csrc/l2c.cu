@@ -237,10 +237,11 @@ static cudaError_t launch_gemv(l2c_ctx* h, int wf, GemvArgs a, int unit) {
     a.early = h->q8_early;
     a.prefetch_bytes = h->pf_q8;
     const dim3 g(grid), t(Q8_THREADS);
-    if (wf == WF_Q40) {  // gs 32, 64 or 128 (l2c_enable_q40)
-        if (a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64, true>, g, t, smem, a, R);
-        if (a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32, true>, g, t, smem, a, R);
-        return launch(h->cap, true, k_gemv_q8<MODE, 128, true>, g, t, smem, a, R);
+    if (wf == WF_Q40) {  // gs 32, 64 or 128 (l2c_enable_q40); K an odd multiple of 32 only with gs 32
+        if (a.K % 64) return launch(h->cap, true, k_gemv_q8<MODE, 32, 1>, g, t, smem, a, R);
+        if (a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64, 2>, g, t, smem, a, R);
+        if (a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32, 2>, g, t, smem, a, R);
+        return launch(h->cap, true, k_gemv_q8<MODE, 128, 2>, g, t, smem, a, R);
     }
     const bool k64 = a.K % 64 == 0;
     if (k64 && a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64>, g, t, smem, a, R);
@@ -273,16 +274,16 @@ static int set_smem_limits(l2c_ctx* h) {
     CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     L2C_Q8_ATTR(0) L2C_Q8_ATTR(32) L2C_Q8_ATTR(64) L2C_Q8_ATTR(128)
 #undef L2C_Q8_ATTR
-#define L2C_Q4_ATTR(GS_)                                                                                                \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_QKV, GS_, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID, GS_, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096)); \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_W13, GS_, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
-    CK(max_carveout(k_gemv_q8<M_QKV, GS_, true>));                                                                      \
-    CK(max_carveout(k_gemv_q8<M_RESID, GS_, true>));                                                                    \
-    CK(max_carveout(k_gemv_q8<M_W13, GS_, true>));                                                                      \
-    CK(max_carveout(k_gemv_q8<M_CLS, GS_, true>));
-    L2C_Q4_ATTR(32) L2C_Q4_ATTR(64) L2C_Q4_ATTR(128)
+#define L2C_Q4_ATTR(GS_, W4_)                                                                                           \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_QKV, GS_, W4_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID, GS_, W4_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096)); \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_W13, GS_, W4_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_, W4_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(max_carveout(k_gemv_q8<M_QKV, GS_, W4_>));                                                                      \
+    CK(max_carveout(k_gemv_q8<M_RESID, GS_, W4_>));                                                                    \
+    CK(max_carveout(k_gemv_q8<M_W13, GS_, W4_>));                                                                      \
+    CK(max_carveout(k_gemv_q8<M_CLS, GS_, W4_>));
+    L2C_Q4_ATTR(32, 1) L2C_Q4_ATTR(32, 2) L2C_Q4_ATTR(64, 2) L2C_Q4_ATTR(128, 2)
 #undef L2C_Q4_ATTR
     {
         cudaError_t e = attn_set_smem_limits();
@@ -934,10 +935,12 @@ static int make_q4(l2c_ctx* h, Q8Mat& m, const float* W, size_t rows, int K, boo
     int rc = dalloc(h, (void**)&m.p, rows * m.rb);
     if (rc) return rc;
     CK(cudaMemsetAsync(m.p, 0, rows * m.rb, h->stream));
-    long long groups = (long long)rows * (K / h->gs4);
+    long long groups = (long long)rows * (K / h->gs4);  // warp tasks: at most one per group
     long long blocks = (groups + 7) / 8;
     int grid = (int)(blocks < 65535LL * 16 ? blocks : 65535LL * 16);
-    k_quantize_rows_q4<<<grid, 256, 0, h->stream>>>(W, (long long)rows, K, h->gs4, m.p, m.rb, wide ? 1 : 0);
+    // mode: 1 the Q8_0 layout (embedding); 2 the 64-value chunk layout; 0 the 32-value one
+    const int mode = wide ? 1 : (K % 64 == 0 ? 2 : 0);
+    k_quantize_rows_q4<<<grid, 256, 0, h->stream>>>(W, (long long)rows, K, h->gs4, m.p, m.rb, mode);
     CK(cudaGetLastError());
     return L2C_OK;
 }
