@@ -1009,7 +1009,10 @@ __host__ __device__ inline Q8Smem q8_smem(int ns, uint32_t unit_bytes, int K, in
 template <int MODE, int GS, int W4 = 0>
 __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, const Q8Ring R) {
     extern __shared__ __align__(128) uint8_t smem[];
-    constexpr int UNIT = (MODE == M_QKV || MODE == M_W13) ? 2 : 1;
+    // rows per unit: Q8_0 pairs for QKV and W1/W3 (RoPE / SwiGLU pairs), single rows
+    // otherwise; the 4-bit rows are half the bytes, so a unit takes twice the rows
+    // (more independent dot chains per warp for the same ring bytes)
+    constexpr int UNIT = ((MODE == M_QKV || MODE == M_W13) ? 2 : 1) * (W4 ? 2 : 1);
     __shared__ double red[Q8_WARPS];
     __shared__ unsigned long long best_s[Q8_WARPS];
     __shared__ double2 rope_cs[MODE == M_QKV ? 128 : 1];
@@ -1072,9 +1075,13 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
         }
     }
     if (MODE == M_QKV && a.amax && blockIdx.x == 0 && threadIdx.x == 0) *a.amax = 0ull;
-    // residual: lane j fetches the x of this warp's j-th unit, for the epilogue
-    float xres = 0.f;
-    if (MODE == M_RESID && lane < nmine) xres = __ldcg(a.out + u0 + warp + lane * Q8_WARPS);
+    // residual: lane j fetches the x of this warp's j-th unit (its UNIT rows), for the epilogue
+    float xres = 0.f, xres1 = 0.f;
+    if (MODE == M_RESID && lane < nmine) {
+        const size_t r0 = (size_t)(u0 + warp + lane * Q8_WARPS) * UNIT;
+        xres = __ldcg(a.out + r0);
+        if (UNIT == 2) xres1 = __ldcg(a.out + r0 + 1);
+    }
     if (fast) pro.post(a, eq, es, xq, xsc, red);
     else q8_quantize_input<NORM>(a, eq, es, xq, xsc, red);
     __syncthreads();
@@ -1150,24 +1157,33 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
             mbar_arrive_expect_tx(&full[s], ub);
             bulk_g2s(slots + (size_t)s * ub, unit_src(k + ns), ub, &full[s], pol);
         }
-        const double tot = warp_sum_scatter<UNIT>(acc);  // UNIT = 2: lanes 16..31 hold row 1
+        // lanes [32r/UNIT, 32(r+1)/UNIT) hold the sum of the unit's row r
+        const double tot = warp_sum_scatter<UNIT>(acc);
         const int u = u0 + warp + k * Q8_WARPS;
-        const float xo = MODE == M_RESID ? __shfl_sync(0xffffffffu, xres, k & 31) : 0.f;
-        if (UNIT == 2) {
-            const double odd = __shfl_down_sync(0xffffffffu, tot, 16);
-            if (lane == 0) {
-                if (MODE == M_QKV) epi_qkv(a, u, (float)tot, (float)odd, pos, rope_cs);
-                else epi_w13(a, u, (float)tot, (float)odd);
+        constexpr int LPR = 32 / UNIT;  // lanes per row after the scatter
+        if (MODE == M_QKV || MODE == M_W13) {
+            // pairs (rows 2i, 2i+1): lane 0 (and lane 16 when UNIT = 4) takes one pair
+            const double odd = __shfl_down_sync(0xffffffffu, tot, LPR);
+            if ((lane & (2 * LPR - 1)) == 0) {
+                const int pr = u * (UNIT / 2) + lane / (2 * LPR);
+                if (MODE == M_QKV) epi_qkv(a, pr, (float)tot, (float)odd, pos, rope_cs);
+                else epi_w13(a, pr, (float)tot, (float)odd);
             }
-        } else if (lane == 0) {
-            if (MODE == M_RESID) {
-                a.out[u] = (k < 32 ? xo : __ldcg(a.out + u)) + (float)tot;
-            } else {
-                const float v = (float)tot;
-                a.out[u] = v;
-                if (v != v) set_error(a.err, DERR_NAN);
-                const unsigned long long key = argmax_key(v, u);
-                best = key > best ? key : best;
+        } else {
+            const float xo = MODE == M_RESID ? __shfl_sync(0xffffffffu, xres, k & 31) : 0.f;
+            const float xo1 = MODE == M_RESID && UNIT == 2 ? __shfl_sync(0xffffffffu, xres1, k & 31) : 0.f;
+            if ((lane & (LPR - 1)) == 0) {
+                const int row = u * UNIT + lane / LPR;
+                if (MODE == M_RESID) {
+                    const float x0 = lane == 0 ? xo : xo1;
+                    a.out[row] = (k < 32 ? x0 : __ldcg(a.out + row)) + (float)tot;
+                } else {
+                    const float v = (float)tot;
+                    a.out[row] = v;
+                    if (v != v) set_error(a.err, DERR_NAN);
+                    const unsigned long long key = argmax_key(v, row);
+                    best = key > best ? key : best;
+                }
             }
         }
     }
@@ -1177,6 +1193,10 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
         for (int j = k; j < nmine && j < k + ns; j++)
             if (!(j == 0 && skip0)) mbar_wait_bounded(&full[j % ns], (j / ns) & 1, a.err, a.wait_ns);
     if (MODE == M_CLS) {
+        if (UNIT == 2) {  // lanes 0 and 16 hold keys
+            const unsigned long long o = __shfl_xor_sync(0xffffffffu, best, 16);
+            best = o > best ? o : best;
+        }
         if (lane == 0) best_s[warp] = best;
         __syncthreads();
         if (threadIdx.x == 0) {

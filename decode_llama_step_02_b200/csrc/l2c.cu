@@ -203,6 +203,7 @@ enum WeightFormat : int { WF_F32 = 0, WF_Q80 = 1, WF_Q40 = 2 };
 
 template <int MODE>
 static cudaError_t launch_gemv(l2c_ctx* h, int wf, GemvArgs a, int unit) {
+    if (wf == WF_Q40) unit *= 2;  // the 4-bit GEMV's units: 4 rows for QKV and W1/W3, else 2
     const int units = a.rows / unit;
     a.late_trigger = (h->late_trigger >> (wf != WF_F32 ? 1 : 0)) & 1;
     if (wf == WF_F32) {
@@ -950,6 +951,8 @@ extern "C" int l2c_enable_q40(l2c_ctx* h, int gs) {
     if (h->gs4) return h->gs4 == gs ? L2C_OK : fail(h, L2C_E_STATE, "Q4_0 already enabled with gs=%d", h->gs4);
     if ((gs != 32 && gs != 64 && gs != 128) || h->d % gs || h->h % gs)
         return fail(h, L2C_E_ARG, "Q4_0: gs=%d must be 32, 64 or 128 and divide dim and hidden_dim", gs);
+    if ((h->d + 2 * h->kvd) % 4 || h->V % 2)  // the 4-bit GEMV takes rows 4 (q/k/v) or 2 (classifier) at a time
+        return fail(h, L2C_E_ARG, "Q4_0: dim + 2 * kv_dim must be a multiple of 4 and vocab_size even");
     h->gs4 = gs;
     const size_t d = h->d, hh = h->h, L = h->L, kvd = h->kvd, V = h->V;
     int rc;
