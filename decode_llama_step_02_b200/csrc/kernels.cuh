@@ -1010,8 +1010,9 @@ template <int MODE, int GS, int W4 = 0>
 __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, const Q8Ring R) {
     extern __shared__ __align__(128) uint8_t smem[];
     // rows per unit: Q8_0 pairs for QKV and W1/W3 (RoPE / SwiGLU pairs), single rows
-    // otherwise; the 4-bit rows are half the bytes, so a unit takes twice the rows
-    // (more independent dot chains per warp for the same ring bytes)
+    // otherwise; twice that for the 4-bit rows (half the bytes, so a ring slot of the
+    // same size holds twice the rows) and for Q8_0 rows with W4 = 3: more independent
+    // dot chains per warp
     constexpr int UNIT = ((MODE == M_QKV || MODE == M_W13) ? 2 : 1) * (W4 ? 2 : 1);
     __shared__ double red[Q8_WARPS];
     __shared__ unsigned long long best_s[Q8_WARPS];
@@ -1050,7 +1051,7 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
     const float* es = nullptr;
     if (a.emb) {
         // the embedding rows are Q8_0-layout records (holding 4-bit codes beside Q4_0 weights)
-        const size_t erb = W4 ? (size_t)K + (((size_t)(K / gs) * 4 + 15) & ~size_t(15)) : rb;
+        const size_t erb = (W4 == 1 || W4 == 2) ? (size_t)K + (((size_t)(K / gs) * 4 + 15) & ~size_t(15)) : rb;
         const uint8_t* rec = static_cast<const uint8_t*>(a.emb) + (size_t)token * erb;
         eq = reinterpret_cast<const int8_t*>(rec);
         es = reinterpret_cast<const float*>(rec + K);
@@ -1090,7 +1091,7 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
         __syncthreads();
     }
     int* corr = reinterpret_cast<int*>(smem + lay.sxd);  // Q4_0: 8 * (sum of the input codes) per 32-chunk
-    if (W4) {
+    if (W4 == 1 || W4 == 2) {
         for (int t = threadIdx.x; t < K / 32; t += Q8_THREADS) {
             const int4 c0 = *reinterpret_cast<const int4*>(xq + 32 * t);
             const int4 c1 = *reinterpret_cast<const int4*>(xq + 32 * t + 16);

@@ -102,6 +102,7 @@ struct l2c_ctx {
     int f32_ctas_per_sm = 1;
     size_t q8_smem_budget = 220 << 10;  // dynamic shared memory of one Q8_0 GEMV CTA (its rings)
     int q8_early = 0;    // 1: Q8_0 GEMVs let the next kernel launch as soon as they start (else at their end)
+    int q8_wide_ns = 0;  // > 0: Q8_0 GEMVs take twice the rows per unit where that many ring slots fit
     unsigned long long wait_ns = kWaitNs;  // limit of every bounded wait in the kernels
     int* stall = nullptr;  // test switch read by the Q8_0 q/k/v kernel of layer 0
     long long oom_after = -1;  // test switch: device allocations after this many fail
@@ -226,14 +227,27 @@ static cudaError_t launch_gemv(l2c_ctx* h, int wf, GemvArgs a, int unit) {
         const size_t smem = (size_t)a.K * 4 + (size_t)rows_max * ks * 4;
         return launch(h->cap, true, k_gemv_f32<MODE>, dim3(grid), dim3(F32_THREADS), smem, a, ks);
     }
-    // units of UNIT rows, as many ring slots per warp as fit (2..8)
-    const int grid = h->sms < units ? h->sms : units;
+    // ring slots per warp for units of u rows (0 if none fit the budget)
+    auto slots_for = [&](int u) {
+        const uint32_t ub = (uint32_t)((size_t)u * a.ld);
+        const size_t fixed = q8_smem(0, ub, a.K, a.gs).total;
+        const size_t per = (size_t)Q8_WARPS * (ub + 8);
+        return h->q8_smem_budget > fixed ? (int)((h->q8_smem_budget - fixed) / per) : 0;
+    };
+    // Q8_0 with twice the rows per unit (W4 = 3) where at least q8_wide_ns slots of them fit
+    bool wide = false;
+    if (wf == WF_Q80 && h->q8_wide_ns > 0 && a.K % 64 == 0 && (a.gs == 32 || a.gs == 64 || a.gs == 128) &&
+        a.rows % (2 * unit) == 0 && slots_for(2 * unit) >= h->q8_wide_ns) {
+        wide = true;
+        unit *= 2;
+    }
+    // units of UNIT rows, as many ring slots per warp as fit (2..8; wide Q8_0 units: 1..8)
+    const int units_q = a.rows / unit;
+    const int grid = h->sms < units_q ? h->sms : units_q;
     Q8Ring R = {};
     R.unit_bytes = (uint32_t)((size_t)unit * a.ld);
-    const size_t fixed = q8_smem(0, R.unit_bytes, a.K, a.gs).total;
-    const size_t per = (size_t)Q8_WARPS * (R.unit_bytes + 8);
-    const int ns = h->q8_smem_budget > fixed ? (int)((h->q8_smem_budget - fixed) / per) : 0;
-    R.ns = ns < 2 ? 2 : (ns > 8 ? 8 : ns);
+    const int ns = slots_for(unit), ns_min = wide ? 1 : 2;
+    R.ns = ns < ns_min ? ns_min : (ns > 8 ? 8 : ns);
     const size_t smem = q8_smem(R.ns, R.unit_bytes, a.K, a.gs).total;
     a.early = h->q8_early;
     a.prefetch_bytes = h->pf_q8;
@@ -243,6 +257,11 @@ static cudaError_t launch_gemv(l2c_ctx* h, int wf, GemvArgs a, int unit) {
         if (a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64, 2>, g, t, smem, a, R);
         if (a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32, 2>, g, t, smem, a, R);
         return launch(h->cap, true, k_gemv_q8<MODE, 128, 2>, g, t, smem, a, R);
+    }
+    if (wide) {
+        if (a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64, 3>, g, t, smem, a, R);
+        if (a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32, 3>, g, t, smem, a, R);
+        return launch(h->cap, true, k_gemv_q8<MODE, 128, 3>, g, t, smem, a, R);
     }
     const bool k64 = a.K % 64 == 0;
     if (k64 && a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64>, g, t, smem, a, R);
@@ -285,6 +304,7 @@ static int set_smem_limits(l2c_ctx* h) {
     CK(max_carveout(k_gemv_q8<M_W13, GS_, W4_>));                                                                      \
     CK(max_carveout(k_gemv_q8<M_CLS, GS_, W4_>));
     L2C_Q4_ATTR(32, 1) L2C_Q4_ATTR(32, 2) L2C_Q4_ATTR(64, 2) L2C_Q4_ATTR(128, 2)
+    L2C_Q4_ATTR(32, 3) L2C_Q4_ATTR(64, 3) L2C_Q4_ATTR(128, 3)
 #undef L2C_Q4_ATTR
     {
         cudaError_t e = attn_set_smem_limits();
@@ -760,6 +780,7 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
     h->attn_min_chunk = (int)env_size("L2C_ATTN_MIN_CHUNK", (size_t)h->attn_min_chunk);
     if (h->attn_min_chunk < 1) h->attn_min_chunk = 1;
     h->q8_early = (int)env_size("L2C_Q8_EARLY", (size_t)h->q8_early);
+    h->q8_wide_ns = (int)env_size("L2C_Q8_WIDE_NS", (size_t)h->q8_wide_ns);
     h->bgemm_stages = (int)env_size("L2C_BGEMM_STAGES", (size_t)h->bgemm_stages);
     if (h->bgemm_stages < 2) h->bgemm_stages = 2;
     h->wait_ns = env_size("L2C_WAIT_NS", h->wait_ns);
