@@ -102,7 +102,7 @@ struct l2c_ctx {
     int f32_ctas_per_sm = 1;
     size_t q8_smem_budget = 220 << 10;  // dynamic shared memory of one Q8_0 GEMV CTA (its rings)
     int q8_early = 0;    // 1: Q8_0 GEMVs let the next kernel launch as soon as they start (else at their end)
-    int q8_wide_ns = 0;  // > 0: Q8_0 GEMVs take twice the rows per unit where that many ring slots fit
+    int q8_wide = 1;     // Q8_0 GEMVs take twice the rows per unit where the ring allows (launch_gemv)
     unsigned long long wait_ns = kWaitNs;  // limit of every bounded wait in the kernels
     int* stall = nullptr;  // test switch read by the Q8_0 q/k/v kernel of layer 0
     long long oom_after = -1;  // test switch: device allocations after this many fail
@@ -234,12 +234,20 @@ static cudaError_t launch_gemv(l2c_ctx* h, int wf, GemvArgs a, int unit) {
         const size_t per = (size_t)Q8_WARPS * (ub + 8);
         return h->q8_smem_budget > fixed ? (int)((h->q8_smem_budget - fixed) / per) : 0;
     };
-    // Q8_0 with twice the rows per unit (W4 = 3) where at least q8_wide_ns slots of them fit
+    // Q8_0 with twice the rows per unit (W4 = 3): where two ring slots of them fit, or
+    // one and every warp still gets at least two units (measured on the 7B widths: q/k/v
+    // 17.1 -> 14.4 us, W1/W3 20.5 -> 19.4, wo 8.8 -> 7.6, classifier 30.2 -> 26.6; W2 with
+    // one slot and 1.7 units per warp 14.8 -> 15.9, so it keeps its single rows)
     bool wide = false;
-    if (wf == WF_Q80 && h->q8_wide_ns > 0 && a.K % 64 == 0 && (a.gs == 32 || a.gs == 64 || a.gs == 128) &&
-        a.rows % (2 * unit) == 0 && slots_for(2 * unit) >= h->q8_wide_ns) {
-        wide = true;
-        unit *= 2;
+    if (wf == WF_Q80 && h->q8_wide && a.K % 64 == 0 && (a.gs == 32 || a.gs == 64 || a.gs == 128) &&
+        a.rows % (2 * unit) == 0) {
+        const int ns_w = slots_for(2 * unit);
+        const int units_w = a.rows / (2 * unit);
+        const int warps = (h->sms < units_w ? h->sms : units_w) * Q8_WARPS;
+        if (ns_w >= 2 || (ns_w == 1 && units_w >= 2 * warps)) {
+            wide = true;
+            unit *= 2;
+        }
     }
     // units of UNIT rows, as many ring slots per warp as fit (2..8; wide Q8_0 units: 1..8)
     const int units_q = a.rows / unit;
@@ -780,7 +788,7 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
     h->attn_min_chunk = (int)env_size("L2C_ATTN_MIN_CHUNK", (size_t)h->attn_min_chunk);
     if (h->attn_min_chunk < 1) h->attn_min_chunk = 1;
     h->q8_early = (int)env_size("L2C_Q8_EARLY", (size_t)h->q8_early);
-    h->q8_wide_ns = (int)env_size("L2C_Q8_WIDE_NS", (size_t)h->q8_wide_ns);
+    h->q8_wide = (int)env_size("L2C_Q8_WIDE", (size_t)h->q8_wide);
     h->bgemm_stages = (int)env_size("L2C_BGEMM_STAGES", (size_t)h->bgemm_stages);
     if (h->bgemm_stages < 2) h->bgemm_stages = 2;
     h->wait_ns = env_size("L2C_WAIT_NS", h->wait_ns);
