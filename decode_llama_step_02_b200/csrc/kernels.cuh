@@ -1006,14 +1006,14 @@ __host__ __device__ inline Q8Smem q8_smem(int ns, uint32_t unit_bytes, int K, in
     return m;
 }
 
-template <int MODE, int GS, int W4 = 0>
+template <int MODE, int GS, int W4 = 0, int UM = 1>
 __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, const Q8Ring R) {
     extern __shared__ __align__(128) uint8_t smem[];
-    // rows per unit: Q8_0 pairs for QKV and W1/W3 (RoPE / SwiGLU pairs), single rows
-    // otherwise; twice that for the 4-bit rows (half the bytes, so a ring slot of the
-    // same size holds twice the rows) and for Q8_0 rows with W4 = 3: more independent
-    // dot chains per warp
-    constexpr int UNIT = ((MODE == M_QKV || MODE == M_W13) ? 2 : 1) * (W4 ? 2 : 1);
+    // rows per unit: pairs for QKV and W1/W3 (RoPE / SwiGLU pairs), single rows
+    // otherwise, times UM (1, 2 or 4): more rows per unit give a warp more independent
+    // dot chains for the same ring bytes (the 4-bit rows are half the bytes)
+    constexpr int UNIT = ((MODE == M_QKV || MODE == M_W13) ? 2 : 1) * UM;
+    static_assert(UNIT <= 8, "warp_sum_scatter takes at most 8 rows");
     __shared__ double red[Q8_WARPS];
     __shared__ unsigned long long best_s[Q8_WARPS];
     __shared__ double2 rope_cs[MODE == M_QKV ? 128 : 1];
@@ -1051,7 +1051,7 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
     const float* es = nullptr;
     if (a.emb) {
         // the embedding rows are Q8_0-layout records (holding 4-bit codes beside Q4_0 weights)
-        const size_t erb = (W4 == 1 || W4 == 2) ? (size_t)K + (((size_t)(K / gs) * 4 + 15) & ~size_t(15)) : rb;
+        const size_t erb = W4 ? (size_t)K + (((size_t)(K / gs) * 4 + 15) & ~size_t(15)) : rb;
         const uint8_t* rec = static_cast<const uint8_t*>(a.emb) + (size_t)token * erb;
         eq = reinterpret_cast<const int8_t*>(rec);
         es = reinterpret_cast<const float*>(rec + K);
@@ -1077,11 +1077,14 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
     }
     if (MODE == M_QKV && a.amax && blockIdx.x == 0 && threadIdx.x == 0) *a.amax = 0ull;
     // residual: lane j fetches the x of this warp's j-th unit (its UNIT rows), for the epilogue
-    float xres = 0.f, xres1 = 0.f;
+    constexpr int XR = MODE == M_RESID ? UNIT : 1;
+    float xres[XR];
+#pragma unroll
+    for (int r = 0; r < XR; r++) xres[r] = 0.f;
     if (MODE == M_RESID && lane < nmine) {
         const size_t r0 = (size_t)(u0 + warp + lane * Q8_WARPS) * UNIT;
-        xres = __ldcg(a.out + r0);
-        if (UNIT == 2) xres1 = __ldcg(a.out + r0 + 1);
+#pragma unroll
+        for (int r = 0; r < XR; r++) xres[r] = __ldcg(a.out + r0 + r);
     }
     if (fast) pro.post(a, eq, es, xq, xsc, red);
     else q8_quantize_input<NORM>(a, eq, es, xq, xsc, red);
@@ -1091,7 +1094,7 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
         __syncthreads();
     }
     int* corr = reinterpret_cast<int*>(smem + lay.sxd);  // Q4_0: 8 * (sum of the input codes) per 32-chunk
-    if (W4 == 1 || W4 == 2) {
+    if (W4) {
         for (int t = threadIdx.x; t < K / 32; t += Q8_THREADS) {
             const int4 c0 = *reinterpret_cast<const int4*>(xq + 32 * t);
             const int4 c1 = *reinterpret_cast<const int4*>(xq + 32 * t + 16);
@@ -1171,12 +1174,18 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
                 else epi_w13(a, pr, (float)tot, (float)odd);
             }
         } else {
-            const float xo = MODE == M_RESID ? __shfl_sync(0xffffffffu, xres, k & 31) : 0.f;
-            const float xo1 = MODE == M_RESID && UNIT == 2 ? __shfl_sync(0xffffffffu, xres1, k & 31) : 0.f;
+            // the x of this lane's row (row lane / LPR of the unit)
+            float x0 = 0.f;
+            if (MODE == M_RESID) {
+#pragma unroll
+                for (int r = 0; r < XR; r++) {
+                    const float xr = __shfl_sync(0xffffffffu, xres[r], k & 31);
+                    if (lane / LPR == r) x0 = xr;
+                }
+            }
             if ((lane & (LPR - 1)) == 0) {
                 const int row = u * UNIT + lane / LPR;
                 if (MODE == M_RESID) {
-                    const float x0 = lane == 0 ? xo : xo1;
                     a.out[row] = (k < 32 ? x0 : __ldcg(a.out + row)) + (float)tot;
                 } else {
                     const float v = (float)tot;
@@ -1194,9 +1203,11 @@ __global__ void __launch_bounds__(Q8_THREADS, 1) k_gemv_q8(const GemvArgs a, con
         for (int j = k; j < nmine && j < k + ns; j++)
             if (!(j == 0 && skip0)) mbar_wait_bounded(&full[j % ns], (j / ns) & 1, a.err, a.wait_ns);
     if (MODE == M_CLS) {
-        if (UNIT == 2) {  // lanes 0 and 16 hold keys
-            const unsigned long long o = __shfl_xor_sync(0xffffffffu, best, 16);
-            best = o > best ? o : best;
+        // lanes 0, 32/UNIT, ... hold keys
+#pragma unroll
+        for (int o = 16; o >= 32 / UNIT; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+            best = other > best ? other : best;
         }
         if (lane == 0) best_s[warp] = best;
         __syncthreads();

@@ -103,6 +103,7 @@ struct l2c_ctx {
     size_t q8_smem_budget = 220 << 10;  // dynamic shared memory of one Q8_0 GEMV CTA (its rings)
     int q8_early = 0;    // 1: Q8_0 GEMVs let the next kernel launch as soon as they start (else at their end)
     int q8_wide = 1;     // Q8_0 GEMVs take twice the rows per unit where the ring allows (launch_gemv)
+    int q4_unit4 = 0;    // Q4_0 GEMVs take four times the rows per unit where the ring allows
     unsigned long long wait_ns = kWaitNs;  // limit of every bounded wait in the kernels
     int* stall = nullptr;  // test switch read by the Q8_0 q/k/v kernel of layer 0
     long long oom_after = -1;  // test switch: device allocations after this many fail
@@ -204,7 +205,6 @@ enum WeightFormat : int { WF_F32 = 0, WF_Q80 = 1, WF_Q40 = 2 };
 
 template <int MODE>
 static cudaError_t launch_gemv(l2c_ctx* h, int wf, GemvArgs a, int unit) {
-    if (wf == WF_Q40) unit *= 2;  // the 4-bit GEMV's units: 4 rows for QKV and W1/W3, else 2
     const int units = a.rows / unit;
     a.late_trigger = (h->late_trigger >> (wf != WF_F32 ? 1 : 0)) & 1;
     if (wf == WF_F32) {
@@ -234,13 +234,22 @@ static cudaError_t launch_gemv(l2c_ctx* h, int wf, GemvArgs a, int unit) {
         const size_t per = (size_t)Q8_WARPS * (ub + 8);
         return h->q8_smem_budget > fixed ? (int)((h->q8_smem_budget - fixed) / per) : 0;
     };
-    // Q8_0 with twice the rows per unit (W4 = 3): where two ring slots of them fit, or
+    // Q8_0 with twice the rows per unit (UM = 2): where two ring slots of them fit, or
     // one and every warp still gets at least two units (measured on the 7B widths: q/k/v
     // 17.1 -> 14.4 us, W1/W3 20.5 -> 19.4, wo 8.8 -> 7.6, classifier 30.2 -> 26.6; W2 with
     // one slot and 1.7 units per warp 14.8 -> 15.9, so it keeps its single rows)
     bool wide = false;
-    if (wf == WF_Q80 && h->q8_wide && a.K % 64 == 0 && (a.gs == 32 || a.gs == 64 || a.gs == 128) &&
-        a.rows % (2 * unit) == 0) {
+    int q4um = 2;  // Q4_0: rows per unit times 2, or 4 where the policy below allows
+    if (wf == WF_Q40) {
+        const int ns4 = slots_for(4 * unit);
+        const int units4 = a.rows / (4 * unit);
+        const int warps4 = (h->sms < units4 ? h->sms : units4) * Q8_WARPS;
+        if (h->q4_unit4 && a.K % 64 == 0 && a.rows % (4 * unit) == 0 &&
+            (ns4 >= 2 || (ns4 == 1 && units4 >= 2 * warps4)))
+            q4um = 4;
+        unit *= q4um;
+    } else if (wf == WF_Q80 && h->q8_wide && a.K % 64 == 0 && (a.gs == 32 || a.gs == 64 || a.gs == 128) &&
+               a.rows % (2 * unit) == 0) {
         const int ns_w = slots_for(2 * unit);
         const int units_w = a.rows / (2 * unit);
         const int warps = (h->sms < units_w ? h->sms : units_w) * Q8_WARPS;
@@ -261,15 +270,20 @@ static cudaError_t launch_gemv(l2c_ctx* h, int wf, GemvArgs a, int unit) {
     a.prefetch_bytes = h->pf_q8;
     const dim3 g(grid), t(Q8_THREADS);
     if (wf == WF_Q40) {  // gs 32, 64 or 128 (l2c_enable_q40); K an odd multiple of 32 only with gs 32
-        if (a.K % 64) return launch(h->cap, true, k_gemv_q8<MODE, 32, 1>, g, t, smem, a, R);
-        if (a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64, 2>, g, t, smem, a, R);
-        if (a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32, 2>, g, t, smem, a, R);
-        return launch(h->cap, true, k_gemv_q8<MODE, 128, 2>, g, t, smem, a, R);
+        if (a.K % 64) return launch(h->cap, true, k_gemv_q8<MODE, 32, 1, 2>, g, t, smem, a, R);
+        if (q4um == 4) {
+            if (a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64, 2, 4>, g, t, smem, a, R);
+            if (a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32, 2, 4>, g, t, smem, a, R);
+            return launch(h->cap, true, k_gemv_q8<MODE, 128, 2, 4>, g, t, smem, a, R);
+        }
+        if (a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64, 2, 2>, g, t, smem, a, R);
+        if (a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32, 2, 2>, g, t, smem, a, R);
+        return launch(h->cap, true, k_gemv_q8<MODE, 128, 2, 2>, g, t, smem, a, R);
     }
     if (wide) {
-        if (a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64, 3>, g, t, smem, a, R);
-        if (a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32, 3>, g, t, smem, a, R);
-        return launch(h->cap, true, k_gemv_q8<MODE, 128, 3>, g, t, smem, a, R);
+        if (a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64, 0, 2>, g, t, smem, a, R);
+        if (a.gs == 32) return launch(h->cap, true, k_gemv_q8<MODE, 32, 0, 2>, g, t, smem, a, R);
+        return launch(h->cap, true, k_gemv_q8<MODE, 128, 0, 2>, g, t, smem, a, R);
     }
     const bool k64 = a.K % 64 == 0;
     if (k64 && a.gs == 64) return launch(h->cap, true, k_gemv_q8<MODE, 64>, g, t, smem, a, R);
@@ -302,17 +316,18 @@ static int set_smem_limits(l2c_ctx* h) {
     CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));
     L2C_Q8_ATTR(0) L2C_Q8_ATTR(32) L2C_Q8_ATTR(64) L2C_Q8_ATTR(128)
 #undef L2C_Q8_ATTR
-#define L2C_Q4_ATTR(GS_, W4_)                                                                                           \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_QKV, GS_, W4_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID, GS_, W4_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096)); \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_W13, GS_, W4_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
-    CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_, W4_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
-    CK(max_carveout(k_gemv_q8<M_QKV, GS_, W4_>));                                                                      \
-    CK(max_carveout(k_gemv_q8<M_RESID, GS_, W4_>));                                                                    \
-    CK(max_carveout(k_gemv_q8<M_W13, GS_, W4_>));                                                                      \
-    CK(max_carveout(k_gemv_q8<M_CLS, GS_, W4_>));
-    L2C_Q4_ATTR(32, 1) L2C_Q4_ATTR(32, 2) L2C_Q4_ATTR(64, 2) L2C_Q4_ATTR(128, 2)
-    L2C_Q4_ATTR(32, 3) L2C_Q4_ATTR(64, 3) L2C_Q4_ATTR(128, 3)
+#define L2C_Q4_ATTR(GS_, W4_, UM_)                                                                                           \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_QKV, GS_, W4_, UM_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_RESID, GS_, W4_, UM_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096)); \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_W13, GS_, W4_, UM_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(cudaFuncSetAttribute(k_gemv_q8<M_CLS, GS_, W4_, UM_>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxopt - 4096));   \
+    CK(max_carveout(k_gemv_q8<M_QKV, GS_, W4_, UM_>));                                                                      \
+    CK(max_carveout(k_gemv_q8<M_RESID, GS_, W4_, UM_>));                                                                    \
+    CK(max_carveout(k_gemv_q8<M_W13, GS_, W4_, UM_>));                                                                      \
+    CK(max_carveout(k_gemv_q8<M_CLS, GS_, W4_, UM_>));
+    L2C_Q4_ATTR(32, 1, 2) L2C_Q4_ATTR(32, 2, 2) L2C_Q4_ATTR(64, 2, 2) L2C_Q4_ATTR(128, 2, 2)
+    L2C_Q4_ATTR(32, 2, 4) L2C_Q4_ATTR(64, 2, 4) L2C_Q4_ATTR(128, 2, 4)
+    L2C_Q4_ATTR(32, 0, 2) L2C_Q4_ATTR(64, 0, 2) L2C_Q4_ATTR(128, 0, 2)
 #undef L2C_Q4_ATTR
     {
         cudaError_t e = attn_set_smem_limits();
@@ -789,6 +804,7 @@ extern "C" int l2c_create(const l2c_config* cfg, const float* blob, size_t blob_
     if (h->attn_min_chunk < 1) h->attn_min_chunk = 1;
     h->q8_early = (int)env_size("L2C_Q8_EARLY", (size_t)h->q8_early);
     h->q8_wide = (int)env_size("L2C_Q8_WIDE", (size_t)h->q8_wide);
+    h->q4_unit4 = (int)env_size("L2C_Q4_UNIT4", (size_t)h->q4_unit4);
     h->bgemm_stages = (int)env_size("L2C_BGEMM_STAGES", (size_t)h->bgemm_stages);
     if (h->bgemm_stages < 2) h->bgemm_stages = 2;
     h->wait_ns = env_size("L2C_WAIT_NS", h->wait_ns);
