@@ -713,6 +713,14 @@ def measure_q40(torch, dec, stream, peak, reps=20):
         kern[name] = {"avg_launch_us": 1e3 * kms, "bytes_per_launch": by, "gbs": by / kms / 1e6,
                       "frac_of_measured_hbm": by / kms / 1e6 / peak, "launches_timed": iters}
     out["kernels_pos%d" % kpos] = kern
+    # the Q4_0 W1/W3 kernel against the copy peak (weights at half a byte plus the scales)
+    d, h = SPEC.dim, SPEC.hidden_dim
+    wb = 2 * h * d * (0.5 + 4.0 / GS) + 4.0 * (2 * d + h)
+    avg_ms = kern["rmsnorm_w13_swiglu"]["avg_launch_us"] / 1e3
+    out["roofline_w13"] = {"bound": "hbm", "achieved": wb / avg_ms / 1e6, "peak": peak, "unit": "GB/s",
+                           "frac": wb / avg_ms / 1e6 / peak, "traffic": traffic_record("k_gemv_q8<W13,Q4_0>"),
+                           "kernel": "k_gemv_q8<W13,Q4_0>", "algorithmic_bytes_per_launch": wb,
+                           "avg_launch_ms": avg_ms}
     out["gs"] = GS
     dec.sync()
     return out

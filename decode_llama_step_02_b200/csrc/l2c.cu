@@ -258,12 +258,12 @@ static cudaError_t launch_gemv(l2c_ctx* h, int wf, GemvArgs a, int unit) {
             unit *= 2;
         }
     }
-    // units of UNIT rows, as many ring slots per warp as fit (2..8; wide Q8_0 units: 1..8)
+    // units of UNIT rows, as many ring slots per warp as fit (2..8; the widened units: 1..8)
     const int units_q = a.rows / unit;
     const int grid = h->sms < units_q ? h->sms : units_q;
     Q8Ring R = {};
     R.unit_bytes = (uint32_t)((size_t)unit * a.ld);
-    const int ns = slots_for(unit), ns_min = wide ? 1 : 2;
+    const int ns = slots_for(unit), ns_min = (wide || q4um == 4) ? 1 : 2;
     R.ns = ns < ns_min ? ns_min : (ns > 8 ? 8 : ns);
     const size_t smem = q8_smem(R.ns, R.unit_bytes, a.K, a.gs).total;
     a.early = h->q8_early;
