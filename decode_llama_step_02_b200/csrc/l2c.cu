@@ -103,7 +103,7 @@ struct l2c_ctx {
     size_t q8_smem_budget = 220 << 10;  // dynamic shared memory of one Q8_0 GEMV CTA (its rings)
     int q8_early = 0;    // 1: Q8_0 GEMVs let the next kernel launch as soon as they start (else at their end)
     int q8_wide = 1;     // Q8_0 GEMVs take twice the rows per unit where the ring allows (launch_gemv)
-    int q4_unit4 = 0;    // Q4_0 GEMVs take four times the rows per unit where the ring allows
+    int q4_unit4 = 1;    // Q4_0 GEMVs take four times the rows per unit where the ring allows
     unsigned long long wait_ns = kWaitNs;  // limit of every bounded wait in the kernels
     int* stall = nullptr;  // test switch read by the Q8_0 q/k/v kernel of layer 0
     long long oom_after = -1;  // test switch: device allocations after this many fail
@@ -239,14 +239,12 @@ static cudaError_t launch_gemv(l2c_ctx* h, int wf, GemvArgs a, int unit) {
     // 17.1 -> 14.4 us, W1/W3 20.5 -> 19.4, wo 8.8 -> 7.6, classifier 30.2 -> 26.6; W2 with
     // one slot and 1.7 units per warp 14.8 -> 15.9, so it keeps its single rows)
     bool wide = false;
-    int q4um = 2;  // Q4_0: rows per unit times 2, or 4 where the policy below allows
+    // Q4_0: rows per unit times 2, or 4 where two ring slots of those still fit (on the
+    // 7B widths wo 6.9 -> 6.2 us and the classifier 23.5 -> 18.4; W1/W3 with one slot of
+    // 8 rows measured no faster, so it keeps 4)
+    int q4um = 2;
     if (wf == WF_Q40) {
-        const int ns4 = slots_for(4 * unit);
-        const int units4 = a.rows / (4 * unit);
-        const int warps4 = (h->sms < units4 ? h->sms : units4) * Q8_WARPS;
-        if (h->q4_unit4 && a.K % 64 == 0 && a.rows % (4 * unit) == 0 &&
-            (ns4 >= 2 || (ns4 == 1 && units4 >= 2 * warps4)))
-            q4um = 4;
+        if (h->q4_unit4 && a.K % 64 == 0 && a.rows % (4 * unit) == 0 && slots_for(4 * unit) >= 2) q4um = 4;
         unit *= q4um;
     } else if (wf == WF_Q80 && h->q8_wide && a.K % 64 == 0 && (a.gs == 32 || a.gs == 64 || a.gs == 128) &&
                a.rows % (2 * unit) == 0) {
@@ -263,7 +261,7 @@ static cudaError_t launch_gemv(l2c_ctx* h, int wf, GemvArgs a, int unit) {
     const int grid = h->sms < units_q ? h->sms : units_q;
     Q8Ring R = {};
     R.unit_bytes = (uint32_t)((size_t)unit * a.ld);
-    const int ns = slots_for(unit), ns_min = (wide || q4um == 4) ? 1 : 2;
+    const int ns = slots_for(unit), ns_min = wide ? 1 : 2;
     R.ns = ns < ns_min ? ns_min : (ns > 8 ? 8 : ns);
     const size_t smem = q8_smem(R.ns, R.unit_bytes, a.K, a.gs).total;
     a.early = h->q8_early;
