@@ -970,8 +970,8 @@ struct Q8Ring {
     uint32_t unit_bytes;  // UNIT * record bytes
 };
 
-// Q8_0 GEMV.  A unit is one row record, or a row pair for QKV and W1/W3
-// (UNIT rows); the CTA owns a contiguous range of units and warp w takes its
+// Q8_0 / Q4_0 GEMV.  A unit is UM row records, or UM row pairs for QKV and
+// W1/W3 (UNIT rows); the CTA owns a contiguous range of units and warp w takes its
 // units w, w + 8, ..., streaming them with 1-D bulk copies through its own
 // ring of `ns` shared-memory slots: its parity waits follow its own copies in
 // order, and it refills a slot as soon as it has read it.  Before the
@@ -983,7 +983,9 @@ struct Q8Ring {
 // by dp4a, (ival * sw) * sx summed per lane in double, one reduce-scatter for
 // the unit's row sums, the epilogue.  GS is the group size of the
 // 64-byte-per-lane dot (32, 64 or 128, K % 64 == 0), or 0 for the generic
-// 16-byte-per-lane loop.  Every wait is bounded (a.wait_ns); a warp that gives
+// 16-byte-per-lane loop.  W4 = 0: Q8_0 row records; 1, 2: Q4_0 records in the
+// 32- or 64-value chunk layout (q4_rows_dot32 / q4_rows_dot64), whose input
+// code sums are computed once per CTA after the quantization.  Every wait is bounded (a.wait_ns); a warp that gives
 // up records DERR_TIMEOUT, makes the others stop (a shared abort flag) and
 // lets its copies in flight land before the CTA leaves.  Dynamic shared
 // memory: the rings [Q8_WARPS][ns][unit], the input codes and scales, the
