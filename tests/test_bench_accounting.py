@@ -54,3 +54,23 @@ def test_7b_figures_of_the_plan():
     # one W1/W3 launch: both matrices, gain, input and output
     assert bench.w13_bytes(False, s) / 1e6 == pytest.approx(360.8, abs=0.1)
     assert bench.w13_bytes(True, s) / 1e6 == pytest.approx(95.9, abs=0.1)
+
+
+@pytest.mark.parametrize("gs", [32, 64, 128])
+def test_q40_bytes_are_nibbles_scales_and_fp32_gains(gs):
+    """Q4_0: every matrix and the classifier at half a byte per weight plus an fp32 scale
+    per group; the embedding row in the int8-wide layout (a byte per code); gains fp32."""
+    spec = synth.L7B
+    d, h, L, H, Hkv, V, S = spec.cfg
+    kvd = Hkv * (d // H)
+    gains = L * 2 * d + d
+    mats = _fp32_weight_floats(spec) - gains - d  # without the embedding row
+    want = mats * (0.5 + 4.0 / gs) + d * (1 + 4.0 / gs) + 4.0 * gains + 8.0 * L * 1 * kvd
+    assert bench.q40_bytes_per_token(0, spec, gs) == pytest.approx(want, rel=1e-12)
+    # the kernels' weight bytes (q/k/v, wo, W1/W3, W2 per layer; the classifier) add up to
+    # the step's quantized matrices
+    vec = {0: 4.0 * (2 * d + d + 2 * kvd), 2: 4.0 * 3 * d, 3: 4.0 * (2 * d + h), 4: 4.0 * (h + 2 * d),
+           5: 4.0 * (2 * d + V)}
+    kw = L * sum(bench.kernel_bytes(k, 2, 0, spec, gs) - vec[k] for k in (0, 2, 3, 4))
+    kw += bench.kernel_bytes(5, 2, 0, spec, gs) - vec[5]
+    assert kw == pytest.approx(mats * (0.5 + 4.0 / gs), rel=1e-12)
