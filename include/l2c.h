@@ -111,7 +111,9 @@ L2C_API int l2c_enable_q80(l2c_ctx* h, int gs);
  * max|x| / 7 (fp32) and code = round(x / scale), in [-7, 7].  The same
  * tensors as l2c_enable_q80 (every matvec weight and the embedding table);
  * the GEMVs stream two codes per byte plus one fp32 scale per group.  gs must
- * be 32, 64 or 128 and divide dim and hidden_dim (else L2C_E_ARG).  Calling
+ * be 32, 64 or 128 and divide dim and hidden_dim, dim + 2 * kv_dim must be a
+ * multiple of 4 and vocab_size even (the 4-bit GEMV takes rows in groups of 4
+ * and 2); otherwise L2C_E_ARG.  Calling
  * it again with the same gs is a no-op; another gs gives L2C_E_STATE.
  * L2C_E_OOM if the device memory runs out.  Blocks.
  */
